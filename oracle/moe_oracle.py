@@ -1,0 +1,226 @@
+"""CPU fp64 oracle of the fused MoE expert layer.
+
+TEST INFRASTRUCTURE.  Only the test suite, the package smoke check and the
+benchmark's CPU-baseline leg may import or run this module.  The product path
+(the CUDA library and its Python binding) never calls it, and it shares no
+code with that path: no kernels, helpers, tables or pre/post-processing.
+
+Plain, slow and obviously correct: every step is the definition written out,
+with numpy sort and matmul as the only library primitives.  Floating point is
+fp64 throughout, over the exact fp32 router logits and the exact bf16 values
+of activations and weights.  Nothing is rounded to bf16 on the way.
+
+Sources (web pages on fused MoE kernels):
+
+* "Fused MoE Kernel Optimization" (skillmd, zjli2013/fused-moe-kernel):
+  section "Token-Expert Routing" (top-k gating, sort by expert, pad each
+  expert to a multiple of BLOCK_SIZE_M), "Grouped GEMM Structure"
+  (sorted_token_ids, expert_ids, num_tokens_post_padded), "Verification"
+  (compare against sequential per-expert matmuls with top-k selection) and
+  "Common Pitfalls" (slot // top_k is the token, padding ids are at least
+  num_valid_tokens, [E, N, K] weight layout, top-k weights on the right rows).
+* axolotl vendor-moe diff, src/axolotl/monkeypatch/deepseek_v3/__init__.py,
+  ``_moe_triton_forward``: gate and up projections, ``act_fn(gate) * up``,
+  down projection, then the weighted sum over the k expert outputs.
+* the same diff, scripts/benchmarks/build_deepseek_v3_8b.py ``build_config``:
+  n_group / topk_group grouped routing, norm_topk_prob, routed_scaling_factor
+  and one shared expert.
+* mlxcel PR "perf(moe): preserve squared-ReLU fused MoE kernel behind a
+  dedicated flag", Summary: fc1 -> relu^2 -> fc2 experts with no gate.
+
+Readings where the pages are silent (each is also listed in the design notes):
+
+* Selection key is (logit descending, expert index ascending); softmax is
+  monotone so selecting on logits selects the same set as on probabilities.
+* Group score ``max``: the largest logit of the group.  Group score ``top2``:
+  the sum of the two largest logits of the group, rounded to fp32 (one fp32
+  addition), so that the group choice, an integer decision, is taken in the
+  same precision as the kernel takes it.  Groups are ranked by (score
+  descending, group index ascending).
+* Renormalised weights: softmax over the k chosen logits.  Otherwise: the
+  softmax over all E logits, taken at the chosen experts.  Both are then
+  multiplied by routed_scaling.
+* Align: slots s = t*k + j are sorted by expert, stably (ascending s); each
+  expert's run is padded to a multiple of block_m with the value S = T*k;
+  experts with no slot get no block; unused positions also hold S and unused
+  block ids hold -1.
+* The shared expert is added with weight 1 to every token, unscaled.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+ACT_SWIGLU = 0
+ACT_RELU2 = 1
+GROUP_MAX = 0
+GROUP_TOP2SUM = 1
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact value of bf16 bit patterns (uint16) as fp64."""
+    u32 = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return u32.view(np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# Route
+# --------------------------------------------------------------------------
+
+def _order_desc(values: np.ndarray) -> np.ndarray:
+    """Indices ordered by (value descending, index ascending)."""
+    # A stable sort of the negated values keeps equal values in index order.
+    return np.argsort(-np.asarray(values), kind="stable")
+
+
+def group_scores(l32: np.ndarray, n_group: int, group_score: int) -> np.ndarray:
+    """Score of each contiguous expert group of one token's fp32 logits."""
+    E = l32.shape[0]
+    g = l32.reshape(n_group, E // n_group)
+    if group_score == GROUP_MAX:
+        return g.max(axis=1)
+    if group_score == GROUP_TOP2SUM:
+        srt = np.sort(g, axis=1)[:, ::-1]
+        if srt.shape[1] < 2:
+            return srt[:, 0].astype(np.float32)
+        return (srt[:, 0].astype(np.float32) + srt[:, 1].astype(np.float32)).astype(np.float32)
+    raise ValueError("unknown group score")
+
+
+def route(logits: np.ndarray, k: int, n_group: int = 1, topk_group: int = 1,
+          group_score: int = GROUP_MAX, renormalize: bool = True,
+          routed_scaling: float = 1.0):
+    """Top-k gating over router logits ("Token-Expert Routing", step 1).
+
+    Returns (topk_ids int32 [T,k], topk_weights float64 [T,k]).  ids of a
+    token are listed in selection order (logit descending, index ascending).
+    """
+    logits = np.asarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    assert E % n_group == 0 and 1 <= topk_group <= n_group
+    assert 1 <= k <= (E // n_group) * topk_group
+    assert np.isfinite(logits).all(), "non-finite router logits are unsupported"
+    ids = np.empty((T, k), dtype=np.int32)
+    wts = np.empty((T, k), dtype=np.float64)
+    gsize = E // n_group
+    for t in range(T):
+        l32 = logits[t]
+        l = l32.astype(np.float64)
+        if n_group > 1:
+            gs = group_scores(l32, n_group, group_score)
+            keep_groups = _order_desc(gs)[:topk_group]
+            allowed = np.zeros(E, dtype=bool)
+            for gidx in keep_groups:
+                allowed[gidx * gsize:(gidx + 1) * gsize] = True
+        else:
+            allowed = np.ones(E, dtype=bool)
+        cand = np.nonzero(allowed)[0]                 # ascending expert ids
+        chosen = cand[_order_desc(l[cand])][:k]
+        ids[t] = chosen
+        if renormalize:
+            m = l[chosen].max()
+            e = np.exp(l[chosen] - m)
+            w = e / e.sum()
+        else:
+            m = l.max()
+            p = np.exp(l - m)
+            w = p[chosen] / p.sum()
+        wts[t] = w * float(routed_scaling)
+    return ids, wts
+
+
+# --------------------------------------------------------------------------
+# Align
+# --------------------------------------------------------------------------
+
+def max_padded(T: int, k: int, E: int, block_m: int) -> int:
+    """Worst-case padded length: S + E*(block_m-1), rounded up to block_m."""
+    S = T * k
+    p = S + E * (block_m - 1)
+    return (p + block_m - 1) // block_m * block_m
+
+
+def align(topk_ids: np.ndarray, E: int, block_m: int):
+    """Sort token-slots by expert and pad each expert to block_m.
+
+    "Token-Expert Routing" steps 2-3 and "Grouped GEMM Structure" of the
+    fused-moe-kernel page.  Returns (sorted_token_ids [P_max],
+    expert_ids [P_max/block_m], num_tokens_post_padded (int),
+    inv_pos [S]), all int32 except the count.
+    """
+    ids2 = np.asarray(topk_ids, dtype=np.int64)
+    T, k = ids2.shape
+    flat = ids2.reshape(-1)
+    S = T * k
+    P = max_padded(T, k, E, block_m)
+    sorted_ids = np.full(P, S, dtype=np.int32)
+    expert_ids = np.full(P // block_m, -1, dtype=np.int32)
+    inv_pos = np.full(S, -1, dtype=np.int32)
+    pos = 0
+    for e in range(E):
+        members = np.nonzero(flat == e)[0]        # ascending slot ids
+        n = members.size
+        if n == 0:
+            continue
+        nblk = (n + block_m - 1) // block_m
+        sorted_ids[pos:pos + n] = members
+        inv_pos[members] = pos + np.arange(n)
+        expert_ids[pos // block_m: pos // block_m + nblk] = e
+        pos += nblk * block_m
+    return sorted_ids, expert_ids, pos, inv_pos
+
+
+# --------------------------------------------------------------------------
+# Forward
+# --------------------------------------------------------------------------
+
+def silu(z: np.ndarray) -> np.ndarray:
+    return z / (1.0 + np.exp(-z))
+
+
+def expert_mlp(x: np.ndarray, w13_e: np.ndarray, w2_e: np.ndarray, act: int) -> np.ndarray:
+    """One expert on rows x [n, d] (fp64), weights as bf16 bits.
+
+    SwiGLU: w13_e rows [0, F) are the gate projection, rows [F, 2F) the up
+    projection; h = silu(gate) * up.  Squared ReLU: w13_e is fc1 [F, d] and
+    h = max(fc1 x, 0)^2.  Output: w2_e [d, F] applied to h.
+    """
+    W1 = bf16_to_f64(w13_e)
+    W2 = bf16_to_f64(w2_e)
+    F = W2.shape[1]
+    if act == ACT_SWIGLU:
+        g = x @ W1[:F].T
+        u = x @ W1[F:].T
+        h = silu(g) * u
+    elif act == ACT_RELU2:
+        a = x @ W1.T
+        h = np.maximum(a, 0.0) ** 2
+    else:
+        raise ValueError("unknown activation")
+    return h @ W2.T
+
+
+def forward(x_bits: np.ndarray, w13: np.ndarray, w2: np.ndarray,
+            topk_ids: np.ndarray, topk_weights: np.ndarray, act: int,
+            w13_shared: np.ndarray | None = None,
+            w2_shared: np.ndarray | None = None) -> np.ndarray:
+    """out[t] = sum_j w[t,j] * expert_{ids[t,j]}(x[t])  (+ shared(x[t])).
+
+    Sequential per-expert matmuls with top-k selection ("Verification" of the
+    fused-moe-kernel page); returns fp64 [T, d].
+    """
+    x = bf16_to_f64(x_bits)
+    ids = np.asarray(topk_ids)
+    wts = np.asarray(topk_weights, dtype=np.float64)
+    T, d = x.shape
+    out = np.zeros((T, d), dtype=np.float64)
+    E = w13.shape[0]
+    for e in range(E):
+        t_idx, j_idx = np.nonzero(ids == e)
+        if t_idx.size == 0:
+            continue
+        y = expert_mlp(x[t_idx], w13[e], w2[e], act)
+        np.add.at(out, t_idx, wts[t_idx, j_idx][:, None] * y)
+    if w13_shared is not None:
+        for s in range(w13_shared.shape[0]):
+            out += expert_mlp(x, w13_shared[s], w2_shared[s], act)
+    return out
