@@ -1,0 +1,248 @@
+// Sort token-slots by expert and pad every expert to a multiple of block_m.
+//
+// Steps 2-3 of "Token-Expert Routing" and the indirection arrays of
+// "Grouped GEMM Structure" on the fused-moe-kernel page ("Fused MoE Kernel
+// Optimization", skillmd zjli2013): sorted_token_ids (slot ids s = t*k + j,
+// so that s // top_k is the token, "Common Pitfalls" 1), expert_ids (one
+// expert per block), num_tokens_post_padded, and padding ids equal to
+// S = T*k, i.e. at least num_valid_tokens ("Common Pitfalls" 2).  The
+// per-expert counts rounded up to the alignment and their running offsets
+// play the role of m_sizes / write_offsets in the axolotl vendor-moe diff
+// (src/axolotl/kernels/moe/indices/indices.py, generate_permute_indices),
+// except that an expert with no slot gets no block.
+//
+// The sort is a stable counting sort: within an expert, slots keep their
+// ascending order, so the result is unique and both code paths below give
+// the same bits.
+//   * S <= kSingleBlockMax: one 1024-thread block does histogram, scan,
+//     padding fill and the stable scatter in one launch (decode latency).
+//   * larger S: per-chunk histograms (one block per chunk), one block for
+//     the scan over (expert, chunk), and a per-chunk stable scatter.
+// Within a round of slots, the rank of a slot among equal experts comes from
+// __match_any_sync inside the warp plus an exclusive prefix over the warps.
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kSingleBlockMax = 8192;
+constexpr int kSmallThreads = 1024;
+constexpr int kChunk = 2048;        // slots per chunk on the multi-block path
+constexpr int kChunkThreads = 256;  // threads per chunk block
+
+__device__ __forceinline__ int load_expert(const int32_t* ids, int s, int S, int E, int32_t* status) {
+  if (s >= S) return -1;
+  const int e = ids[s];
+  if (e < 0 || e >= E) {
+    set_status(status, MOE_ERR_BAD_EXPERT_ID);
+    return -1;
+  }
+  return e;
+}
+
+// Exclusive prefix of padded counts over experts, by one warp.  off[E] is
+// the padded total.
+__device__ void warp_padded_scan(const int* cnt, int* off, int E, int bm, int lane) {
+  constexpr int kPer = MOE_MAX_EXPERTS / 32;
+  int local[kPer];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = lane * kPer + i;
+    const int c = e < E ? cnt[e] : 0;
+    local[i] = (c + bm - 1) / bm * bm;
+    sum += local[i];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  int run = incl - sum;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = lane * kPer + i;
+    if (e < E) off[e] = run;
+    run += local[i];
+  }
+  if (lane == 31) off[E] = incl;
+}
+
+// Block b (rows [b*bm, (b+1)*bm)) belongs to the expert e with
+// off[e] <= b*bm < off[e+1]; -1 past the padded total.
+__device__ __forceinline__ int block_expert(const int* off, int E, int p) {
+  if (p >= off[E]) return -1;
+  int lo = 0, hi = E - 1;  // last e with off[e] <= p
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= p)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+// One round of the stable scatter over `nthreads` consecutive slots.  wcnt
+// is [nwarps][E] of zeros on entry and on exit; run[e] is advanced.
+template <int NWARPS>
+__device__ __forceinline__ void scatter_round(int e, int s, int (*wcnt)[MOE_MAX_EXPERTS], int* run, int* tot, int E,
+                                              int32_t* sorted_ids, int32_t* inv_pos) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const unsigned peers = __match_any_sync(0xffffffffu, e);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  if (e >= 0 && rank == 0) wcnt[warp][e] = __popc(peers);
+  __syncthreads();
+  if (threadIdx.x < E) {
+    int acc = 0;
+#pragma unroll 4
+    for (int w = 0; w < NWARPS; ++w) {
+      const int c = wcnt[w][threadIdx.x];
+      wcnt[w][threadIdx.x] = acc;
+      acc += c;
+    }
+    tot[threadIdx.x] = acc;
+  }
+  __syncthreads();
+  if (e >= 0) {
+    const int pos = run[e] + wcnt[warp][e] + rank;
+    sorted_ids[pos] = s;
+    inv_pos[s] = pos;
+  }
+  __syncthreads();
+  if (threadIdx.x < E) {
+    run[threadIdx.x] += tot[threadIdx.x];
+#pragma unroll 4
+    for (int w = 0; w < NWARPS; ++w) wcnt[w][threadIdx.x] = 0;
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSmallThreads)
+    align_single_kernel(const int32_t* __restrict__ ids, int S, int E, int bm, int P_max,
+                        int32_t* __restrict__ sorted_ids, int32_t* __restrict__ expert_ids, int32_t* ntpp,
+                        int32_t* __restrict__ inv_pos, int32_t* status) {
+  constexpr int kWarps = kSmallThreads / 32;
+  __shared__ int cnt[MOE_MAX_EXPERTS];
+  __shared__ int off[MOE_MAX_EXPERTS + 1];
+  __shared__ int run[MOE_MAX_EXPERTS];
+  __shared__ int tot[MOE_MAX_EXPERTS];
+  __shared__ int wcnt[kWarps][MOE_MAX_EXPERTS];
+  const int tid = threadIdx.x;
+  for (int i = tid; i < MOE_MAX_EXPERTS; i += kSmallThreads) cnt[i] = 0;
+  for (int i = tid; i < kWarps * MOE_MAX_EXPERTS; i += kSmallThreads) (&wcnt[0][0])[i] = 0;
+  __syncthreads();
+  for (int s = tid; s < S; s += kSmallThreads) {
+    const int e = load_expert(ids, s, S, E, status);
+    if (e >= 0) atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  if (tid < 32) warp_padded_scan(cnt, off, E, bm, tid);
+  __syncthreads();
+  if (tid < E) run[tid] = off[tid];
+  if (tid == 0) *ntpp = off[E];
+  for (int p = tid; p < P_max; p += kSmallThreads) sorted_ids[p] = S;
+  for (int b = tid; b < P_max / bm; b += kSmallThreads) expert_ids[b] = block_expert(off, E, b * bm);
+  __syncthreads();
+  for (int base = 0; base < S; base += kSmallThreads) {
+    const int s = base + tid;
+    const int e = load_expert(ids, s, S, E, nullptr);
+    scatter_round<kWarps>(e, s, wcnt, run, tot, E, sorted_ids, inv_pos);
+  }
+}
+
+// ---- multi-block path ----------------------------------------------------
+
+__global__ void __launch_bounds__(kChunkThreads)
+    align_count_kernel(const int32_t* __restrict__ ids, int S, int E, int32_t* __restrict__ counts,
+                       int32_t* status) {
+  __shared__ int cnt[MOE_MAX_EXPERTS];
+  const int c = blockIdx.x;
+  for (int i = threadIdx.x; i < E; i += kChunkThreads) cnt[i] = 0;
+  __syncthreads();
+  const int end = min(S, (c + 1) * kChunk);
+  for (int s = c * kChunk + threadIdx.x; s < end; s += kChunkThreads) {
+    const int e = load_expert(ids, s, S, E, status);
+    if (e >= 0) atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < E; i += kChunkThreads) counts[static_cast<size_t>(c) * E + i] = cnt[i];
+}
+
+__global__ void __launch_bounds__(1024)
+    align_scan_kernel(const int32_t* __restrict__ counts, int nchunks, int S, int E, int bm, int P_max,
+                      int32_t* __restrict__ bases, int32_t* __restrict__ sorted_ids,
+                      int32_t* __restrict__ expert_ids, int32_t* ntpp) {
+  __shared__ int cnt[MOE_MAX_EXPERTS];
+  __shared__ int off[MOE_MAX_EXPERTS + 1];
+  const int tid = threadIdx.x;
+  if (tid < E) {
+    int total = 0;
+    for (int c = 0; c < nchunks; ++c) total += counts[static_cast<size_t>(c) * E + tid];
+    cnt[tid] = total;
+  }
+  __syncthreads();
+  if (tid < 32) warp_padded_scan(cnt, off, E, bm, tid);
+  __syncthreads();
+  if (tid < E) {
+    int run = off[tid];
+    for (int c = 0; c < nchunks; ++c) {
+      bases[static_cast<size_t>(c) * E + tid] = run;
+      run += counts[static_cast<size_t>(c) * E + tid];
+    }
+    // padding inside this expert's last block
+    for (int p = off[tid] + cnt[tid]; p < off[tid + 1]; ++p) sorted_ids[p] = S;
+  }
+  if (tid == 0) *ntpp = off[E];
+  for (int p = off[E] + tid; p < P_max; p += blockDim.x) sorted_ids[p] = S;
+  for (int b = tid; b < P_max / bm; b += blockDim.x) expert_ids[b] = block_expert(off, E, b * bm);
+}
+
+__global__ void __launch_bounds__(kChunkThreads)
+    align_scatter_kernel(const int32_t* __restrict__ ids, int S, int E, const int32_t* __restrict__ bases,
+                         int32_t* __restrict__ sorted_ids, int32_t* __restrict__ inv_pos) {
+  constexpr int kWarps = kChunkThreads / 32;
+  __shared__ int run[MOE_MAX_EXPERTS];
+  __shared__ int tot[MOE_MAX_EXPERTS];
+  __shared__ int wcnt[kWarps][MOE_MAX_EXPERTS];
+  const int c = blockIdx.x;
+  for (int i = threadIdx.x; i < E; i += kChunkThreads) run[i] = bases[static_cast<size_t>(c) * E + i];
+  for (int i = threadIdx.x; i < kWarps * MOE_MAX_EXPERTS; i += kChunkThreads) (&wcnt[0][0])[i] = 0;
+  __syncthreads();
+  const int end = min(S, (c + 1) * kChunk);
+  for (int base = c * kChunk; base < end; base += kChunkThreads) {
+    const int s = base + threadIdx.x;
+    const int e = s < end ? load_expert(ids, s, S, E, nullptr) : -1;
+    scatter_round<kWarps>(e, s, wcnt, run, tot, E, sorted_ids, inv_pos);
+  }
+}
+
+}  // namespace
+
+bool align_uses_single_block(int S) { return S <= kSingleBlockMax; }
+
+int align_num_chunks(int S) { return (S + kChunk - 1) / kChunk; }
+
+cudaError_t launch_align(const int32_t* topk_ids, int S, int E, int block_m, int P_max, int32_t* sorted_ids,
+                         int32_t* expert_ids, int32_t* ntpp, int32_t* inv_pos, int32_t* ws, int32_t* status,
+                         cudaStream_t stream, int* launches) {
+  if (align_uses_single_block(S)) {
+    align_single_kernel<<<1, kSmallThreads, 0, stream>>>(topk_ids, S, E, block_m, P_max, sorted_ids, expert_ids,
+                                                         ntpp, inv_pos, status);
+    ++*launches;
+    return cudaGetLastError();
+  }
+  const int nchunks = align_num_chunks(S);
+  int32_t* counts = ws;
+  int32_t* bases = ws + static_cast<size_t>(nchunks) * E;
+  align_count_kernel<<<nchunks, kChunkThreads, 0, stream>>>(topk_ids, S, E, counts, status);
+  align_scan_kernel<<<1, 1024, 0, stream>>>(counts, nchunks, S, E, block_m, P_max, bases, sorted_ids, expert_ids,
+                                            ntpp);
+  align_scatter_kernel<<<nchunks, kChunkThreads, 0, stream>>>(topk_ids, S, E, bases, sorted_ids, inv_pos);
+  *launches += 3;
+  return cudaGetLastError();
+}
+
+}  // namespace moe

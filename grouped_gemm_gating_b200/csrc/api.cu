@@ -1,0 +1,304 @@
+// C ABI of the fused MoE layer: argument checks, workspace layout, TMA
+// tensor-map encoding and the launch sequence.  See include/moe.h for the
+// contract of every entry point.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "common.cuh"
+#include "gemm.h"
+
+namespace {
+
+thread_local int g_last_launches = 0;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int num_sms_current_device() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// bf16 tensor [depth, rows, K] (K innermost) as a 3-D map with 64 x box_rows
+// boxes and 128-byte swizzle; zero fill out of bounds.
+bool encode_3d(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint64_t depth, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {K, rows, depth};
+  const cuuint64_t strides[2] = {K * 2, rows * K * 2};
+  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_2d(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {K, rows};
+  const cuuint64_t strides[1] = {K * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_block_m(int bm) { return bm == 16 || bm == 32 || bm == 64 || bm == 128; }
+
+constexpr size_t kWsAlign = 256;
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int64_t padded_total(int T, int k, int E, int bm, int n_shared) {
+  const int64_t pmax = moe_max_padded(T, k, E, bm);
+  if (pmax < 0) return -1;
+  const int64_t shared_rows = n_shared ? (static_cast<int64_t>(T) + bm - 1) / bm * bm : 0;
+  return pmax + shared_rows;
+}
+
+moe_status check_dims(int T, int d, int F, int E, int k) {
+  if (T < 0 || E < 1 || k < 1 || d < 1 || F < 1) return MOE_ERR_INVALID_ARG;
+  if (k > E) return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  if (d % 64 || F % 64 || d > 16384 || F > 16384) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(T) * k >= (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status finish(cudaError_t err, int launches) {
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t moe_max_padded(int T, int k, int E, int block_m) {
+  if (T < 0 || k < 1 || E < 1 || !valid_block_m(block_m)) return -1;
+  const int64_t S = static_cast<int64_t>(T) * k;
+  const int64_t p = S + static_cast<int64_t>(E) * (block_m - 1);
+  return (p + block_m - 1) / block_m * block_m;
+}
+
+size_t moe_align_workspace_size(int T, int k, int E) {
+  if (T < 0 || k < 1 || E < 1 || E > MOE_MAX_EXPERTS) return 0;
+  const int64_t S = static_cast<int64_t>(T) * k;
+  if (S >= (int64_t(1) << 30)) return 0;
+  if (moe::align_uses_single_block(static_cast<int>(S))) return 0;
+  return static_cast<size_t>(moe::align_num_chunks(static_cast<int>(S))) * E * 2 * sizeof(int32_t);
+}
+
+size_t moe_workspace_size(int T, int d, int F, int E, int k, int block_m, moe_act act, int n_shared) {
+  if (check_dims(T, d, F, E, k) != MOE_OK || !valid_block_m(block_m)) return 0;
+  if ((act != MOE_ACT_SWIGLU && act != MOE_ACT_RELU2) || (n_shared != 0 && n_shared != 1)) return 0;
+  const int64_t P = padded_total(T, k, E, block_m, n_shared);
+  const size_t h = round_up(static_cast<size_t>(P) * F * 2, kWsAlign);
+  const size_t y = round_up(static_cast<size_t>(P) * d * 2, kWsAlign);
+  return h + y + kWsAlign;
+}
+
+moe_status moe_route(const float* logits, int T, int E, int k, int n_group, int topk_group,
+                     moe_group_score group_score, int renormalize, float routed_scaling, int32_t* topk_ids,
+                     float* topk_weights, int32_t* dev_status, moe_stream_t stream) {
+  if (T < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  if (n_group < 1 || E % n_group != 0 || topk_group < 1 || topk_group > n_group) return MOE_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(k) > static_cast<int64_t>(topk_group) * (E / n_group)) return MOE_ERR_INVALID_ARG;
+  if (group_score != MOE_GROUP_MAX && group_score != MOE_GROUP_TOP2SUM) return MOE_ERR_INVALID_ARG;
+  if (!(routed_scaling > 0.0f) || routed_scaling > 3.0e38f) return MOE_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(T) * k >= (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return finish(cudaSuccess, 0);
+  if (!logits || !topk_ids || !topk_weights) return MOE_ERR_INVALID_ARG;
+  int launches = 0;
+  cudaError_t err = moe::launch_route(logits, T, E, k, n_group, topk_group, static_cast<int>(group_score),
+                                      renormalize ? 1 : 0, routed_scaling, topk_ids, topk_weights, dev_status,
+                                      reinterpret_cast<cudaStream_t>(stream), &launches);
+  return finish(err, launches);
+}
+
+moe_status moe_align(const int32_t* topk_ids, int T, int k, int E, int block_m, int32_t* sorted_token_ids,
+                     int32_t* expert_ids, int32_t* num_tokens_post_padded, int32_t* inv_pos, void* ws,
+                     size_t ws_bytes, int32_t* dev_status, moe_stream_t stream) {
+  if (T < 0 || E < 1 || k < 1 || k > E || !valid_block_m(block_m)) return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(T) * k >= (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
+  if (!sorted_token_ids || !expert_ids || !num_tokens_post_padded) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_ids || !inv_pos)) return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_align_workspace_size(T, k, E);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return MOE_ERR_WORKSPACE;
+  const int S = T * k;
+  const int64_t P_max = moe_max_padded(T, k, E, block_m);
+  int launches = 0;
+  cudaError_t err = moe::launch_align(topk_ids, S, E, block_m, static_cast<int>(P_max), sorted_token_ids,
+                                      expert_ids, num_tokens_post_padded, inv_pos, static_cast<int32_t*>(ws),
+                                      dev_status, reinterpret_cast<cudaStream_t>(stream), &launches);
+  return finish(err, launches);
+}
+
+moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, const uint16_t* w2, int E, int F,
+                       const uint16_t* w13_shared, const uint16_t* w2_shared, int n_shared,
+                       const float* topk_weights, int k, const int32_t* sorted_token_ids,
+                       const int32_t* expert_ids, const int32_t* num_tokens_post_padded, const int32_t* inv_pos,
+                       int block_m, moe_act act, uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
+                       moe_stream_t stream) {
+  moe_status st = check_dims(T, d, F, E, k);
+  if (st != MOE_OK) return st;
+  if (!valid_block_m(block_m)) return MOE_ERR_UNSUPPORTED;
+  if (act != MOE_ACT_SWIGLU && act != MOE_ACT_RELU2) return MOE_ERR_INVALID_ARG;
+  if (n_shared != 0 && n_shared != 1) return MOE_ERR_UNSUPPORTED;
+  if (n_shared && (!w13_shared || !w2_shared)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return finish(cudaSuccess, 0);
+  if (!x || !w13 || !w2 || !topk_weights || !sorted_token_ids || !expert_ids || !num_tokens_post_padded ||
+      !inv_pos || !out)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w13) || !aligned16(w2) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (n_shared && (!aligned16(w13_shared) || !aligned16(w2_shared))) return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_workspace_size(T, d, F, E, k, block_m, act, n_shared);
+  if (ws == nullptr || ws_bytes < need) return MOE_ERR_WORKSPACE;
+
+  const int bm = block_m;
+  const int64_t P_max = moe_max_padded(T, k, E, bm);
+  const int64_t P_total = padded_total(T, k, E, bm, n_shared);
+  const int n_shared_blocks = n_shared ? (T + bm - 1) / bm : 0;
+  const int max_routed_blocks = static_cast<int>(P_max / bm);
+  uint8_t* wsb = reinterpret_cast<uint8_t*>(round_up(reinterpret_cast<uintptr_t>(ws), kWsAlign));
+  uint16_t* h = reinterpret_cast<uint16_t*>(wsb);
+  uint16_t* y = reinterpret_cast<uint16_t*>(wsb + round_up(static_cast<size_t>(P_total) * F * 2, kWsAlign));
+  const int n1 = act == MOE_ACT_SWIGLU ? 2 * F : F;
+  const int num_sms = num_sms_current_device();
+  if (num_sms <= 0) return MOE_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int launches = 0;
+
+  // gate/up (or fc1) GEMM with the activation epilogue: h [P_total, F]
+  moe::GemmArgs a1;
+  std::memset(&a1, 0, sizeof(a1));
+  const int epi1 = act == MOE_ACT_SWIGLU ? moe::kEpiSwiGLU : moe::kEpiRelu2;
+  const uint32_t box1 = static_cast<uint32_t>(moe::gemm_box_rows(epi1, bm));
+  if (!encode_3d(&a1.tm_w, w13, d, n1, E, box1)) return MOE_ERR_CUDA;
+  if (n_shared) {
+    if (!encode_3d(&a1.tm_ws, w13_shared, d, n1, 1, box1)) return MOE_ERR_CUDA;
+  } else {
+    a1.tm_ws = a1.tm_w;
+  }
+  a1.x = x;
+  a1.sorted_ids = sorted_token_ids;
+  a1.expert_ids = expert_ids;
+  a1.ntpp = num_tokens_post_padded;
+  a1.topk_w = topk_weights;
+  a1.out = h;
+  a1.status = dev_status;
+  a1.T = T;
+  a1.k = k;
+  a1.S = T * k;
+  a1.E = E;
+  a1.K = d;
+  a1.n_out = F;
+  a1.up_row_offset = F;
+  a1.block_m = bm;
+  a1.max_routed_blocks = max_routed_blocks;
+  a1.n_shared_blocks = n_shared_blocks;
+  int64_t tiles = moe::gemm_max_tiles(epi1, bm, max_routed_blocks, n_shared_blocks, F);
+  int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+  if (grid < 1) grid = 1;
+  cudaError_t err = moe::launch_grouped_gemm(epi1, bm, a1, grid, s);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  ++launches;
+
+  // down GEMM with the top-k weight epilogue: y [P_total, d]
+  moe::GemmArgs a2;
+  std::memset(&a2, 0, sizeof(a2));
+  const uint32_t box2 = static_cast<uint32_t>(moe::gemm_box_rows(moe::kEpiScale, bm));
+  if (!encode_3d(&a2.tm_w, w2, F, d, E, box2)) return MOE_ERR_CUDA;
+  if (n_shared) {
+    if (!encode_3d(&a2.tm_ws, w2_shared, F, d, 1, box2)) return MOE_ERR_CUDA;
+  } else {
+    a2.tm_ws = a2.tm_w;
+  }
+  if (!encode_2d(&a2.tm_x, h, F, static_cast<uint64_t>(P_total), static_cast<uint32_t>(bm))) return MOE_ERR_CUDA;
+  a2.x = nullptr;
+  a2.sorted_ids = sorted_token_ids;
+  a2.expert_ids = expert_ids;
+  a2.ntpp = num_tokens_post_padded;
+  a2.topk_w = topk_weights;
+  a2.out = y;
+  a2.status = dev_status;
+  a2.T = T;
+  a2.k = k;
+  a2.S = T * k;
+  a2.E = E;
+  a2.K = F;
+  a2.n_out = d;
+  a2.up_row_offset = 0;
+  a2.block_m = bm;
+  a2.max_routed_blocks = max_routed_blocks;
+  a2.n_shared_blocks = n_shared_blocks;
+  tiles = moe::gemm_max_tiles(moe::kEpiScale, bm, max_routed_blocks, n_shared_blocks, d);
+  grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+  if (grid < 1) grid = 1;
+  err = moe::launch_grouped_gemm(moe::kEpiScale, bm, a2, grid, s);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  ++launches;
+
+  err = moe::launch_combine(y, inv_pos, num_tokens_post_padded, T, k, d, n_shared, out, s, &launches);
+  return finish(err, launches);
+}
+
+moe_status moe_read_status(const int32_t* dev_status, moe_stream_t stream) {
+  if (dev_status == nullptr) return MOE_ERR_INVALID_ARG;
+  int32_t v = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&v, dev_status, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  return static_cast<moe_status>(v);
+}
+
+const char* moe_status_string(moe_status status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_NONFINITE: return "MOE_ERR_NONFINITE";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+    case MOE_ERR_BAD_EXPERT_ID: return "MOE_ERR_BAD_EXPERT_ID";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+int moe_last_launch_count(void) { return g_last_launches; }
+
+}  // extern "C"

@@ -1,0 +1,48 @@
+// Shared definitions of the CUDA side of the fused MoE layer.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kWarp = 32;
+// Pipeline waits inside a kernel give up after this much wall time, set an
+// error in the status word and let the kernel return (no trap, no hang).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
+  if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+  __nv_bfloat16 v = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&v);
+}
+
+// Internal launchers (one translation unit each).
+cudaError_t launch_route(const float* logits, int T, int E, int k, int n_group, int topk_group, int group_score,
+                         int renormalize, float routed_scaling, int32_t* topk_ids, float* topk_weights,
+                         int32_t* status, cudaStream_t stream, int* launches);
+
+int align_num_chunks(int S);
+bool align_uses_single_block(int S);
+cudaError_t launch_align(const int32_t* topk_ids, int S, int E, int block_m, int P_max, int32_t* sorted_ids,
+                         int32_t* expert_ids, int32_t* ntpp, int32_t* inv_pos, int32_t* ws, int32_t* status,
+                         cudaStream_t stream, int* launches);
+
+cudaError_t launch_combine(const uint16_t* y, const int32_t* inv_pos, const int32_t* ntpp, int T, int k, int d,
+                           int has_shared, uint16_t* out, cudaStream_t stream, int* launches);
+
+}  // namespace moe

@@ -1,0 +1,48 @@
+// Host-visible interface of the tcgen05 grouped GEMM kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace moe {
+
+enum EpiKind : int {
+  kEpiSwiGLU = 0,  // gate/up GEMM, h = silu(gate) * up
+  kEpiRelu2 = 1,   // fc1 GEMM, h = max(a, 0)^2
+  kEpiScale = 2    // down GEMM, y = topk_weight(row) * acc
+};
+
+// Arguments of one grouped GEMM launch.  Rows of the token operand are the
+// padded positions p = blk * block_m + r of the expert-sorted layout; block
+// blk < routed_blocks belongs to expert expert_ids[blk], blocks after that
+// (n_shared_blocks of them) to the shared expert, whose token is
+// (blk - routed_blocks) * block_m + r.
+struct GemmArgs {
+  CUtensorMap tm_w;   // routed expert weights, 3-D {K, rows per expert, E}, 128B swizzle
+  CUtensorMap tm_ws;  // shared expert weights, 3-D {K, rows, 1}
+  CUtensorMap tm_x;   // down GEMM only: h, 2-D {K, P_total}
+  const uint16_t* x;  // gate/up GEMM only: token rows gathered from x [T, K]
+  const int32_t* sorted_ids;
+  const int32_t* expert_ids;
+  const int32_t* ntpp;
+  const float* topk_w;  // [T * k], indexed by slot
+  uint16_t* out;        // [P_total, n_out] bf16
+  int32_t* status;
+  int T, k, S, E;
+  int K;                // reduction length (multiple of 64)
+  int n_out;            // output columns (multiple of 16)
+  int up_row_offset;    // SwiGLU: first up-projection row of an expert (= F)
+  int block_m;
+  int max_routed_blocks;
+  int n_shared_blocks;
+};
+
+// Rows of one weight TMA box and output columns of one tile for a variant.
+int gemm_box_rows(int epi, int block_m);
+// Token rows per tile (== block_m).
+int gemm_token_rows(int block_m);
+// Upper bound on tiles of one launch, for grid sizing.
+int64_t gemm_max_tiles(int epi, int block_m, int max_routed_blocks, int n_shared_blocks, int n_out);
+cudaError_t launch_grouped_gemm(int epi, int block_m, const GemmArgs& args, int grid, cudaStream_t stream);
+
+}  // namespace moe

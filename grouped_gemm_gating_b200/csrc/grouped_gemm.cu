@@ -1,0 +1,483 @@
+// Persistent, warp-specialised grouped GEMM on the 5th-generation tensor
+// cores (tcgen05) of sm_100a, with the MoE epilogues fused in.
+//
+// This is the "Grouped GEMM Structure" of the fused-moe-kernel page ("Fused
+// MoE Kernel Optimization", skillmd zjli2013): a tiled GEMM with an extra
+// indirection, where sorted_token_ids maps each block of block_m rows to
+// token rows, expert_ids maps the block to the expert whose [N, K] weight
+// slice is used, and blocks at or past num_tokens_post_padded do no work.
+// The gate/up projections and `act_fn(gate) * up` of the axolotl
+// `_moe_triton_forward` (src/axolotl/monkeypatch/deepseek_v3/__init__.py) are
+// one GEMM here with the activation in the epilogue; the squared-ReLU fc1 of
+// the mlxcel PR ("fc1 -> relu^2 -> fc2") is the same GEMM with a relu^2
+// epilogue; the down projection applies the top-k weight of each row in its
+// epilogue ("Common Pitfalls" 4: routed weights on the right rows).
+//
+// Two tile forms share this template:
+//  * token-major (block_m = 128): MMA M = 128 token rows, N = 256 weight rows
+//    (SwiGLU: 128 gate rows followed by the matching 128 up rows, so one
+//    thread holds both halves of its h columns).
+//  * weight-major "swap-AB" (block_m = 16..64, few tokens per expert): MMA
+//    M = 128 weight rows, N = block_m token rows; SwiGLU issues one MMA for
+//    the gate rows and one for the up rows into adjacent TMEM columns.
+//
+// Warp roles (one CTA per SM, persistent over a static tile stride):
+//   warp 0       TMA producer: weight tiles (and h tiles for the down GEMM)
+//   warp 1       TMEM allocator and MMA issuer (one thread)
+//   warps 2..5   epilogue: TMEM -> registers -> activation -> bf16 -> global
+//   warps 6..9   gate/up GEMM only: row gather of x through sorted_token_ids
+//                with 16-byte cp.async into the 128B-swizzled layout
+// Shared-memory stages are guarded by full/empty mbarriers, the two TMEM
+// accumulator buffers by tmem-full/tmem-empty mbarriers.  Every wait is
+// bounded in time; on expiry the kernel records MOE_ERR_DEVICE_TIMEOUT and
+// all roles leave their loops so the CTA frees its TMEM and exits.
+#include "common.cuh"
+#include "gemm.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+template <bool SWAP, int EPI, int TOK>
+struct GemmCfg {
+  static constexpr bool kGated = (EPI == kEpiSwiGLU);
+  static constexpr bool kGather = (EPI != kEpiScale);
+  static constexpr int kBoxRows = (!SWAP && !kGated) ? 256 : 128;
+  static constexpr int kBoxes = kGated ? 2 : 1;
+  static constexpr int kWRows = kBoxRows * kBoxes;
+  static constexpr int kOutCols = kBoxRows;
+  static constexpr int kWBytes = kWRows * 128;
+  static constexpr int kXBytes = TOK * 128;
+  static constexpr int kStageBytes = kWBytes + kXBytes;
+  static constexpr int kStagesRaw = (225 * 1024) / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+  static constexpr int kAccCols = SWAP ? (kGated ? 2 * TOK : TOK) : 256;
+  static constexpr int kTmemNeed = 2 * kAccCols;
+  static constexpr int kTmemCols = kTmemNeed <= 32    ? 32
+                                   : kTmemNeed <= 64  ? 64
+                                   : kTmemNeed <= 128 ? 128
+                                   : kTmemNeed <= 256 ? 256
+                                                      : 512;
+  static constexpr int kNumThreads = kGather ? 320 : 192;
+  static constexpr int kGatherLag = 2;
+  static constexpr uint32_t kTxBytes = kWBytes + (kGather ? 0 : kXBytes);
+  static constexpr int kBarrierBytes = 256;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes;
+  static constexpr uint32_t kIdesc = SWAP ? ptx::idesc_bf16_f32(128, TOK) : ptx::idesc_bf16_f32(128, 256);
+
+  static_assert(TOK % 16 == 0 && TOK >= 16 && TOK <= 128, "token rows per tile");
+  static_assert(SWAP || TOK == 128, "token-major tiles hold 128 token rows");
+  static_assert(kStages >= kGatherLag + 2, "pipeline depth");
+  static_assert(kAccCols * 2 <= 512, "two accumulator buffers must fit TMEM");
+  static_assert((2 * kStages + 4) * 8 + 8 <= kBarrierBytes, "barrier area");
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+};
+
+struct TileCoord {
+  int blk, wt;
+  bool shared_blk;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(int tile, int n_wt, int routed_blocks) {
+  TileCoord c;
+  c.blk = tile / n_wt;
+  c.wt = tile - c.blk * n_wt;
+  c.shared_blk = c.blk >= routed_blocks;
+  return c;
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+template <bool SWAP, int EPI, int TOK>
+__global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
+  using C = GemmCfg<SWAP, EPI, TOK>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x / kWarp;
+  const int lane = threadIdx.x % kWarp;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      ptx::mbar_init(&full[s], 1 + (C::kGather ? 128 : 0));
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&tfull[b], 1);
+      ptx::mbar_init(&tempty[b], 4);
+    }
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_holder, C::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  int ntpp = *args.ntpp;
+  int routed_blocks = ntpp / args.block_m;
+  if (routed_blocks < 0) routed_blocks = 0;
+  if (routed_blocks > args.max_routed_blocks) routed_blocks = args.max_routed_blocks;
+  const int total_blocks = routed_blocks + args.n_shared_blocks;
+  const int n_wt = (args.n_out + C::kOutCols - 1) / C::kOutCols;
+  const int total_tiles = total_blocks * n_wt;
+  const int nk = args.K / 64;
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    set_status(args.status, MOE_ERR_DEVICE_TIMEOUT);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&args.tm_w);
+      if (args.n_shared_blocks) ptx::prefetch_tmap(&args.tm_ws);
+      if (!C::kGather) ptx::prefetch_tmap(&args.tm_x);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        const TileCoord tc = tile_coord(tile, n_wt, routed_blocks);
+        const CUtensorMap* tm = tc.shared_blk ? &args.tm_ws : &args.tm_w;
+        int e = 0;
+        if (!tc.shared_blk) {
+          e = args.expert_ids[tc.blk];
+          if (e < 0 || e >= args.E) set_status(args.status, MOE_ERR_BAD_EXPERT_ID);
+        }
+        const int row0 = tc.wt * C::kBoxRows;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+            fail();
+            ok = false;
+            break;
+          }
+          uint8_t* sW = smem + stage * C::kStageBytes;
+          ptx::mbar_arrive_expect_tx(&full[stage], C::kTxBytes);
+          ptx::tma_load_3d(sW, tm, &full[stage], kb * 64, row0, e);
+          if (C::kGated)
+            ptx::tma_load_3d(sW + C::kBoxRows * 128, tm, &full[stage], kb * 64, args.up_row_offset + row0, e);
+          if (!C::kGather) ptx::tma_load_2d(sW + C::kWBytes, &args.tm_x, &full[stage], kb * 64, tc.blk * args.block_m);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int abuf = 0;
+      uint32_t aphase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        if (!ptx::mbar_wait_bounded(&tempty[abuf], aphase ^ 1u, abort_flag, kWaitLimitNs)) {
+          fail();
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * C::kAccCols);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait_bounded(&full[stage], phase, abort_flag, kWaitLimitNs)) {
+            fail();
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sW = ptx::smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t sX = sW + C::kWBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            const uint64_t dw = ptx::sw128_kmajor_desc(sW + kk * 32);
+            const uint64_t dx = ptx::sw128_kmajor_desc(sX + kk * 32);
+            if (!SWAP) {
+              ptx::mma_bf16(d_tmem, dx, dw, C::kIdesc, acc);
+            } else {
+              ptx::mma_bf16(d_tmem, dw, dx, C::kIdesc, acc);
+              if (C::kGated) {
+                const uint64_t du = ptx::sw128_kmajor_desc(sW + C::kBoxRows * 128 + kk * 32);
+                ptx::mma_bf16(d_tmem + TOK, du, dx, C::kIdesc, acc);
+              }
+            }
+          }
+          ptx::mma_commit(&empty[stage]);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        ptx::mma_commit(&tfull[abuf]);
+        if (++abuf == 2) {
+          abuf = 0;
+          aphase ^= 1u;
+        }
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row = q * 32 + lane;
+    int abuf = 0;
+    uint32_t aphase = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      const TileCoord tc = tile_coord(tile, n_wt, routed_blocks);
+      if (!ptx::mbar_wait_bounded(&tfull[abuf], aphase, abort_flag, kWaitLimitNs)) {
+        fail();
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(abuf * C::kAccCols);
+      const int pos0 = tc.blk * args.block_m;
+      if (!SWAP) {
+        // thread = token row `row` of the tile, columns = weight rows
+        const int p = pos0 + row;
+        bool valid;
+        float wrow = 1.0f;
+        if (!tc.shared_blk) {
+          const int slot = args.sorted_ids[p];
+          valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
+          if (EPI == kEpiScale && valid) wrow = args.topk_w[slot];
+        } else {
+          valid = (tc.blk - routed_blocks) * args.block_m + row < args.T;
+        }
+        if (EPI != kEpiScale) valid = true;  // h rows are always written (padding rows are zero)
+        uint16_t* orow = args.out + static_cast<size_t>(p) * args.n_out;
+        if (EPI == kEpiSwiGLU) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < 128; c0 += 16) {
+            uint32_t g[16], u[16];
+            ptx::tmem_ld16(t_acc + c0, g);
+            ptx::tmem_ld16(t_acc + 128 + c0, u);
+            ptx::tmem_wait_ld();
+            const int col = tc.wt * 128 + c0;
+            if (col < args.n_out) {
+              uint32_t pk[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float h0 = silu_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+                const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+                pk[i] = pack_bf16x2(h0, h1);
+              }
+              uint4* dst = reinterpret_cast<uint4*>(orow + col);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int c0 = 0; c0 < 256; c0 += 16) {
+            uint32_t a[16];
+            ptx::tmem_ld16(t_acc + c0, a);
+            ptx::tmem_wait_ld();
+            const int col = tc.wt * 256 + c0;
+            if (col < args.n_out && valid) {
+              uint32_t pk[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                float v0 = __uint_as_float(a[2 * i]), v1 = __uint_as_float(a[2 * i + 1]);
+                if (EPI == kEpiRelu2) {
+                  v0 = fmaxf(v0, 0.0f);
+                  v1 = fmaxf(v1, 0.0f);
+                  v0 *= v0;
+                  v1 *= v1;
+                } else {
+                  v0 *= wrow;
+                  v1 *= wrow;
+                }
+                pk[i] = pack_bf16x2(v0, v1);
+              }
+              uint4* dst = reinterpret_cast<uint4*>(orow + col);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+          }
+        }
+      } else {
+        // thread = weight row `row` (output column), columns = token rows
+        const int col = tc.wt * 128 + row;
+        const bool col_ok = col < args.n_out;
+#pragma unroll 1
+        for (int j0 = 0; j0 < TOK; j0 += 16) {
+          uint32_t a[16], u[16];
+          ptx::tmem_ld16(t_acc + j0, a);
+          if (EPI == kEpiSwiGLU) ptx::tmem_ld16(t_acc + TOK + j0, u);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int p = pos0 + j0 + jj;
+            float v = __uint_as_float(a[jj]);
+            bool valid = true;
+            if (EPI == kEpiSwiGLU) {
+              v = silu_f(v) * __uint_as_float(u[jj]);
+            } else if (EPI == kEpiRelu2) {
+              v = fmaxf(v, 0.0f);
+              v *= v;
+            } else {
+              if (!tc.shared_blk) {
+                const int slot = args.sorted_ids[p];
+                valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
+                v *= valid ? args.topk_w[slot] : 0.0f;
+              } else {
+                valid = (tc.blk - routed_blocks) * args.block_m + j0 + jj < args.T;
+              }
+            }
+            if (col_ok && valid) args.out[static_cast<size_t>(p) * args.n_out + col] = float_to_bf16_bits(v);
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&tempty[abuf]);
+      if (++abuf == 2) {
+        abuf = 0;
+        aphase ^= 1u;
+      }
+    }
+  } else if (C::kGather) {
+    // ------------------------------------------------ row gather of x
+    constexpr int kRowsPerThread = TOK / 16;
+    constexpr int kLag = C::kGatherLag;
+    const int gtid = threadIdx.x - 192;
+    const int chunk = gtid & 7;
+    const int r0 = gtid >> 3;
+    int stage = 0, astage = 0, pend = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      const TileCoord tc = tile_coord(tile, n_wt, routed_blocks);
+      const uint16_t* src[kRowsPerThread];
+      uint32_t nbytes[kRowsPerThread];
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int r = r0 + 16 * i;
+        int tok;
+        bool valid;
+        if (!tc.shared_blk) {
+          const int slot = args.sorted_ids[tc.blk * args.block_m + r];
+          valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
+          tok = valid ? slot / args.k : 0;
+        } else {
+          tok = (tc.blk - routed_blocks) * args.block_m + r;
+          valid = tok < args.T;
+          if (!valid) tok = 0;
+        }
+        src[i] = args.x + static_cast<size_t>(tok) * args.K + chunk * 8;
+        nbytes[i] = valid ? 16u : 0u;
+      }
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+          fail();
+          ok = false;
+          break;
+        }
+        const uint32_t sX = ptx::smem_u32(smem + stage * C::kStageBytes + C::kWBytes);
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          const int r = r0 + 16 * i;
+          const uint32_t dst = sX + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4);
+          ptx::cp_async_16(dst, src[i] + kb * 64, nbytes[i]);
+        }
+        ptx::cp_async_commit();
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        if (++pend > kLag) {
+          ptx::cp_async_wait<kLag>();
+          ptx::fence_proxy_async_smem();
+          ptx::mbar_arrive(&full[astage]);
+          if (++astage == C::kStages) astage = 0;
+          --pend;
+        }
+      }
+    }
+    ptx::cp_async_wait<0>();
+    ptx::fence_proxy_async_smem();
+    for (; pend > 0; --pend) {
+      ptx::mbar_arrive(&full[astage]);
+      if (++astage == C::kStages) astage = 0;
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+namespace {
+
+template <bool SWAP, int EPI, int TOK>
+cudaError_t launch_variant(const GemmArgs& args, int grid, cudaStream_t stream) {
+  using C = GemmCfg<SWAP, EPI, TOK>;
+  auto kern = grouped_gemm_kernel<SWAP, EPI, TOK>;
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_done[dev]) {
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (err != cudaSuccess) return err;
+    attr_done[dev] = true;
+  }
+  kern<<<grid, C::kNumThreads, C::kSmemBytes, stream>>>(args);
+  return cudaGetLastError();
+}
+
+template <bool SWAP, int TOK>
+cudaError_t launch_epi(int epi, const GemmArgs& a, int grid, cudaStream_t s) {
+  switch (epi) {
+    case kEpiSwiGLU: return launch_variant<SWAP, kEpiSwiGLU, TOK>(a, grid, s);
+    case kEpiRelu2: return launch_variant<SWAP, kEpiRelu2, TOK>(a, grid, s);
+    case kEpiScale: return launch_variant<SWAP, kEpiScale, TOK>(a, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+int gemm_token_rows(int block_m) { return block_m; }
+
+int gemm_box_rows(int epi, int block_m) {
+  const bool swap = block_m < 128;
+  const bool gated = epi == kEpiSwiGLU;
+  return (!swap && !gated) ? 256 : 128;
+}
+
+int64_t gemm_max_tiles(int epi, int block_m, int max_routed_blocks, int n_shared_blocks, int n_out) {
+  const int cols = gemm_box_rows(epi, block_m);
+  const int64_t n_wt = (n_out + cols - 1) / cols;
+  return static_cast<int64_t>(max_routed_blocks + n_shared_blocks) * n_wt;
+}
+
+cudaError_t launch_grouped_gemm(int epi, int block_m, const GemmArgs& a, int grid, cudaStream_t s) {
+  switch (block_m) {
+    case 16: return launch_epi<true, 16>(epi, a, grid, s);
+    case 32: return launch_epi<true, 32>(epi, a, grid, s);
+    case 64: return launch_epi<true, 64>(epi, a, grid, s);
+    case 128: return launch_epi<false, 128>(epi, a, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace moe

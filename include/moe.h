@@ -1,0 +1,201 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) fused Mixture-of-Experts expert layer.
+ *
+ * The layer computes, for T tokens x[T, d] and router logits[T, E]:
+ *
+ *   1. moe_route   top-k gating: per token, the k experts with the largest
+ *                  logits (optionally restricted to the topk_group best of
+ *                  n_group contiguous expert groups) and their softmax
+ *                  weights (renormalised over the chosen k, or the full
+ *                  softmax), times routed_scaling.
+ *   2. moe_align   the token-slots s = t*k + j sorted by expert (stable in
+ *                  s), each expert's run padded to a multiple of block_m:
+ *                  sorted_token_ids, expert_ids (one per block of block_m
+ *                  rows), num_tokens_post_padded and the inverse map inv_pos.
+ *   3. moe_forward the grouped gate/up GEMM over [E, N, K] expert weights
+ *                  with a fused SwiGLU or squared-ReLU epilogue, the grouped
+ *                  down GEMM with the top-k weight applied per row, and the
+ *                  weighted scatter-reduce back to out[T, d] (plus an
+ *                  optional always-on shared expert).
+ *
+ * Sources.  "Fused MoE Kernel Optimization" (skillmd zjli2013/fused-moe-
+ * kernel): "Token-Expert Routing" (top-k gating; sort tokens by expert; pad
+ * each expert's count to a multiple of BLOCK_SIZE_M), "Grouped GEMM
+ * Structure" (sorted_token_ids maps blocks to token rows, expert_ids maps
+ * each M-block to its expert, blocks at or past num_tokens_post_padded do no
+ * work) and "Common Pitfalls" (slot // top_k is the token; padding ids are at
+ * least num_valid_tokens; [E, N, K] expert-major weights; top-k weights on
+ * the right rows).  The axolotl vendor-moe diff,
+ * src/axolotl/monkeypatch/deepseek_v3/__init__.py `_moe_triton_forward`
+ * (gate/up GEMMs, act_fn(gate) * up, down GEMM, weighted sum over k) and
+ * scripts/benchmarks/build_deepseek_v3_8b.py `build_config` (n_group,
+ * topk_group, routed_scaling_factor, norm_topk_prob, one shared expert).
+ * The mlxcel PR "perf(moe): preserve squared-ReLU fused MoE kernel behind a
+ * dedicated flag", Summary (fc1 -> relu^2 -> fc2 experts with no gate).
+ *
+ * Conventions for every call.
+ *   - Pointers named `dev`/tensors are DEVICE pointers (cudaMalloc'd or
+ *     torch-owned), row-major, contiguous and 16-byte aligned.  The caller
+ *     owns every buffer; the library allocates nothing and keeps no state
+ *     between calls apart from one-time per-device kernel attribute set-up.
+ *   - bf16 values are passed as raw 16-bit patterns (uint16_t).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and never synchronise the host; device-side results
+ *     such as num_tokens_post_padded stay on the device.
+ *   - Every argument is checked on the host first.  A failed check returns
+ *     an error code and launches nothing.  T == 0 is MOE_OK and a no-op
+ *     (moe_align still writes its padding outputs).
+ *   - `dev_status` (nullable) is one int32 on the device.  Kernels that
+ *     detect an error at run time (non-finite logits, an out-of-range expert
+ *     id, a pipeline wait that exceeded its time limit) store the first such
+ *     code there with an atomic compare-and-swap; they never trap.  Clear it
+ *     to 0 before use; read it with moe_read_status.
+ */
+#ifndef MOE_B200_H_
+#define MOE_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,    /* shape, pointer, alignment or range check failed */
+  MOE_ERR_UNSUPPORTED = 2,    /* valid arguments outside this build's limits */
+  MOE_ERR_WORKSPACE = 3,      /* workspace pointer missing or too small */
+  MOE_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed (launch, attribute, tensor map) */
+  MOE_ERR_NONFINITE = 5,      /* device: a router logit was NaN or infinite */
+  MOE_ERR_DEVICE_TIMEOUT = 6, /* device: a pipeline wait exceeded its time limit; outputs are invalid */
+  MOE_ERR_BAD_EXPERT_ID = 7   /* device: a topk_ids entry was outside [0, E) */
+} moe_status;
+
+typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_RELU2 = 1 } moe_act;
+
+typedef enum {
+  MOE_GROUP_MAX = 0,     /* group score = largest logit in the group */
+  MOE_GROUP_TOP2SUM = 1  /* group score = fp32 sum of the two largest logits in the group */
+} moe_group_score;
+
+/* Limits of this build (checked; MOE_ERR_UNSUPPORTED beyond them):
+ *   1 <= E <= 256, 1 <= k <= min(E, 16), d and F multiples of 64 with
+ *   64 <= d, F <= 16384, block_m in {16, 32, 64, 128}, n_shared in {0, 1},
+ *   T * k < 2^30. */
+#define MOE_MAX_EXPERTS 256
+#define MOE_MAX_TOPK 16
+
+/* Worst-case padded length of sorted_token_ids for (T, k, E, block_m):
+ * P_max = T*k + E*(block_m - 1), rounded up to a multiple of block_m.
+ * Returns -1 on invalid arguments. */
+MOE_API int64_t moe_max_padded(int T, int k, int E, int block_m);
+
+/* Bytes of device scratch moe_align needs (0 when T*k is small enough for
+ * the single-block path).  Returns 0 on invalid arguments. */
+MOE_API size_t moe_align_workspace_size(int T, int k, int E);
+
+/* Bytes of device scratch moe_forward needs: the activation h
+ * [P_total, F] and the scaled expert outputs y [P_total, d], both bf16,
+ * where P_total = P_max + n_shared * ceil(T / block_m) * block_m.
+ * Returns 0 on invalid arguments. */
+MOE_API size_t moe_workspace_size(int T, int d, int F, int E, int k, int block_m,
+                          moe_act act, int n_shared);
+
+/*
+ * moe_route — top-k gating ("Token-Expert Routing", step 1).
+ *   logits        [T, E] fp32, device.
+ *   n_group       number of contiguous expert groups (1 = ungrouped); E % n_group == 0.
+ *   topk_group    groups kept per token, 1 <= topk_group <= n_group;
+ *                 k <= topk_group * E / n_group.
+ *   group_score   how a group is scored (ignored when n_group == 1).
+ *   renormalize   1: softmax over the k chosen logits; 0: full softmax over E.
+ *   routed_scaling multiplies every weight (finite, > 0).
+ *   topk_ids      [T, k] int32 out, device: ids in selection order (logit
+ *                 descending, ties to the lower expert id).
+ *   topk_weights  [T, k] fp32 out, device.
+ * Groups are ranked by (score descending, group index ascending).  Errors:
+ * MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED on the host; MOE_ERR_NONFINITE
+ * in dev_status if a logit is NaN/Inf (outputs then unspecified).
+ */
+MOE_API moe_status moe_route(const float* logits, int T, int E, int k,
+                     int n_group, int topk_group, moe_group_score group_score,
+                     int renormalize, float routed_scaling,
+                     int32_t* topk_ids, float* topk_weights,
+                     int32_t* dev_status, moe_stream_t stream);
+
+/*
+ * moe_align — sort token-slots by expert and pad to block_m ("Token-Expert
+ * Routing" steps 2-3, "Grouped GEMM Structure", "Common Pitfalls" 1-2).
+ *   topk_ids               [T, k] int32, device, values in [0, E).
+ *   sorted_token_ids       [P_max] int32 out: slot ids s = t*k + j grouped by
+ *                          expert (ascending expert, ascending s within an
+ *                          expert); every other entry holds S = T*k.
+ *   expert_ids             [P_max / block_m] int32 out: the expert of each
+ *                          block; -1 for blocks at or past the padded total.
+ *   num_tokens_post_padded [1] int32 out: sum_e ceil(count_e/block_m)*block_m.
+ *   inv_pos                [T*k] int32 out: position of slot s in sorted_token_ids.
+ *   ws, ws_bytes           scratch of moe_align_workspace_size bytes (may be
+ *                          NULL when that size is 0).
+ * Experts with no slot get no block.  Results are unique and deterministic.
+ * An id outside [0, E) sets MOE_ERR_BAD_EXPERT_ID in dev_status.
+ */
+MOE_API moe_status moe_align(const int32_t* topk_ids, int T, int k, int E, int block_m,
+                     int32_t* sorted_token_ids, int32_t* expert_ids,
+                     int32_t* num_tokens_post_padded, int32_t* inv_pos,
+                     void* ws, size_t ws_bytes,
+                     int32_t* dev_status, moe_stream_t stream);
+
+/*
+ * moe_forward — grouped expert GEMMs and weighted scatter-reduce.
+ *   x            [T, d] bf16.
+ *   w13          SwiGLU: [E, 2F, d] bf16, rows [0, F) the gate projection,
+ *                rows [F, 2F) the up projection.  relu^2: [E, F, d] (fc1).
+ *   w2           [E, d, F] bf16 (down projection / fc2).
+ *   w13_shared, w2_shared  the shared expert, same layouts with E = 1
+ *                (required iff n_shared == 1).
+ *   topk_weights [T, k] fp32; sorted_token_ids, expert_ids,
+ *                num_tokens_post_padded, inv_pos: moe_align's outputs for
+ *                the same (T, k, E, block_m).
+ *   out          [T, d] bf16 out:
+ *                out[t] = sum_j topk_weights[t,j] * W2_e (act(W13_e x[t]))
+ *                         (+ shared(x[t]) with weight 1),
+ *                with fp32 accumulation, h and the per-slot scaled outputs
+ *                rounded to bf16, the k-sum in fp32 in slot order.
+ *   ws, ws_bytes scratch of moe_workspace_size bytes.
+ * Errors: host checks as above; MOE_ERR_DEVICE_TIMEOUT in dev_status if a
+ * pipeline wait inside a GEMM kernel exceeded its limit (out is then invalid).
+ */
+MOE_API moe_status moe_forward(const uint16_t* x, int T, int d,
+                       const uint16_t* w13, const uint16_t* w2, int E, int F,
+                       const uint16_t* w13_shared, const uint16_t* w2_shared, int n_shared,
+                       const float* topk_weights, int k,
+                       const int32_t* sorted_token_ids, const int32_t* expert_ids,
+                       const int32_t* num_tokens_post_padded, const int32_t* inv_pos,
+                       int block_m, moe_act act,
+                       uint16_t* out, void* ws, size_t ws_bytes,
+                       int32_t* dev_status, moe_stream_t stream);
+
+/* Synchronises `stream`, then returns the code stored in dev_status (MOE_OK
+ * when 0), or MOE_ERR_CUDA if the synchronisation or the copy failed. */
+MOE_API moe_status moe_read_status(const int32_t* dev_status, moe_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+MOE_API const char* moe_status_string(moe_status status);
+
+/* Number of kernel launches the most recent successful call on this host
+ * thread issued (for launch accounting in benchmarks). */
+MOE_API int moe_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H_ */

@@ -1,0 +1,102 @@
+"""Helpers shared by the GPU parity tests: move seeded inputs to the device,
+run the layer through the C ABI, run the oracle, and compare."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from grouped_gemm_gating_b200 import moe as M
+from grouped_gemm_gating_b200 import workloads as W
+
+# Output tolerance of the layer against the fp64 oracle: max |diff| within
+# 2e-2 * rms(oracle) and relative L2 error within 5e-3.
+OUT_MAX_ABS_REL_RMS = 2e-2
+OUT_REL_L2 = 5e-3
+# Routing weights: fp32 exp, a shuffle-tree sum over <= 256 terms and one
+# division, against fp64: a few ulp of fp32 relative error (see design notes).
+WEIGHT_TOL = 2e-6
+
+
+def bf16_dev(bits: np.ndarray, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def bf16_host(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def route_kwargs(cfg: W.MoEConfig) -> dict:
+    return dict(n_group=cfg.n_group, topk_group=cfg.topk_group, group_score=cfg.group_score,
+                renormalize=bool(cfg.renormalize), routed_scaling=cfg.routed_scaling)
+
+
+def oracle_route(inp: W.MoEInputs):
+    c = inp.cfg
+    return oracle.route(inp.logits, c.k, c.n_group, c.topk_group, c.group_score,
+                        bool(c.renormalize), c.routed_scaling)
+
+
+class DeviceLayer:
+    """Seeded inputs on the device plus the layer's buffers."""
+
+    def __init__(self, inp: W.MoEInputs, device="cuda"):
+        c = inp.cfg
+        self.inp, self.cfg = inp, c
+        self.x = bf16_dev(inp.x, device)
+        self.logits = torch.from_numpy(inp.logits).to(device)
+        self.w13 = bf16_dev(inp.w13, device)
+        self.w2 = bf16_dev(inp.w2, device)
+        self.w13s = bf16_dev(inp.w13_shared, device) if c.n_shared else None
+        self.w2s = bf16_dev(inp.w2_shared, device) if c.n_shared else None
+        self.buf = M.MoEBuffers(c.T, c.d, c.F, c.E, c.k, c.block_m, c.act, c.n_shared, device)
+
+    def run(self, route=True, align=True):
+        b = self.buf
+        if route:
+            b.route(self.logits, **route_kwargs(self.cfg))
+        if align:
+            b.align()
+        return b.forward(self.x, self.w13, self.w2, self.w13s, self.w2s)
+
+    def status(self) -> int:
+        return M.moe_read_status(self.buf.status)
+
+    def h_rows(self) -> np.ndarray:
+        """The activation h [P_total, F] from the forward workspace (fp32)."""
+        c = self.cfg
+        P_total = self.buf.P_max + (c.n_shared * ((c.T + c.block_m - 1) // c.block_m) * c.block_m)
+        base = (self.buf.ws.data_ptr() + 255) // 256 * 256 - self.buf.ws.data_ptr()
+        raw = self.buf.ws[base: base + P_total * c.F * 2].view(torch.int16).reshape(P_total, c.F)
+        return W.bf16_bits_to_f32(raw.cpu().numpy().view(np.uint16))
+
+
+def compare_out(gpu_bits: np.ndarray, ref: np.ndarray, label: str = ""):
+    got = W.bf16_bits_to_f32(gpu_bits).astype(np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.isfinite(got).all(), f"{label}: non-finite output"
+    diff = got - ref
+    rms = float(np.sqrt((ref ** 2).mean()))
+    max_abs = float(np.abs(diff).max()) if diff.size else 0.0
+    rel_l2 = float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300))
+    assert rms > 0.0, f"{label}: degenerate oracle output"
+    assert max_abs <= OUT_MAX_ABS_REL_RMS * rms, f"{label}: max|diff|={max_abs:.3e} > 2e-2*rms={rms:.3e}"
+    assert rel_l2 <= OUT_REL_L2, f"{label}: rel L2={rel_l2:.3e}"
+    return max_abs / rms, rel_l2
+
+
+def compare_route(ids_gpu, w_gpu, ids_ref, w_ref, label=""):
+    assert np.array_equal(ids_gpu, ids_ref), f"{label}: topk_ids differ at {np.argwhere(ids_gpu != ids_ref)[:5]}"
+    tol = WEIGHT_TOL * np.maximum(1.0, np.abs(w_ref))
+    bad = np.abs(w_gpu.astype(np.float64) - w_ref) > tol
+    assert not bad.any(), f"{label}: topk_weights differ at {np.argwhere(bad)[:5]}"
+
+
+def compare_align(buf: M.MoEBuffers, ref, label=""):
+    st, ex, n, inv = ref
+    S = buf.T * buf.k
+    assert int(buf.ntpp.item()) == n, f"{label}: num_tokens_post_padded {buf.ntpp.item()} != {n}"
+    assert np.array_equal(buf.sorted_token_ids.cpu().numpy(), st), f"{label}: sorted_token_ids differ"
+    assert np.array_equal(buf.expert_ids.cpu().numpy(), ex), f"{label}: expert_ids differ"
+    if S:
+        assert np.array_equal(buf.inv_pos.cpu().numpy()[:S], inv), f"{label}: inv_pos differ"

@@ -1,0 +1,238 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Routing ids, align outputs: bit-exact.  Routing weights: within
+WEIGHT_TOL * max(1, |w|).  Layer output: max |diff| <= 2e-2 * rms(oracle)
+and relative L2 <= 5e-3.  Small cases are compared element by element over
+the whole output; the full-size workloads on a seeded sample of tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from grouped_gemm_gating_b200 import moe as M
+from grouped_gemm_gating_b200 import workloads as W
+from moe_testlib import (DeviceLayer, compare_align, compare_out, compare_route, oracle_route,
+                         route_kwargs)
+
+pytestmark = pytest.mark.gpu
+
+CFG = W.CONFIGS
+
+# Reduced versions of every configuration: the oracle finishes them in
+# seconds, yet they span several tiles in both dimensions and ragged tails.
+SMALL = {
+    "tiny": CFG["tiny"],
+    "decode": CFG["decode"],
+    "decode_d512": CFG["decode"].with_(name="decode_d512", d=512, F=384, seed=2002),
+    "relu2_small": CFG["relu2"].with_(name="relu2_small", T=64, E=16, seed=2004),
+    "dsv3_small": CFG["dsv3"].with_(name="dsv3_small", T=300, d=512, F=384, seed=2003),
+    "zipf_small": CFG["zipf"].with_(name="zipf_small", T=1000, d=256, F=192, E=32, seed=2005,
+                                    logits_kind="normal"),
+    "swap_bm32": CFG["tiny"].with_(name="swap_bm32", T=200, d=256, F=320, E=8, k=3, block_m=32, seed=2006,
+                                   logits_kind="normal"),
+    "swap_bm64_relu2": CFG["relu2"].with_(name="swap_bm64_relu2", T=150, d=192, F=192, E=6, k=2, block_m=64,
+                                          seed=2007),
+    "tokm_relu2": CFG["relu2"].with_(name="tokm_relu2", T=333, d=320, F=448, E=5, k=2, block_m=128,
+                                     seed=2008),
+    "one_expert_hot": CFG["tiny"].with_(name="one_expert_hot", T=700, d=128, F=128, E=4, k=1, block_m=128,
+                                        seed=2009, logits_kind="decode_hot"),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    M.load_library()
+
+
+def _full_check(cfg):
+    inp = W.make_inputs(cfg)
+    lay = DeviceLayer(inp)
+    out = lay.run()
+    torch.cuda.synchronize()
+    assert lay.status() == 0, M.status_name(lay.status())
+    ids, w = oracle_route(inp)
+    compare_route(lay.buf.topk_ids.cpu().numpy(), lay.buf.topk_weights.cpu().numpy(), ids, w, cfg.name)
+    compare_align(lay.buf, oracle.align(ids, cfg.E, cfg.block_m), cfg.name)
+    ref = oracle.forward(inp.x, inp.w13, inp.w2, ids, w, cfg.act, inp.w13_shared, inp.w2_shared)
+    return compare_out(M_bits(out), ref, cfg.name)
+
+
+def M_bits(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_layer_small_full_output(name):
+    _full_check(SMALL[name])
+
+
+def test_hidden_activation_matches_oracle():
+    """h rows (first GEMM + activation) checked on their own."""
+    cfg = SMALL["dsv3_small"]
+    inp = W.make_inputs(cfg)
+    lay = DeviceLayer(inp)
+    lay.run()
+    torch.cuda.synchronize()
+    ids, _ = oracle_route(inp)
+    st = lay.buf.sorted_token_ids.cpu().numpy()
+    ex = lay.buf.expert_ids.cpu().numpy()
+    ntpp = int(lay.buf.ntpp.item())
+    h = lay.h_rows()
+    x = oracle.bf16_to_f64(inp.x)
+    S = cfg.T * cfg.k
+    rng = np.random.default_rng(0)
+    for p in rng.choice(ntpp, size=64, replace=False):
+        s = st[p]
+        if s >= S:
+            assert np.all(h[p] == 0.0), "padding rows of h must be zero"
+            continue
+        ref = oracle.expert_hidden(x[s // cfg.k][None, :], inp.w13[ex[p // cfg.block_m]], cfg.act)[0]
+        err = np.abs(h[p] - ref).max()
+        assert err <= 1e-2 * max(np.abs(ref).max(), 1e-3), (p, err)
+    # shared-expert rows follow the routed rows
+    for t in (0, cfg.T - 1):
+        ref = oracle.expert_hidden(x[t][None, :], inp.w13_shared[0], cfg.act)[0]
+        assert np.abs(h[ntpp + t] - ref).max() <= 1e-2 * np.abs(ref).max()
+
+
+# ------------------------------------------------------------ routing -----
+
+@pytest.mark.parametrize("name", list(CFG))
+def test_route_parity_configs(name):
+    cfg = CFG[name]
+    rng_inp = W.make_inputs(cfg.with_(d=64, F=64, E=cfg.E)) if name != "tiny" else W.make_inputs(cfg)
+    lg = rng_inp.logits
+    dev = torch.from_numpy(lg).cuda()
+    ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M.moe_route(dev, cfg.k, ids, w, dev_status=st, **route_kwargs(cfg))
+    assert M.moe_read_status(st) == 0
+    ref = oracle.route(lg, cfg.k, cfg.n_group, cfg.topk_group, cfg.group_score, bool(cfg.renormalize),
+                       cfg.routed_scaling)
+    compare_route(ids.cpu().numpy(), w.cpu().numpy(), *ref, name)
+
+
+@pytest.mark.parametrize("E,k,n_group,topk_group,score,renorm,scale", [
+    (8, 2, 1, 1, 0, 1, 1.0),
+    (16, 4, 4, 2, 0, 1, 2.5),
+    (16, 4, 4, 2, 1, 1, 1.0),
+    (18, 4, 6, 4, 1, 0, 1.0),
+    (64, 6, 8, 3, 0, 0, 1.0),
+    (128, 8, 1, 1, 0, 0, 2.5),
+    (256, 16, 8, 4, 1, 1, 1.0),
+    (256, 8, 256, 8, 0, 1, 1.0),
+    (5, 5, 1, 1, 0, 1, 1.0),
+    (1, 1, 1, 1, 0, 1, 1.0),
+])
+@pytest.mark.parametrize("ties", [False, True])
+def test_route_parity_variants(E, k, n_group, topk_group, score, renorm, scale, ties):
+    T = 333
+    lg = W.tie_logits(T, E, seed=E + k, levels=3) if ties else \
+        np.random.default_rng(E * 7 + k).standard_normal((T, E)).astype(np.float32)
+    dev = torch.from_numpy(lg).cuda()
+    ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    M.moe_route(dev, k, ids, w, n_group, topk_group, score, bool(renorm), scale)
+    ref = oracle.route(lg, k, n_group, topk_group, score, bool(renorm), scale)
+    compare_route(ids.cpu().numpy(), w.cpu().numpy(), *ref, f"E{E}k{k}g{n_group}")
+
+
+def test_route_nonfinite_sets_status():
+    lg = np.zeros((4, 8), np.float32)
+    lg[2, 3] = np.nan
+    ids = torch.empty((4, 2), dtype=torch.int32, device="cuda")
+    w = torch.empty((4, 2), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M.moe_route(torch.from_numpy(lg).cuda(), 2, ids, w, dev_status=st)
+    assert M.moe_read_status(st) == 5
+
+
+# ------------------------------------------------------------- align ------
+
+def _align_gpu(ids_np, E, bm):
+    T, k = ids_np.shape
+    buf = M.MoEBuffers(T, 64, 64, E, k, bm)
+    buf.topk_ids.copy_(torch.from_numpy(ids_np))
+    buf.align()
+    torch.cuda.synchronize()
+    assert M.moe_read_status(buf.status) == 0
+    return buf
+
+
+@pytest.mark.parametrize("bm", [16, 32, 64, 128])
+@pytest.mark.parametrize("T,E,k,skew", [
+    (1, 8, 1, 0.0), (3, 128, 8, 0.0), (256, 128, 6, 0.0), (1024, 8, 8, 3.0), (1023, 256, 8, 0.0),
+    (1025, 256, 8, 50.0), (2048, 128, 8, 0.0), (4096, 18, 4, 0.0), (16384, 128, 8, 5.0),
+    (5000, 32, 3, 0.0),
+])
+def test_align_parity(bm, T, E, k, skew):
+    ids = W.random_topk_ids(T, E, k, seed=T + E + bm, skew=skew)
+    buf = _align_gpu(ids, E, bm)
+    compare_align(buf, oracle.align(ids, E, bm), f"T{T}E{E}k{k}bm{bm}")
+
+
+def test_align_all_slots_one_expert_and_empty():
+    T, E, k, bm = 9000, 64, 1, 128          # multi-chunk path, one expert owns all slots
+    ids = np.full((T, k), 17, np.int32)
+    compare_align(_align_gpu(ids, E, bm), oracle.align(ids, E, bm), "one-expert")
+    ids = np.zeros((0, 4), np.int32)
+    buf = M.MoEBuffers(0, 64, 64, 16, 4, 16)
+    buf.align()
+    torch.cuda.synchronize()
+    compare_align(buf, oracle.align(ids, 16, 16), "empty")
+
+
+def test_align_bad_expert_id_sets_status():
+    ids = np.array([[0, 1], [2, 99]], np.int32)
+    buf = M.MoEBuffers(2, 64, 64, 8, 2, 16)
+    buf.topk_ids.copy_(torch.from_numpy(ids))
+    buf.align()
+    assert M.moe_read_status(buf.status) == 7
+
+
+# -------------------------------------------------------- full size -------
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["decode", "relu2", "dsv3", "zipf"])
+def test_layer_full_size_sampled(name):
+    """Full-size workload in the benchmark's launch configuration; the oracle
+    checks routing and align in full and the output on sampled tokens."""
+    cfg = CFG[name]
+    inp = W.make_inputs(cfg)
+    lay = DeviceLayer(inp)
+    out = lay.run()
+    torch.cuda.synchronize()
+    assert lay.status() == 0, M.status_name(lay.status())
+    ids, w = oracle_route(inp)
+    compare_route(lay.buf.topk_ids.cpu().numpy(), lay.buf.topk_weights.cpu().numpy(), ids, w, name)
+    compare_align(lay.buf, oracle.align(ids, cfg.E, cfg.block_m), name)
+    n = min(cfg.T, 96)
+    sample = np.sort(np.random.default_rng(cfg.seed).choice(cfg.T, size=n, replace=False))
+    ref = oracle.forward(inp.x[sample], inp.w13, inp.w2, ids[sample], w[sample], cfg.act,
+                         inp.w13_shared, inp.w2_shared)
+    compare_out(M_bits(out)[sample], ref, name)
+    if name == "zipf":
+        counts = np.bincount(ids.reshape(-1), minlength=cfg.E)
+        assert (counts == 0).sum() == 8
+
+
+def test_repeated_calls_are_deterministic():
+    cfg = SMALL["zipf_small"]
+    lay = DeviceLayer(W.make_inputs(cfg))
+    a = M_bits(lay.run()).copy()
+    for _ in range(3):
+        b = M_bits(lay.run())
+        assert np.array_equal(a, b)
+
+
+def test_forward_zero_tokens_is_noop():
+    buf = M.MoEBuffers(0, 128, 128, 8, 2, 16)
+    x = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    w13 = torch.zeros((8, 256, 128), dtype=torch.bfloat16, device="cuda")
+    w2 = torch.zeros((8, 128, 128), dtype=torch.bfloat16, device="cuda")
+    buf.align()
+    buf.forward(x, w13, w2)
+    torch.cuda.synchronize()
