@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 fused MoE expert layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole layer over one batch of the workload:
+route (top-k gating) -> align (sort/pad by expert) -> gate/up GEMM with the
+activation epilogue -> down GEMM with the top-k weights -> scatter-reduce.
+Inputs and weights are resident in HBM when the timed region starts; L2 is
+flushed (a buffer of twice the L2 size is written) before every timed step,
+outside the step's events.  Steps are timed with CUDA events on the launch
+stream; every kernel of the step is bracketed by library-recorded events so
+the dominant kernel's duration is measured live over the same region.
+
+Multi-GPU (torchrun, one process per GPU): the layer does not shard, so each
+rank runs an independent replica of the workload ("scaling": "weak"); ranks
+meet at barriers and the slowest rank's time is reported.
+
+--impl reference times the CPU fp64 oracle (test infrastructure) on the host
+cores on a bounded sample of the same workload; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from grouped_gemm_gating_b200 import workloads as W  # noqa: E402
+
+METRIC = "MoE layer TFLOPS and tokens/s on 1 B200; % of bf16 tensor peak / HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+CLOCK_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+# tokens per oracle step for the CPU baseline / reference arm (bounded sample)
+CPU_SAMPLE_TOKENS = {"tiny": 32, "decode": 1, "relu2": 2, "dsv3": 8, "zipf": 8}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="decode", choices=sorted(W.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if a.steps < 1:
+        ap.error("--steps must be at least 1")
+    return a
+
+
+def workload_desc(cfg: W.MoEConfig) -> str:
+    act = "SwiGLU" if cfg.act == W.ACT_SWIGLU else "relu2"
+    s = (f"{cfg.name}: T={cfg.T} d_model={cfg.d} d_ff={cfg.F} E={cfg.E} top_k={cfg.k} {act} "
+         f"block_m={cfg.block_m}")
+    if cfg.n_group > 1:
+        s += f" n_group={cfg.n_group} topk_group={cfg.topk_group}"
+    if cfg.n_shared:
+        s += f" shared_experts={cfg.n_shared}"
+    return s
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic(cfg: W.MoEConfig, topk_ids: np.ndarray):
+    """FLOPs and bytes of the step and of each GEMM launch (no padding, no re-reads)."""
+    S = cfg.T * cfg.k
+    U = int(np.unique(topk_ids).size)
+    rows = S + cfg.T * cfg.n_shared          # rows through the expert GEMMs
+    n_w = U + cfg.n_shared                   # weight matrices read
+    n1 = cfg.n1
+    g1_flops = 2 * rows * n1 * cfg.d
+    g2_flops = 2 * rows * cfg.d * cfg.F
+    g1_bytes = n_w * n1 * cfg.d * 2 + cfg.T * cfg.d * 2 + rows * cfg.F * 2
+    g2_bytes = n_w * cfg.d * cfg.F * 2 + rows * cfg.F * 2 + rows * cfg.d * 4
+    return dict(S=S, U=U, flops_routed=cfg.flops_routed(), flops_total=cfg.flops_total(),
+                gate_up_gemm=(g1_flops, g1_bytes), down_gemm=(g2_flops, g2_bytes),
+                weight_bytes=n_w * (n1 * cfg.d + cfg.d * cfg.F) * 2)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU works."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={CLOCK_QUERY}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, active = [], [], set()
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(CLOCK_REASONS, f[5:9]):
+                if v.lower().startswith("active"):
+                    active.add(name)
+        busy = [s for s in sm if s > 0.5 * max(smax or [1])] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(active), "samples": len(sm)}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_step(inp: W.MoEInputs, tokens: np.ndarray):
+    """One oracle pass (route, align, forward) over the sampled tokens."""
+    import oracle
+    c = inp.cfg
+    lg = inp.logits[tokens]
+    ids, w = oracle.route(lg, c.k, c.n_group, c.topk_group, c.group_score, bool(c.renormalize),
+                          c.routed_scaling)
+    oracle.align(ids, c.E, c.block_m)
+    return oracle.forward(inp.x[tokens], inp.w13, inp.w2, ids, w, c.act, inp.w13_shared, inp.w2_shared)
+
+
+def time_oracle(inp: W.MoEInputs, steps: int, warmup: int, min_seconds: float = 0.0):
+    """Time the oracle on seeded token samples: at least `steps` steps, and
+    more (up to 10x) until `min_seconds` of CPU work has been measured."""
+    c = inp.cfg
+    n = min(c.T, CPU_SAMPLE_TOKENS.get(c.name, 8))
+    rng = np.random.default_rng(c.seed)
+    times = []
+    i = 0
+    while True:
+        tokens = np.sort(rng.choice(c.T, size=n, replace=False))
+        t0 = time.perf_counter()
+        oracle_step(inp, tokens)
+        if i >= warmup:
+            times.append(time.perf_counter() - t0)
+        i += 1
+        if len(times) >= steps and (sum(times) >= min_seconds or len(times) >= 10 * steps):
+            break
+    sec = float(np.mean(times))
+    flops = c.flops_total() * n / c.T
+    return {"value": flops / sec / 1e12, "unit": "TFLOPS", "tokens_per_s": n / sec, "cores": cpu_threads(),
+            "kind": "oracle", "steps": len(times),
+            "sample": f"{n} of {c.T} tokens per step (seeded), {len(times)} steps after {warmup} warm-up "
+                      f"({sum(times):.1f} s); route+align+forward in fp64 numpy"}
+
+
+# --------------------------------------------------------------------------
+
+def dist_setup(gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != gpus:
+        raise SystemExit(f"--gpus {gpus} but WORLD_SIZE={world}")
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local, pg
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+def max_over_ranks(pg, value: float) -> float:
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args):
+    import torch
+
+    from grouped_gemm_gating_b200 import moe as M
+
+    world, rank, local, pg = dist_setup(args.gpus)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    M.load_library()
+    cfg = W.CONFIGS[args.workload]
+    inp = W.make_inputs(cfg)
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    x = to_dev(inp.x)
+    logits = torch.from_numpy(inp.logits).to(dev)
+    w13, w2 = to_dev(inp.w13), to_dev(inp.w2)
+    w13s = to_dev(inp.w13_shared) if cfg.n_shared else None
+    w2s = to_dev(inp.w2_shared) if cfg.n_shared else None
+    buf = M.MoEBuffers(cfg.T, cfg.d, cfg.F, cfg.E, cfg.k, cfg.block_m, cfg.act, cfg.n_shared, dev)
+    rk = dict(n_group=cfg.n_group, topk_group=cfg.topk_group, group_score=cfg.group_score,
+              renormalize=bool(cfg.renormalize), routed_scaling=cfg.routed_scaling)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
+
+    def step(xin, lgin):
+        n = 0
+        buf.route(lgin, **rk)
+        n += M.moe_last_launch_count()
+        buf.align()
+        n += M.moe_last_launch_count()
+        buf.forward(xin, w13, w2, w13s, w2s)
+        n += M.moe_last_launch_count()
+        return n
+
+    stream = torch.cuda.current_stream(dev)
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks.start()
+    for _ in range(args.warmup):
+        step(x, logits)
+    torch.cuda.synchronize(dev)
+    assert M.moe_read_status(buf.status) == 0, "device status set during warm-up"
+    topk_ids = buf.topk_ids.cpu().numpy()
+
+    # ---- device-timed region: inputs resident in HBM ----
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    launches = 0
+    barrier(pg)
+    torch.cuda.synchronize(dev)
+    M.moe_profile_enable(True)
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        launches += step(x, logits)
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(pg)
+    stages = M.moe_profile_collect()
+    M.moe_profile_enable(False)
+    clk = clocks.stop()
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    total_ms = max_over_ranks(pg, total_ms)
+    assert M.moe_read_status(buf.status) == 0, "device status set during the timed region"
+
+    # ---- end to end through the public API with pinned host buffers ----
+    x_h = torch.from_numpy(np.ascontiguousarray(inp.x).view(np.int16)).view(torch.bfloat16).pin_memory()
+    lg_h = torch.from_numpy(inp.logits).pin_memory()
+    out_h = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(x)
+    lg_d = torch.empty_like(logits)
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(pg)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        e_starts[i].record(stream)
+        x_d.copy_(x_h, non_blocking=True)
+        lg_d.copy_(lg_h, non_blocking=True)
+        step(x_d, lg_d)
+        out_h.copy_(buf.out, non_blocking=True)
+        e_ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(pg)
+    e2e_ms = max_over_ranks(pg, sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)))
+    assert torch.equal(out_h.view(torch.int16), buf.out.cpu().view(torch.int16))
+
+    alg = algorithmic(cfg, topk_ids)
+    sec_per_step = total_ms / args.steps / 1e3
+    value = world * alg["flops_total"] / sec_per_step / 1e12
+    e2e_value = world * alg["flops_total"] / (e2e_ms / args.steps / 1e3) / 1e12
+
+    # ---- roofline of the dominant kernel ----
+    peaks, peak_src = load_peaks()
+    dom = max(("gate_up_gemm", "down_gemm"), key=lambda s: stages[s][0])
+    dom_ms, dom_calls = stages[dom]
+    per_launch_s = dom_ms / max(dom_calls, 1) / 1e3
+    fl, by = alg[dom]
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if fl / by >= ridge:
+        achieved = fl / per_launch_s / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "unit": "TFLOP/s"}
+    else:
+        achieved = by / per_launch_s / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "unit": "GB/s"}
+    roof.update({"kernel": dom, "achieved": round(achieved, 2), "peak": peak,
+                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
+                 "frac": round(achieved / peak, 4), "traffic": None,
+                 "per_launch_us": round(per_launch_s * 1e6, 2),
+                 "algorithmic_flops": fl, "algorithmic_bytes": by})
+
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
+        "tokens_per_s": round(world * cfg.T / sec_per_step, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random-init expert weights ~N(0,0.02))",
+        "config": {"workload": workload_desc(cfg), "global_batch": world * cfg.T,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed before every timed step (write of 2x L2)",
+                   "experts_hit": alg["U"], "flops_per_step": alg["flops_total"],
+                   "flops_routed_per_step": alg["flops_routed"]},
+        "stages_us": {k: round(v[0] / max(v[1], 1) * 1e3, 2) for k, v in stages.items()},
+        "roofline": roof,
+        "e2e": {"value": round(e2e_value, 4), "unit": "TFLOPS",
+                "h2d_bytes_per_step": int(inp.x.nbytes + inp.logits.nbytes),
+                "d2h_bytes_per_step": int(cfg.T * cfg.d * 2)},
+        "gpu_launches": int(launches),
+        "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = time_oracle(inp, steps=2, warmup=1, min_seconds=10.0)
+        line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    if pg is not None:
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = W.CONFIGS[args.workload]
+    inp = W.make_inputs(cfg)
+    steps = min(args.steps, 20)
+    warm = min(args.warmup, 3)
+    cb = time_oracle(inp, steps=steps, warmup=warm)
+    steps = cb["steps"]
+    n = min(cfg.T, CPU_SAMPLE_TOKENS.get(cfg.name, 8))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(cb["value"], 6), "unit": "TFLOPS",
+        "n_gpus": world, "steps": steps, "warmup": warm,
+        "ms_per_step": round(n / cb["tokens_per_s"] * 1e3, 3), "tokens_per_s": round(cb["tokens_per_s"], 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": workload_desc(cfg), "global_batch": cfg.T, "parallelism": "host CPU"},
+        "cpu_baseline": {"value": round(cb["value"], 6), "unit": "TFLOPS", "cores": cb["cores"],
+                         "kind": "oracle", "sample": cb["sample"]},
+        "e2e": {"value": round(cb["value"], 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/moe.h"
 #include "common.cuh"
@@ -15,6 +16,39 @@
 namespace {
 
 thread_local int g_last_launches = 0;
+
+// ---- stage profiling: event pairs recorded around each kernel launch ----
+struct StageRecord {
+  int stage;
+  cudaEvent_t start, stop;
+};
+thread_local bool g_profile = false;
+thread_local std::vector<StageRecord> g_records;
+
+struct StageScope {
+  StageRecord rec{};
+  cudaStream_t stream;
+  bool active;
+  StageScope(int stage, cudaStream_t s) : stream(s), active(g_profile) {
+    if (!active) return;
+    rec.stage = stage;
+    if (cudaEventCreate(&rec.start) != cudaSuccess || cudaEventCreate(&rec.stop) != cudaSuccess ||
+        cudaEventRecord(rec.start, stream) != cudaSuccess)
+      active = false;
+  }
+  ~StageScope() {
+    if (!active) return;
+    if (cudaEventRecord(rec.stop, stream) == cudaSuccess) g_records.push_back(rec);
+  }
+};
+
+void release_records() {
+  for (auto& r : g_records) {
+    cudaEventDestroy(r.start);
+    cudaEventDestroy(r.stop);
+  }
+  g_records.clear();
+}
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -125,7 +159,7 @@ size_t moe_workspace_size(int T, int d, int F, int E, int k, int block_m, moe_ac
   if ((act != MOE_ACT_SWIGLU && act != MOE_ACT_RELU2) || (n_shared != 0 && n_shared != 1)) return 0;
   const int64_t P = padded_total(T, k, E, block_m, n_shared);
   const size_t h = round_up(static_cast<size_t>(P) * F * 2, kWsAlign);
-  const size_t y = round_up(static_cast<size_t>(P) * d * 2, kWsAlign);
+  const size_t y = round_up(static_cast<size_t>(P) * d * 4, kWsAlign);
   return h + y + kWsAlign;
 }
 
@@ -142,6 +176,7 @@ moe_status moe_route(const float* logits, int T, int E, int k, int n_group, int 
   if (T == 0) return finish(cudaSuccess, 0);
   if (!logits || !topk_ids || !topk_weights) return MOE_ERR_INVALID_ARG;
   int launches = 0;
+  StageScope scope(0, reinterpret_cast<cudaStream_t>(stream));
   cudaError_t err = moe::launch_route(logits, T, E, k, n_group, topk_group, static_cast<int>(group_score),
                                       renormalize ? 1 : 0, routed_scaling, topk_ids, topk_weights, dev_status,
                                       reinterpret_cast<cudaStream_t>(stream), &launches);
@@ -161,6 +196,7 @@ moe_status moe_align(const int32_t* topk_ids, int T, int k, int E, int block_m, 
   const int S = T * k;
   const int64_t P_max = moe_max_padded(T, k, E, block_m);
   int launches = 0;
+  StageScope scope(1, reinterpret_cast<cudaStream_t>(stream));
   cudaError_t err = moe::launch_align(topk_ids, S, E, block_m, static_cast<int>(P_max), sorted_token_ids,
                                       expert_ids, num_tokens_post_padded, inv_pos, static_cast<int32_t*>(ws),
                                       dev_status, reinterpret_cast<cudaStream_t>(stream), &launches);
@@ -195,7 +231,7 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   const int max_routed_blocks = static_cast<int>(P_max / bm);
   uint8_t* wsb = reinterpret_cast<uint8_t*>(round_up(reinterpret_cast<uintptr_t>(ws), kWsAlign));
   uint16_t* h = reinterpret_cast<uint16_t*>(wsb);
-  uint16_t* y = reinterpret_cast<uint16_t*>(wsb + round_up(static_cast<size_t>(P_total) * F * 2, kWsAlign));
+  float* y = reinterpret_cast<float*>(wsb + round_up(static_cast<size_t>(P_total) * F * 2, kWsAlign));
   const int n1 = act == MOE_ACT_SWIGLU ? 2 * F : F;
   const int num_sms = num_sms_current_device();
   if (num_sms <= 0) return MOE_ERR_CUDA;
@@ -233,11 +269,15 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   int64_t tiles = moe::gemm_max_tiles(epi1, bm, max_routed_blocks, n_shared_blocks, F);
   int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
   if (grid < 1) grid = 1;
-  cudaError_t err = moe::launch_grouped_gemm(epi1, bm, a1, grid, s);
+  cudaError_t err;
+  {
+    StageScope scope(2, s);
+    err = moe::launch_grouped_gemm(epi1, bm, a1, grid, s);
+  }
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   ++launches;
 
-  // down GEMM with the top-k weight epilogue: y [P_total, d]
+  // down GEMM with the top-k weight epilogue: y [P_total, d] fp32
   moe::GemmArgs a2;
   std::memset(&a2, 0, sizeof(a2));
   const uint32_t box2 = static_cast<uint32_t>(moe::gemm_box_rows(moe::kEpiScale, bm));
@@ -268,11 +308,17 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   tiles = moe::gemm_max_tiles(moe::kEpiScale, bm, max_routed_blocks, n_shared_blocks, d);
   grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
   if (grid < 1) grid = 1;
-  err = moe::launch_grouped_gemm(moe::kEpiScale, bm, a2, grid, s);
+  {
+    StageScope scope(3, s);
+    err = moe::launch_grouped_gemm(moe::kEpiScale, bm, a2, grid, s);
+  }
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   ++launches;
 
-  err = moe::launch_combine(y, inv_pos, num_tokens_post_padded, T, k, d, n_shared, out, s, &launches);
+  {
+    StageScope scope(4, s);
+    err = moe::launch_combine(y, inv_pos, num_tokens_post_padded, T, k, d, n_shared, out, s, &launches);
+  }
   return finish(err, launches);
 }
 
@@ -300,5 +346,33 @@ const char* moe_status_string(moe_status status) {
 }
 
 int moe_last_launch_count(void) { return g_last_launches; }
+
+moe_status moe_profile_enable(int on) {
+  release_records();
+  g_profile = on != 0;
+  return MOE_OK;
+}
+
+moe_status moe_profile_collect(double* stage_ms, int* stage_calls, int n_stages) {
+  if (stage_ms == nullptr || n_stages < 0) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n_stages; ++i) {
+    stage_ms[i] = 0.0;
+    if (stage_calls) stage_calls[i] = 0;
+  }
+  moe_status st = MOE_OK;
+  for (auto& r : g_records) {
+    float ms = 0.0f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) {
+      st = MOE_ERR_CUDA;
+      continue;
+    }
+    if (r.stage >= 0 && r.stage < n_stages) {
+      stage_ms[r.stage] += ms;
+      if (stage_calls) ++stage_calls[r.stage];
+    }
+  }
+  release_records();
+  return st;
+}
 
 }  // extern "C"

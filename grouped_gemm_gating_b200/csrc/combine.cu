@@ -2,14 +2,15 @@
 //
 // out[t, :] = sum_{j<k} y[inv_pos[t*k + j], :]  (+ y[ntpp + t, :] for the
 // shared expert), where each y row already carries its top-k weight (applied
-// in the down GEMM epilogue).  This is the final
+// in the down GEMM epilogue; y is fp32).  This is the final
 // `(expert_outputs * topk_weights).sum(dim=1)` of the axolotl
 // `_moe_triton_forward` (src/axolotl/monkeypatch/deepseek_v3/__init__.py)
 // and "Common Pitfalls" 4 of the fused-moe-kernel page (weights on the right
 // rows).  The sum is fp32 in slot order, so the result is deterministic.
 //
-// HBM-bound: each thread moves 16-byte vectors (8 bf16); one block per
-// token row, columns strided over the block.
+// HBM-bound: each thread moves 8 columns (two 16-byte fp32 vectors in per
+// row, one 16-byte bf16 vector out); one block per token row, columns
+// strided over the block.
 #include "common.cuh"
 
 namespace moe {
@@ -19,7 +20,7 @@ namespace {
 constexpr int kCombineThreads = 256;
 
 __global__ void __launch_bounds__(kCombineThreads)
-    combine_kernel(const uint16_t* __restrict__ y, const int32_t* __restrict__ inv_pos,
+    combine_kernel(const float* __restrict__ y, const int32_t* __restrict__ inv_pos,
                    const int32_t* __restrict__ ntpp, int T, int k, int d, int has_shared,
                    uint16_t* __restrict__ out) {
   const int t = blockIdx.x;
@@ -34,13 +35,16 @@ __global__ void __launch_bounds__(kCombineThreads)
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
     for (int r = 0; r < nrows; ++r) {
-      const uint4 q = *reinterpret_cast<const uint4*>(y + static_cast<size_t>(rows[r]) * d + v * 8);
-      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc[2 * i] += __uint_as_float(w[i] << 16);
-        acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
-      }
+      const float4* src = reinterpret_cast<const float4*>(y + static_cast<size_t>(rows[r]) * d + v * 8);
+      const float4 a = src[0], b = src[1];
+      acc[0] += a.x;
+      acc[1] += a.y;
+      acc[2] += a.z;
+      acc[3] += a.w;
+      acc[4] += b.x;
+      acc[5] += b.y;
+      acc[6] += b.z;
+      acc[7] += b.w;
     }
     uint4 o;
     o.x = pack_bf16x2(acc[0], acc[1]);
@@ -53,7 +57,7 @@ __global__ void __launch_bounds__(kCombineThreads)
 
 }  // namespace
 
-cudaError_t launch_combine(const uint16_t* y, const int32_t* inv_pos, const int32_t* ntpp, int T, int k, int d,
+cudaError_t launch_combine(const float* y, const int32_t* inv_pos, const int32_t* ntpp, int T, int k, int d,
                            int has_shared, uint16_t* out, cudaStream_t stream, int* launches) {
   combine_kernel<<<T, kCombineThreads, 0, stream>>>(y, inv_pos, ntpp, T, k, d, has_shared, out);
   ++*launches;

@@ -42,7 +42,7 @@ cudaError_t launch_align(const int32_t* topk_ids, int S, int E, int block_m, int
                          int32_t* expert_ids, int32_t* ntpp, int32_t* inv_pos, int32_t* ws, int32_t* status,
                          cudaStream_t stream, int* launches);
 
-cudaError_t launch_combine(const uint16_t* y, const int32_t* inv_pos, const int32_t* ntpp, int T, int k, int d,
+cudaError_t launch_combine(const float* y, const int32_t* inv_pos, const int32_t* ntpp, int T, int k, int d,
                            int has_shared, uint16_t* out, cudaStream_t stream, int* launches);
 
 }  // namespace moe

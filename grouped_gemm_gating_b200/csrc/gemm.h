@@ -9,7 +9,7 @@ namespace moe {
 enum EpiKind : int {
   kEpiSwiGLU = 0,  // gate/up GEMM, h = silu(gate) * up
   kEpiRelu2 = 1,   // fc1 GEMM, h = max(a, 0)^2
-  kEpiScale = 2    // down GEMM, y = topk_weight(row) * acc
+  kEpiScale = 2    // down GEMM, y = topk_weight(row) * acc, stored fp32
 };
 
 // Arguments of one grouped GEMM launch.  Rows of the token operand are the
@@ -26,7 +26,7 @@ struct GemmArgs {
   const int32_t* expert_ids;
   const int32_t* ntpp;
   const float* topk_w;  // [T * k], indexed by slot
-  uint16_t* out;        // [P_total, n_out] bf16
+  void* out;            // [P_total, n_out]: bf16 h (gate/up GEMM) or fp32 y (down GEMM)
   int32_t* status;
   int T, k, S, E;
   int K;                // reduction length (multiple of 64)

@@ -256,8 +256,8 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
           valid = (tc.blk - routed_blocks) * args.block_m + row < args.T;
         }
         if (EPI != kEpiScale) valid = true;  // h rows are always written (padding rows are zero)
-        uint16_t* orow = args.out + static_cast<size_t>(p) * args.n_out;
         if (EPI == kEpiSwiGLU) {
+          uint16_t* orow = static_cast<uint16_t*>(args.out) + static_cast<size_t>(p) * args.n_out;
 #pragma unroll 1
           for (int c0 = 0; c0 < 128; c0 += 16) {
             uint32_t g[16], u[16];
@@ -278,7 +278,29 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
               dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
           }
+        } else if (EPI == kEpiRelu2) {
+          uint16_t* orow = static_cast<uint16_t*>(args.out) + static_cast<size_t>(p) * args.n_out;
+#pragma unroll 1
+          for (int c0 = 0; c0 < 256; c0 += 16) {
+            uint32_t a[16];
+            ptx::tmem_ld16(t_acc + c0, a);
+            ptx::tmem_wait_ld();
+            const int col = tc.wt * 256 + c0;
+            if (col < args.n_out) {
+              uint32_t pk[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float v0 = fmaxf(__uint_as_float(a[2 * i]), 0.0f);
+                const float v1 = fmaxf(__uint_as_float(a[2 * i + 1]), 0.0f);
+                pk[i] = pack_bf16x2(v0 * v0, v1 * v1);
+              }
+              uint4* dst = reinterpret_cast<uint4*>(orow + col);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+          }
         } else {
+          float* orow = static_cast<float*>(args.out) + static_cast<size_t>(p) * args.n_out;
 #pragma unroll 1
           for (int c0 = 0; c0 < 256; c0 += 16) {
             uint32_t a[16];
@@ -286,24 +308,11 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
             ptx::tmem_wait_ld();
             const int col = tc.wt * 256 + c0;
             if (col < args.n_out && valid) {
-              uint32_t pk[8];
+              float4* dst = reinterpret_cast<float4*>(orow + col);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                float v0 = __uint_as_float(a[2 * i]), v1 = __uint_as_float(a[2 * i + 1]);
-                if (EPI == kEpiRelu2) {
-                  v0 = fmaxf(v0, 0.0f);
-                  v1 = fmaxf(v1, 0.0f);
-                  v0 *= v0;
-                  v1 *= v1;
-                } else {
-                  v0 *= wrow;
-                  v1 *= wrow;
-                }
-                pk[i] = pack_bf16x2(v0, v1);
-              }
-              uint4* dst = reinterpret_cast<uint4*>(orow + col);
-              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_float4(__uint_as_float(a[4 * i]) * wrow, __uint_as_float(a[4 * i + 1]) * wrow,
+                                     __uint_as_float(a[4 * i + 2]) * wrow, __uint_as_float(a[4 * i + 3]) * wrow);
             }
           }
         }
@@ -336,7 +345,13 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
                 valid = (tc.blk - routed_blocks) * args.block_m + j0 + jj < args.T;
               }
             }
-            if (col_ok && valid) args.out[static_cast<size_t>(p) * args.n_out + col] = float_to_bf16_bits(v);
+            if (col_ok && valid) {
+              const size_t idx = static_cast<size_t>(p) * args.n_out + col;
+              if (EPI == kEpiScale)
+                static_cast<float*>(args.out)[idx] = v;
+              else
+                static_cast<uint16_t*>(args.out)[idx] = float_to_bf16_bits(v);
+            }
           }
         }
       }

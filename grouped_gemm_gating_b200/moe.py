@@ -43,7 +43,11 @@ _SIG = {
     "moe_read_status": (_I, [_P, _P]),
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_last_launch_count": (_I, []),
+    "moe_profile_enable": (_I, [_I]),
+    "moe_profile_collect": (_I, [_P, _P, _I]),
 }
+
+STAGES = ("route", "align", "gate_up_gemm", "down_gemm", "combine")
 
 _lib = None
 _lock = threading.Lock()
@@ -122,6 +126,20 @@ def moe_workspace_size(T, d, F, E, k, block_m, act, n_shared) -> int:
 
 def moe_last_launch_count() -> int:
     return int(load_library().moe_last_launch_count())
+
+
+def moe_profile_enable(on: bool = True) -> None:
+    """Start (or stop) recording CUDA events around every kernel launch."""
+    _check("moe_profile_enable", load_library().moe_profile_enable(1 if on else 0))
+
+
+def moe_profile_collect() -> dict:
+    """Summed milliseconds and launch counts per stage since enable; clears."""
+    n = len(STAGES)
+    ms = (ctypes.c_double * n)()
+    calls = (ctypes.c_int * n)()
+    _check("moe_profile_collect", load_library().moe_profile_collect(ms, calls, n))
+    return {name: (float(ms[i]), int(calls[i])) for i, name in enumerate(STAGES)}
 
 
 # ---------------------------------------------------------------- calls ---

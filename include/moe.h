@@ -104,7 +104,7 @@ MOE_API int64_t moe_max_padded(int T, int k, int E, int block_m);
 MOE_API size_t moe_align_workspace_size(int T, int k, int E);
 
 /* Bytes of device scratch moe_forward needs: the activation h
- * [P_total, F] and the scaled expert outputs y [P_total, d], both bf16,
+ * [P_total, F] in bf16 and the scaled expert outputs y [P_total, d] in fp32,
  * where P_total = P_max + n_shared * ceil(T / block_m) * block_m.
  * Returns 0 on invalid arguments. */
 MOE_API size_t moe_workspace_size(int T, int d, int F, int E, int k, int block_m,
@@ -168,8 +168,9 @@ MOE_API moe_status moe_align(const int32_t* topk_ids, int T, int k, int E, int b
  *   out          [T, d] bf16 out:
  *                out[t] = sum_j topk_weights[t,j] * W2_e (act(W13_e x[t]))
  *                         (+ shared(x[t]) with weight 1),
- *                with fp32 accumulation, h and the per-slot scaled outputs
- *                rounded to bf16, the k-sum in fp32 in slot order.
+ *                with fp32 accumulation; h is rounded to bf16 (it feeds the
+ *                bf16 down GEMM), the per-slot scaled outputs stay fp32 and
+ *                the k-sum is fp32 in slot order, rounded once to bf16.
  *   ws, ws_bytes scratch of moe_workspace_size bytes.
  * Errors: host checks as above; MOE_ERR_DEVICE_TIMEOUT in dev_status if a
  * pipeline wait inside a GEMM kernel exceeded its limit (out is then invalid).
@@ -194,6 +195,19 @@ MOE_API const char* moe_status_string(moe_status status);
 /* Number of kernel launches the most recent successful call on this host
  * thread issued (for launch accounting in benchmarks). */
 MOE_API int moe_last_launch_count(void);
+
+/* Stage profiling (host-thread local).  While enabled, every moe_route,
+ * moe_align and moe_forward call records a pair of CUDA events on its stream
+ * around each of its kernels; the events are created by the library.
+ * Stages: 0 route, 1 align, 2 gate/up (fc1) GEMM, 3 down GEMM, 4 combine.
+ * moe_profile_enable(1) starts a fresh record, (0) stops recording.
+ * moe_profile_collect waits for the recorded events, writes into
+ * stage_ms[i] (i < n_stages) the summed milliseconds of stage i and into
+ * stage_calls[i] (nullable) how many launches were summed, then releases the
+ * events and clears the record.  MOE_ERR_CUDA if an event call failed. */
+#define MOE_NUM_STAGES 5
+MOE_API moe_status moe_profile_enable(int on);
+MOE_API moe_status moe_profile_collect(double* stage_ms, int* stage_calls, int n_stages);
 
 #ifdef __cplusplus
 }
