@@ -9,10 +9,23 @@ import oracle
 from grouped_gemm_gating_b200 import moe as M
 from grouped_gemm_gating_b200 import workloads as W
 
-# Output tolerance of the layer against the fp64 oracle: max |diff| within
-# 2e-2 * rms(oracle) and relative L2 error within 5e-3.
+# Output tolerance of the layer against the fp64 oracle: relative L2 error
+# within 5e-3, and max |diff| within 2e-2 * rms(oracle) beyond the bf16
+# output format's own quantum.  The output is bf16, so rounding even the
+# exact result costs up to half a bf16 ulp (2^-8 relative at the bottom of a
+# binade); for outputs several rms large that alone exceeds 2e-2 * rms, so
+# the bound is read as |diff| <= 2e-2 * rms + half_ulp_bf16(oracle).
 OUT_MAX_ABS_REL_RMS = 2e-2
 OUT_REL_L2 = 5e-3
+
+
+def bf16_half_ulp(v: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 numbers at |v| (8 significant bits)."""
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, np.exp2(e - 8), 0.0)
+
+
 # Routing weights: fp32 exp, a shuffle-tree sum over <= 256 terms and one
 # division, against fp64: a few ulp of fp32 relative error (see design notes).
 WEIGHT_TOL = 2e-6
@@ -77,12 +90,14 @@ def compare_out(gpu_bits: np.ndarray, ref: np.ndarray, label: str = ""):
     assert np.isfinite(got).all(), f"{label}: non-finite output"
     diff = got - ref
     rms = float(np.sqrt((ref ** 2).mean()))
-    max_abs = float(np.abs(diff).max()) if diff.size else 0.0
-    rel_l2 = float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300))
     assert rms > 0.0, f"{label}: degenerate oracle output"
-    assert max_abs <= OUT_MAX_ABS_REL_RMS * rms, f"{label}: max|diff|={max_abs:.3e} > 2e-2*rms={rms:.3e}"
+    max_abs = float(np.abs(diff).max()) if diff.size else 0.0
+    excess = float((np.abs(diff) - bf16_half_ulp(ref)).max()) if diff.size else 0.0
+    rel_l2 = float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300))
+    assert excess <= OUT_MAX_ABS_REL_RMS * rms, \
+        f"{label}: max(|diff| - half_ulp) = {excess / rms:.3e} * rms > 2e-2 * rms (literal {max_abs / rms:.3e})"
     assert rel_l2 <= OUT_REL_L2, f"{label}: rel L2={rel_l2:.3e}"
-    return max_abs / rms, rel_l2
+    return max_abs / rms, excess / rms, rel_l2
 
 
 def compare_route(ids_gpu, w_gpu, ids_ref, w_ref, label=""):
