@@ -177,26 +177,28 @@ def silu(z: np.ndarray) -> np.ndarray:
     return z / (1.0 + np.exp(-z))
 
 
-def expert_mlp(x: np.ndarray, w13_e: np.ndarray, w2_e: np.ndarray, act: int) -> np.ndarray:
-    """One expert on rows x [n, d] (fp64), weights as bf16 bits.
+def expert_hidden(x: np.ndarray, w13_e: np.ndarray, act: int) -> np.ndarray:
+    """Hidden activation of one expert on rows x [n, d] (fp64).
 
     SwiGLU: w13_e rows [0, F) are the gate projection, rows [F, 2F) the up
     projection; h = silu(gate) * up.  Squared ReLU: w13_e is fc1 [F, d] and
-    h = max(fc1 x, 0)^2.  Output: w2_e [d, F] applied to h.
+    h = max(fc1 x, 0)^2.
     """
     W1 = bf16_to_f64(w13_e)
-    W2 = bf16_to_f64(w2_e)
-    F = W2.shape[1]
     if act == ACT_SWIGLU:
+        F = W1.shape[0] // 2
         g = x @ W1[:F].T
         u = x @ W1[F:].T
-        h = silu(g) * u
-    elif act == ACT_RELU2:
+        return silu(g) * u
+    if act == ACT_RELU2:
         a = x @ W1.T
-        h = np.maximum(a, 0.0) ** 2
-    else:
-        raise ValueError("unknown activation")
-    return h @ W2.T
+        return np.maximum(a, 0.0) ** 2
+    raise ValueError("unknown activation")
+
+
+def expert_mlp(x: np.ndarray, w13_e: np.ndarray, w2_e: np.ndarray, act: int) -> np.ndarray:
+    """One expert on rows x [n, d] (fp64): w2_e [d, F] applied to h."""
+    return expert_hidden(x, w13_e, act) @ bf16_to_f64(w2_e).T
 
 
 def forward(x_bits: np.ndarray, w13: np.ndarray, w2: np.ndarray,
