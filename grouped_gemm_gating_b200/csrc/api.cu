@@ -137,6 +137,10 @@ moe_status finish(cudaError_t err, int launches) {
 
 }  // namespace
 
+namespace moe {
+void record_launches(int n) { g_last_launches = n; }
+}  // namespace moe
+
 extern "C" {
 
 int64_t moe_max_padded(int T, int k, int E, int block_m) {

@@ -38,6 +38,7 @@ _SIG = {
     "moe_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "moe_route": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _P, _P]),
     "moe_align": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
+    "moe_align_noalloc": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "moe_forward": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _P, _I, _P, _I, _P, _P, _P, _P, _I, _I,
                          _P, _P, ctypes.c_size_t, _P, _P]),
     "moe_read_status": (_I, [_P, _P]),
@@ -169,6 +170,22 @@ def moe_align(topk_ids, E, block_m, sorted_token_ids, expert_ids, num_tokens_pos
                                     _ptr(expert_ids), _ptr(num_tokens_post_padded), _ptr(inv_pos),
                                     _ptr(ws), ws_bytes, _ptr(dev_status), _stream(topk_ids.device))
     _check("moe_align", code)
+
+
+def moe_align_noalloc(topk_ids, E, block_m, sorted_token_ids, expert_ids, num_tokens_post_padded,
+                      inv_pos, dev_status=None):
+    """moe_align without a workspace, for callers that cannot allocate device
+    memory: the library keeps the scratch in a fixed static device array
+    (limit ceil(T*k/2048)*E <= 131072).  Calls that overlap on the GPU race
+    on that array."""
+    T, k = topk_ids.shape
+    for t in (topk_ids, sorted_token_ids, expert_ids, num_tokens_post_padded, inv_pos):
+        if t.dtype != torch.int32:
+            raise ValueError("moe_align_noalloc: int32 tensors expected")
+    code = load_library().moe_align_noalloc(_ptr(topk_ids), T, k, E, block_m, _ptr(sorted_token_ids),
+                                            _ptr(expert_ids), _ptr(num_tokens_post_padded), _ptr(inv_pos),
+                                            _ptr(dev_status), _stream(topk_ids.device))
+    _check("moe_align_noalloc", code)
 
 
 def moe_forward(x, w13, w2, topk_weights, sorted_token_ids, expert_ids, num_tokens_post_padded,

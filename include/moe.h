@@ -185,6 +185,31 @@ MOE_API moe_status moe_forward(const uint16_t* x, int T, int d,
                        uint16_t* out, void* ws, size_t ws_bytes,
                        int32_t* dev_status, moe_stream_t stream);
 
+/*
+ * moe_align_noalloc — moe_align for callers that cannot allocate device
+ * memory.  No passage of the source pages has a counterpart: it is the same
+ * sort and pad as moe_align, with the same arguments minus the workspace.
+ * Callers that cannot call cudaMalloc (a runtime that reserves all device
+ * memory up front, code running while a stream is captured into a CUDA
+ * graph, a plugin whose host framework owns every allocation) cannot supply
+ * moe_align's workspace; this entry point keeps the multi-block path's
+ * scratch in a fixed 1 MiB static device array instead.
+ *   Limit: ceil(T*k / 2048) * E <= 131072 (e.g. T*k <= 2^21 at E = 128);
+ *   larger problems return MOE_ERR_UNSUPPORTED and launch nothing.
+ *   Every GPU that loads the library holds the 1 MiB until the process exits.
+ *   The first call on a device looks up the array's device address (one
+ *   cudaGetSymbolAddress, cached per device); make that first call before
+ *   any stream capture.  It allocates nothing, ever.
+ *   All calls share the one array and it keeps the last call's contents
+ *   (nothing in it needs to start at zero); calls whose kernels overlap on
+ *   the GPU (other streams, other host threads) race on it and must be
+ *   serialised by the caller.
+ */
+MOE_API moe_status moe_align_noalloc(const int32_t* topk_ids, int T, int k, int E, int block_m,
+                             int32_t* sorted_token_ids, int32_t* expert_ids,
+                             int32_t* num_tokens_post_padded, int32_t* inv_pos,
+                             int32_t* dev_status, moe_stream_t stream);
+
 /* Synchronises `stream`, then returns the code stored in dev_status (MOE_OK
  * when 0), or MOE_ERR_CUDA if the synchronisation or the copy failed. */
 MOE_API moe_status moe_read_status(const int32_t* dev_status, moe_stream_t stream);
