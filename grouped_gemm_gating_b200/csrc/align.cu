@@ -133,6 +133,8 @@ __global__ void __launch_bounds__(kSmallThreads)
   const int tid = threadIdx.x;
   for (int i = tid; i < MOE_MAX_EXPERTS; i += kSmallThreads) cnt[i] = 0;
   for (int i = tid; i < kWarps * MOE_MAX_EXPERTS; i += kSmallThreads) (&wcnt[0][0])[i] = 0;
+  pdl_wait();
+  pdl_launch_dependents();
   __syncthreads();
   for (int s = tid; s < S; s += kSmallThreads) {
     const int e = load_expert(ids, s, S, E, status);
@@ -161,6 +163,8 @@ __global__ void __launch_bounds__(kChunkThreads)
   __shared__ int cnt[MOE_MAX_EXPERTS];
   const int c = blockIdx.x;
   for (int i = threadIdx.x; i < E; i += kChunkThreads) cnt[i] = 0;
+  pdl_wait();
+  pdl_launch_dependents();
   __syncthreads();
   const int end = min(S, (c + 1) * kChunk);
   for (int s = c * kChunk + threadIdx.x; s < end; s += kChunkThreads) {
@@ -178,6 +182,8 @@ __global__ void __launch_bounds__(1024)
   __shared__ int cnt[MOE_MAX_EXPERTS];
   __shared__ int off[MOE_MAX_EXPERTS + 1];
   const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
   if (tid < E) {
     int total = 0;
     for (int c = 0; c < nchunks; ++c) total += counts[static_cast<size_t>(c) * E + tid];
@@ -208,6 +214,8 @@ __global__ void __launch_bounds__(kChunkThreads)
   __shared__ int tot[MOE_MAX_EXPERTS];
   __shared__ int wcnt[kWarps][MOE_MAX_EXPERTS];
   const int c = blockIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
   for (int i = threadIdx.x; i < E; i += kChunkThreads) run[i] = bases[static_cast<size_t>(c) * E + i];
   for (int i = threadIdx.x; i < kWarps * MOE_MAX_EXPERTS; i += kChunkThreads) (&wcnt[0][0])[i] = 0;
   __syncthreads();
@@ -229,20 +237,23 @@ cudaError_t launch_align(const int32_t* topk_ids, int S, int E, int block_m, int
                          int32_t* expert_ids, int32_t* ntpp, int32_t* inv_pos, int32_t* ws, int32_t* status,
                          cudaStream_t stream, int* launches) {
   if (align_uses_single_block(S)) {
-    align_single_kernel<<<1, kSmallThreads, 0, stream>>>(topk_ids, S, E, block_m, P_max, sorted_ids, expert_ids,
-                                                         ntpp, inv_pos, status);
     ++*launches;
-    return cudaGetLastError();
+    return launch_pdl(align_single_kernel, dim3(1), dim3(kSmallThreads), 0, stream, topk_ids, S, E, block_m, P_max,
+                      sorted_ids, expert_ids, ntpp, inv_pos, status);
   }
   const int nchunks = align_num_chunks(S);
   int32_t* counts = ws;
   int32_t* bases = ws + static_cast<size_t>(nchunks) * E;
-  align_count_kernel<<<nchunks, kChunkThreads, 0, stream>>>(topk_ids, S, E, counts, status);
-  align_scan_kernel<<<1, 1024, 0, stream>>>(counts, nchunks, S, E, block_m, P_max, bases, sorted_ids, expert_ids,
-                                            ntpp);
-  align_scatter_kernel<<<nchunks, kChunkThreads, 0, stream>>>(topk_ids, S, E, bases, sorted_ids, inv_pos);
+  cudaError_t err = launch_pdl(align_count_kernel, dim3(nchunks), dim3(kChunkThreads), 0, stream, topk_ids, S, E,
+                               counts, status);
+  if (err != cudaSuccess) return err;
+  err = launch_pdl(align_scan_kernel, dim3(1), dim3(1024), 0, stream, static_cast<const int32_t*>(counts), nchunks,
+                   S, E, block_m, P_max, bases, sorted_ids, expert_ids, ntpp);
+  if (err != cudaSuccess) return err;
+  err = launch_pdl(align_scatter_kernel, dim3(nchunks), dim3(kChunkThreads), 0, stream, topk_ids, S, E,
+                   static_cast<const int32_t*>(bases), sorted_ids, inv_pos);
   *launches += 3;
-  return cudaGetLastError();
+  return err;
 }
 
 }  // namespace moe

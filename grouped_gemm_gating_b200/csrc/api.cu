@@ -18,12 +18,26 @@ namespace {
 thread_local int g_last_launches = 0;
 
 // ---- stage profiling: event pairs recorded around each kernel launch ----
+// Events come from a per-thread pool, so that recording (also while a stream
+// is being captured into a CUDA graph) creates no event once the pool is
+// primed by moe_profile_enable.
 struct StageRecord {
   int stage;
   cudaEvent_t start, stop;
 };
 thread_local bool g_profile = false;
 thread_local std::vector<StageRecord> g_records;
+thread_local std::vector<cudaEvent_t> g_event_pool;
+constexpr int kEventPoolPrime = 64;
+
+bool take_event(cudaEvent_t* ev) {
+  if (!g_event_pool.empty()) {
+    *ev = g_event_pool.back();
+    g_event_pool.pop_back();
+    return true;
+  }
+  return cudaEventCreate(ev) == cudaSuccess;
+}
 
 struct StageScope {
   StageRecord rec{};
@@ -32,20 +46,36 @@ struct StageScope {
   StageScope(int stage, cudaStream_t s) : stream(s), active(g_profile) {
     if (!active) return;
     rec.stage = stage;
-    if (cudaEventCreate(&rec.start) != cudaSuccess || cudaEventCreate(&rec.stop) != cudaSuccess ||
-        cudaEventRecord(rec.start, stream) != cudaSuccess)
+    if (!take_event(&rec.start)) {
       active = false;
+      return;
+    }
+    if (!take_event(&rec.stop)) {
+      g_event_pool.push_back(rec.start);
+      active = false;
+      return;
+    }
+    if (cudaEventRecord(rec.start, stream) != cudaSuccess) {
+      g_event_pool.push_back(rec.start);
+      g_event_pool.push_back(rec.stop);
+      active = false;
+    }
   }
   ~StageScope() {
     if (!active) return;
-    if (cudaEventRecord(rec.stop, stream) == cudaSuccess) g_records.push_back(rec);
+    if (cudaEventRecord(rec.stop, stream) == cudaSuccess) {
+      g_records.push_back(rec);
+    } else {
+      g_event_pool.push_back(rec.start);
+      g_event_pool.push_back(rec.stop);
+    }
   }
 };
 
 void release_records() {
   for (auto& r : g_records) {
-    cudaEventDestroy(r.start);
-    cudaEventDestroy(r.stop);
+    g_event_pool.push_back(r.start);
+    g_event_pool.push_back(r.stop);
   }
   g_records.clear();
 }
@@ -352,12 +382,17 @@ const char* moe_status_string(moe_status status) {
 int moe_last_launch_count(void) { return g_last_launches; }
 
 moe_status moe_profile_enable(int on) {
-  release_records();
+  if (on) release_records();  // a fresh record; disabling keeps the records readable
   g_profile = on != 0;
+  while (g_profile && g_event_pool.size() < kEventPoolPrime) {
+    cudaEvent_t ev;
+    if (cudaEventCreate(&ev) != cudaSuccess) return MOE_ERR_CUDA;
+    g_event_pool.push_back(ev);
+  }
   return MOE_OK;
 }
 
-moe_status moe_profile_collect(double* stage_ms, int* stage_calls, int n_stages) {
+moe_status moe_profile_collect(double* stage_ms, int* stage_calls, int n_stages, int release) {
   if (stage_ms == nullptr || n_stages < 0) return MOE_ERR_INVALID_ARG;
   for (int i = 0; i < n_stages; ++i) {
     stage_ms[i] = 0.0;
@@ -375,7 +410,7 @@ moe_status moe_profile_collect(double* stage_ms, int* stage_calls, int n_stages)
       if (stage_calls) ++stage_calls[r.stage];
     }
   }
-  release_records();
+  if (release) release_records();
   return st;
 }
 

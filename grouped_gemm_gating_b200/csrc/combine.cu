@@ -24,6 +24,8 @@ __global__ void __launch_bounds__(kCombineThreads)
                    const int32_t* __restrict__ ntpp, int T, int k, int d, int has_shared,
                    uint16_t* __restrict__ out) {
   const int t = blockIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
   if (t >= T) return;
   const int nvec = d / 8;
   int rows[MOE_MAX_TOPK + 1];
@@ -59,9 +61,9 @@ __global__ void __launch_bounds__(kCombineThreads)
 
 cudaError_t launch_combine(const float* y, const int32_t* inv_pos, const int32_t* ntpp, int T, int k, int d,
                            int has_shared, uint16_t* out, cudaStream_t stream, int* launches) {
-  combine_kernel<<<T, kCombineThreads, 0, stream>>>(y, inv_pos, ntpp, T, k, d, has_shared, out);
   ++*launches;
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(T), dim3(kCombineThreads), 0, stream, y, inv_pos, ntpp, T, k, d, has_shared,
+                    out);
 }
 
 }  // namespace moe

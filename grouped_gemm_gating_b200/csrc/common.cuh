@@ -3,6 +3,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <utility>
 
 #include "../../include/moe.h"
 
@@ -12,6 +13,34 @@ constexpr int kWarp = 32;
 // Pipeline waits inside a kernel give up after this much wall time, set an
 // error in the status word and let the kernel return (no trap, no hang).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Programmatic dependent launch: every kernel of the layer is launched with
+// programmatic stream serialisation, so it may start (prologue: barrier
+// init, TMEM allocation, tensor-map prefetch) while the previous kernel in
+// the stream drains.  Before its first global-memory access it waits for the
+// previous grid to complete and flush (griddepcontrol.wait; a no-op when the
+// kernel was launched without the attribute), and it lets the next kernel
+// launch early (griddepcontrol.launch_dependents).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
   if (status != nullptr) atomicCAS(status, 0, code);

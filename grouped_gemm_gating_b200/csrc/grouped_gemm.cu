@@ -119,11 +119,19 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
     ptx::tmem_alloc(tmem_holder, C::kTmemCols);
     ptx::tmem_relinquish();
   }
+  if (threadIdx.x == 0) {
+    ptx::prefetch_tmap(&args.tm_w);
+    if (args.n_shared_blocks) ptx::prefetch_tmap(&args.tm_ws);
+    if (EPI == kEpiScale) ptx::prefetch_tmap(&args.tm_x);
+  }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
+  // everything above overlaps the previous kernel; global reads start here
+  pdl_wait();
+  pdl_launch_dependents();
   int ntpp = *args.ntpp;
   int routed_blocks = ntpp / args.block_m;
   if (routed_blocks < 0) routed_blocks = 0;
@@ -141,9 +149,6 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
-      ptx::prefetch_tmap(&args.tm_w);
-      if (args.n_shared_blocks) ptx::prefetch_tmap(&args.tm_ws);
-      if (!C::kGather) ptx::prefetch_tmap(&args.tm_x);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -455,8 +460,7 @@ cudaError_t launch_variant(const GemmArgs& args, int grid, cudaStream_t stream) 
     if (err != cudaSuccess) return err;
     attr_done[dev] = true;
   }
-  kern<<<grid, C::kNumThreads, C::kSmemBytes, stream>>>(args);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(C::kNumThreads), C::kSmemBytes, stream, args);
 }
 
 template <bool SWAP, int TOK>

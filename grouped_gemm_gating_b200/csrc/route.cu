@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   __shared__ unsigned char s_gkeep[kWarpsPerBlock][MOE_MAX_EXPERTS];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int t = blockIdx.x * kWarpsPerBlock + warp;
+  pdl_wait();
+  pdl_launch_dependents();
   if (t >= T) return;
 
   const float* row = logits + static_cast<size_t>(t) * E;
@@ -182,20 +184,11 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int n_group, 
                          int32_t* status, cudaStream_t stream, int* launches) {
   const int grid = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
   const int block = kWarpsPerBlock * 32;
-#define MOE_ROUTE_LAUNCH(VPL)                                                                                   \
-  route_kernel<VPL><<<grid, block, 0, stream>>>(logits, T, E, k, n_group, topk_group, group_score, renormalize, \
-                                                routed_scaling, topk_ids, topk_weights, status)
-  if (E <= 32)
-    MOE_ROUTE_LAUNCH(1);
-  else if (E <= 64)
-    MOE_ROUTE_LAUNCH(2);
-  else if (E <= 128)
-    MOE_ROUTE_LAUNCH(4);
-  else
-    MOE_ROUTE_LAUNCH(8);
-#undef MOE_ROUTE_LAUNCH
+  auto kern = E <= 32 ? route_kernel<1> : E <= 64 ? route_kernel<2> : E <= 128 ? route_kernel<4> : route_kernel<8>;
+  cudaError_t err = launch_pdl(kern, dim3(grid), dim3(block), 0, stream, logits, T, E, k, n_group, topk_group,
+                               group_score, renormalize, routed_scaling, topk_ids, topk_weights, status);
   ++*launches;
-  return cudaGetLastError();
+  return err;
 }
 
 }  // namespace moe

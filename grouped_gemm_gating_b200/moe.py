@@ -45,7 +45,7 @@ _SIG = {
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_last_launch_count": (_I, []),
     "moe_profile_enable": (_I, [_I]),
-    "moe_profile_collect": (_I, [_P, _P, _I]),
+    "moe_profile_collect": (_I, [_P, _P, _I, _I]),
 }
 
 STAGES = ("route", "align", "gate_up_gemm", "down_gemm", "combine")
@@ -134,12 +134,15 @@ def moe_profile_enable(on: bool = True) -> None:
     _check("moe_profile_enable", load_library().moe_profile_enable(1 if on else 0))
 
 
-def moe_profile_collect() -> dict:
-    """Summed milliseconds and launch counts per stage since enable; clears."""
+def moe_profile_collect(release: bool = True) -> dict:
+    """Summed milliseconds and launch counts per stage of the recorded events.
+
+    release=False keeps the records (read a captured graph's events again
+    after its next replay)."""
     n = len(STAGES)
     ms = (ctypes.c_double * n)()
     calls = (ctypes.c_int * n)()
-    _check("moe_profile_collect", load_library().moe_profile_collect(ms, calls, n))
+    _check("moe_profile_collect", load_library().moe_profile_collect(ms, calls, n, 1 if release else 0))
     return {name: (float(ms[i]), int(calls[i])) for i, name in enumerate(STAGES)}
 
 

@@ -223,16 +223,20 @@ MOE_API int moe_last_launch_count(void);
 
 /* Stage profiling (host-thread local).  While enabled, every moe_route,
  * moe_align and moe_forward call records a pair of CUDA events on its stream
- * around each of its kernels; the events are created by the library.
+ * around each of its kernels (events come from a pool the library owns; the
+ * calls may be captured into a CUDA graph, where the records become event
+ * nodes that are re-recorded at every replay).
  * Stages: 0 route, 1 align, 2 gate/up (fc1) GEMM, 3 down GEMM, 4 combine.
- * moe_profile_enable(1) starts a fresh record, (0) stops recording.
- * moe_profile_collect waits for the recorded events, writes into
- * stage_ms[i] (i < n_stages) the summed milliseconds of stage i and into
- * stage_calls[i] (nullable) how many launches were summed, then releases the
- * events and clears the record.  MOE_ERR_CUDA if an event call failed. */
+ * moe_profile_enable(1) starts a fresh record (and primes the event pool),
+ * (0) stops recording and keeps what was recorded.  moe_profile_collect waits for the recorded events,
+ * writes into stage_ms[i] (i < n_stages) the summed milliseconds of stage i
+ * and into stage_calls[i] (nullable) how many launches were summed; with
+ * release != 0 it then returns the events to the pool and clears the record
+ * (release == 0 keeps them, e.g. to read a graph's events after each
+ * replay).  MOE_ERR_CUDA if an event call failed. */
 #define MOE_NUM_STAGES 5
 MOE_API moe_status moe_profile_enable(int on);
-MOE_API moe_status moe_profile_collect(double* stage_ms, int* stage_calls, int n_stages);
+MOE_API moe_status moe_profile_collect(double* stage_ms, int* stage_calls, int n_stages, int release);
 
 #ifdef __cplusplus
 }
