@@ -316,6 +316,7 @@ def run_ours(args):
             stages[k_][0] += ms
             stages[k_][1] += n
     M.moe_profile_collect(release=True)
+    stage_source = "CUDA events around each kernel in a replayed graph of the step"
     clk = clocks.stop()
 
     # ---- the same step enqueued eagerly from Python (no graph), for context ----
@@ -383,6 +384,7 @@ def run_ours(args):
                    "flops_routed_per_step": alg["flops_routed"]},
         "ms_per_step_eager": round(eager_ms / args.steps, 5),
         "stages_us": {k: round(v[0] / max(v[1], 1) * 1e3, 2) for k, v in stages.items()},
+        "stages_source": stage_source,
         "roofline": roof,
         "e2e": {"value": round(e2e_value, 4), "unit": "TFLOPS", "ms_per_step": round(e2e_ms / args.steps, 5),
                 "h2d_bytes_per_step": int(inp.x.nbytes + inp.logits.nbytes),

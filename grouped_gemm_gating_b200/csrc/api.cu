@@ -30,6 +30,16 @@ thread_local std::vector<StageRecord> g_records;
 thread_local std::vector<cudaEvent_t> g_event_pool;
 constexpr int kEventPoolPrime = 64;
 
+// Under stream capture a plain event record only orders work inside the
+// capture; the external flag makes it an event-record node of the graph, so
+// the event is recorded (with its timestamp) at every replay.
+cudaError_t record_event(cudaEvent_t ev, cudaStream_t stream) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return cudaErrorUnknown;
+  if (cs == cudaStreamCaptureStatusActive) return cudaEventRecordWithFlags(ev, stream, cudaEventRecordExternal);
+  return cudaEventRecord(ev, stream);
+}
+
 bool take_event(cudaEvent_t* ev) {
   if (!g_event_pool.empty()) {
     *ev = g_event_pool.back();
@@ -55,7 +65,7 @@ struct StageScope {
       active = false;
       return;
     }
-    if (cudaEventRecord(rec.start, stream) != cudaSuccess) {
+    if (record_event(rec.start, stream) != cudaSuccess) {
       g_event_pool.push_back(rec.start);
       g_event_pool.push_back(rec.stop);
       active = false;
@@ -63,7 +73,7 @@ struct StageScope {
   }
   ~StageScope() {
     if (!active) return;
-    if (cudaEventRecord(rec.stop, stream) == cudaSuccess) {
+    if (record_event(rec.stop, stream) == cudaSuccess) {
       g_records.push_back(rec);
     } else {
       g_event_pool.push_back(rec.start);
