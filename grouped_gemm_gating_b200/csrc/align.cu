@@ -20,105 +20,18 @@
 //     the scan over (expert, chunk), and a per-chunk stable scatter.
 // Within a round of slots, the rank of a slot among equal experts comes from
 // __match_any_sync inside the warp plus an exclusive prefix over the warps.
-#include "common.cuh"
+#include "align_impl.cuh"
 
 namespace moe {
 
 namespace {
 
+using namespace align_detail;
+
 constexpr int kSingleBlockMax = 8192;
 constexpr int kSmallThreads = 1024;
 constexpr int kChunk = 2048;        // slots per chunk on the multi-block path
 constexpr int kChunkThreads = 256;  // threads per chunk block
-
-__device__ __forceinline__ int load_expert(const int32_t* ids, int s, int S, int E, int32_t* status) {
-  if (s >= S) return -1;
-  const int e = ids[s];
-  if (e < 0 || e >= E) {
-    set_status(status, MOE_ERR_BAD_EXPERT_ID);
-    return -1;
-  }
-  return e;
-}
-
-// Exclusive prefix of padded counts over experts, by one warp.  off[E] is
-// the padded total.
-__device__ void warp_padded_scan(const int* cnt, int* off, int E, int bm, int lane) {
-  constexpr int kPer = MOE_MAX_EXPERTS / 32;
-  int local[kPer];
-  int sum = 0;
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int e = lane * kPer + i;
-    const int c = e < E ? cnt[e] : 0;
-    local[i] = (c + bm - 1) / bm * bm;
-    sum += local[i];
-  }
-  int incl = sum;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += n;
-  }
-  int run = incl - sum;
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int e = lane * kPer + i;
-    if (e < E) off[e] = run;
-    run += local[i];
-  }
-  if (lane == 31) off[E] = incl;
-}
-
-// Block b (rows [b*bm, (b+1)*bm)) belongs to the expert e with
-// off[e] <= b*bm < off[e+1]; -1 past the padded total.
-__device__ __forceinline__ int block_expert(const int* off, int E, int p) {
-  if (p >= off[E]) return -1;
-  int lo = 0, hi = E - 1;  // last e with off[e] <= p
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (off[mid] <= p)
-      lo = mid;
-    else
-      hi = mid - 1;
-  }
-  return lo;
-}
-
-// One round of the stable scatter over `nthreads` consecutive slots.  wcnt
-// is [nwarps][E] of zeros on entry and on exit; run[e] is advanced.
-template <int NWARPS>
-__device__ __forceinline__ void scatter_round(int e, int s, int (*wcnt)[MOE_MAX_EXPERTS], int* run, int* tot, int E,
-                                              int32_t* sorted_ids, int32_t* inv_pos) {
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const unsigned peers = __match_any_sync(0xffffffffu, e);
-  const int rank = __popc(peers & ((1u << lane) - 1u));
-  if (e >= 0 && rank == 0) wcnt[warp][e] = __popc(peers);
-  __syncthreads();
-  if (threadIdx.x < E) {
-    int acc = 0;
-#pragma unroll 4
-    for (int w = 0; w < NWARPS; ++w) {
-      const int c = wcnt[w][threadIdx.x];
-      wcnt[w][threadIdx.x] = acc;
-      acc += c;
-    }
-    tot[threadIdx.x] = acc;
-  }
-  __syncthreads();
-  if (e >= 0) {
-    const int pos = run[e] + wcnt[warp][e] + rank;
-    sorted_ids[pos] = s;
-    inv_pos[s] = pos;
-  }
-  __syncthreads();
-  if (threadIdx.x < E) {
-    run[threadIdx.x] += tot[threadIdx.x];
-#pragma unroll 4
-    for (int w = 0; w < NWARPS; ++w) wcnt[w][threadIdx.x] = 0;
-  }
-  __syncthreads();
-}
 
 __global__ void __launch_bounds__(kSmallThreads)
     align_single_kernel(const int32_t* __restrict__ ids, int S, int E, int bm, int P_max,
@@ -130,29 +43,12 @@ __global__ void __launch_bounds__(kSmallThreads)
   __shared__ int run[MOE_MAX_EXPERTS];
   __shared__ int tot[MOE_MAX_EXPERTS];
   __shared__ int wcnt[kWarps][MOE_MAX_EXPERTS];
-  const int tid = threadIdx.x;
-  for (int i = tid; i < MOE_MAX_EXPERTS; i += kSmallThreads) cnt[i] = 0;
-  for (int i = tid; i < kWarps * MOE_MAX_EXPERTS; i += kSmallThreads) (&wcnt[0][0])[i] = 0;
+  for (int i = threadIdx.x; i < kWarps * MOE_MAX_EXPERTS; i += kSmallThreads) (&wcnt[0][0])[i] = 0;
   pdl_wait();
   pdl_launch_dependents();
-  __syncthreads();
-  for (int s = tid; s < S; s += kSmallThreads) {
-    const int e = load_expert(ids, s, S, E, status);
-    if (e >= 0) atomicAdd(&cnt[e], 1);
-  }
-  __syncthreads();
-  if (tid < 32) warp_padded_scan(cnt, off, E, bm, tid);
-  __syncthreads();
-  if (tid < E) run[tid] = off[tid];
-  if (tid == 0) *ntpp = off[E];
-  for (int p = tid; p < P_max; p += kSmallThreads) sorted_ids[p] = S;
-  for (int b = tid; b < P_max / bm; b += kSmallThreads) expert_ids[b] = block_expert(off, E, b * bm);
-  __syncthreads();
-  for (int base = 0; base < S; base += kSmallThreads) {
-    const int s = base + tid;
-    const int e = load_expert(ids, s, S, E, nullptr);
-    scatter_round<kWarps>(e, s, wcnt, run, tot, E, sorted_ids, inv_pos);
-  }
+  auto get_expert = [&](int s, bool report) { return load_expert(ids, s, S, E, report ? status : nullptr); };
+  align_one_block<kWarps>(get_expert, S, E, bm, P_max, sorted_ids, expert_ids, ntpp, inv_pos, cnt, off, run, tot,
+                          wcnt);
 }
 
 // ---- multi-block path ----------------------------------------------------

@@ -11,6 +11,7 @@
 
 #include "../../include/moe.h"
 #include "common.cuh"
+#include "fused.h"
 #include "gemm.h"
 
 namespace {
@@ -150,6 +151,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool valid_block_m(int bm) { return bm == 16 || bm == 32 || bm == 64 || bm == 128; }
 
 constexpr size_t kWsAlign = 256;
+// Batches up to this many tokens let the fused expert kernel do the
+// scatter-reduce itself (one CTA per d-column tile sums every token).
+constexpr int kFusedCombineMaxT = 64;
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -172,6 +176,32 @@ moe_status check_dims(int T, int d, int F, int E, int k) {
 moe_status finish(cudaError_t err, int launches) {
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status check_route_args(int T, int E, int k, int n_group, int topk_group, moe_group_score group_score,
+                            float routed_scaling) {
+  if (T < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  if (n_group < 1 || E % n_group != 0 || topk_group < 1 || topk_group > n_group) return MOE_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(k) > static_cast<int64_t>(topk_group) * (E / n_group)) return MOE_ERR_INVALID_ARG;
+  if (group_score != MOE_GROUP_MAX && group_score != MOE_GROUP_TOP2SUM) return MOE_ERR_INVALID_ARG;
+  if (!(routed_scaling > 0.0f) || routed_scaling > 3.0e38f) return MOE_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(T) * k >= (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status check_align_args(const int32_t* topk_ids, int T, int k, int E, int block_m,
+                            const int32_t* sorted_token_ids, const int32_t* expert_ids,
+                            const int32_t* num_tokens_post_padded, const int32_t* inv_pos, const void* ws,
+                            size_t ws_bytes) {
+  if (T < 0 || E < 1 || k < 1 || k > E || !valid_block_m(block_m)) return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(T) * k >= (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
+  if (!sorted_token_ids || !expert_ids || !num_tokens_post_padded) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_ids || !inv_pos)) return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_align_workspace_size(T, k, E);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return MOE_ERR_WORKSPACE;
   return MOE_OK;
 }
 
@@ -204,19 +234,15 @@ size_t moe_workspace_size(int T, int d, int F, int E, int k, int block_m, moe_ac
   const int64_t P = padded_total(T, k, E, block_m, n_shared);
   const size_t h = round_up(static_cast<size_t>(P) * F * 2, kWsAlign);
   const size_t y = round_up(static_cast<size_t>(P) * d * 4, kWsAlign);
-  return h + y + kWsAlign;
+  const size_t counters = round_up(static_cast<size_t>(P / block_m + (d + 127) / 128) * 4, kWsAlign);
+  return h + y + counters + kWsAlign;
 }
 
 moe_status moe_route(const float* logits, int T, int E, int k, int n_group, int topk_group,
                      moe_group_score group_score, int renormalize, float routed_scaling, int32_t* topk_ids,
                      float* topk_weights, int32_t* dev_status, moe_stream_t stream) {
-  if (T < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
-  if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
-  if (n_group < 1 || E % n_group != 0 || topk_group < 1 || topk_group > n_group) return MOE_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(k) > static_cast<int64_t>(topk_group) * (E / n_group)) return MOE_ERR_INVALID_ARG;
-  if (group_score != MOE_GROUP_MAX && group_score != MOE_GROUP_TOP2SUM) return MOE_ERR_INVALID_ARG;
-  if (!(routed_scaling > 0.0f) || routed_scaling > 3.0e38f) return MOE_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(T) * k >= (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
+  moe_status st = check_route_args(T, E, k, n_group, topk_group, group_score, routed_scaling);
+  if (st != MOE_OK) return st;
   if (T == 0) return finish(cudaSuccess, 0);
   if (!logits || !topk_ids || !topk_weights) return MOE_ERR_INVALID_ARG;
   int launches = 0;
@@ -227,16 +253,49 @@ moe_status moe_route(const float* logits, int T, int E, int k, int n_group, int 
   return finish(err, launches);
 }
 
+moe_status moe_route_align(const float* logits, int T, int E, int k, int n_group, int topk_group,
+                           moe_group_score group_score, int renormalize, float routed_scaling, int block_m,
+                           int32_t* topk_ids, float* topk_weights, int32_t* sorted_token_ids, int32_t* expert_ids,
+                           int32_t* num_tokens_post_padded, int32_t* inv_pos, void* ws, size_t ws_bytes,
+                           int32_t* dev_status, moe_stream_t stream) {
+  moe_status st = check_route_args(T, E, k, n_group, topk_group, group_score, routed_scaling);
+  if (st != MOE_OK) return st;
+  st = check_align_args(topk_ids, T, k, E, block_m, sorted_token_ids, expert_ids, num_tokens_post_padded, inv_pos,
+                        ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (T > 0 && (!logits || !topk_weights)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t P_max = moe_max_padded(T, k, E, block_m);
+  int launches = 0;
+  cudaError_t err = cudaSuccess;
+  if (T > 0 && moe::route_align_fusable(T, k, n_group)) {
+    StageScope scope(5, s);
+    err = moe::launch_route_align(logits, T, E, k, n_group, topk_group, static_cast<int>(group_score),
+                                  renormalize ? 1 : 0, routed_scaling, topk_ids, topk_weights, block_m,
+                                  static_cast<int>(P_max), sorted_token_ids, expert_ids, num_tokens_post_padded,
+                                  inv_pos, dev_status, s, &launches);
+    return finish(err, launches);
+  }
+  if (T > 0) {
+    StageScope scope(0, s);
+    err = moe::launch_route(logits, T, E, k, n_group, topk_group, static_cast<int>(group_score), renormalize ? 1 : 0,
+                            routed_scaling, topk_ids, topk_weights, dev_status, s, &launches);
+  }
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  {
+    StageScope scope(1, s);
+    err = moe::launch_align(topk_ids, T * k, E, block_m, static_cast<int>(P_max), sorted_token_ids, expert_ids,
+                            num_tokens_post_padded, inv_pos, static_cast<int32_t*>(ws), dev_status, s, &launches);
+  }
+  return finish(err, launches);
+}
+
 moe_status moe_align(const int32_t* topk_ids, int T, int k, int E, int block_m, int32_t* sorted_token_ids,
                      int32_t* expert_ids, int32_t* num_tokens_post_padded, int32_t* inv_pos, void* ws,
                      size_t ws_bytes, int32_t* dev_status, moe_stream_t stream) {
-  if (T < 0 || E < 1 || k < 1 || k > E || !valid_block_m(block_m)) return MOE_ERR_INVALID_ARG;
-  if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(T) * k >= (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
-  if (!sorted_token_ids || !expert_ids || !num_tokens_post_padded) return MOE_ERR_INVALID_ARG;
-  if (T > 0 && (!topk_ids || !inv_pos)) return MOE_ERR_INVALID_ARG;
-  const size_t need = moe_align_workspace_size(T, k, E);
-  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return MOE_ERR_WORKSPACE;
+  moe_status st = check_align_args(topk_ids, T, k, E, block_m, sorted_token_ids, expert_ids, num_tokens_post_padded,
+                                   inv_pos, ws, ws_bytes);
+  if (st != MOE_OK) return st;
   const int S = T * k;
   const int64_t P_max = moe_max_padded(T, k, E, block_m);
   int launches = 0;
@@ -281,6 +340,63 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   if (num_sms <= 0) return MOE_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int launches = 0;
+  int32_t* counters = reinterpret_cast<int32_t*>(wsb + round_up(static_cast<size_t>(P_total) * F * 2, kWsAlign) +
+                                                 round_up(static_cast<size_t>(P_total) * d * 4, kWsAlign));
+  const int total_blocks_max = static_cast<int>(P_total / bm);
+  const int n_dtiles = (d + 127) / 128;
+
+  if (moe::fused_expert_supported(bm)) {
+    // small token blocks: both GEMMs (and for small batches the combine) in
+    // one persistent kernel; its cross-CTA counters start from zero
+    moe::FusedArgs fa;
+    std::memset(&fa, 0, sizeof(fa));
+    if (!encode_3d(&fa.tm_w13, w13, d, n1, E, 128) || !encode_3d(&fa.tm_w2, w2, F, d, E, 128)) return MOE_ERR_CUDA;
+    if (n_shared) {
+      if (!encode_3d(&fa.tm_w13s, w13_shared, d, n1, 1, 128) || !encode_3d(&fa.tm_w2s, w2_shared, F, d, 1, 128))
+        return MOE_ERR_CUDA;
+    } else {
+      fa.tm_w13s = fa.tm_w13;
+      fa.tm_w2s = fa.tm_w2;
+    }
+    fa.x = x;
+    fa.h = h;
+    fa.y = y;
+    fa.out = out;
+    fa.sorted_ids = sorted_token_ids;
+    fa.expert_ids = expert_ids;
+    fa.ntpp = num_tokens_post_padded;
+    fa.inv_pos = inv_pos;
+    fa.topk_w = topk_weights;
+    fa.ready = counters;
+    fa.done = counters + total_blocks_max;
+    fa.status = dev_status;
+    fa.T = T;
+    fa.k = k;
+    fa.S = T * k;
+    fa.E = E;
+    fa.d = d;
+    fa.F = F;
+    fa.block_m = bm;
+    fa.max_routed_blocks = max_routed_blocks;
+    fa.n_shared_blocks = n_shared_blocks;
+    fa.do_combine = T <= kFusedCombineMaxT ? 1 : 0;
+    const int64_t tiles = static_cast<int64_t>(total_blocks_max) * ((F + 127) / 128 + n_dtiles);
+    const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+    cudaError_t err = cudaMemsetAsync(counters, 0, static_cast<size_t>(total_blocks_max + n_dtiles) * 4, s);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    {
+      StageScope scope(6, s);
+      err = moe::launch_fused_expert(act == MOE_ACT_SWIGLU ? moe::kEpiSwiGLU : moe::kEpiRelu2, bm, fa,
+                                     grid < 1 ? 1 : grid, s);
+    }
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    ++launches;
+    if (!fa.do_combine) {
+      StageScope scope(4, s);
+      err = moe::launch_combine(y, inv_pos, num_tokens_post_padded, T, k, d, n_shared, out, s, &launches);
+    }
+    return finish(err, launches);
+  }
 
   // gate/up (or fc1) GEMM with the activation epilogue: h [P_total, F]
   moe::GemmArgs a1;

@@ -71,6 +71,12 @@ cudaError_t launch_align(const int32_t* topk_ids, int S, int E, int block_m, int
                          int32_t* expert_ids, int32_t* ntpp, int32_t* inv_pos, int32_t* ws, int32_t* status,
                          cudaStream_t stream, int* launches);
 
+bool route_align_fusable(int T, int k, int n_group);
+cudaError_t launch_route_align(const float* logits, int T, int E, int k, int n_group, int topk_group,
+                               int group_score, int renormalize, float routed_scaling, int32_t* topk_ids,
+                               float* topk_weights, int block_m, int P_max, int32_t* sorted_ids, int32_t* expert_ids,
+                               int32_t* ntpp, int32_t* inv_pos, int32_t* status, cudaStream_t stream, int* launches);
+
 cudaError_t launch_combine(const float* y, const int32_t* inv_pos, const int32_t* ntpp, int T, int k, int d,
                            int has_shared, uint16_t* out, cudaStream_t stream, int* launches);
 

@@ -1,0 +1,486 @@
+// Fused expert kernel for small token blocks (block_m = 16..64): the gate/up
+// GEMM with its activation, the down GEMM with the top-k weights and, for
+// small batches, the scatter-reduce, in one persistent launch.
+//
+// This is the same computation as the separate grouped GEMMs (see
+// grouped_gemm.cu for the sources: "Grouped GEMM Structure" of the
+// fused-moe-kernel page, the gate/up, activation, down and weighted-sum
+// sequence of the axolotl `_moe_triton_forward`, the relu^2 experts of the
+// mlxcel PR) specialised for the decode / verifier shape, where the layer is
+// bound by streaming each hit expert's weights once from HBM and every
+// separate launch costs as much as a few microseconds of that stream.
+//
+// Work list: all gate/up tiles (block, h-column tile) first, then all down
+// tiles (block, d-column tile).  Every CTA walks the list with the same
+// static stride, so its own gate/up tiles always come before its down tiles
+// and no CTA waits on work queued behind itself; all CTAs are co-resident
+// (one per SM, grid <= SM count).  A down tile needs the block's full h rows:
+// the gate/up epilogue publishes each finished tile with a release pattern
+// (h stores, __threadfence, atomicAdd on ready[block]); the down tile's
+// gather warps poll ready[block] with ld.acquire before loading h.  The TMA
+// warp streams the down tile's W2 slices without waiting, so the down
+// GEMM's weight traffic overlaps the tail of the gate/up phase.
+//
+// Combine (do_combine): the CTA that finishes the last down tile of a
+// d-column tile (done[column tile] reaches the number of blocks) sums, for
+// that column range, out[t] = sum_j y[inv_pos[t*k + j]] (+ the shared
+// expert's row) in fp32 in slot order and writes bf16: the same arithmetic as
+// the combine kernel.
+//
+// Every wait is bounded in time; on expiry the kernel records
+// MOE_ERR_DEVICE_TIMEOUT and all roles leave their loops.
+#include "common.cuh"
+#include "fused.h"
+#include "gemm.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+template <int EPI1, int TOK>
+struct FusedCfg {
+  static constexpr bool kGated = (EPI1 == kEpiSwiGLU);
+  static constexpr int kW1Rows = kGated ? 256 : 128;  // phase-1 weight rows per stage
+  static constexpr int kW2Rows = 128;                 // phase-2 weight rows per stage
+  static constexpr int kWBytes = kW1Rows * 128;
+  static constexpr int kXBytes = TOK * 128;
+  static constexpr int kStageBytes = kWBytes + kXBytes;
+  static constexpr int kStagesRaw = (225 * 1024) / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+  static constexpr int kAccCols = kGated ? 2 * TOK : TOK;
+  static constexpr int kTmemNeed = 2 * kAccCols;
+  static constexpr int kTmemCols = kTmemNeed <= 32    ? 32
+                                   : kTmemNeed <= 64  ? 64
+                                   : kTmemNeed <= 128 ? 128
+                                   : kTmemNeed <= 256 ? 256
+                                                      : 512;
+  static constexpr int kNumThreads = 320;
+  static constexpr int kGatherLag = 2;
+  static constexpr uint32_t kTx1 = kWBytes;
+  static constexpr uint32_t kTx2 = kW2Rows * 128;
+  static constexpr int kBarrierBytes = 256;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes;
+  static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(128, TOK);
+  static_assert(TOK == 16 || TOK == 32 || TOK == 64, "token rows per tile");
+  static_assert(kStages >= kGatherLag + 2, "pipeline depth");
+  static_assert((2 * kStages + 4) * 8 + 16 <= kBarrierBytes, "barrier area");
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+};
+
+struct Tile {
+  int phase;  // 1: gate/up, 2: down
+  int blk, wt;
+  bool shared_blk;
+};
+
+__device__ __forceinline__ Tile fused_tile(int u, int n1_tiles, int n_wt1, int n_wt2, int routed_blocks) {
+  Tile t;
+  if (u < n1_tiles) {
+    t.phase = 1;
+    t.blk = u / n_wt1;
+    t.wt = u - t.blk * n_wt1;
+  } else {
+    const int v = u - n1_tiles;
+    t.phase = 2;
+    t.blk = v / n_wt2;
+    t.wt = v - t.blk * n_wt2;
+  }
+  t.shared_blk = t.blk >= routed_blocks;
+  return t;
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Named barrier over the four epilogue warps (barrier 0 is __syncthreads).
+__device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int EPI1, int TOK>
+__global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
+    fused_expert_kernel(const __grid_constant__ FusedArgs args) {
+  using C = FusedCfg<EPI1, TOK>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_holder + 2);
+
+  const int warp = threadIdx.x / kWarp;
+  const int lane = threadIdx.x % kWarp;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      ptx::mbar_init(&full[s], 1 + 128);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&tfull[b], 1);
+      ptx::mbar_init(&tempty[b], 4);
+    }
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&args.tm_w13);
+    ptx::prefetch_tmap(&args.tm_w2);
+    if (args.n_shared_blocks) {
+      ptx::prefetch_tmap(&args.tm_w13s);
+      ptx::prefetch_tmap(&args.tm_w2s);
+    }
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_holder, C::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  pdl_wait();
+  pdl_launch_dependents();
+  int routed_blocks = *args.ntpp / args.block_m;
+  if (routed_blocks < 0) routed_blocks = 0;
+  if (routed_blocks > args.max_routed_blocks) routed_blocks = args.max_routed_blocks;
+  const int total_blocks = routed_blocks + args.n_shared_blocks;
+  const int n_wt1 = (args.F + 127) / 128;
+  const int n_wt2 = (args.d + 127) / 128;
+  const int n1_tiles = total_blocks * n_wt1;
+  const int total_tiles = n1_tiles + total_blocks * n_wt2;
+  const int nk1 = args.d / 64;
+  const int nk2 = args.F / 64;
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    set_status(args.status, MOE_ERR_DEVICE_TIMEOUT);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer (weights)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < total_tiles; u += gridDim.x) {
+        const Tile t = fused_tile(u, n1_tiles, n_wt1, n_wt2, routed_blocks);
+        int e = 0;
+        if (!t.shared_blk) {
+          e = args.expert_ids[t.blk];
+          if (e < 0 || e >= args.E) set_status(args.status, MOE_ERR_BAD_EXPERT_ID);
+        }
+        const int nk = t.phase == 1 ? nk1 : nk2;
+        const CUtensorMap* tm = t.phase == 1 ? (t.shared_blk ? &args.tm_w13s : &args.tm_w13)
+                                             : (t.shared_blk ? &args.tm_w2s : &args.tm_w2);
+        const int row0 = t.wt * 128;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+            fail();
+            ok = false;
+            break;
+          }
+          uint8_t* sW = smem + stage * C::kStageBytes;
+          if (t.phase == 1) {
+            ptx::mbar_arrive_expect_tx(&full[stage], C::kTx1);
+            ptx::tma_load_3d(sW, tm, &full[stage], kb * 64, row0, e);
+            if (C::kGated) ptx::tma_load_3d(sW + 128 * 128, tm, &full[stage], kb * 64, args.F + row0, e);
+          } else {
+            ptx::mbar_arrive_expect_tx(&full[stage], C::kTx2);
+            ptx::tma_load_3d(sW, tm, &full[stage], kb * 64, row0, e);
+          }
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int abuf = 0;
+      uint32_t aphase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < total_tiles; u += gridDim.x) {
+        const Tile t = fused_tile(u, n1_tiles, n_wt1, n_wt2, routed_blocks);
+        if (!ptx::mbar_wait_bounded(&tempty[abuf], aphase ^ 1u, abort_flag, kWaitLimitNs)) {
+          fail();
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * C::kAccCols);
+        const int nk = t.phase == 1 ? nk1 : nk2;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait_bounded(&full[stage], phase, abort_flag, kWaitLimitNs)) {
+            fail();
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sW = ptx::smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t sX = sW + C::kWBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            const uint64_t dw = ptx::sw128_kmajor_desc(sW + kk * 32);
+            const uint64_t dx = ptx::sw128_kmajor_desc(sX + kk * 32);
+            ptx::mma_bf16(d_tmem, dw, dx, C::kIdesc, acc);
+            if (C::kGated && t.phase == 1) {
+              const uint64_t du = ptx::sw128_kmajor_desc(sW + 128 * 128 + kk * 32);
+              ptx::mma_bf16(d_tmem + TOK, du, dx, C::kIdesc, acc);
+            }
+          }
+          ptx::mma_commit(&empty[stage]);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        ptx::mma_commit(&tfull[abuf]);
+        if (++abuf == 2) {
+          abuf = 0;
+          aphase ^= 1u;
+        }
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;  // weight row within the tile = output column
+    const int etid = threadIdx.x - 64;
+    int abuf = 0;
+    uint32_t aphase = 0;
+    for (int u = blockIdx.x; u < total_tiles; u += gridDim.x) {
+      const Tile t = fused_tile(u, n1_tiles, n_wt1, n_wt2, routed_blocks);
+      if (!ptx::mbar_wait_bounded(&tfull[abuf], aphase, abort_flag, kWaitLimitNs)) {
+        fail();
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t t_acc =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(abuf * C::kAccCols);
+      const int pos0 = t.blk * args.block_m;
+      const int col = t.wt * 128 + row;
+      if (t.phase == 1) {
+        const bool col_ok = col < args.F;
+#pragma unroll 1
+        for (int j0 = 0; j0 < TOK; j0 += 16) {
+          uint32_t a[16], g[16];
+          ptx::tmem_ld16(t_acc + j0, a);
+          if (C::kGated) ptx::tmem_ld16(t_acc + TOK + j0, g);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            float v = __uint_as_float(a[jj]);
+            if (C::kGated) {
+              v = silu_f(v) * __uint_as_float(g[jj]);
+            } else {
+              v = fmaxf(v, 0.0f);
+              v *= v;
+            }
+            if (col_ok) args.h[static_cast<size_t>(pos0 + j0 + jj) * args.F + col] = float_to_bf16_bits(v);
+          }
+        }
+      } else {
+        const bool col_ok = col < args.d;
+#pragma unroll 1
+        for (int j0 = 0; j0 < TOK; j0 += 16) {
+          uint32_t a[16];
+          ptx::tmem_ld16(t_acc + j0, a);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int p = pos0 + j0 + jj;
+            bool valid;
+            float wv = 1.0f;
+            if (!t.shared_blk) {
+              const int slot = args.sorted_ids[p];
+              valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
+              if (valid) wv = args.topk_w[slot];
+            } else {
+              valid = (t.blk - routed_blocks) * args.block_m + j0 + jj < args.T;
+            }
+            if (col_ok && valid) args.y[static_cast<size_t>(p) * args.d + col] = __uint_as_float(a[jj]) * wv;
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&tempty[abuf]);
+      if (++abuf == 2) {
+        abuf = 0;
+        aphase ^= 1u;
+      }
+      // publish the finished tile
+      __threadfence();
+      epilogue_sync();
+      if (t.phase == 1) {
+        if (etid == 0) atomicAdd(&args.ready[t.blk], 1);
+      } else if (args.do_combine) {
+        if (etid == 0) *last_flag = (atomicAdd(&args.done[t.wt], 1) == total_blocks - 1) ? 1 : 0;
+        epilogue_sync();
+        if (*last_flag) {
+          // this CTA finished the last down tile of column tile t.wt
+          __threadfence();
+          const int c = t.wt * 128 + row;
+          if (c < args.d) {
+            for (int tok = 0; tok < args.T; ++tok) {
+              float acc = 0.0f;
+              for (int j = 0; j < args.k; ++j) {
+                const int pr = args.inv_pos[static_cast<size_t>(tok) * args.k + j];
+                acc += __ldcg(args.y + static_cast<size_t>(pr) * args.d + c);
+              }
+              if (args.n_shared_blocks) acc += __ldcg(args.y + static_cast<size_t>(*args.ntpp + tok) * args.d + c);
+              args.out[static_cast<size_t>(tok) * args.d + c] = float_to_bf16_bits(acc);
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------ row gather (x, then h)
+    constexpr int kRowsPerThread = TOK / 16;
+    constexpr int kLag = C::kGatherLag;
+    const int gtid = threadIdx.x - 192;
+    const int chunk = gtid & 7;
+    const int r0 = gtid >> 3;
+    int stage = 0, astage = 0, pend = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < total_tiles; u += gridDim.x) {
+      const Tile t = fused_tile(u, n1_tiles, n_wt1, n_wt2, routed_blocks);
+      const uint16_t* src[kRowsPerThread];
+      uint32_t nbytes[kRowsPerThread];
+      int K;
+      if (t.phase == 1) {
+        K = args.d;
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          const int r = r0 + 16 * i;
+          int tok;
+          bool valid;
+          if (!t.shared_blk) {
+            const int slot = args.sorted_ids[t.blk * args.block_m + r];
+            valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
+            tok = valid ? slot / args.k : 0;
+          } else {
+            tok = (t.blk - routed_blocks) * args.block_m + r;
+            valid = tok < args.T;
+            if (!valid) tok = 0;
+          }
+          src[i] = args.x + static_cast<size_t>(tok) * K + chunk * 8;
+          nbytes[i] = valid ? 16u : 0u;
+        }
+      } else {
+        K = args.F;
+        // wait until every gate/up tile of this block has published its h
+        if (lane == 0) {
+          const uint64_t t0 = ptx::globaltimer_ns();
+          while (ld_acquire(args.ready + t.blk) < n_wt1) {
+            if (*abort_flag || ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+              fail();
+              ok = false;
+              break;
+            }
+            __nanosleep(64);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        __syncwarp();  // orders every lane's h loads after lane 0's acquire
+        if (!ok) break;
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          const int r = r0 + 16 * i;
+          src[i] = args.h + static_cast<size_t>(t.blk * args.block_m + r) * K + chunk * 8;
+          nbytes[i] = 16u;
+        }
+      }
+      const int nk = K / 64;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+          fail();
+          ok = false;
+          break;
+        }
+        const uint32_t sX = ptx::smem_u32(smem + stage * C::kStageBytes + C::kWBytes);
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          const int r = r0 + 16 * i;
+          const uint32_t dst = sX + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4);
+          ptx::cp_async_16(dst, src[i] + kb * 64, nbytes[i]);
+        }
+        ptx::cp_async_commit();
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        if (++pend > kLag) {
+          ptx::cp_async_wait<kLag>();
+          ptx::fence_proxy_async_smem();
+          ptx::mbar_arrive(&full[astage]);
+          if (++astage == C::kStages) astage = 0;
+          --pend;
+        }
+      }
+    }
+    ptx::cp_async_wait<0>();
+    ptx::fence_proxy_async_smem();
+    for (; pend > 0; --pend) {
+      ptx::mbar_arrive(&full[astage]);
+      if (++astage == C::kStages) astage = 0;
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+template <int EPI1, int TOK>
+cudaError_t launch_fused_variant(const FusedArgs& args, int grid, cudaStream_t stream) {
+  using C = FusedCfg<EPI1, TOK>;
+  auto kern = fused_expert_kernel<EPI1, TOK>;
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_done[dev]) {
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (err != cudaSuccess) return err;
+    attr_done[dev] = true;
+  }
+  return launch_pdl(kern, dim3(grid), dim3(C::kNumThreads), C::kSmemBytes, stream, args);
+}
+
+}  // namespace
+
+bool fused_expert_supported(int block_m) { return block_m == 16 || block_m == 32 || block_m == 64; }
+
+cudaError_t launch_fused_expert(int act_epi, int block_m, const FusedArgs& args, int grid, cudaStream_t stream) {
+  const bool gated = act_epi == kEpiSwiGLU;
+  switch (block_m) {
+    case 16: return gated ? launch_fused_variant<kEpiSwiGLU, 16>(args, grid, stream)
+                          : launch_fused_variant<kEpiRelu2, 16>(args, grid, stream);
+    case 32: return gated ? launch_fused_variant<kEpiSwiGLU, 32>(args, grid, stream)
+                          : launch_fused_variant<kEpiRelu2, 32>(args, grid, stream);
+    case 64: return gated ? launch_fused_variant<kEpiSwiGLU, 64>(args, grid, stream)
+                          : launch_fused_variant<kEpiRelu2, 64>(args, grid, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace moe

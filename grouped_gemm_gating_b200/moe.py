@@ -39,6 +39,8 @@ _SIG = {
     "moe_route": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _P, _P]),
     "moe_align": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
     "moe_align_noalloc": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "moe_route_align": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P, _P, _P, _P, _P, _P, _P,
+                             ctypes.c_size_t, _P, _P]),
     "moe_forward": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _P, _I, _P, _I, _P, _P, _P, _P, _I, _I,
                          _P, _P, ctypes.c_size_t, _P, _P]),
     "moe_read_status": (_I, [_P, _P]),
@@ -48,7 +50,7 @@ _SIG = {
     "moe_profile_collect": (_I, [_P, _P, _I, _I]),
 }
 
-STAGES = ("route", "align", "gate_up_gemm", "down_gemm", "combine")
+STAGES = ("route", "align", "gate_up_gemm", "down_gemm", "combine", "route_align", "fused_expert")
 
 _lib = None
 _lock = threading.Lock()
@@ -175,6 +177,25 @@ def moe_align(topk_ids, E, block_m, sorted_token_ids, expert_ids, num_tokens_pos
     _check("moe_align", code)
 
 
+def moe_route_align(logits, k, block_m, topk_ids, topk_weights, sorted_token_ids, expert_ids,
+                    num_tokens_post_padded, inv_pos, ws=None, n_group=1, topk_group=1, group_score=GROUP_MAX,
+                    renormalize=True, routed_scaling=1.0, dev_status=None):
+    """moe_route then moe_align in one call (one kernel for small batches)."""
+    T, E = logits.shape
+    if logits.dtype != torch.float32 or topk_weights.dtype != torch.float32:
+        raise ValueError("moe_route_align: logits/weights fp32")
+    for t in (topk_ids, sorted_token_ids, expert_ids, num_tokens_post_padded, inv_pos):
+        if t.dtype != torch.int32:
+            raise ValueError("moe_route_align: int32 index tensors expected")
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    code = load_library().moe_route_align(
+        _ptr(logits), T, E, k, n_group, topk_group, group_score, 1 if renormalize else 0,
+        float(routed_scaling), block_m, _ptr(topk_ids), _ptr(topk_weights), _ptr(sorted_token_ids),
+        _ptr(expert_ids), _ptr(num_tokens_post_padded), _ptr(inv_pos), _ptr(ws), ws_bytes,
+        _ptr(dev_status), _stream(logits.device))
+    _check("moe_route_align", code)
+
+
 def moe_align_noalloc(topk_ids, E, block_m, sorted_token_ids, expert_ids, num_tokens_post_padded,
                       inv_pos, dev_status=None):
     """moe_align without a workspace, for callers that cannot allocate device
@@ -260,6 +281,12 @@ class MoEBuffers:
     def align(self):
         moe_align(self.topk_ids, self.E, self.block_m, self.sorted_token_ids, self.expert_ids,
                   self.ntpp, self.inv_pos, self.align_ws, self.status)
+
+    def route_align(self, logits, n_group=1, topk_group=1, group_score=GROUP_MAX, renormalize=True,
+                    routed_scaling=1.0):
+        moe_route_align(logits, self.k, self.block_m, self.topk_ids, self.topk_weights, self.sorted_token_ids,
+                        self.expert_ids, self.ntpp, self.inv_pos, self.align_ws, n_group, topk_group, group_score,
+                        renormalize, routed_scaling, self.status)
 
     def forward(self, x, w13, w2, w13_shared=None, w2_shared=None):
         moe_forward(x, w13, w2, self.topk_weights, self.sorted_token_ids, self.expert_ids, self.ntpp,

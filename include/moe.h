@@ -104,7 +104,8 @@ MOE_API int64_t moe_max_padded(int T, int k, int E, int block_m);
 MOE_API size_t moe_align_workspace_size(int T, int k, int E);
 
 /* Bytes of device scratch moe_forward needs: the activation h
- * [P_total, F] in bf16 and the scaled expert outputs y [P_total, d] in fp32,
+ * [P_total, F] in bf16, the scaled expert outputs y [P_total, d] in fp32 and
+ * P_total / block_m + ceil(d / 128) int32 counters,
  * where P_total = P_max + n_shared * ceil(T / block_m) * block_m.
  * Returns 0 on invalid arguments. */
 MOE_API size_t moe_workspace_size(int T, int d, int F, int E, int k, int block_m,
@@ -210,6 +211,23 @@ MOE_API moe_status moe_align_noalloc(const int32_t* topk_ids, int T, int k, int 
                              int32_t* num_tokens_post_padded, int32_t* inv_pos,
                              int32_t* dev_status, moe_stream_t stream);
 
+/*
+ * moe_route_align — moe_route followed by moe_align, in one call.  Same
+ * arguments, outputs and errors as the two calls; the results are
+ * bit-identical.  For small batches (T <= 64, T*k <= 1024, n_group <= 64)
+ * both steps run in a single one-block kernel, which saves a launch on the
+ * latency-bound decode path; otherwise the two kernels of the separate calls
+ * run back to back.  ws / ws_bytes as for moe_align.
+ */
+MOE_API moe_status moe_route_align(const float* logits, int T, int E, int k,
+                           int n_group, int topk_group, moe_group_score group_score,
+                           int renormalize, float routed_scaling, int block_m,
+                           int32_t* topk_ids, float* topk_weights,
+                           int32_t* sorted_token_ids, int32_t* expert_ids,
+                           int32_t* num_tokens_post_padded, int32_t* inv_pos,
+                           void* ws, size_t ws_bytes,
+                           int32_t* dev_status, moe_stream_t stream);
+
 /* Synchronises `stream`, then returns the code stored in dev_status (MOE_OK
  * when 0), or MOE_ERR_CUDA if the synchronisation or the copy failed. */
 MOE_API moe_status moe_read_status(const int32_t* dev_status, moe_stream_t stream);
@@ -226,7 +244,10 @@ MOE_API int moe_last_launch_count(void);
  * around each of its kernels (events come from a pool the library owns; the
  * calls may be captured into a CUDA graph, where the records become event
  * nodes that are re-recorded at every replay).
- * Stages: 0 route, 1 align, 2 gate/up (fc1) GEMM, 3 down GEMM, 4 combine.
+ * Stages: 0 route, 1 align, 2 gate/up (fc1) GEMM, 3 down GEMM, 4 combine,
+ * 5 fused route+align (moe_route_align on a small batch), 6 fused expert
+ * kernel (moe_forward with block_m <= 64: both GEMMs, and the combine when
+ * T <= 64).
  * moe_profile_enable(1) starts a fresh record (and primes the event pool),
  * (0) stops recording and keeps what was recorded.  moe_profile_collect waits for the recorded events,
  * writes into stage_ms[i] (i < n_stages) the summed milliseconds of stage i
@@ -234,7 +255,7 @@ MOE_API int moe_last_launch_count(void);
  * release != 0 it then returns the events to the pool and clears the record
  * (release == 0 keeps them, e.g. to read a graph's events after each
  * replay).  MOE_ERR_CUDA if an event call failed. */
-#define MOE_NUM_STAGES 5
+#define MOE_NUM_STAGES 7
 MOE_API moe_status moe_profile_enable(int on);
 MOE_API moe_status moe_profile_collect(double* stage_ms, int* stage_calls, int n_stages, int release);
 

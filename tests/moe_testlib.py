@@ -64,12 +64,15 @@ class DeviceLayer:
         self.w2s = bf16_dev(inp.w2_shared, device) if c.n_shared else None
         self.buf = M.MoEBuffers(c.T, c.d, c.F, c.E, c.k, c.block_m, c.act, c.n_shared, device)
 
-    def run(self, route=True, align=True):
+    def run(self, route=True, align=True, fused_route_align=False):
         b = self.buf
-        if route:
-            b.route(self.logits, **route_kwargs(self.cfg))
-        if align:
-            b.align()
+        if fused_route_align:
+            b.route_align(self.logits, **route_kwargs(self.cfg))
+        else:
+            if route:
+                b.route(self.logits, **route_kwargs(self.cfg))
+            if align:
+                b.align()
         return b.forward(self.x, self.w13, self.w2, self.w13s, self.w2s)
 
     def status(self) -> int:

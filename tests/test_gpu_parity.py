@@ -37,6 +37,12 @@ SMALL = {
                                      seed=2008),
     "one_expert_hot": CFG["tiny"].with_(name="one_expert_hot", T=700, d=128, F=128, E=4, k=1, block_m=128,
                                         seed=2009, logits_kind="decode_hot"),
+    # fused expert kernel (block_m <= 64) with a shared expert, with the
+    # in-kernel combine (T <= 64) and with the separate combine (T > 64)
+    "shared_bm16_fused_combine": CFG["dsv3"].with_(name="shared_bm16_fused_combine", T=40, d=256, F=192,
+                                                   block_m=16, seed=2010),
+    "shared_bm32_sep_combine": CFG["dsv3"].with_(name="shared_bm32_sep_combine", T=100, d=320, F=128,
+                                                 block_m=32, seed=2011),
 }
 
 
@@ -272,4 +278,36 @@ def test_profile_events_cover_every_kernel():
     st = M.moe_profile_collect()
     assert st["route"][1] == 1 and st["gate_up_gemm"][1] == 1 and st["down_gemm"][1] == 1
     assert st["combine"][1] == 1 and st["align"][1] == 1
-    assert all(ms > 0.0 for ms, _ in st.values())
+    assert all(ms > 0.0 for ms, n in st.values() if n)
+    # the small-batch path: one fused route+align kernel, one fused expert kernel
+    lay = DeviceLayer(W.make_inputs(SMALL["decode"]))
+    lay.buf.route_align(lay.logits)
+    lay.buf.forward(lay.x, lay.w13, lay.w2)
+    M.moe_profile_enable(True)
+    lay.buf.route_align(lay.logits)
+    lay.buf.forward(lay.x, lay.w13, lay.w2)
+    M.moe_profile_enable(False)
+    st = M.moe_profile_collect()
+    assert st["route_align"][1] == 1 and st["fused_expert"][1] == 1
+    assert st["combine"][1] == 0 and st["gate_up_gemm"][1] == 0
+
+
+@pytest.mark.parametrize("name,T", [("tiny", None), ("decode", None), ("relu2_small", None), ("dsv3_small", 16),
+                                    ("dsv3_small", 300), ("swap_bm32", 64), ("zipf_small", None)])
+def test_route_align_matches_separate_calls(name, T):
+    cfg = SMALL[name] if T is None else SMALL[name].with_(T=T)
+    inp = W.make_inputs(cfg)
+    a = DeviceLayer(inp)
+    b = DeviceLayer(inp)
+    a.buf.route(a.logits, **route_kwargs(cfg))
+    a.buf.align()
+    b.buf.route_align(b.logits, **route_kwargs(cfg))
+    torch.cuda.synchronize()
+    assert b.status() == 0
+    S = cfg.T * cfg.k
+    for attr in ("topk_ids", "topk_weights", "sorted_token_ids", "expert_ids", "ntpp"):
+        x, y = getattr(a.buf, attr), getattr(b.buf, attr)
+        assert torch.equal(x.view(torch.int32), y.view(torch.int32)), attr
+    assert torch.equal(a.buf.inv_pos[:S], b.buf.inv_pos[:S])
+    ids, w = oracle_route(inp)
+    compare_route(b.buf.topk_ids.cpu().numpy(), b.buf.topk_weights.cpu().numpy(), ids, w, name)
