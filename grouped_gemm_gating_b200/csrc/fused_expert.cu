@@ -19,7 +19,9 @@
 // (h stores, __threadfence, atomicAdd on ready[block]); the down tile's
 // gather warps poll ready[block] with ld.acquire before loading h.  The TMA
 // warp streams the down tile's W2 slices without waiting, so the down
-// GEMM's weight traffic overlaps the tail of the gate/up phase.
+// GEMM's weight traffic overlaps the tail of the gate/up phase.  Before a
+// gather warp blocks on ready[], it signals every stage it has filled, so a
+// CTA never waits on others while holding back work they may depend on.
 //
 // Combine (do_combine): the CTA that finishes the last down tile of a
 // d-column tile (done[column tile] reaches the number of blocks) sums, for
@@ -383,19 +385,33 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
         }
       } else {
         K = args.F;
-        // wait until every gate/up tile of this block has published its h
-        if (lane == 0) {
-          const uint64_t t0 = ptx::globaltimer_ns();
-          while (ld_acquire(args.ready + t.blk) < n_wt1) {
-            if (*abort_flag || ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
-              fail();
-              ok = false;
-              break;
-            }
-            __nanosleep(64);
+        // wait until every gate/up tile of this block has published its h.
+        // Never wait on another tile while holding stages this thread has
+        // filled but not yet signalled: this CTA's own gate/up tile may need
+        // them to finish, and other CTAs may be waiting for that tile.
+        int ready = 0;
+        if (lane == 0) ready = ld_acquire(args.ready + t.blk) >= n_wt1 ? 1 : 0;
+        ready = __shfl_sync(0xffffffffu, ready, 0);
+        if (!ready) {
+          ptx::cp_async_wait<0>();
+          ptx::fence_proxy_async_smem();
+          for (; pend > 0; --pend) {
+            ptx::mbar_arrive(&full[astage]);
+            if (++astage == C::kStages) astage = 0;
           }
+          if (lane == 0) {
+            const uint64_t t0 = ptx::globaltimer_ns();
+            while (ld_acquire(args.ready + t.blk) < n_wt1) {
+              if (*abort_flag || ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+                fail();
+                ok = false;
+                break;
+              }
+              __nanosleep(64);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         __syncwarp();  // orders every lane's h loads after lane 0's acquire
         if (!ok) break;
 #pragma unroll
