@@ -58,14 +58,16 @@ struct FusedCfg {
                                    : kTmemNeed <= 256 ? 256
                                                       : 512;
   static constexpr int kNumThreads = 320;
-  static constexpr int kGatherLag = 2;
+  // stages a gather thread keeps in flight before signalling the oldest; at
+  // most kStages - 1, since issuing stage s + lag needs stage s - 1 consumed
+  static constexpr int kGatherLag = kStages - 1;
   static constexpr uint32_t kTx1 = kWBytes;
   static constexpr uint32_t kTx2 = kW2Rows * 128;
   static constexpr int kBarrierBytes = 256;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes;
   static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(128, TOK);
   static_assert(TOK == 16 || TOK == 32 || TOK == 64, "token rows per tile");
-  static_assert(kStages >= kGatherLag + 2, "pipeline depth");
+  static_assert(kGatherLag >= 1 && kGatherLag <= kStages - 1 && kStages >= 3, "pipeline depth");
   static_assert((2 * kStages + 4) * 8 + 16 <= kBarrierBytes, "barrier area");
   static_assert(kSmemBytes <= 232448, "shared memory per block");
 };

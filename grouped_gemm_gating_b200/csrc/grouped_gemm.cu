@@ -58,7 +58,9 @@ struct GemmCfg {
                                    : kTmemNeed <= 256 ? 256
                                                       : 512;
   static constexpr int kNumThreads = kGather ? 320 : 192;
-  static constexpr int kGatherLag = 2;
+  // stages a gather thread keeps in flight before signalling the oldest; at
+  // most kStages - 1, since issuing stage s + lag needs stage s - 1 consumed
+  static constexpr int kGatherLag = kStages - 1;
   static constexpr uint32_t kTxBytes = kWBytes + (kGather ? 0 : kXBytes);
   static constexpr int kBarrierBytes = 256;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes;
@@ -66,7 +68,7 @@ struct GemmCfg {
 
   static_assert(TOK % 16 == 0 && TOK >= 16 && TOK <= 128, "token rows per tile");
   static_assert(SWAP || TOK == 128, "token-major tiles hold 128 token rows");
-  static_assert(kStages >= kGatherLag + 2, "pipeline depth");
+  static_assert(kGatherLag >= 1 && kGatherLag <= kStages - 1 && kStages >= 3, "pipeline depth");
   static_assert(kAccCols * 2 <= 512, "two accumulator buffers must fit TMEM");
   static_assert((2 * kStages + 4) * 8 + 8 <= kBarrierBytes, "barrier area");
   static_assert(kSmemBytes <= 232448, "shared memory per block");
