@@ -358,6 +358,9 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
       fa.tm_w13s = fa.tm_w13;
       fa.tm_w2s = fa.tm_w2;
     }
+    if (!encode_2d(&fa.tm_x, x, d, static_cast<uint64_t>(T), 1) ||
+        !encode_2d(&fa.tm_h, h, F, static_cast<uint64_t>(P_total), static_cast<uint32_t>(bm)))
+      return MOE_ERR_CUDA;
     fa.x = x;
     fa.h = h;
     fa.y = y;
@@ -409,6 +412,7 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   } else {
     a1.tm_ws = a1.tm_w;
   }
+  if (!encode_2d(&a1.tm_x, x, d, static_cast<uint64_t>(T), 1)) return MOE_ERR_CUDA;
   a1.x = x;
   a1.sorted_ids = sorted_token_ids;
   a1.expert_ids = expert_ids;

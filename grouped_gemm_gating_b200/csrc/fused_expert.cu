@@ -16,12 +16,13 @@
 // and no CTA waits on work queued behind itself; all CTAs are co-resident
 // (one per SM, grid <= SM count).  A down tile needs the block's full h rows:
 // the gate/up epilogue publishes each finished tile with a release pattern
-// (h stores, __threadfence, atomicAdd on ready[block]); the down tile's
-// gather warps poll ready[block] with ld.acquire before loading h.  The TMA
-// warp streams the down tile's W2 slices without waiting, so the down
-// GEMM's weight traffic overlaps the tail of the gate/up phase.  Before a
-// gather warp blocks on ready[], it signals every stage it has filled, so a
-// CTA never waits on others while holding back work they may depend on.
+// (h stores, a generic-to-async proxy fence, __threadfence, atomicAdd on
+// ready[block]); the token warp polls ready[block] with ld.acquire, fences
+// the proxies again and only then loads the block's h rows by TMA.  The
+// weight warp streams the down tile's W2 slices without waiting, so the down
+// GEMM's weight traffic overlaps the tail of the gate/up phase.  Both
+// operands of every stage arrive by TMA and complete transaction bytes on
+// the stage's barrier, so no warp holds back a stage another tile needs.
 //
 // Combine (do_combine): the CTA that finishes the last down tile of a
 // d-column tile (done[column tile] reaches the number of blocks) sums, for
@@ -57,17 +58,14 @@ struct FusedCfg {
                                    : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256
                                                       : 512;
-  static constexpr int kNumThreads = 320;
-  // stages a gather thread keeps in flight before signalling the oldest; at
-  // most kStages - 1, since issuing stage s + lag needs stage s - 1 consumed
-  static constexpr int kGatherLag = kStages - 1;
+  static constexpr int kNumThreads = 224;
   static constexpr uint32_t kTx1 = kWBytes;
   static constexpr uint32_t kTx2 = kW2Rows * 128;
   static constexpr int kBarrierBytes = 256;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes;
   static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(128, TOK);
   static_assert(TOK == 16 || TOK == 32 || TOK == 64, "token rows per tile");
-  static_assert(kGatherLag >= 1 && kGatherLag <= kStages - 1 && kStages >= 3, "pipeline depth");
+  static_assert(kStages >= 3, "pipeline depth");
   static_assert((2 * kStages + 4) * 8 + 16 <= kBarrierBytes, "barrier area");
   static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
@@ -124,7 +122,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      ptx::mbar_init(&full[s], 1 + 128);
+      ptx::mbar_init(&full[s], 2);
       ptx::mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -135,6 +133,8 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&args.tm_w13);
     ptx::prefetch_tmap(&args.tm_w2);
+    ptx::prefetch_tmap(&args.tm_x);
+    ptx::prefetch_tmap(&args.tm_h);
     if (args.n_shared_blocks) {
       ptx::prefetch_tmap(&args.tm_w13s);
       ptx::prefetch_tmap(&args.tm_w2s);
@@ -326,6 +326,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
         aphase ^= 1u;
       }
       // publish the finished tile
+      if (t.phase == 1) ptx::fence_proxy_async_global();  // h is read back by TMA
       __threadfence();
       epilogue_sync();
       if (t.phase == 1) {
@@ -351,111 +352,70 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
         }
       }
     }
-  } else {
-    // ------------------------------------------------ row gather (x, then h)
-    constexpr int kRowsPerThread = TOK / 16;
-    constexpr int kLag = C::kGatherLag;
-    const int gtid = threadIdx.x - 192;
-    const int chunk = gtid & 7;
-    const int r0 = gtid >> 3;
-    int stage = 0, astage = 0, pend = 0;
+  } else if (warp == 6) {
+    // ------------------------------------------------ token operand (TMA)
+    // gate/up tiles: lane l gathers x rows 4l..4l+3 of the block;
+    // down tiles: lane 0 loads the block's h rows once they are published
+    const bool active = 4 * lane < TOK;
+    int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < total_tiles; u += gridDim.x) {
       const Tile t = fused_tile(u, n1_tiles, n_wt1, n_wt2, routed_blocks);
-      const uint16_t* src[kRowsPerThread];
-      uint32_t nbytes[kRowsPerThread];
-      int K;
+      int rows[4] = {args.T, args.T, args.T, args.T};
       if (t.phase == 1) {
-        K = args.d;
 #pragma unroll
-        for (int i = 0; i < kRowsPerThread; ++i) {
-          const int r = r0 + 16 * i;
-          int tok;
-          bool valid;
+        for (int i = 0; i < 4; ++i) {
+          const int r = 4 * lane + i;
+          if (!active) continue;
           if (!t.shared_blk) {
             const int slot = args.sorted_ids[t.blk * args.block_m + r];
-            valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
-            tok = valid ? slot / args.k : 0;
+            if (static_cast<unsigned>(slot) < static_cast<unsigned>(args.S)) rows[i] = slot / args.k;
           } else {
-            tok = (t.blk - routed_blocks) * args.block_m + r;
-            valid = tok < args.T;
-            if (!valid) tok = 0;
+            const int tok = (t.blk - routed_blocks) * args.block_m + r;
+            if (tok < args.T) rows[i] = tok;
           }
-          src[i] = args.x + static_cast<size_t>(tok) * K + chunk * 8;
-          nbytes[i] = valid ? 16u : 0u;
         }
-      } else {
-        K = args.F;
-        // wait until every gate/up tile of this block has published its h.
-        // Never wait on another tile while holding stages this thread has
-        // filled but not yet signalled: this CTA's own gate/up tile may need
-        // them to finish, and other CTAs may be waiting for that tile.
-        int ready = 0;
-        if (lane == 0) ready = ld_acquire(args.ready + t.blk) >= n_wt1 ? 1 : 0;
-        ready = __shfl_sync(0xffffffffu, ready, 0);
-        if (!ready) {
-          ptx::cp_async_wait<0>();
-          ptx::fence_proxy_async_smem();
-          for (; pend > 0; --pend) {
-            ptx::mbar_arrive(&full[astage]);
-            if (++astage == C::kStages) astage = 0;
+      } else if (lane == 0) {
+        // wait until every gate/up tile of this block has published its h
+        const uint64_t t0 = ptx::globaltimer_ns();
+        while (ld_acquire(args.ready + t.blk) < n_wt1) {
+          if (*abort_flag || ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+            fail();
+            ok = false;
+            break;
           }
-          if (lane == 0) {
-            const uint64_t t0 = ptx::globaltimer_ns();
-            while (ld_acquire(args.ready + t.blk) < n_wt1) {
-              if (*abort_flag || ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
-                fail();
-                ok = false;
-                break;
-              }
-              __nanosleep(64);
-            }
-          }
-          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          __nanosleep(64);
         }
-        __syncwarp();  // orders every lane's h loads after lane 0's acquire
-        if (!ok) break;
-#pragma unroll
-        for (int i = 0; i < kRowsPerThread; ++i) {
-          const int r = r0 + 16 * i;
-          src[i] = args.h + static_cast<size_t>(t.blk * args.block_m + r) * K + chunk * 8;
-          nbytes[i] = 16u;
-        }
+        ptx::fence_proxy_async_global();
       }
-      const int nk = K / 64;
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      const int nk = t.phase == 1 ? nk1 : nk2;
       for (int kb = 0; kb < nk; ++kb) {
-        if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
-          fail();
+        int good = 1;
+        if (lane == 0) {
+          good = ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs) ? 1 : 0;
+          if (good) ptx::mbar_arrive_expect_tx(&full[stage], C::kXBytes);
+        }
+        good = __shfl_sync(0xffffffffu, good, 0);
+        if (!good) {
+          if (lane == 0) fail();
           ok = false;
           break;
         }
-        const uint32_t sX = ptx::smem_u32(smem + stage * C::kStageBytes + C::kWBytes);
-#pragma unroll
-        for (int i = 0; i < kRowsPerThread; ++i) {
-          const int r = r0 + 16 * i;
-          const uint32_t dst = sX + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4);
-          ptx::cp_async_16(dst, src[i] + kb * 64, nbytes[i]);
+        uint8_t* sX = smem + stage * C::kStageBytes + C::kWBytes;
+        if (t.phase == 1) {
+          if (active)
+            ptx::tma_gather4(sX + lane * 512, &args.tm_x, &full[stage], kb * 64, rows[0], rows[1], rows[2], rows[3]);
+        } else if (lane == 0) {
+          ptx::tma_load_2d(sX, &args.tm_h, &full[stage], kb * 64, t.blk * args.block_m);
         }
-        ptx::cp_async_commit();
         if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;
         }
-        if (++pend > kLag) {
-          ptx::cp_async_wait<kLag>();
-          ptx::fence_proxy_async_smem();
-          ptx::mbar_arrive(&full[astage]);
-          if (++astage == C::kStages) astage = 0;
-          --pend;
-        }
       }
-    }
-    ptx::cp_async_wait<0>();
-    ptx::fence_proxy_async_smem();
-    for (; pend > 0; --pend) {
-      ptx::mbar_arrive(&full[astage]);
-      if (++astage == C::kStages) astage = 0;
     }
   }
 

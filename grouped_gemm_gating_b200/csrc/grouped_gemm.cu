@@ -25,10 +25,14 @@
 //   warp 0       TMA producer: weight tiles (and h tiles for the down GEMM)
 //   warp 1       TMEM allocator and MMA issuer (one thread)
 //   warps 2..5   epilogue: TMEM -> registers -> activation -> bf16 -> global
-//   warps 6..9   gate/up GEMM only: row gather of x through sorted_token_ids
-//                with 16-byte cp.async into the 128B-swizzled layout
-// Shared-memory stages are guarded by full/empty mbarriers, the two TMEM
-// accumulator buffers by tmem-full/tmem-empty mbarriers.  Every wait is
+//   warp 6       gate/up GEMM only: row gather of x through sorted_token_ids
+//                with TMA gather4 loads (each lane fetches 4 token rows of a
+//                64-column slice; padding rows use an out-of-range row index
+//                and arrive as zeros)
+// Shared-memory stages are guarded by full/empty mbarriers (every operand
+// arrives by TMA and completes transaction bytes on the stage's full
+// barrier), the two TMEM accumulator buffers by tmem-full/tmem-empty
+// mbarriers.  Every wait is
 // bounded in time; on expiry the kernel records MOE_ERR_DEVICE_TIMEOUT and
 // all roles leave their loops so the CTA frees its TMEM and exits.
 #include "common.cuh"
@@ -57,10 +61,7 @@ struct GemmCfg {
                                    : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256
                                                       : 512;
-  static constexpr int kNumThreads = kGather ? 320 : 192;
-  // stages a gather thread keeps in flight before signalling the oldest; at
-  // most kStages - 1, since issuing stage s + lag needs stage s - 1 consumed
-  static constexpr int kGatherLag = kStages - 1;
+  static constexpr int kNumThreads = kGather ? 224 : 192;
   static constexpr uint32_t kTxBytes = kWBytes + (kGather ? 0 : kXBytes);
   static constexpr int kBarrierBytes = 256;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes;
@@ -68,7 +69,7 @@ struct GemmCfg {
 
   static_assert(TOK % 16 == 0 && TOK >= 16 && TOK <= 128, "token rows per tile");
   static_assert(SWAP || TOK == 128, "token-major tiles hold 128 token rows");
-  static_assert(kGatherLag >= 1 && kGatherLag <= kStages - 1 && kStages >= 3, "pipeline depth");
+  static_assert(kStages >= 3, "pipeline depth");
   static_assert(kAccCols * 2 <= 512, "two accumulator buffers must fit TMEM");
   static_assert((2 * kStages + 4) * 8 + 8 <= kBarrierBytes, "barrier area");
   static_assert(kSmemBytes <= 232448, "shared memory per block");
@@ -107,7 +108,7 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      ptx::mbar_init(&full[s], 1 + (C::kGather ? 128 : 0));
+      ptx::mbar_init(&full[s], C::kGather ? 2 : 1);
       ptx::mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
   if (threadIdx.x == 0) {
     ptx::prefetch_tmap(&args.tm_w);
     if (args.n_shared_blocks) ptx::prefetch_tmap(&args.tm_ws);
-    if (EPI == kEpiScale) ptx::prefetch_tmap(&args.tm_x);
+    ptx::prefetch_tmap(&args.tm_x);
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -370,69 +371,50 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
         aphase ^= 1u;
       }
     }
-  } else if (C::kGather) {
-    // ------------------------------------------------ row gather of x
-    constexpr int kRowsPerThread = TOK / 16;
-    constexpr int kLag = C::kGatherLag;
-    const int gtid = threadIdx.x - 192;
-    const int chunk = gtid & 7;
-    const int r0 = gtid >> 3;
-    int stage = 0, astage = 0, pend = 0;
+  } else if (C::kGather && warp == 6) {
+    // ------------------------------------------------ row gather of x (TMA)
+    // lane l fetches token rows 4l..4l+3 of the tile's block
+    const bool active = 4 * lane < TOK;
+    int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
       const TileCoord tc = tile_coord(tile, n_wt, routed_blocks);
-      const uint16_t* src[kRowsPerThread];
-      uint32_t nbytes[kRowsPerThread];
+      int rows[4];
 #pragma unroll
-      for (int i = 0; i < kRowsPerThread; ++i) {
-        const int r = r0 + 16 * i;
-        int tok;
-        bool valid;
-        if (!tc.shared_blk) {
-          const int slot = args.sorted_ids[tc.blk * args.block_m + r];
-          valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
-          tok = valid ? slot / args.k : 0;
-        } else {
-          tok = (tc.blk - routed_blocks) * args.block_m + r;
-          valid = tok < args.T;
-          if (!valid) tok = 0;
+      for (int i = 0; i < 4; ++i) {
+        const int r = 4 * lane + i;
+        int tok = args.T;  // out of range: the row arrives as zeros
+        if (active) {
+          if (!tc.shared_blk) {
+            const int slot = args.sorted_ids[tc.blk * args.block_m + r];
+            if (static_cast<unsigned>(slot) < static_cast<unsigned>(args.S)) tok = slot / args.k;
+          } else {
+            const int t = (tc.blk - routed_blocks) * args.block_m + r;
+            if (t < args.T) tok = t;
+          }
         }
-        src[i] = args.x + static_cast<size_t>(tok) * args.K + chunk * 8;
-        nbytes[i] = valid ? 16u : 0u;
+        rows[i] = tok;
       }
       for (int kb = 0; kb < nk; ++kb) {
-        if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
-          fail();
+        int good = 1;
+        if (lane == 0) {
+          good = ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs) ? 1 : 0;
+          if (good) ptx::mbar_arrive_expect_tx(&full[stage], C::kXBytes);
+        }
+        good = __shfl_sync(0xffffffffu, good, 0);
+        if (!good) {
+          if (lane == 0) fail();
           ok = false;
           break;
         }
-        const uint32_t sX = ptx::smem_u32(smem + stage * C::kStageBytes + C::kWBytes);
-#pragma unroll
-        for (int i = 0; i < kRowsPerThread; ++i) {
-          const int r = r0 + 16 * i;
-          const uint32_t dst = sX + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4);
-          ptx::cp_async_16(dst, src[i] + kb * 64, nbytes[i]);
-        }
-        ptx::cp_async_commit();
+        uint8_t* sX = smem + stage * C::kStageBytes + C::kWBytes;
+        if (active) ptx::tma_gather4(sX + lane * 512, &args.tm_x, &full[stage], kb * 64, rows[0], rows[1], rows[2], rows[3]);
         if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;
         }
-        if (++pend > kLag) {
-          ptx::cp_async_wait<kLag>();
-          ptx::fence_proxy_async_smem();
-          ptx::mbar_arrive(&full[astage]);
-          if (++astage == C::kStages) astage = 0;
-          --pend;
-        }
       }
-    }
-    ptx::cp_async_wait<0>();
-    ptx::fence_proxy_async_smem();
-    for (; pend > 0; --pend) {
-      ptx::mbar_arrive(&full[astage]);
-      if (++astage == C::kStages) astage = 0;
     }
   }
 
