@@ -151,9 +151,6 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool valid_block_m(int bm) { return bm == 16 || bm == 32 || bm == 64 || bm == 128; }
 
 constexpr size_t kWsAlign = 256;
-// Batches up to this many tokens let the fused expert kernel do the
-// scatter-reduce itself (one CTA per d-column tile sums every token).
-constexpr int kFusedCombineMaxT = 64;
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -358,9 +355,7 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
       fa.tm_w13s = fa.tm_w13;
       fa.tm_w2s = fa.tm_w2;
     }
-    if (!encode_2d(&fa.tm_x, x, d, static_cast<uint64_t>(T), 1) ||
-        !encode_2d(&fa.tm_h, h, F, static_cast<uint64_t>(P_total), static_cast<uint32_t>(bm)))
-      return MOE_ERR_CUDA;
+    if (!encode_2d(&fa.tm_h, h, F, static_cast<uint64_t>(P_total), static_cast<uint32_t>(bm))) return MOE_ERR_CUDA;
     fa.x = x;
     fa.h = h;
     fa.y = y;
@@ -382,7 +377,7 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
     fa.block_m = bm;
     fa.max_routed_blocks = max_routed_blocks;
     fa.n_shared_blocks = n_shared_blocks;
-    fa.do_combine = T <= kFusedCombineMaxT ? 1 : 0;
+    fa.do_combine = moe::fused_expert_combines(T, k, n_shared) ? 1 : 0;
     const int64_t tiles = static_cast<int64_t>(total_blocks_max) * ((F + 127) / 128 + n_dtiles);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
     cudaError_t err = cudaMemsetAsync(counters, 0, static_cast<size_t>(total_blocks_max + n_dtiles) * 4, s);
@@ -412,7 +407,7 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   } else {
     a1.tm_ws = a1.tm_w;
   }
-  if (!encode_2d(&a1.tm_x, x, d, static_cast<uint64_t>(T), 1)) return MOE_ERR_CUDA;
+  a1.tm_x = a1.tm_w;  // unused by the gate/up GEMM (rows are gathered with cp.async)
   a1.x = x;
   a1.sorted_ids = sorted_token_ids;
   a1.expert_ids = expert_ids;

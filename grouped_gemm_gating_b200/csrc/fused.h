@@ -12,7 +12,6 @@ struct FusedArgs {
   CUtensorMap tm_w13s;  // shared expert, 3-D {d, N1, 1}
   CUtensorMap tm_w2;    // routed down weights, 3-D {F, d, E}, 128-row boxes
   CUtensorMap tm_w2s;   // shared expert, 3-D {F, d, 1}
-  CUtensorMap tm_x;     // x, 2-D {d, T}, 64 x 1 boxes (row gather)
   CUtensorMap tm_h;     // h, 2-D {F, P_total}, 64 x block_m boxes
   const uint16_t* x;    // [T, d] bf16
   uint16_t* h;          // [P_total, F] bf16 (workspace)
@@ -30,10 +29,12 @@ struct FusedArgs {
   int block_m;
   int max_routed_blocks;
   int n_shared_blocks;
-  int do_combine;       // 1: the kernel also writes out (small batches)
+  int do_combine;       // 1: the kernel also writes out (fused_expert_combines)
 };
 
 bool fused_expert_supported(int block_m);
+// True when the fused kernel also does the scatter-reduce (T*k <= 64, no shared expert).
+bool fused_expert_combines(int T, int k, int n_shared);
 cudaError_t launch_fused_expert(int act_epi, int block_m, const FusedArgs& args, int grid, cudaStream_t stream);
 
 }  // namespace moe

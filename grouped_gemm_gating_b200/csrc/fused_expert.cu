@@ -17,18 +17,20 @@
 // (one per SM, grid <= SM count).  A down tile needs the block's full h rows:
 // the gate/up epilogue publishes each finished tile with a release pattern
 // (h stores, a generic-to-async proxy fence, __threadfence, atomicAdd on
-// ready[block]); the token warp polls ready[block] with ld.acquire, fences
-// the proxies again and only then loads the block's h rows by TMA.  The
-// weight warp streams the down tile's W2 slices without waiting, so the down
-// GEMM's weight traffic overlaps the tail of the gate/up phase.  Both
-// operands of every stage arrive by TMA and complete transaction bytes on
-// the stage's barrier, so no warp holds back a stage another tile needs.
+// ready[block]); one token-loader thread polls ready[block] with ld.acquire,
+// fences the proxies again and only then loads the block's h rows by TMA.
+// The weight warp streams the down tile's W2 slices without waiting, so the
+// down GEMM's weight traffic overlaps the tail of the gate/up phase.  Every
+// stage is signalled as soon as its bytes land (TMA transaction bytes;
+// cp.async.mbarrier.arrive.noinc for gathered rows), so no warp holds back a
+// stage that another tile needs while it waits.
 //
-// Combine (do_combine): the CTA that finishes the last down tile of a
-// d-column tile (done[column tile] reaches the number of blocks) sums, for
-// that column range, out[t] = sum_j y[inv_pos[t*k + j]] (+ the shared
-// expert's row) in fp32 in slot order and writes bf16: the same arithmetic as
-// the combine kernel.
+// Combine (do_combine, T*k <= 64, no shared expert): the CTA that finishes
+// the last down tile of a d-column tile (done[column tile] reaches the
+// number of blocks) sums, for that column range, out[t] = sum_j
+// y[inv_pos[t*k + j]] in fp32 in slot order and writes bf16 -- the same
+// arithmetic as the combine kernel; all its loads are issued before the
+// first sum so the tail costs two memory round trips.
 //
 // Every wait is bounded in time; on expiry the kernel records
 // MOE_ERR_DEVICE_TIMEOUT and all roles leave their loops.
@@ -58,7 +60,7 @@ struct FusedCfg {
                                    : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256
                                                       : 512;
-  static constexpr int kNumThreads = 224;
+  static constexpr int kNumThreads = 320;
   static constexpr uint32_t kTx1 = kWBytes;
   static constexpr uint32_t kTx2 = kW2Rows * 128;
   static constexpr int kBarrierBytes = 256;
@@ -94,6 +96,9 @@ __device__ __forceinline__ Tile fused_tile(int u, int n1_tiles, int n_wt1, int n
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
+// Slots (T * k) up to which the kernel does the scatter-reduce itself.
+constexpr int kCombineMaxSlots = 64;
+
 __device__ __forceinline__ int ld_acquire(const int32_t* p) {
   int v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -122,7 +127,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      ptx::mbar_init(&full[s], 2);
+      ptx::mbar_init(&full[s], 1 + 128);
       ptx::mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -133,7 +138,6 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&args.tm_w13);
     ptx::prefetch_tmap(&args.tm_w2);
-    ptx::prefetch_tmap(&args.tm_x);
     ptx::prefetch_tmap(&args.tm_h);
     if (args.n_shared_blocks) {
       ptx::prefetch_tmap(&args.tm_w13s);
@@ -230,6 +234,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
             break;
           }
           ptx::tc_fence_after();
+          ptx::fence_proxy_async_smem();
           const uint32_t sW = ptx::smem_u32(smem + stage * C::kStageBytes);
           const uint32_t sX = sW + C::kWBytes;
 #pragma unroll
@@ -335,48 +340,73 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
         if (etid == 0) *last_flag = (atomicAdd(&args.done[t.wt], 1) == total_blocks - 1) ? 1 : 0;
         epilogue_sync();
         if (*last_flag) {
-          // this CTA finished the last down tile of column tile t.wt
+          // this CTA finished the last down tile of column tile t.wt: every
+          // load first (independent), then the sums in slot order
           __threadfence();
           const int c = t.wt * 128 + row;
+          const int nslot = args.T * args.k;
           if (c < args.d) {
-            for (int tok = 0; tok < args.T; ++tok) {
-              float acc = 0.0f;
-              for (int j = 0; j < args.k; ++j) {
-                const int pr = args.inv_pos[static_cast<size_t>(tok) * args.k + j];
-                acc += __ldcg(args.y + static_cast<size_t>(pr) * args.d + c);
+            int pr[kCombineMaxSlots];
+            float v[kCombineMaxSlots];
+#pragma unroll
+            for (int i = 0; i < kCombineMaxSlots; ++i)
+              if (i < nslot) pr[i] = __ldcg(args.inv_pos + i);
+#pragma unroll
+            for (int i = 0; i < kCombineMaxSlots; ++i)
+              if (i < nslot) v[i] = __ldcg(args.y + static_cast<size_t>(pr[i]) * args.d + c);
+            float acc = 0.0f;
+            int j = 0, tok = 0;
+#pragma unroll
+            for (int i = 0; i < kCombineMaxSlots; ++i) {
+              if (i < nslot) {
+                acc += v[i];
+                if (++j == args.k) {
+                  args.out[static_cast<size_t>(tok) * args.d + c] = float_to_bf16_bits(acc);
+                  acc = 0.0f;
+                  j = 0;
+                  ++tok;
+                }
               }
-              if (args.n_shared_blocks) acc += __ldcg(args.y + static_cast<size_t>(*args.ntpp + tok) * args.d + c);
-              args.out[static_cast<size_t>(tok) * args.d + c] = float_to_bf16_bits(acc);
             }
           }
         }
       }
     }
-  } else if (warp == 6) {
-    // ------------------------------------------------ token operand (TMA)
-    // gate/up tiles: lane l gathers x rows 4l..4l+3 of the block;
-    // down tiles: lane 0 loads the block's h rows once they are published
-    const bool active = 4 * lane < TOK;
+  } else {
+    // ------------------------------------------------ token operand
+    // gate/up tiles: 128 threads gather the block's x rows with cp.async;
+    // down tiles: thread 0 loads the block's h rows by TMA once published,
+    // the others only arrive
+    constexpr int kRowsPerThread = TOK / 16;
+    const int gtid = threadIdx.x - 192;
+    const int chunk = gtid & 7;
+    const int r0 = gtid >> 3;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < total_tiles; u += gridDim.x) {
       const Tile t = fused_tile(u, n1_tiles, n_wt1, n_wt2, routed_blocks);
-      int rows[4] = {args.T, args.T, args.T, args.T};
+      const uint16_t* src[kRowsPerThread];
+      uint32_t nbytes[kRowsPerThread];
       if (t.phase == 1) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = 4 * lane + i;
-          if (!active) continue;
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          const int r = r0 + 16 * i;
+          int tok = 0;
+          bool valid;
           if (!t.shared_blk) {
             const int slot = args.sorted_ids[t.blk * args.block_m + r];
-            if (static_cast<unsigned>(slot) < static_cast<unsigned>(args.S)) rows[i] = slot / args.k;
+            valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
+            if (valid) tok = slot / args.k;
           } else {
-            const int tok = (t.blk - routed_blocks) * args.block_m + r;
-            if (tok < args.T) rows[i] = tok;
+            tok = (t.blk - routed_blocks) * args.block_m + r;
+            valid = tok < args.T;
+            if (!valid) tok = 0;
           }
+          src[i] = args.x + static_cast<size_t>(tok) * args.d + chunk * 8;
+          nbytes[i] = valid ? 16u : 0u;
         }
-      } else if (lane == 0) {
+      } else if (gtid == 0) {
         // wait until every gate/up tile of this block has published its h
         const uint64_t t0 = ptx::globaltimer_ns();
         while (ld_acquire(args.ready + t.blk) < n_wt1) {
@@ -389,27 +419,28 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
         }
         ptx::fence_proxy_async_global();
       }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
       const int nk = t.phase == 1 ? nk1 : nk2;
-      for (int kb = 0; kb < nk; ++kb) {
-        int good = 1;
-        if (lane == 0) {
-          good = ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs) ? 1 : 0;
-          if (good) ptx::mbar_arrive_expect_tx(&full[stage], C::kXBytes);
-        }
-        good = __shfl_sync(0xffffffffu, good, 0);
-        if (!good) {
-          if (lane == 0) fail();
+      for (int kb = 0; ok && kb < nk; ++kb) {
+        if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+          fail();
           ok = false;
           break;
         }
-        uint8_t* sX = smem + stage * C::kStageBytes + C::kWBytes;
+        const uint32_t sX = ptx::smem_u32(smem + stage * C::kStageBytes + C::kWBytes);
         if (t.phase == 1) {
-          if (active)
-            ptx::tma_gather4(sX + lane * 512, &args.tm_x, &full[stage], kb * 64, rows[0], rows[1], rows[2], rows[3]);
-        } else if (lane == 0) {
-          ptx::tma_load_2d(sX, &args.tm_h, &full[stage], kb * 64, t.blk * args.block_m);
+#pragma unroll
+          for (int i = 0; i < kRowsPerThread; ++i) {
+            const int r = r0 + 16 * i;
+            const uint32_t dst = sX + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4);
+            ptx::cp_async_16(dst, src[i] + kb * 64, nbytes[i]);
+          }
+          ptx::cp_async_arrive_noinc(&full[stage]);
+        } else if (gtid == 0) {
+          ptx::mbar_arrive_expect_tx(&full[stage], C::kXBytes);
+          ptx::tma_load_2d(smem + stage * C::kStageBytes + C::kWBytes, &args.tm_h, &full[stage], kb * 64,
+                           t.blk * args.block_m);
+        } else {
+          ptx::mbar_arrive(&full[stage]);
         }
         if (++stage == C::kStages) {
           stage = 0;
@@ -447,6 +478,10 @@ cudaError_t launch_fused_variant(const FusedArgs& args, int grid, cudaStream_t s
 }  // namespace
 
 bool fused_expert_supported(int block_m) { return block_m == 16 || block_m == 32 || block_m == 64; }
+
+bool fused_expert_combines(int T, int k, int n_shared) {
+  return n_shared == 0 && static_cast<int64_t>(T) * k <= kCombineMaxSlots;
+}
 
 cudaError_t launch_fused_expert(int act_epi, int block_m, const FusedArgs& args, int grid, cudaStream_t stream) {
   const bool gated = act_epi == kEpiSwiGLU;

@@ -20,9 +20,8 @@ enum EpiKind : int {
 struct GemmArgs {
   CUtensorMap tm_w;   // routed expert weights, 3-D {K, rows per expert, E}, 128B swizzle
   CUtensorMap tm_ws;  // shared expert weights, 3-D {K, rows, 1}
-  CUtensorMap tm_x;   // token operand: gate/up GEMM x, 2-D {K, T} with 64 x 1 boxes (row
-                      // gather); down GEMM h, 2-D {K, P_total} with 64 x block_m boxes
-  const uint16_t* x;  // gate/up GEMM only: x [T, K] (rows are fetched through tm_x)
+  CUtensorMap tm_x;   // down GEMM only: h, 2-D {K, P_total} with 64 x block_m boxes
+  const uint16_t* x;  // gate/up GEMM only: token rows gathered from x [T, K]
   const int32_t* sorted_ids;
   const int32_t* expert_ids;
   const int32_t* ntpp;

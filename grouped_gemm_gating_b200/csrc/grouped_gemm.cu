@@ -25,14 +25,15 @@
 //   warp 0       TMA producer: weight tiles (and h tiles for the down GEMM)
 //   warp 1       TMEM allocator and MMA issuer (one thread)
 //   warps 2..5   epilogue: TMEM -> registers -> activation -> bf16 -> global
-//   warp 6       gate/up GEMM only: row gather of x through sorted_token_ids
-//                with TMA gather4 loads (each lane fetches 4 token rows of a
-//                64-column slice; padding rows use an out-of-range row index
-//                and arrive as zeros)
-// Shared-memory stages are guarded by full/empty mbarriers (every operand
-// arrives by TMA and completes transaction bytes on the stage's full
-// barrier), the two TMEM accumulator buffers by tmem-full/tmem-empty
-// mbarriers.  Every wait is
+//   warps 6..9   gate/up GEMM only: row gather of x through sorted_token_ids
+//                with 16-byte cp.async into the 128B-swizzled layout (padding
+//                rows zero-filled); each thread's copies of a stage arrive on
+//                the stage's full barrier by cp.async.mbarrier.arrive.noinc
+// Shared-memory stages are guarded by full/empty mbarriers (TMA operands
+// complete transaction bytes on the full barrier, gathered rows arrive on it
+// when their copies land; the MMA thread fences the generic and async
+// proxies before reading a stage), the two TMEM accumulator buffers by
+// tmem-full/tmem-empty mbarriers.  Every wait is
 // bounded in time; on expiry the kernel records MOE_ERR_DEVICE_TIMEOUT and
 // all roles leave their loops so the CTA frees its TMEM and exits.
 #include "common.cuh"
@@ -61,7 +62,7 @@ struct GemmCfg {
                                    : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256
                                                       : 512;
-  static constexpr int kNumThreads = kGather ? 224 : 192;
+  static constexpr int kNumThreads = kGather ? 320 : 192;
   static constexpr uint32_t kTxBytes = kWBytes + (kGather ? 0 : kXBytes);
   static constexpr int kBarrierBytes = 256;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes;
@@ -108,7 +109,7 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      ptx::mbar_init(&full[s], C::kGather ? 2 : 1);
+      ptx::mbar_init(&full[s], C::kGather ? 1 + 128 : 1);
       ptx::mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -205,6 +206,7 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
             break;
           }
           ptx::tc_fence_after();
+          if (C::kGather) ptx::fence_proxy_async_smem();
           const uint32_t sW = ptx::smem_u32(smem + stage * C::kStageBytes);
           const uint32_t sX = sW + C::kWBytes;
 #pragma unroll
@@ -371,45 +373,50 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
         aphase ^= 1u;
       }
     }
-  } else if (C::kGather && warp == 6) {
-    // ------------------------------------------------ row gather of x (TMA)
-    // lane l fetches token rows 4l..4l+3 of the tile's block
-    const bool active = 4 * lane < TOK;
+  } else if (C::kGather) {
+    // ------------------------------------------------ row gather of x
+    constexpr int kRowsPerThread = TOK / 16;
+    const int gtid = threadIdx.x - 192;
+    const int chunk = gtid & 7;
+    const int r0 = gtid >> 3;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
       const TileCoord tc = tile_coord(tile, n_wt, routed_blocks);
-      int rows[4];
+      const uint16_t* src[kRowsPerThread];
+      uint32_t nbytes[kRowsPerThread];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = 4 * lane + i;
-        int tok = args.T;  // out of range: the row arrives as zeros
-        if (active) {
-          if (!tc.shared_blk) {
-            const int slot = args.sorted_ids[tc.blk * args.block_m + r];
-            if (static_cast<unsigned>(slot) < static_cast<unsigned>(args.S)) tok = slot / args.k;
-          } else {
-            const int t = (tc.blk - routed_blocks) * args.block_m + r;
-            if (t < args.T) tok = t;
-          }
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int r = r0 + 16 * i;
+        int tok = 0;
+        bool valid;
+        if (!tc.shared_blk) {
+          const int slot = args.sorted_ids[tc.blk * args.block_m + r];
+          valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
+          if (valid) tok = slot / args.k;
+        } else {
+          tok = (tc.blk - routed_blocks) * args.block_m + r;
+          valid = tok < args.T;
+          if (!valid) tok = 0;
         }
-        rows[i] = tok;
+        src[i] = args.x + static_cast<size_t>(tok) * args.K + chunk * 8;
+        nbytes[i] = valid ? 16u : 0u;
       }
       for (int kb = 0; kb < nk; ++kb) {
-        int good = 1;
-        if (lane == 0) {
-          good = ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs) ? 1 : 0;
-          if (good) ptx::mbar_arrive_expect_tx(&full[stage], C::kXBytes);
-        }
-        good = __shfl_sync(0xffffffffu, good, 0);
-        if (!good) {
-          if (lane == 0) fail();
+        if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+          fail();
           ok = false;
           break;
         }
-        uint8_t* sX = smem + stage * C::kStageBytes + C::kWBytes;
-        if (active) ptx::tma_gather4(sX + lane * 512, &args.tm_x, &full[stage], kb * 64, rows[0], rows[1], rows[2], rows[3]);
+        const uint32_t sX = ptx::smem_u32(smem + stage * C::kStageBytes + C::kWBytes);
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          const int r = r0 + 16 * i;
+          const uint32_t dst = sX + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4);
+          ptx::cp_async_16(dst, src[i] + kb * 64, nbytes[i]);
+        }
+        ptx::cp_async_arrive_noinc(&full[stage]);
         if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;

@@ -1,4 +1,4 @@
-// Inline-PTX wrappers for sm_100a: mbarriers, TMA tile and row-gather loads,
+// Inline-PTX wrappers for sm_100a: mbarriers, TMA tile loads, cp.async,
 // proxy fences and the 5th-generation tensor core (tcgen05: TMEM
 // allocation, MMA issue, commit and TMEM loads).
 #pragma once
@@ -89,24 +89,32 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// Row gather: four rows (r0..r3, any order, out-of-range rows read as zero)
-// of a 2-D tensor map whose box is 64 columns x 1 row, starting at column
-// c0, into 4 consecutive 128-byte rows of shared memory (512 B at dst),
-// completing 512 bytes of transaction count on `bar`.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int r0, int r1,
-                                            int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
-      "%5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-      : "memory");
-}
-
 // Orders this thread's generic-proxy global accesses with its async-proxy
 // (TMA) accesses: writers call it after their stores, readers before their
 // bulk tensor loads.
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- cp.async
+
+// 16-byte global->shared copy (L2 only); src_bytes == 0 zero-fills.
+__device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+// Arrives on `bar` (without raising its expected count) once every cp.async
+// this thread issued so far has landed in shared memory.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Orders shared-memory data this thread has observed (through an mbarrier)
+// as written by the generic proxy before its subsequent async-proxy reads
+// (tensor-core operand fetches).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05

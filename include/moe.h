@@ -247,7 +247,7 @@ MOE_API int moe_last_launch_count(void);
  * Stages: 0 route, 1 align, 2 gate/up (fc1) GEMM, 3 down GEMM, 4 combine,
  * 5 fused route+align (moe_route_align on a small batch), 6 fused expert
  * kernel (moe_forward with block_m <= 64: both GEMMs, and the combine when
- * T <= 64).
+ * T*k <= 64 without a shared expert).
  * moe_profile_enable(1) starts a fresh record (and primes the event pool),
  * (0) stops recording and keeps what was recorded.  moe_profile_collect waits for the recorded events,
  * writes into stage_ms[i] (i < n_stages) the summed milliseconds of stage i
