@@ -347,9 +347,11 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
     // one persistent kernel; its cross-CTA counters start from zero
     moe::FusedArgs fa;
     std::memset(&fa, 0, sizeof(fa));
-    if (!encode_3d(&fa.tm_w13, w13, d, n1, E, 128) || !encode_3d(&fa.tm_w2, w2, F, d, E, 128)) return MOE_ERR_CUDA;
+    // gate/up boxes: 64 gate rows + 64 up rows per tile (SwiGLU) or 128 fc1 rows
+    const uint32_t box13 = act == MOE_ACT_SWIGLU ? 64 : 128;
+    if (!encode_3d(&fa.tm_w13, w13, d, n1, E, box13) || !encode_3d(&fa.tm_w2, w2, F, d, E, 128)) return MOE_ERR_CUDA;
     if (n_shared) {
-      if (!encode_3d(&fa.tm_w13s, w13_shared, d, n1, 1, 128) || !encode_3d(&fa.tm_w2s, w2_shared, F, d, 1, 128))
+      if (!encode_3d(&fa.tm_w13s, w13_shared, d, n1, 1, box13) || !encode_3d(&fa.tm_w2s, w2_shared, F, d, 1, 128))
         return MOE_ERR_CUDA;
     } else {
       fa.tm_w13s = fa.tm_w13;
@@ -378,7 +380,8 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
     fa.max_routed_blocks = max_routed_blocks;
     fa.n_shared_blocks = n_shared_blocks;
     fa.do_combine = moe::fused_expert_combines(T, k, n_shared) ? 1 : 0;
-    const int64_t tiles = static_cast<int64_t>(total_blocks_max) * ((F + 127) / 128 + n_dtiles);
+    const int h_cols = act == MOE_ACT_SWIGLU ? 64 : 128;
+    const int64_t tiles = static_cast<int64_t>(total_blocks_max) * ((F + h_cols - 1) / h_cols + n_dtiles);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
     cudaError_t err = cudaMemsetAsync(counters, 0, static_cast<size_t>(total_blocks_max + n_dtiles) * 4, s);
     if (err != cudaSuccess) return MOE_ERR_CUDA;

@@ -46,14 +46,18 @@ namespace {
 template <int EPI1, int TOK>
 struct FusedCfg {
   static constexpr bool kGated = (EPI1 == kEpiSwiGLU);
-  static constexpr int kW1Rows = kGated ? 256 : 128;  // phase-1 weight rows per stage
-  static constexpr int kW2Rows = 128;                 // phase-2 weight rows per stage
-  static constexpr int kWBytes = kW1Rows * 128;
+  // Every stage holds 128 weight rows: SwiGLU gate/up tiles stack 64 gate
+  // rows on the 64 matching up rows (one M = 128 MMA, 64 h columns per
+  // tile); relu^2 fc1 tiles and down tiles hold 128 rows of one matrix.
+  static constexpr int kWRows = 128;
+  static constexpr int kH1Cols = kGated ? 64 : 128;  // h columns per gate/up tile
+  static constexpr int kWBytes = kWRows * 128;
   static constexpr int kXBytes = TOK * 128;
   static constexpr int kStageBytes = kWBytes + kXBytes;
-  static constexpr int kStagesRaw = (225 * 1024) / kStageBytes;
+  static constexpr int kXbufBytes = kGated ? 64 * TOK * 4 : 0;  // up half handed to the gate half
+  static constexpr int kStagesRaw = (225 * 1024 - kXbufBytes) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
-  static constexpr int kAccCols = kGated ? 2 * TOK : TOK;
+  static constexpr int kAccCols = TOK;
   static constexpr int kTmemNeed = 2 * kAccCols;
   static constexpr int kTmemCols = kTmemNeed <= 32    ? 32
                                    : kTmemNeed <= 64  ? 64
@@ -61,12 +65,13 @@ struct FusedCfg {
                                    : kTmemNeed <= 256 ? 256
                                                       : 512;
   static constexpr int kNumThreads = 320;
-  static constexpr uint32_t kTx1 = kWBytes;
-  static constexpr uint32_t kTx2 = kW2Rows * 128;
+  static constexpr uint32_t kTx = kWBytes;
   static constexpr int kBarrierBytes = 256;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes;
+  static constexpr int kSlotBytes = 256;  // inv_pos of the in-kernel combine (64 slots)
+  static constexpr int kSmemBytes = kStages * kStageBytes + kXbufBytes + kSlotBytes + 1024 + kBarrierBytes;
   static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(128, TOK);
   static_assert(TOK == 16 || TOK == 32 || TOK == 64, "token rows per tile");
+  static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned");
   static_assert(kStages >= 3, "pipeline depth");
   static_assert((2 * kStages + 4) * 8 + 16 <= kBarrierBytes, "barrier area");
   static_assert(kSmemBytes <= 232448, "shared memory per block");
@@ -105,8 +110,12 @@ __device__ __forceinline__ int ld_acquire(const int32_t* p) {
   return v;
 }
 
-// Named barrier over the four epilogue warps (barrier 0 is __syncthreads).
-__device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier over the four epilogue warps (barrier 0 is __syncthreads);
+// each warp reconverges first, as the aligned barrier requires.
+__device__ __forceinline__ void epilogue_sync() {
+  __syncwarp();
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
 
 template <int EPI1, int TOK>
 __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
@@ -114,7 +123,10 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
   using C = FusedCfg<EPI1, TOK>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  float* xbuf = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);  // [TOK][64]
+  int* s_slot = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes + C::kXbufBytes);
+  uint64_t* full =
+      reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes + C::kXbufBytes + C::kSlotBytes);
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
@@ -159,7 +171,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
   if (routed_blocks < 0) routed_blocks = 0;
   if (routed_blocks > args.max_routed_blocks) routed_blocks = args.max_routed_blocks;
   const int total_blocks = routed_blocks + args.n_shared_blocks;
-  const int n_wt1 = (args.F + 127) / 128;
+  const int n_wt1 = (args.F + C::kH1Cols - 1) / C::kH1Cols;
   const int n_wt2 = (args.d + 127) / 128;
   const int n1_tiles = total_blocks * n_wt1;
   const int total_tiles = n1_tiles + total_blocks * n_wt2;
@@ -187,7 +199,6 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
         const int nk = t.phase == 1 ? nk1 : nk2;
         const CUtensorMap* tm = t.phase == 1 ? (t.shared_blk ? &args.tm_w13s : &args.tm_w13)
                                              : (t.shared_blk ? &args.tm_w2s : &args.tm_w2);
-        const int row0 = t.wt * 128;
         for (int kb = 0; kb < nk; ++kb) {
           if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
             fail();
@@ -195,13 +206,13 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
             break;
           }
           uint8_t* sW = smem + stage * C::kStageBytes;
-          if (t.phase == 1) {
-            ptx::mbar_arrive_expect_tx(&full[stage], C::kTx1);
-            ptx::tma_load_3d(sW, tm, &full[stage], kb * 64, row0, e);
-            if (C::kGated) ptx::tma_load_3d(sW + 128 * 128, tm, &full[stage], kb * 64, args.F + row0, e);
+          ptx::mbar_arrive_expect_tx(&full[stage], C::kTx);
+          if (t.phase == 1 && C::kGated) {
+            // 64 gate rows, then the 64 matching up rows (64-row boxes)
+            ptx::tma_load_3d(sW, tm, &full[stage], kb * 64, t.wt * 64, e);
+            ptx::tma_load_3d(sW + 64 * 128, tm, &full[stage], kb * 64, args.F + t.wt * 64, e);
           } else {
-            ptx::mbar_arrive_expect_tx(&full[stage], C::kTx2);
-            ptx::tma_load_3d(sW, tm, &full[stage], kb * 64, row0, e);
+            ptx::tma_load_3d(sW, tm, &full[stage], kb * 64, t.wt * 128, e);
           }
           if (++stage == C::kStages) {
             stage = 0;
@@ -243,10 +254,6 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
             const uint64_t dw = ptx::sw128_kmajor_desc(sW + kk * 32);
             const uint64_t dx = ptx::sw128_kmajor_desc(sX + kk * 32);
             ptx::mma_bf16(d_tmem, dw, dx, C::kIdesc, acc);
-            if (C::kGated && t.phase == 1) {
-              const uint64_t du = ptx::sw128_kmajor_desc(sW + 128 * 128 + kk * 32);
-              ptx::mma_bf16(d_tmem + TOK, du, dx, C::kIdesc, acc);
-            }
           }
           ptx::mma_commit(&empty[stage]);
           if (++stage == C::kStages) {
@@ -279,28 +286,49 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
       const uint32_t t_acc =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(abuf * C::kAccCols);
       const int pos0 = t.blk * args.block_m;
-      const int col = t.wt * 128 + row;
-      if (t.phase == 1) {
+      if (t.phase == 1 && C::kGated) {
+        // lanes 0-63 hold the gate and lanes 64-127 the up pre-activations
+        // of h columns wt*64 + (row % 64): the up half goes through xbuf
+        const int col = t.wt * 64 + (row & 63);
         const bool col_ok = col < args.F;
-#pragma unroll 1
+        float gate[TOK];
+#pragma unroll
         for (int j0 = 0; j0 < TOK; j0 += 16) {
-          uint32_t a[16], g[16];
+          uint32_t a[16];
           ptx::tmem_ld16(t_acc + j0, a);
-          if (C::kGated) ptx::tmem_ld16(t_acc + TOK + j0, g);
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
-            float v = __uint_as_float(a[jj]);
-            if (C::kGated) {
-              v = silu_f(v) * __uint_as_float(g[jj]);
-            } else {
-              v = fmaxf(v, 0.0f);
-              v *= v;
-            }
+            if (q >= 2)
+              xbuf[(j0 + jj) * 64 + (row - 64)] = __uint_as_float(a[jj]);
+            else
+              gate[j0 + jj] = __uint_as_float(a[jj]);
+          }
+        }
+        epilogue_sync();
+        if (q < 2 && col_ok) {
+#pragma unroll
+          for (int j = 0; j < TOK; ++j)
+            args.h[static_cast<size_t>(pos0 + j) * args.F + col] =
+                float_to_bf16_bits(silu_f(gate[j]) * xbuf[j * 64 + row]);
+        }
+      } else if (t.phase == 1) {
+        const int col = t.wt * 128 + row;
+        const bool col_ok = col < args.F;
+#pragma unroll 1
+        for (int j0 = 0; j0 < TOK; j0 += 16) {
+          uint32_t a[16];
+          ptx::tmem_ld16(t_acc + j0, a);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            float v = fmaxf(__uint_as_float(a[jj]), 0.0f);
+            v *= v;
             if (col_ok) args.h[static_cast<size_t>(pos0 + j0 + jj) * args.F + col] = float_to_bf16_bits(v);
           }
         }
       } else {
+        const int col = t.wt * 128 + row;
         const bool col_ok = col < args.d;
 #pragma unroll 1
         for (int j0 = 0; j0 < TOK; j0 += 16) {
@@ -345,15 +373,13 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
           __threadfence();
           const int c = t.wt * 128 + row;
           const int nslot = args.T * args.k;
+          for (int i = etid; i < nslot; i += 128) s_slot[i] = __ldcg(args.inv_pos + i);
+          epilogue_sync();
           if (c < args.d) {
-            int pr[kCombineMaxSlots];
             float v[kCombineMaxSlots];
 #pragma unroll
             for (int i = 0; i < kCombineMaxSlots; ++i)
-              if (i < nslot) pr[i] = __ldcg(args.inv_pos + i);
-#pragma unroll
-            for (int i = 0; i < kCombineMaxSlots; ++i)
-              if (i < nslot) v[i] = __ldcg(args.y + static_cast<size_t>(pr[i]) * args.d + c);
+              if (i < nslot) v[i] = __ldcg(args.y + static_cast<size_t>(s_slot[i]) * args.d + c);
             float acc = 0.0f;
             int j = 0, tok = 0;
 #pragma unroll
@@ -450,6 +476,9 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
     }
   }
 
+  // every warp reconverges (the idle lanes of the producer and MMA warps
+  // wait for their working lane) before the block-wide barrier
+  __syncwarp();
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -425,6 +425,9 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
     }
   }
 
+  // every warp reconverges (the idle lanes of the producer and MMA warps
+  // wait for their working lane) before the block-wide barrier
+  __syncwarp();
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
