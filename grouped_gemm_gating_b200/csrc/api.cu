@@ -151,6 +151,13 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool valid_block_m(int bm) { return bm == 16 || bm == 32 || bm == 64 || bm == 128; }
 
 constexpr size_t kWsAlign = 256;
+// The forward workspace starts with a fixed block of int32 counters that the
+// fused expert kernel keeps at zero between calls (the last CTA of every
+// launch resets them): [0] finished CTAs, [1, 1 + kMaxDTiles) done per
+// d-column tile, then ready per block.  h and y follow it.
+constexpr size_t kCounterInts = 16384;
+constexpr int kMaxDTiles = 255;
+constexpr int kMaxFusedBlocks = static_cast<int>(kCounterInts) - 1 - kMaxDTiles;
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -231,8 +238,7 @@ size_t moe_workspace_size(int T, int d, int F, int E, int k, int block_m, moe_ac
   const int64_t P = padded_total(T, k, E, block_m, n_shared);
   const size_t h = round_up(static_cast<size_t>(P) * F * 2, kWsAlign);
   const size_t y = round_up(static_cast<size_t>(P) * d * 4, kWsAlign);
-  const size_t counters = round_up(static_cast<size_t>(P / block_m + (d + 127) / 128) * 4, kWsAlign);
-  return h + y + counters + kWsAlign;
+  return kCounterInts * 4 + h + y + kWsAlign;
 }
 
 moe_status moe_route(const float* logits, int T, int E, int k, int n_group, int topk_group,
@@ -330,21 +336,22 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   const int n_shared_blocks = n_shared ? (T + bm - 1) / bm : 0;
   const int max_routed_blocks = static_cast<int>(P_max / bm);
   uint8_t* wsb = reinterpret_cast<uint8_t*>(round_up(reinterpret_cast<uintptr_t>(ws), kWsAlign));
-  uint16_t* h = reinterpret_cast<uint16_t*>(wsb);
-  float* y = reinterpret_cast<float*>(wsb + round_up(static_cast<size_t>(P_total) * F * 2, kWsAlign));
+  int32_t* counters = reinterpret_cast<int32_t*>(wsb);
+  uint16_t* h = reinterpret_cast<uint16_t*>(wsb + kCounterInts * 4);
+  float* y =
+      reinterpret_cast<float*>(wsb + kCounterInts * 4 + round_up(static_cast<size_t>(P_total) * F * 2, kWsAlign));
   const int n1 = act == MOE_ACT_SWIGLU ? 2 * F : F;
   const int num_sms = num_sms_current_device();
   if (num_sms <= 0) return MOE_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int launches = 0;
-  int32_t* counters = reinterpret_cast<int32_t*>(wsb + round_up(static_cast<size_t>(P_total) * F * 2, kWsAlign) +
-                                                 round_up(static_cast<size_t>(P_total) * d * 4, kWsAlign));
   const int total_blocks_max = static_cast<int>(P_total / bm);
   const int n_dtiles = (d + 127) / 128;
 
-  if (moe::fused_expert_supported(bm)) {
+  if (moe::fused_expert_supported(bm) && total_blocks_max <= kMaxFusedBlocks && n_dtiles <= kMaxDTiles) {
     // small token blocks: both GEMMs (and for small batches the combine) in
-    // one persistent kernel; its cross-CTA counters start from zero
+    // one persistent kernel; its cross-CTA counters are zero on entry and
+    // are returned to zero by the kernel's last CTA
     moe::FusedArgs fa;
     std::memset(&fa, 0, sizeof(fa));
     // gate/up boxes: 64 gate rows + 64 up rows per tile (SwiGLU) or 128 fc1 rows
@@ -367,8 +374,9 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
     fa.ntpp = num_tokens_post_padded;
     fa.inv_pos = inv_pos;
     fa.topk_w = topk_weights;
-    fa.ready = counters;
-    fa.done = counters + total_blocks_max;
+    fa.finished = counters;
+    fa.done = counters + 1;
+    fa.ready = counters + 1 + kMaxDTiles;
     fa.status = dev_status;
     fa.T = T;
     fa.k = k;
@@ -383,8 +391,7 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
     const int h_cols = act == MOE_ACT_SWIGLU ? 64 : 128;
     const int64_t tiles = static_cast<int64_t>(total_blocks_max) * ((F + h_cols - 1) / h_cols + n_dtiles);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-    cudaError_t err = cudaMemsetAsync(counters, 0, static_cast<size_t>(total_blocks_max + n_dtiles) * 4, s);
-    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    cudaError_t err;
     {
       StageScope scope(6, s);
       err = moe::launch_fused_expert(act == MOE_ACT_SWIGLU ? moe::kEpiSwiGLU : moe::kEpiRelu2, bm, fa,

@@ -22,8 +22,10 @@ struct FusedArgs {
   const int32_t* ntpp;
   const int32_t* inv_pos;
   const float* topk_w;  // [T * k]
-  int32_t* ready;       // [blocks]   gate/up tiles published per block (zeroed before launch)
-  int32_t* done;        // [d tiles]  down tiles finished per d-column tile (zeroed before launch)
+  // Cross-CTA counters, zero on entry; the last CTA to finish resets them.
+  int32_t* ready;       // [blocks]   gate/up tiles published per block
+  int32_t* done;        // [d tiles]  down tiles finished per d-column tile
+  int32_t* finished;    // [1]        CTAs that have finished
   int32_t* status;
   int T, k, S, E, d, F;
   int block_m;

@@ -485,6 +485,19 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, C::kTmemCols);
   }
+  // Check out; the last CTA returns every counter to zero for the next
+  // launch (no other CTA touches them any more).
+  if (threadIdx.x == 0) {
+    __threadfence();
+    *last_flag = atomicAdd(args.finished, 1) == static_cast<int>(gridDim.x) - 1 ? 1 : 0;
+  }
+  __syncthreads();
+  if (*last_flag) {
+    __threadfence();
+    for (int i = threadIdx.x; i < total_blocks; i += blockDim.x) args.ready[i] = 0;
+    for (int i = threadIdx.x; i < n_wt2; i += blockDim.x) args.done[i] = 0;
+    if (threadIdx.x == 0) *args.finished = 0;
+  }
 }
 
 template <int EPI1, int TOK>

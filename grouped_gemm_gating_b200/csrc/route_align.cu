@@ -14,14 +14,13 @@ namespace moe {
 
 namespace {
 
-constexpr int kFusedThreads = 1024;
-constexpr int kFusedWarps = kFusedThreads / 32;
 constexpr int kFusedMaxT = 64;
 constexpr int kFusedMaxS = 1024;
 constexpr int kFusedMaxGroups = 64;
 
-template <int VPL>
-__global__ void __launch_bounds__(kFusedThreads)
+// NWARPS warps: 8 for up to 256 slots (decode), 32 above.
+template <int VPL, int NWARPS>
+__global__ void __launch_bounds__(NWARPS * 32)
     route_align_kernel(const float* __restrict__ logits, int T, int E, int k, int n_group, int topk_group,
                        int group_score, int renormalize, float routed_scaling, int32_t* __restrict__ topk_ids,
                        float* __restrict__ topk_weights, int bm, int P_max, int32_t* __restrict__ sorted_ids,
@@ -32,6 +31,8 @@ __global__ void __launch_bounds__(kFusedThreads)
   __shared__ int off[MOE_MAX_EXPERTS + 1];
   __shared__ int run[MOE_MAX_EXPERTS];
   __shared__ int tot[MOE_MAX_EXPERTS];
+  constexpr int kFusedWarps = NWARPS;
+  constexpr int kFusedThreads = NWARPS * 32;
   __shared__ int wcnt[kFusedWarps][MOE_MAX_EXPERTS];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   // While routing, each warp's row of wcnt doubles as its group-score
@@ -66,12 +67,17 @@ cudaError_t launch_route_align(const float* logits, int T, int E, int k, int n_g
                                float* topk_weights, int block_m, int P_max, int32_t* sorted_ids, int32_t* expert_ids,
                                int32_t* ntpp, int32_t* inv_pos, int32_t* status, cudaStream_t stream,
                                int* launches) {
-  auto kern = E <= 32    ? route_align_kernel<1>
-              : E <= 64  ? route_align_kernel<2>
-              : E <= 128 ? route_align_kernel<4>
-                         : route_align_kernel<8>;
+  const bool small = T * k <= 256;
+  auto kern = small ? (E <= 32    ? route_align_kernel<1, 8>
+                       : E <= 64  ? route_align_kernel<2, 8>
+                       : E <= 128 ? route_align_kernel<4, 8>
+                                  : route_align_kernel<8, 8>)
+                    : (E <= 32    ? route_align_kernel<1, 32>
+                       : E <= 64  ? route_align_kernel<2, 32>
+                       : E <= 128 ? route_align_kernel<4, 32>
+                                  : route_align_kernel<8, 32>);
   ++*launches;
-  return launch_pdl(kern, dim3(1), dim3(kFusedThreads), 0, stream, logits, T, E, k, n_group, topk_group, group_score,
+  return launch_pdl(kern, dim3(1), dim3(small ? 256 : 1024), 0, stream, logits, T, E, k, n_group, topk_group, group_score,
                     renormalize, routed_scaling, topk_ids, topk_weights, block_m, P_max, sorted_ids, expert_ids, ntpp,
                     inv_pos, status);
 }

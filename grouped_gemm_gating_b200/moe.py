@@ -269,7 +269,8 @@ class MoEBuffers:
         fws = moe_workspace_size(T, d, F, E, k, block_m, act, n_shared)
         if fws == 0:
             raise ValueError("unsupported layer shape")
-        self.ws = torch.empty(fws, dtype=torch.uint8, device=dev)
+        # zero-filled: the workspace's leading counter block must start at zero
+        self.ws = torch.zeros(fws, dtype=torch.uint8, device=dev)
         self.out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
         self.status = torch.zeros(1, **i32)
 

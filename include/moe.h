@@ -103,11 +103,15 @@ MOE_API int64_t moe_max_padded(int T, int k, int E, int block_m);
  * the single-block path).  Returns 0 on invalid arguments. */
 MOE_API size_t moe_align_workspace_size(int T, int k, int E);
 
-/* Bytes of device scratch moe_forward needs: the activation h
- * [P_total, F] in bf16, the scaled expert outputs y [P_total, d] in fp32 and
- * P_total / block_m + ceil(d / 128) int32 counters,
- * where P_total = P_max + n_shared * ceil(T / block_m) * block_m.
- * Returns 0 on invalid arguments. */
+/* Bytes of device scratch moe_forward needs: a 64 KiB block of int32
+ * counters, then the activation h [P_total, F] in bf16 and the scaled expert
+ * outputs y [P_total, d] in fp32, where
+ * P_total = P_max + n_shared * ceil(T / block_m) * block_m.
+ * The counter block (the first 64 KiB after rounding ws up to 256 bytes)
+ * must be zero before the first moe_forward on a workspace (allocate it
+ * zero-filled or cudaMemset it once); every moe_forward leaves it at zero
+ * again, so a workspace can be reused across calls and layer shapes as long
+ * as nothing else writes that block.  Returns 0 on invalid arguments. */
 MOE_API size_t moe_workspace_size(int T, int d, int F, int E, int k, int block_m,
                           moe_act act, int n_shared);
 
@@ -172,7 +176,9 @@ MOE_API moe_status moe_align(const int32_t* topk_ids, int T, int k, int E, int b
  *                with fp32 accumulation; h is rounded to bf16 (it feeds the
  *                bf16 down GEMM), the per-slot scaled outputs stay fp32 and
  *                the k-sum is fp32 in slot order, rounded once to bf16.
- *   ws, ws_bytes scratch of moe_workspace_size bytes.
+ *   ws, ws_bytes scratch of moe_workspace_size bytes (its counter block zero,
+ *                see moe_workspace_size); calls sharing a workspace must not
+ *                overlap on the GPU.
  * Errors: host checks as above; MOE_ERR_DEVICE_TIMEOUT in dev_status if a
  * pipeline wait inside a GEMM kernel exceeded its limit (out is then invalid).
  */

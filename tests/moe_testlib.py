@@ -82,7 +82,8 @@ class DeviceLayer:
         """The activation h [P_total, F] from the forward workspace (fp32)."""
         c = self.cfg
         P_total = self.buf.P_max + (c.n_shared * ((c.T + c.block_m - 1) // c.block_m) * c.block_m)
-        base = (self.buf.ws.data_ptr() + 255) // 256 * 256 - self.buf.ws.data_ptr()
+        # after rounding up to 256 bytes: 64 KiB of counters, then h
+        base = (self.buf.ws.data_ptr() + 255) // 256 * 256 - self.buf.ws.data_ptr() + 65536
         raw = self.buf.ws[base: base + P_total * c.F * 2].view(torch.int16).reshape(P_total, c.F)
         return W.bf16_bits_to_f32(raw.cpu().numpy().view(np.uint16))
 

@@ -51,7 +51,7 @@ def test_workspace_sizes(lib):
     T, d, F, E, k, bm = 4096, 3072, 2560, 18, 4, 128
     P = oracle.max_padded(T, k, E, bm) + T  # shared rows (T is a multiple of bm)
     size = M.moe_workspace_size(T, d, F, E, k, bm, M.ACT_SWIGLU, 1)
-    counters = (P // bm + (d + 127) // 128) * 4
+    counters = 65536
     assert size >= P * (2 * F + 4 * d) + counters
     assert size <= P * (2 * F + 4 * d) + counters + 1024
     assert M.moe_workspace_size(T, d + 32, F, E, k, bm, M.ACT_SWIGLU, 0) == 0   # d % 64

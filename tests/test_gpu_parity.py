@@ -311,3 +311,24 @@ def test_route_align_matches_separate_calls(name, T):
     assert torch.equal(a.buf.inv_pos[:S], b.buf.inv_pos[:S])
     ids, w = oracle_route(inp)
     compare_route(b.buf.topk_ids.cpu().numpy(), b.buf.topk_weights.cpu().numpy(), ids, w, name)
+
+
+def test_fused_counters_return_to_zero_and_workspace_is_shareable():
+    """The fused kernel's counter block is zero after every call, so one
+    workspace serves calls of different shapes in turn."""
+    cfg_a = SMALL["decode_d512"]
+    cfg_b = SMALL["swap_bm32"]
+    lay_a = DeviceLayer(W.make_inputs(cfg_a))
+    lay_b = DeviceLayer(W.make_inputs(cfg_b))
+    shared_ws = lay_a.buf.ws if lay_a.buf.ws.numel() >= lay_b.buf.ws.numel() else lay_b.buf.ws
+    lay_a.buf.ws = shared_ws
+    lay_b.buf.ws = shared_ws
+    ref_a = M_bits(lay_a.run()).copy()
+    ref_b = M_bits(lay_b.run()).copy()
+    for _ in range(2):
+        assert np.array_equal(M_bits(lay_a.run()), ref_a)
+        torch.cuda.synchronize()
+        base = (shared_ws.data_ptr() + 255) // 256 * 256 - shared_ws.data_ptr()
+        assert int(shared_ws[base: base + 65536].count_nonzero()) == 0
+        assert np.array_equal(M_bits(lay_b.run()), ref_b)
+    assert lay_a.status() == 0 and lay_b.status() == 0
