@@ -364,7 +364,6 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
       fa.tm_w13s = fa.tm_w13;
       fa.tm_w2s = fa.tm_w2;
     }
-    if (!encode_2d(&fa.tm_h, h, F, static_cast<uint64_t>(P_total), static_cast<uint32_t>(bm))) return MOE_ERR_CUDA;
     fa.x = x;
     fa.h = h;
     fa.y = y;

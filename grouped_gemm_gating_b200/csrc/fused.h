@@ -12,7 +12,6 @@ struct FusedArgs {
   CUtensorMap tm_w13s;  // shared expert, 3-D {d, N1, 1}
   CUtensorMap tm_w2;    // routed down weights, 3-D {F, d, E}, 128-row boxes
   CUtensorMap tm_w2s;   // shared expert, 3-D {F, d, 1}
-  CUtensorMap tm_h;     // h, 2-D {F, P_total}, 64 x block_m boxes
   const uint16_t* x;    // [T, d] bf16
   uint16_t* h;          // [P_total, F] bf16 (workspace)
   float* y;             // [P_total, d] fp32 (workspace)

@@ -15,14 +15,15 @@
 // static stride, so its own gate/up tiles always come before its down tiles
 // and no CTA waits on work queued behind itself; all CTAs are co-resident
 // (one per SM, grid <= SM count).  A down tile needs the block's full h rows:
-// the gate/up epilogue publishes each finished tile with a release pattern
-// (h stores, a generic-to-async proxy fence, __threadfence, atomicAdd on
-// ready[block]); one token-loader thread polls ready[block] with ld.acquire,
-// fences the proxies again and only then loads the block's h rows by TMA.
-// The weight warp streams the down tile's W2 slices without waiting, so the
-// down GEMM's weight traffic overlaps the tail of the gate/up phase.  Every
-// stage is signalled as soon as its bytes land (TMA transaction bytes;
-// cp.async.mbarrier.arrive.noinc for gathered rows), so no warp holds back a
+// the gate/up epilogue publishes each finished tile (h stores, a barrier of
+// the epilogue warps, then one red.release.gpu add on ready[block]); every
+// token-loader thread polls ready[block] with ld.acquire.gpu and then loads
+// its share of the block's h rows with cp.async.  No GPU-scope fence sits on this path: such fences wait
+// behind the SM's queue of in-flight weight loads.  The weight warp streams
+// the down tile's W2 slices without waiting, so the down GEMM's weight
+// traffic overlaps the tail of the gate/up phase.  Every stage is signalled
+// as soon as its bytes land (TMA transaction bytes for weights,
+// cp.async.mbarrier.arrive.noinc for token rows), so no warp holds back a
 // stage that another tile needs while it waits.
 //
 // Combine (do_combine, T*k <= 64, no shared expert): the CTA that finishes
@@ -73,7 +74,7 @@ struct FusedCfg {
   static_assert(TOK == 16 || TOK == 32 || TOK == 64, "token rows per tile");
   static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned");
   static_assert(kStages >= 3, "pipeline depth");
-  static_assert((2 * kStages + 4) * 8 + 16 <= kBarrierBytes, "barrier area");
+  static_assert((2 * kStages + 4) * 8 + 16 <= kBarrierBytes, "barrier area");  // + 4 words
   static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
 
@@ -104,17 +105,28 @@ __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)
 // Slots (T * k) up to which the kernel does the scatter-reduce itself.
 constexpr int kCombineMaxSlots = 64;
 
-__device__ __forceinline__ int ld_acquire(const int32_t* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Named barrier over the four epilogue warps (barrier 0 is __syncthreads);
-// each warp reconverges first, as the aligned barrier requires.
+// Named barrier 1 over the four epilogue warps (barrier 0 is
+// __syncthreads).  Each warp reconverges first, as the aligned barrier
+// requires.  epilogue_any() is the same barrier with an OR reduction: the
+// epilogue takes its leave-on-timeout decision uniformly, so no epilogue
+// thread can be left waiting at a later barrier for one that left.
 __device__ __forceinline__ void epilogue_sync() {
   __syncwarp();
   asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+__device__ __forceinline__ bool epilogue_any(bool v) {
+  uint32_t r;
+  __syncwarp();
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u)
+      : "memory");
+  return r != 0;
 }
 
 template <int EPI1, int TOK>
@@ -150,7 +162,6 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&args.tm_w13);
     ptx::prefetch_tmap(&args.tm_w2);
-    ptx::prefetch_tmap(&args.tm_h);
     if (args.n_shared_blocks) {
       ptx::prefetch_tmap(&args.tm_w13s);
       ptx::prefetch_tmap(&args.tm_w2s);
@@ -278,8 +289,9 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
     uint32_t aphase = 0;
     for (int u = blockIdx.x; u < total_tiles; u += gridDim.x) {
       const Tile t = fused_tile(u, n1_tiles, n_wt1, n_wt2, routed_blocks);
-      if (!ptx::mbar_wait_bounded(&tfull[abuf], aphase, abort_flag, kWaitLimitNs)) {
-        fail();
+      const bool got = ptx::mbar_wait_bounded(&tfull[abuf], aphase, abort_flag, kWaitLimitNs);
+      if (epilogue_any(!got)) {
+        if (!got) fail();
         break;
       }
       ptx::tc_fence_after();
@@ -358,19 +370,18 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
         abuf = 0;
         aphase ^= 1u;
       }
-      // publish the finished tile
-      if (t.phase == 1) ptx::fence_proxy_async_global();  // h is read back by TMA
-      __threadfence();
+      // publish the finished tile: the barrier orders every epilogue
+      // thread's stores before thread 0's GPU-scope release
       epilogue_sync();
       if (t.phase == 1) {
-        if (etid == 0) atomicAdd(&args.ready[t.blk], 1);
+        if (etid == 0) ptx::red_release_gpu_add(&args.ready[t.blk], 1);
       } else if (args.do_combine) {
-        if (etid == 0) *last_flag = (atomicAdd(&args.done[t.wt], 1) == total_blocks - 1) ? 1 : 0;
+        if (etid == 0) *last_flag = (ptx::atom_acq_rel_gpu_add(&args.done[t.wt], 1) == total_blocks - 1) ? 1 : 0;
         epilogue_sync();
         if (*last_flag) {
-          // this CTA finished the last down tile of column tile t.wt: every
-          // load first (independent), then the sums in slot order
-          __threadfence();
+          // this CTA finished the last down tile of column tile t.wt (its
+          // acquire plus the barrier order the loads below after every
+          // other CTA's y stores): every load first, then the sums in order
           const int c = t.wt * 128 + row;
           const int nslot = args.T * args.k;
           for (int i = etid; i < nslot; i += 128) s_slot[i] = __ldcg(args.inv_pos + i);
@@ -400,9 +411,8 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
     }
   } else {
     // ------------------------------------------------ token operand
-    // gate/up tiles: 128 threads gather the block's x rows with cp.async;
-    // down tiles: thread 0 loads the block's h rows by TMA once published,
-    // the others only arrive
+    // 128 threads copy the tile's token rows with cp.async: gathered x rows
+    // for gate/up tiles, the block's h rows for down tiles once published
     constexpr int kRowsPerThread = TOK / 16;
     const int gtid = threadIdx.x - 192;
     const int chunk = gtid & 7;
@@ -414,7 +424,9 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
       const Tile t = fused_tile(u, n1_tiles, n_wt1, n_wt2, routed_blocks);
       const uint16_t* src[kRowsPerThread];
       uint32_t nbytes[kRowsPerThread];
+      int K;
       if (t.phase == 1) {
+        K = args.d;
 #pragma unroll
         for (int i = 0; i < kRowsPerThread; ++i) {
           const int r = r0 + 16 * i;
@@ -429,45 +441,45 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
             valid = tok < args.T;
             if (!valid) tok = 0;
           }
-          src[i] = args.x + static_cast<size_t>(tok) * args.d + chunk * 8;
+          src[i] = args.x + static_cast<size_t>(tok) * K + chunk * 8;
           nbytes[i] = valid ? 16u : 0u;
         }
-      } else if (gtid == 0) {
+      } else {
+        K = args.F;
         // wait until every gate/up tile of this block has published its h
+        // (this thread holds no unsignalled stage while it waits)
         const uint64_t t0 = ptx::globaltimer_ns();
-        while (ld_acquire(args.ready + t.blk) < n_wt1) {
+        while (ptx::ld_acquire_gpu(args.ready + t.blk) < n_wt1) {
           if (*abort_flag || ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
             fail();
             ok = false;
             break;
           }
-          __nanosleep(64);
+          __nanosleep(128);
         }
-        ptx::fence_proxy_async_global();
+        if (!ok) break;
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          const int r = r0 + 16 * i;
+          src[i] = args.h + static_cast<size_t>(t.blk * args.block_m + r) * K + chunk * 8;
+          nbytes[i] = 16u;
+        }
       }
-      const int nk = t.phase == 1 ? nk1 : nk2;
-      for (int kb = 0; ok && kb < nk; ++kb) {
+      const int nk = K / 64;
+      for (int kb = 0; kb < nk; ++kb) {
         if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
           fail();
           ok = false;
           break;
         }
         const uint32_t sX = ptx::smem_u32(smem + stage * C::kStageBytes + C::kWBytes);
-        if (t.phase == 1) {
 #pragma unroll
-          for (int i = 0; i < kRowsPerThread; ++i) {
-            const int r = r0 + 16 * i;
-            const uint32_t dst = sX + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4);
-            ptx::cp_async_16(dst, src[i] + kb * 64, nbytes[i]);
-          }
-          ptx::cp_async_arrive_noinc(&full[stage]);
-        } else if (gtid == 0) {
-          ptx::mbar_arrive_expect_tx(&full[stage], C::kXBytes);
-          ptx::tma_load_2d(smem + stage * C::kStageBytes + C::kWBytes, &args.tm_h, &full[stage], kb * 64,
-                           t.blk * args.block_m);
-        } else {
-          ptx::mbar_arrive(&full[stage]);
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          const int r = r0 + 16 * i;
+          const uint32_t dst = sX + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4);
+          ptx::cp_async_16(dst, src[i] + kb * 64, nbytes[i]);
         }
+        ptx::cp_async_arrive_noinc(&full[stage]);
         if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;
@@ -487,13 +499,10 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
   }
   // Check out; the last CTA returns every counter to zero for the next
   // launch (no other CTA touches them any more).
-  if (threadIdx.x == 0) {
-    __threadfence();
-    *last_flag = atomicAdd(args.finished, 1) == static_cast<int>(gridDim.x) - 1 ? 1 : 0;
-  }
+  if (threadIdx.x == 0)
+    *last_flag = ptx::atom_acq_rel_gpu_add(args.finished, 1) == static_cast<int>(gridDim.x) - 1 ? 1 : 0;
   __syncthreads();
   if (*last_flag) {
-    __threadfence();
     for (int i = threadIdx.x; i < total_blocks; i += blockDim.x) args.ready[i] = 0;
     for (int i = threadIdx.x; i < n_wt2; i += blockDim.x) args.done[i] = 0;
     if (threadIdx.x == 0) *args.finished = 0;
