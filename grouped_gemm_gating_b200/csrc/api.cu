@@ -153,11 +153,9 @@ bool valid_block_m(int bm) { return bm == 16 || bm == 32 || bm == 64 || bm == 12
 constexpr size_t kWsAlign = 256;
 // The forward workspace starts with a fixed block of int32 counters that the
 // fused expert kernel keeps at zero between calls (the last CTA of every
-// launch resets them): [0] finished CTAs, [1, 1 + kMaxDTiles) done per
-// d-column tile, then ready per block.  h and y follow it.
+// launch resets them; it uses the first three as grid counters, the rest is
+// reserved).  h and y follow it.
 constexpr size_t kCounterInts = 16384;
-constexpr int kMaxDTiles = 255;
-constexpr int kMaxFusedBlocks = static_cast<int>(kCounterInts) - 1 - kMaxDTiles;
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -346,12 +344,11 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int launches = 0;
   const int total_blocks_max = static_cast<int>(P_total / bm);
-  const int n_dtiles = (d + 127) / 128;
 
-  if (moe::fused_expert_supported(bm) && total_blocks_max <= kMaxFusedBlocks && n_dtiles <= kMaxDTiles) {
-    // small token blocks: both GEMMs (and for small batches the combine) in
-    // one persistent kernel; its cross-CTA counters are zero on entry and
-    // are returned to zero by the kernel's last CTA
+  if (moe::fused_expert_supported(bm)) {
+    // small token blocks: both GEMMs and the scatter-reduce in one persistent
+    // kernel that accumulates into the fp32 y region; its three grid
+    // counters are zero on entry and are returned to zero by its last CTA
     moe::FusedArgs fa;
     std::memset(&fa, 0, sizeof(fa));
     // gate/up boxes: 64 gate rows + 64 up rows per tile (SwiGLU) or 128 fc1 rows
@@ -365,17 +362,13 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
       fa.tm_w2s = fa.tm_w2;
     }
     fa.x = x;
-    fa.h = h;
-    fa.y = y;
+    fa.acc = y;
     fa.out = out;
     fa.sorted_ids = sorted_token_ids;
     fa.expert_ids = expert_ids;
     fa.ntpp = num_tokens_post_padded;
-    fa.inv_pos = inv_pos;
     fa.topk_w = topk_weights;
-    fa.finished = counters;
-    fa.done = counters + 1;
-    fa.ready = counters + 1 + kMaxDTiles;
+    fa.sync = counters;
     fa.status = dev_status;
     fa.T = T;
     fa.k = k;
@@ -386,22 +379,16 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
     fa.block_m = bm;
     fa.max_routed_blocks = max_routed_blocks;
     fa.n_shared_blocks = n_shared_blocks;
-    fa.do_combine = moe::fused_expert_combines(T, k, n_shared) ? 1 : 0;
-    const int h_cols = act == MOE_ACT_SWIGLU ? 64 : 128;
-    const int64_t tiles = static_cast<int64_t>(total_blocks_max) * ((F + h_cols - 1) / h_cols + n_dtiles);
+    const int epi = act == MOE_ACT_SWIGLU ? moe::kEpiSwiGLU : moe::kEpiRelu2;
+    const int64_t tiles = moe::fused_expert_max_tiles(epi, total_blocks_max, F);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
     cudaError_t err;
     {
       StageScope scope(6, s);
-      err = moe::launch_fused_expert(act == MOE_ACT_SWIGLU ? moe::kEpiSwiGLU : moe::kEpiRelu2, bm, fa,
-                                     grid < 1 ? 1 : grid, s);
+      err = moe::launch_fused_expert(epi, bm, fa, grid < 1 ? 1 : grid, s);
     }
     if (err != cudaSuccess) return MOE_ERR_CUDA;
     ++launches;
-    if (!fa.do_combine) {
-      StageScope scope(4, s);
-      err = moe::launch_combine(y, inv_pos, num_tokens_post_padded, T, k, d, n_shared, out, s, &launches);
-    }
     return finish(err, launches);
   }
 

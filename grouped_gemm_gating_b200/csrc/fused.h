@@ -1,5 +1,6 @@
-// Host-visible interface of the fused expert kernel (gate/up GEMM + act,
-// down GEMM + top-k weight, optional scatter-reduce) for block_m <= 64.
+// Host-visible interface of the fused expert kernel for block_m <= 64: the
+// gate/up GEMM with its activation, the down GEMM split along d_ff with the
+// top-k weights, and the scatter-reduce, in one persistent launch.
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -8,34 +9,29 @@
 namespace moe {
 
 struct FusedArgs {
-  CUtensorMap tm_w13;   // routed gate/up (or fc1) weights, 3-D {d, N1, E}, 128-row boxes
-  CUtensorMap tm_w13s;  // shared expert, 3-D {d, N1, 1}
-  CUtensorMap tm_w2;    // routed down weights, 3-D {F, d, E}, 128-row boxes
+  CUtensorMap tm_w13;   // routed gate/up (or fc1) weights, 3-D {d, N1, E}; boxes of 64 x 64 rows
+                        // (SwiGLU: 64 gate rows, then the matching 64 up rows) or 64 x 128 (relu^2)
+  CUtensorMap tm_w13s;  // shared expert, 3-D {d, N1, 1}, same boxes
+  CUtensorMap tm_w2;    // routed down weights, 3-D {F, d, E}, 64 x 128 boxes
   CUtensorMap tm_w2s;   // shared expert, 3-D {F, d, 1}
   const uint16_t* x;    // [T, d] bf16
-  uint16_t* h;          // [P_total, F] bf16 (workspace)
-  float* y;             // [P_total, d] fp32 (workspace)
+  float* acc;           // [T, d] fp32 accumulator (workspace; zeroed by the kernel)
   uint16_t* out;        // [T, d] bf16
   const int32_t* sorted_ids;
   const int32_t* expert_ids;
   const int32_t* ntpp;
-  const int32_t* inv_pos;
   const float* topk_w;  // [T * k]
-  // Cross-CTA counters, zero on entry; the last CTA to finish resets them.
-  int32_t* ready;       // [blocks]   gate/up tiles published per block
-  int32_t* done;        // [d tiles]  down tiles finished per d-column tile
-  int32_t* finished;    // [1]        CTAs that have finished
+  int32_t* sync;        // [3] grid counters (zeroed, finished, departed); zero at rest
   int32_t* status;
   int T, k, S, E, d, F;
   int block_m;
   int max_routed_blocks;
   int n_shared_blocks;
-  int do_combine;       // 1: the kernel also writes out (fused_expert_combines)
 };
 
 bool fused_expert_supported(int block_m);
-// True when the fused kernel also does the scatter-reduce (T*k <= 64, no shared expert).
-bool fused_expert_combines(int T, int k, int n_shared);
+// Upper bound on the fused kernel's tiles, for grid sizing.
+int64_t fused_expert_max_tiles(int act_epi, int total_blocks_max, int F);
 cudaError_t launch_fused_expert(int act_epi, int block_m, const FusedArgs& args, int grid, cudaStream_t stream);
 
 }  // namespace moe

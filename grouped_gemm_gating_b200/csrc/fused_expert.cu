@@ -1,40 +1,51 @@
-// Fused expert kernel for small token blocks (block_m = 16..64): the gate/up
-// GEMM with its activation, the down GEMM with the top-k weights and, for
-// small batches, the scatter-reduce, in one persistent launch.
+// Fused expert kernel for small token blocks (block_m = 16..64): gate/up GEMM
+// with its activation, down GEMM with the top-k weights and the
+// scatter-reduce, in one persistent launch.
 //
-// This is the same computation as the separate grouped GEMMs (see
-// grouped_gemm.cu for the sources: "Grouped GEMM Structure" of the
-// fused-moe-kernel page, the gate/up, activation, down and weighted-sum
-// sequence of the axolotl `_moe_triton_forward`, the relu^2 experts of the
-// mlxcel PR) specialised for the decode / verifier shape, where the layer is
-// bound by streaming each hit expert's weights once from HBM and every
-// separate launch costs as much as a few microseconds of that stream.
+// The computation is the layer of the fused-moe-kernel page ("Fused MoE
+// Kernel Optimization": "Grouped GEMM Structure", "Common Pitfalls" 4) and of
+// the axolotl `_moe_triton_forward` (src/axolotl/monkeypatch/deepseek_v3/
+// __init__.py: gate/up projections, act_fn(gate) * up, down projection,
+// weighted sum over the k experts), with the relu^2 experts of the mlxcel PR
+// ("fc1 -> relu^2 -> fc2").  For the decode / verifier shape the layer is
+// bound by streaming each hit expert's weights once, so the design avoids
+// anything that stalls that stream.
 //
-// Work list: all gate/up tiles (block, h-column tile) first, then all down
-// tiles (block, d-column tile).  Every CTA walks the list with the same
-// static stride, so its own gate/up tiles always come before its down tiles
-// and no CTA waits on work queued behind itself; all CTAs are co-resident
-// (one per SM, grid <= SM count).  A down tile needs the block's full h rows:
-// the gate/up epilogue publishes each finished tile (h stores, a barrier of
-// the epilogue warps, then one red.release.gpu add on ready[block]); every
-// token-loader thread polls ready[block] with ld.acquire.gpu and then loads
-// its share of the block's h rows with cp.async.  No GPU-scope fence sits on this path: such fences wait
-// behind the SM's queue of in-flight weight loads.  The weight warp streams
-// the down tile's W2 slices without waiting, so the down GEMM's weight
-// traffic overlaps the tail of the gate/up phase.  Every stage is signalled
-// as soon as its bytes land (TMA transaction bytes for weights,
-// cp.async.mbarrier.arrive.noinc for token rows), so no warp holds back a
-// stage that another tile needs while it waits.
+// Split along d_ff.  A tile is (block of block_m token rows, one slice of
+// the hidden dimension: 64 h columns for SwiGLU, 128 for relu^2).  A CTA
+//   1. computes the slice's pre-activations with the weights as the MMA's
+//      M = 128 rows (SwiGLU stacks 64 gate rows on the matching 64 up rows;
+//      the epilogue hands the up half to the gate half through shared
+//      memory),
+//   2. writes h = act(...) for the slice into shared memory, already in the
+//      K-major 128-byte-swizzled layout the tensor core reads,
+//   3. streams the matching columns of W2 for every 128-row d tile and
+//      multiplies them by that h slice,
+//   4. adds topk_weight * partial into an fp32 [T, d] accumulator with
+//      red.global.add (fire-and-forget).
+// No tile waits for another CTA's work while weights stream (a GPU-scope
+// handoff from an SM whose TMA queue is full takes several microseconds).
+// The fp32 partials are summed in an order that depends on timing, so the
+// output is reproducible to fp32 rounding of the sum, not bit for bit.
 //
-// Combine (do_combine, T*k <= 64, no shared expert): the CTA that finishes
-// the last down tile of a d-column tile (done[column tile] reaches the
-// number of blocks) sums, for that column range, out[t] = sum_j
-// y[inv_pos[t*k + j]] in fp32 in slot order and writes bf16 -- the same
-// arithmetic as the combine kernel; all its loads are issued before the
-// first sum so the tail costs two memory round trips.
+// Each CTA runs its tiles software-pipelined: gate/up of tile i+1 is issued
+// before the down GEMM of tile i, so the tensor core never idles while the
+// epilogue turns tile i's accumulator into its h slice.
 //
-// Every wait is bounded in time; on expiry the kernel records
-// MOE_ERR_DEVICE_TIMEOUT and all roles leave their loops.
+// Grid protocol (all CTAs co-resident: one per SM, grid <= SM count):
+//   start: the gather warps zero this CTA's slice of the accumulator and
+//          count the CTA on sync[0]; the epilogue waits for all CTAs there
+//          before its first reduction (the weight stream does not wait).
+//   end:   every CTA counts itself on sync[1] once its reductions are issued,
+//          waits for all, converts its slice of the accumulator to bf16 and
+//          counts itself on sync[2]; the last one resets the counters.
+//
+// Warp roles: warp 0 TMA producer (weights), warp 1 TMEM allocator + MMA
+// issuer, warps 2-5 epilogue, warps 6-9 token-row gather (cp.async; each
+// thread's copies arrive on the stage's full barrier when they land).  TMEM:
+// two gate/up accumulators of block_m columns, then a ring of down-GEMM
+// accumulators (groups of 64 columns).  Every wait is bounded in time; on expiry the kernel records
+// MOE_ERR_DEVICE_TIMEOUT and all roles leave.
 #include "common.cuh"
 #include "fused.h"
 #include "gemm.h"
@@ -47,72 +58,78 @@ namespace {
 template <int EPI1, int TOK>
 struct FusedCfg {
   static constexpr bool kGated = (EPI1 == kEpiSwiGLU);
-  // Every stage holds 128 weight rows: SwiGLU gate/up tiles stack 64 gate
-  // rows on the 64 matching up rows (one M = 128 MMA, 64 h columns per
-  // tile); relu^2 fc1 tiles and down tiles hold 128 rows of one matrix.
-  static constexpr int kWRows = 128;
-  static constexpr int kH1Cols = kGated ? 64 : 128;  // h columns per gate/up tile
-  static constexpr int kWBytes = kWRows * 128;
-  static constexpr int kXBytes = TOK * 128;
+  static constexpr int kH = kGated ? 64 : 128;  // h columns per tile
+  static constexpr int kHk = kH / 64;           // 64-wide K blocks of the down GEMM per tile
+  static constexpr int kWBytes = 128 * 128;     // 128 weight rows x 64 bf16 per stage
+  static constexpr int kXBytes = TOK * 128;     // token rows x 64 bf16 per stage
   static constexpr int kStageBytes = kWBytes + kXBytes;
+  static constexpr int kHBufBytes = kHk * TOK * 128;            // one h slice (B operand of the down GEMM)
   static constexpr int kXbufBytes = kGated ? 64 * TOK * 4 : 0;  // up half handed to the gate half
-  static constexpr int kStagesRaw = (225 * 1024 - kXbufBytes) / kStageBytes;
+  static constexpr int kTokBytes = 2 * 2 * 64 * 4;              // token id and weight per row, two tiles
+  static constexpr int kBarrierBytes = 1024;
+  static constexpr int kFixedBytes = 2 * kHBufBytes + kXbufBytes + kTokBytes + kBarrierBytes + 1024;
+  static constexpr int kStagesRaw = (227 * 1024 - kFixedBytes) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
-  static constexpr int kAccCols = TOK;
-  static constexpr int kTmemNeed = 2 * kAccCols;
-  static constexpr int kTmemCols = kTmemNeed <= 32    ? 32
-                                   : kTmemNeed <= 64  ? 64
-                                   : kTmemNeed <= 128 ? 128
-                                   : kTmemNeed <= 256 ? 256
-                                                      : 512;
+  // Down-GEMM accumulators: groups of kGroup d tiles (64 TMEM columns) form
+  // one slot of a TMEM ring, so the epilogue synchronises once per group.
+  static constexpr int kGroup = 64 / TOK;
+  static constexpr int kD2Raw = (512 - 2 * TOK) / 64;
+  static constexpr int kD2Slots = kD2Raw > 8 ? 8 : kD2Raw;
   static constexpr int kNumThreads = 320;
-  static constexpr uint32_t kTx = kWBytes;
-  static constexpr int kBarrierBytes = 256;
-  static constexpr int kSlotBytes = 256;  // inv_pos of the in-kernel combine (64 slots)
-  static constexpr int kSmemBytes = kStages * kStageBytes + kXbufBytes + kSlotBytes + 1024 + kBarrierBytes;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kFixedBytes;
   static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(128, TOK);
   static_assert(TOK == 16 || TOK == 32 || TOK == 64, "token rows per tile");
-  static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned");
+  static_assert(kStageBytes % 1024 == 0 && kHBufBytes % 1024 == 0, "1024-byte aligned operand tiles");
   static_assert(kStages >= 3, "pipeline depth");
-  static_assert((2 * kStages + 4) * 8 + 16 <= kBarrierBytes, "barrier area");  // + 4 words
+  static_assert((2 * kStages + 9 + 2 * kD2Slots) * 8 + 16 <= kBarrierBytes, "barrier area");
   static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
 
-struct Tile {
-  int phase;  // 1: gate/up, 2: down
+struct TileInfo {
   int blk, wt;
   bool shared_blk;
 };
 
-__device__ __forceinline__ Tile fused_tile(int u, int n1_tiles, int n_wt1, int n_wt2, int routed_blocks) {
-  Tile t;
-  if (u < n1_tiles) {
-    t.phase = 1;
-    t.blk = u / n_wt1;
-    t.wt = u - t.blk * n_wt1;
-  } else {
-    const int v = u - n1_tiles;
-    t.phase = 2;
-    t.blk = v / n_wt2;
-    t.wt = v - t.blk * n_wt2;
-  }
+__device__ __forceinline__ TileInfo tile_info(int u, int n_h, int routed_blocks) {
+  TileInfo t;
+  t.blk = u / n_h;
+  t.wt = u - t.blk * n_h;
   t.shared_blk = t.blk >= routed_blocks;
   return t;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+// silu(g) = g * sigmoid(g); the quotient with the fast approximate divide
+// (h is rounded to bf16 right after, far coarser than its error).
+__device__ __forceinline__ float silu_fast(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-// Slots (T * k) up to which the kernel does the scatter-reduce itself.
-constexpr int kCombineMaxSlots = 64;
+// The d tiles of a tile's down GEMM are walked starting at a tile-dependent
+// offset, so that CTAs working at the same time add into different lines of
+// the accumulator instead of all hitting the same ones.
+__device__ __forceinline__ int d_rotation(int u, int n_d) { return u % n_d; }
+__device__ __forceinline__ int d_tile(int k, int rot, int n_d) {
+  const int di = k + rot;
+  return di >= n_d ? di - n_d : di;
+}
 
-// Named barrier 1 over the four epilogue warps (barrier 0 is
-// __syncthreads).  Each warp reconverges first, as the aligned barrier
-// requires.  epilogue_any() is the same barrier with an OR reduction: the
-// epilogue takes its leave-on-timeout decision uniformly, so no epilogue
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Named barrier 1 over the four epilogue warps, 2 over the four gather warps
+// (barrier 0 is __syncthreads).  Each warp reconverges first, as the aligned
+// barrier requires.  epilogue_any() is barrier 1 with an OR reduction: the
+// epilogue takes every leave-on-timeout decision uniformly, so no epilogue
 // thread can be left waiting at a later barrier for one that left.
 __device__ __forceinline__ void epilogue_sync() {
   __syncwarp();
   asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+__device__ __forceinline__ void gather_sync() {
+  __syncwarp();
+  asm volatile("bar.sync 2, 128;" ::: "memory");
 }
 
 __device__ __forceinline__ bool epilogue_any(bool v) {
@@ -129,22 +146,38 @@ __device__ __forceinline__ bool epilogue_any(bool v) {
   return r != 0;
 }
 
+// Bounded spin until *p >= target (acquire).  False on timeout or abort.
+__device__ __forceinline__ bool spin_until(const int32_t* p, int target, volatile int* abort_flag) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (ptx::ld_acquire_gpu(p) < target) {
+    if (*abort_flag || ptx::globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    __nanosleep(64);
+  }
+  return true;
+}
+
 template <int EPI1, int TOK>
 __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
     fused_expert_kernel(const __grid_constant__ FusedArgs args) {
   using C = FusedCfg<EPI1, TOK>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* xbuf = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);  // [TOK][64]
-  int* s_slot = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes + C::kXbufBytes);
-  uint64_t* full =
-      reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes + C::kXbufBytes + C::kSlotBytes);
+  uint8_t* hbuf = smem + C::kStages * C::kStageBytes;                // [2][kHk][TOK rows x 128 B]
+  float* xbuf = reinterpret_cast<float*>(hbuf + 2 * C::kHBufBytes);  // [TOK][64]
+  int* tok_s = reinterpret_cast<int*>(hbuf + 2 * C::kHBufBytes + C::kXbufBytes);  // [2][64]
+  float* w_s = reinterpret_cast<float*>(tok_s + 2 * 64);                           // [2][64]
+  uint64_t* full = reinterpret_cast<uint64_t*>(w_s + 2 * 64);
   uint64_t* empty = full + C::kStages;
-  uint64_t* tfull = empty + C::kStages;
-  uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* d1_full = empty + C::kStages;
+  uint64_t* d1_empty = d1_full + 2;
+  uint64_t* hb_full = d1_empty + 2;
+  uint64_t* hb_empty = hb_full + 2;
+  uint64_t* mma_done = hb_empty + 2;
+  uint64_t* d2_full = mma_done + 1;
+  uint64_t* d2_empty = d2_full + C::kD2Slots;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(d2_empty + C::kD2Slots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_holder + 2);
+  volatile int* flag = reinterpret_cast<volatile int*>(tmem_holder + 2);
 
   const int warp = threadIdx.x / kWarp;
   const int lane = threadIdx.x % kWarp;
@@ -155,10 +188,18 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
       ptx::mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(&tfull[b], 1);
-      ptx::mbar_init(&tempty[b], 4);
+      ptx::mbar_init(&d1_full[b], 1);
+      ptx::mbar_init(&d1_empty[b], 4);
+      ptx::mbar_init(&hb_full[b], 1);
+      ptx::mbar_init(&hb_empty[b], 1);
+    }
+    ptx::mbar_init(mma_done, 1);
+    for (int s = 0; s < C::kD2Slots; ++s) {
+      ptx::mbar_init(&d2_full[s], 1);
+      ptx::mbar_init(&d2_empty[s], 4);
     }
     *abort_flag = 0;
+    *flag = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&args.tm_w13);
     ptx::prefetch_tmap(&args.tm_w2);
@@ -168,7 +209,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
     }
   }
   if (warp == 1) {
-    ptx::tmem_alloc(tmem_holder, C::kTmemCols);
+    ptx::tmem_alloc(tmem_holder, 512);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -182,52 +223,83 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
   if (routed_blocks < 0) routed_blocks = 0;
   if (routed_blocks > args.max_routed_blocks) routed_blocks = args.max_routed_blocks;
   const int total_blocks = routed_blocks + args.n_shared_blocks;
-  const int n_wt1 = (args.F + C::kH1Cols - 1) / C::kH1Cols;
-  const int n_wt2 = (args.d + 127) / 128;
-  const int n1_tiles = total_blocks * n_wt1;
-  const int total_tiles = n1_tiles + total_blocks * n_wt2;
+  const int n_h = (args.F + C::kH - 1) / C::kH;
+  const int n_d = (args.d + 127) / 128;
+  const int total_tiles = total_blocks * n_h;
+  // tiles of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
+  const int n_my = static_cast<int>(blockIdx.x) < total_tiles
+                       ? (total_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                             static_cast<int>(gridDim.x)
+                       : 0;
   const int nk1 = args.d / 64;
-  const int nk2 = args.F / 64;
+  const int nk2 = n_d * C::kHk;  // down-GEMM stages per tile
+  const int nacc = args.T * args.d;
 
   auto fail = [&]() {
     *abort_flag = 1;
     set_status(args.status, MOE_ERR_DEVICE_TIMEOUT);
   };
+  auto tile_of = [&](int i) { return tile_info(static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x), n_h, routed_blocks); };
 
+  // Stage order of every role: gate/up of tile 0; then for i >= 1 gate/up of
+  // tile i followed by the down GEMM of tile i-1; last the down GEMM of the
+  // final tile.
   if (warp == 0) {
     // ------------------------------------------------ TMA producer (weights)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < total_tiles; u += gridDim.x) {
-        const Tile t = fused_tile(u, n1_tiles, n_wt1, n_wt2, routed_blocks);
-        int e = 0;
-        if (!t.shared_blk) {
-          e = args.expert_ids[t.blk];
-          if (e < 0 || e >= args.E) set_status(args.status, MOE_ERR_BAD_EXPERT_ID);
+      auto expert_of = [&](const TileInfo& t) {
+        if (t.shared_blk) return 0;
+        const int e = args.expert_ids[t.blk];
+        if (e < 0 || e >= args.E) set_status(args.status, MOE_ERR_BAD_EXPERT_ID);  // TMA fills zeros
+        return e;
+      };
+      auto acquire = [&]() {
+        if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+          fail();
+          ok = false;
         }
-        const int nk = t.phase == 1 ? nk1 : nk2;
-        const CUtensorMap* tm = t.phase == 1 ? (t.shared_blk ? &args.tm_w13s : &args.tm_w13)
-                                             : (t.shared_blk ? &args.tm_w2s : &args.tm_w2);
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
-            fail();
-            ok = false;
-            break;
+        return ok;
+      };
+      auto advance = [&]() {
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      };
+      // Streamed weight lines are used once: mark them first to leave L2.
+      const uint64_t evict_first = ptx::l2_policy_evict_first();
+      for (int i = 0; ok && i <= n_my; ++i) {
+        if (i < n_my) {
+          const TileInfo t = tile_of(i);
+          const int e = expert_of(t);
+          const CUtensorMap* tm = t.shared_blk ? &args.tm_w13s : &args.tm_w13;
+          for (int s = 0; s < nk1 && acquire(); ++s) {
+            uint8_t* sW = smem + stage * C::kStageBytes;
+            ptx::mbar_arrive_expect_tx(&full[stage], C::kWBytes);
+            if (C::kGated) {
+              ptx::tma_load_3d_hint(sW, tm, &full[stage], s * 64, t.wt * 64, e, evict_first);
+              ptx::tma_load_3d_hint(sW + 64 * 128, tm, &full[stage], s * 64, args.F + t.wt * 64, e, evict_first);
+            } else {
+              ptx::tma_load_3d_hint(sW, tm, &full[stage], s * 64, t.wt * 128, e, evict_first);
+            }
+            advance();
           }
-          uint8_t* sW = smem + stage * C::kStageBytes;
-          ptx::mbar_arrive_expect_tx(&full[stage], C::kTx);
-          if (t.phase == 1 && C::kGated) {
-            // 64 gate rows, then the 64 matching up rows (64-row boxes)
-            ptx::tma_load_3d(sW, tm, &full[stage], kb * 64, t.wt * 64, e);
-            ptx::tma_load_3d(sW + 64 * 128, tm, &full[stage], kb * 64, args.F + t.wt * 64, e);
-          } else {
-            ptx::tma_load_3d(sW, tm, &full[stage], kb * 64, t.wt * 128, e);
-          }
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
+        }
+        if (ok && i >= 1) {
+          const TileInfo t = tile_of(i - 1);
+          const int e = expert_of(t);
+          const CUtensorMap* tm = t.shared_blk ? &args.tm_w2s : &args.tm_w2;
+          const int rot = d_rotation(static_cast<int>(blockIdx.x) + (i - 1) * static_cast<int>(gridDim.x), n_d);
+          for (int s = 0; s < nk2 && acquire(); ++s) {
+            const int dk = s / C::kHk, kk = s - dk * C::kHk;
+            const int di = d_tile(dk, rot, n_d);
+            uint8_t* sW = smem + stage * C::kStageBytes;
+            ptx::mbar_arrive_expect_tx(&full[stage], C::kWBytes);
+            ptx::tma_load_3d_hint(sW, tm, &full[stage], t.wt * C::kH + kk * 64, di * 128, e, evict_first);
+            advance();
           }
         }
       }
@@ -237,255 +309,327 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int abuf = 0;
-      uint32_t aphase = 0;
+      int d2c = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < total_tiles; u += gridDim.x) {
-        const Tile t = fused_tile(u, n1_tiles, n_wt1, n_wt2, routed_blocks);
-        if (!ptx::mbar_wait_bounded(&tempty[abuf], aphase ^ 1u, abort_flag, kWaitLimitNs)) {
+      auto wait = [&](uint64_t* bar, uint32_t parity) {
+        if (!ptx::mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs)) {
           fail();
-          break;
+          ok = false;
         }
-        ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * C::kAccCols);
-        const int nk = t.phase == 1 ? nk1 : nk2;
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!ptx::mbar_wait_bounded(&full[stage], phase, abort_flag, kWaitLimitNs)) {
-            fail();
-            ok = false;
-            break;
-          }
+        return ok;
+      };
+      for (int i = 0; ok && i <= n_my; ++i) {
+        if (i < n_my) {
+          const int b = i & 1;
+          const uint32_t bph = static_cast<uint32_t>((i >> 1) & 1);
+          if (!wait(&d1_empty[b], bph ^ 1u)) break;
           ptx::tc_fence_after();
-          ptx::fence_proxy_async_smem();
-          const uint32_t sW = ptx::smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t sX = sW + C::kWBytes;
+          const uint32_t d1 = tmem_base + static_cast<uint32_t>(b * TOK);
+          for (int kb = 0; kb < nk1; ++kb) {
+            if (!wait(&full[stage], phase)) break;
+            ptx::tc_fence_after();
+            ptx::fence_proxy_async_smem();  // token rows were written by cp.async
+            const uint32_t sW = ptx::smem_u32(smem + stage * C::kStageBytes);
+            const uint32_t sX = sW + C::kWBytes;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
-            const uint64_t dw = ptx::sw128_kmajor_desc(sW + kk * 32);
-            const uint64_t dx = ptx::sw128_kmajor_desc(sX + kk * 32);
-            ptx::mma_bf16(d_tmem, dw, dx, C::kIdesc, acc);
+            for (int q = 0; q < 4; ++q)
+              ptx::mma_bf16(d1, ptx::sw128_kmajor_desc(sW + q * 32), ptx::sw128_kmajor_desc(sX + q * 32), C::kIdesc,
+                            (kb | q) != 0 ? 1u : 0u);
+            ptx::mma_commit(&empty[stage]);
+            if (++stage == C::kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-          ptx::mma_commit(&empty[stage]);
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+          if (!ok) break;
+          ptx::mma_commit(&d1_full[b]);
         }
-        if (!ok) break;
-        ptx::mma_commit(&tfull[abuf]);
-        if (++abuf == 2) {
-          abuf = 0;
-          aphase ^= 1u;
+        if (i >= 1) {
+          const int p = i - 1;
+          const int b = p & 1;
+          if (!wait(&hb_full[b], static_cast<uint32_t>((p >> 1) & 1))) break;
+          ptx::tc_fence_after();
+          const uint32_t sH = ptx::smem_u32(hbuf + b * C::kHBufBytes);
+          const int n_g = (n_d + C::kGroup - 1) / C::kGroup;
+          for (int g = 0; ok && g < n_g; ++g, ++d2c) {
+            const int slot = d2c % C::kD2Slots;
+            const uint32_t sph = static_cast<uint32_t>((d2c / C::kD2Slots) & 1);
+            if (!wait(&d2_empty[slot], sph ^ 1u)) break;
+            ptx::tc_fence_after();
+            for (int w = 0; ok && w < C::kGroup && g * C::kGroup + w < n_d; ++w) {
+              const uint32_t d2 = tmem_base + static_cast<uint32_t>(2 * TOK + slot * 64 + w * TOK);
+              for (int kk = 0; kk < C::kHk; ++kk) {
+                if (!wait(&full[stage], phase)) break;
+                ptx::tc_fence_after();
+                const uint32_t sW = ptx::smem_u32(smem + stage * C::kStageBytes);
+                const uint32_t sB = sH + kk * TOK * 128;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  ptx::mma_bf16(d2, ptx::sw128_kmajor_desc(sW + q * 32), ptx::sw128_kmajor_desc(sB + q * 32),
+                                C::kIdesc, (kk | q) != 0 ? 1u : 0u);
+                ptx::mma_commit(&empty[stage]);
+                if (++stage == C::kStages) {
+                  stage = 0;
+                  phase ^= 1u;
+                }
+              }
+            }
+            if (!ok) break;
+            ptx::mma_commit(&d2_full[slot]);
+          }
+          if (!ok) break;
+          ptx::mma_commit(&hb_empty[b]);  // the h slice may be overwritten once these MMAs finish
         }
       }
+      // no MMA of this CTA may still run when TMEM is freed (this wait
+      // ignores the abort flag; *flag stays zero until the block barrier)
+      ptx::mma_commit(mma_done);
+      if (!ptx::mbar_wait_bounded(mma_done, 0u, flag, kWaitLimitNs)) fail();
     }
   } else if (warp < 6) {
     // ------------------------------------------------ epilogue
-    const int q = warp & 3;
-    const int row = q * 32 + lane;  // weight row within the tile = output column
+    const int q = warp & 3;         // TMEM lane quadrant this warp may access
+    const int row = q * 32 + lane;  // accumulator row: weight row / d row within the tile
     const int etid = threadIdx.x - 64;
-    int abuf = 0;
-    uint32_t aphase = 0;
-    for (int u = blockIdx.x; u < total_tiles; u += gridDim.x) {
-      const Tile t = fused_tile(u, n1_tiles, n_wt1, n_wt2, routed_blocks);
-      const bool got = ptx::mbar_wait_bounded(&tfull[abuf], aphase, abort_flag, kWaitLimitNs);
-      if (epilogue_any(!got)) {
-        if (!got) fail();
-        break;
-      }
-      ptx::tc_fence_after();
-      const uint32_t t_acc =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(abuf * C::kAccCols);
-      const int pos0 = t.blk * args.block_m;
-      if (t.phase == 1 && C::kGated) {
-        // lanes 0-63 hold the gate and lanes 64-127 the up pre-activations
-        // of h columns wt*64 + (row % 64): the up half goes through xbuf
-        const int col = t.wt * 64 + (row & 63);
-        const bool col_ok = col < args.F;
-        float gate[TOK];
-#pragma unroll
-        for (int j0 = 0; j0 < TOK; j0 += 16) {
-          uint32_t a[16];
-          ptx::tmem_ld16(t_acc + j0, a);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            if (q >= 2)
-              xbuf[(j0 + jj) * 64 + (row - 64)] = __uint_as_float(a[jj]);
-            else
-              gate[j0 + jj] = __uint_as_float(a[jj]);
-          }
-        }
-        epilogue_sync();
-        if (q < 2 && col_ok) {
-#pragma unroll
-          for (int j = 0; j < TOK; ++j)
-            args.h[static_cast<size_t>(pos0 + j) * args.F + col] =
-                float_to_bf16_bits(silu_f(gate[j]) * xbuf[j * 64 + row]);
-        }
-      } else if (t.phase == 1) {
-        const int col = t.wt * 128 + row;
-        const bool col_ok = col < args.F;
-#pragma unroll 1
-        for (int j0 = 0; j0 < TOK; j0 += 16) {
-          uint32_t a[16];
-          ptx::tmem_ld16(t_acc + j0, a);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            float v = fmaxf(__uint_as_float(a[jj]), 0.0f);
-            v *= v;
-            if (col_ok) args.h[static_cast<size_t>(pos0 + j0 + jj) * args.F + col] = float_to_bf16_bits(v);
-          }
-        }
-      } else {
-        const int col = t.wt * 128 + row;
-        const bool col_ok = col < args.d;
-#pragma unroll 1
-        for (int j0 = 0; j0 < TOK; j0 += 16) {
-          uint32_t a[16];
-          ptx::tmem_ld16(t_acc + j0, a);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int p = pos0 + j0 + jj;
-            bool valid;
-            float wv = 1.0f;
-            if (!t.shared_blk) {
-              const int slot = args.sorted_ids[p];
-              valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
-              if (valid) wv = args.topk_w[slot];
-            } else {
-              valid = (t.blk - routed_blocks) * args.block_m + j0 + jj < args.T;
+    bool zero_seen = false;
+    int d2c = 0;
+    // Same order as the MMA: the gate/up accumulator of tile i is turned
+    // into h before the down-GEMM partials of tile i-1 are reduced, so the
+    // tensor core finds h(i) ready when it reaches the down GEMM of tile i.
+    for (int i = 0; i <= n_my; ++i) {
+      if (i < n_my) {
+        const TileInfo t = tile_of(i);
+        const int b = i & 1;
+        const uint32_t bph = static_cast<uint32_t>((i >> 1) & 1);
+        // token and weight of each row of the block (-1: padding), used by
+        // the reduction of this tile one step later
+        if (etid < TOK) {
+          const int j = etid;
+          int tok = -1;
+          float wj = 0.0f;
+          if (!t.shared_blk) {
+            const int slot = args.sorted_ids[t.blk * args.block_m + j];
+            if (static_cast<unsigned>(slot) < static_cast<unsigned>(args.S)) {
+              tok = slot / args.k;
+              wj = args.topk_w[slot];
             }
-            if (col_ok && valid) args.y[static_cast<size_t>(p) * args.d + col] = __uint_as_float(a[jj]) * wv;
+          } else {
+            const int tk = (t.blk - routed_blocks) * args.block_m + j;
+            if (tk < args.T) {
+              tok = tk;
+              wj = 1.0f;
+            }
           }
+          tok_s[b * 64 + j] = tok;
+          w_s[b * 64 + j] = wj;
         }
-      }
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&tempty[abuf]);
-      if (++abuf == 2) {
-        abuf = 0;
-        aphase ^= 1u;
-      }
-      // publish the finished tile: the barrier orders every epilogue
-      // thread's stores before thread 0's GPU-scope release
-      epilogue_sync();
-      if (t.phase == 1) {
-        if (etid == 0) ptx::red_release_gpu_add(&args.ready[t.blk], 1);
-      } else if (args.do_combine) {
-        if (etid == 0) *last_flag = (ptx::atom_acq_rel_gpu_add(&args.done[t.wt], 1) == total_blocks - 1) ? 1 : 0;
-        epilogue_sync();
-        if (*last_flag) {
-          // this CTA finished the last down tile of column tile t.wt (its
-          // acquire plus the barrier order the loads below after every
-          // other CTA's y stores): every load first, then the sums in order
-          const int c = t.wt * 128 + row;
-          const int nslot = args.T * args.k;
-          for (int i = etid; i < nslot; i += 128) s_slot[i] = __ldcg(args.inv_pos + i);
+        const bool got = ptx::mbar_wait_bounded(&d1_full[b], bph, abort_flag, kWaitLimitNs) &&
+                         ptx::mbar_wait_bounded(&hb_empty[b], bph ^ 1u, abort_flag, kWaitLimitNs);
+        if (epilogue_any(!got)) {
+          if (!got) fail();
+          break;
+        }
+        ptx::tc_fence_after();
+        // ---- gate/up accumulator -> h slice in shared memory (MMA operand layout)
+        const uint32_t t1 = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * TOK);
+        uint8_t* hb = hbuf + b * C::kHBufBytes;
+        if (C::kGated) {
+          float gate[TOK];
+#pragma unroll
+          for (int j0 = 0; j0 < TOK; j0 += 16) {
+            uint32_t a[16];
+            ptx::tmem_ld16(t1 + j0, a);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              if (q >= 2)
+                xbuf[(j0 + jj) * 64 + (row - 64)] = __uint_as_float(a[jj]);
+              else
+                gate[j0 + jj] = __uint_as_float(a[jj]);
+            }
+          }
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&d1_empty[b]);
           epilogue_sync();
-          if (c < args.d) {
-            float v[kCombineMaxSlots];
+          if (q < 2) {
+            const int c = row;  // h column within the slice (0..63)
 #pragma unroll
-            for (int i = 0; i < kCombineMaxSlots; ++i)
-              if (i < nslot) v[i] = __ldcg(args.y + static_cast<size_t>(s_slot[i]) * args.d + c);
-            float acc = 0.0f;
-            int j = 0, tok = 0;
+            for (int j = 0; j < TOK; ++j) {
+              const float hv = silu_fast(gate[j]) * xbuf[j * 64 + c];
+              const uint32_t off = (j >> 3) * 1024 + (j & 7) * 128 + (((c >> 3) ^ (j & 7)) << 4) + (c & 7) * 2;
+              *reinterpret_cast<uint16_t*>(hb + off) = float_to_bf16_bits(hv);
+            }
+          }
+        } else {
+          const int c = row & 63, kk = row >> 6;  // h column within its 64-wide K block
 #pragma unroll
-            for (int i = 0; i < kCombineMaxSlots; ++i) {
-              if (i < nslot) {
-                acc += v[i];
-                if (++j == args.k) {
-                  args.out[static_cast<size_t>(tok) * args.d + c] = float_to_bf16_bits(acc);
-                  acc = 0.0f;
-                  j = 0;
-                  ++tok;
-                }
+          for (int j0 = 0; j0 < TOK; j0 += 16) {
+            uint32_t a[16];
+            ptx::tmem_ld16(t1 + j0, a);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int j = j0 + jj;
+              float v = fmaxf(__uint_as_float(a[jj]), 0.0f);
+              v *= v;
+              const uint32_t off =
+                  kk * TOK * 128 + (j >> 3) * 1024 + (j & 7) * 128 + (((c >> 3) ^ (j & 7)) << 4) + (c & 7) * 2;
+              *reinterpret_cast<uint16_t*>(hb + off) = float_to_bf16_bits(v);
+            }
+          }
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&d1_empty[b]);
+        }
+        ptx::fence_proxy_async_smem();  // the tensor core reads the h slice next
+        epilogue_sync();                // (also publishes tok_s / w_s of this tile)
+        if (etid == 0) ptx::mbar_arrive(&hb_full[b]);
+      }
+      if (i >= 1) {
+        const int p = i - 1;
+        const int b = p & 1;
+        // every CTA has zeroed its slice of the accumulator before anyone adds
+        if (!zero_seen) {
+          const bool got = etid != 0 || spin_until(args.sync, static_cast<int>(gridDim.x), abort_flag);
+          if (epilogue_any(!got)) {
+            if (!got) fail();
+            break;
+          }
+          zero_seen = true;
+        }
+        // ---- down-GEMM partial of every d tile -> fp32 accumulator
+        const int rot = d_rotation(static_cast<int>(blockIdx.x) + p * static_cast<int>(gridDim.x), n_d);
+        const int* tk = tok_s + b * 64;
+        const float* wk = w_s + b * 64;
+        // valid rows of a block come first (an expert's padding ends its
+        // last block; shared-expert blocks end at row T), so the reduction
+        // stops at the first padding row
+        int n_valid = TOK;
+#pragma unroll
+        for (int j = TOK - 1; j >= 0; --j)
+          if (tk[j] < 0) n_valid = j;
+        bool left = false;
+        const int n_g = (n_d + C::kGroup - 1) / C::kGroup;
+        for (int g = 0; g < n_g; ++g, ++d2c) {
+          const int slot = d2c % C::kD2Slots;
+          const uint32_t sph = static_cast<uint32_t>((d2c / C::kD2Slots) & 1);
+          const bool got = ptx::mbar_wait_bounded(&d2_full[slot], sph, abort_flag, kWaitLimitNs);
+          if (epilogue_any(!got)) {
+            if (!got) fail();
+            left = true;
+            break;
+          }
+          ptx::tc_fence_after();
+          const int n_w = min(C::kGroup, n_d - g * C::kGroup);
+          const uint32_t t2 =
+              tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(2 * TOK + slot * 64);
+          uint32_t a[C::kGroup][TOK];
+#pragma unroll
+          for (int w = 0; w < C::kGroup; ++w) {
+            if (w < n_w) {
+#pragma unroll
+              for (int j0 = 0; j0 < TOK; j0 += 16)
+                ptx::tmem_ld16(t2 + w * TOK + j0, *reinterpret_cast<uint32_t(*)[16]>(&a[w][j0]));
+            }
+          }
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int w = 0; w < C::kGroup; ++w)
+#pragma unroll
+            for (int j = 0; j < TOK; ++j) asm volatile("" : "+r"(a[w][j]));  // uses stay after the wait
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&d2_empty[slot]);
+#pragma unroll
+          for (int w = 0; w < C::kGroup; ++w) {
+            const int drow = d_tile(g * C::kGroup + w, rot, n_d) * 128 + row;
+            if (w < n_w && drow < args.d) {
+              float* dst = args.acc + drow;
+#pragma unroll
+              for (int j = 0; j < TOK; ++j) {
+                if (j >= n_valid) break;
+                red_add_f32(dst + static_cast<size_t>(tk[j]) * args.d, wk[j] * __uint_as_float(a[w][j]));
               }
             }
           }
         }
+        if (left) break;
+        epilogue_sync();  // all reads of this tok_s / w_s buffer are done before it is rewritten
       }
     }
   } else {
-    // ------------------------------------------------ token operand
-    // 128 threads copy the tile's token rows with cp.async: gathered x rows
-    // for gate/up tiles, the block's h rows for down tiles once published
-    constexpr int kRowsPerThread = TOK / 16;
+    // ------------------------------------------------ token-row gather
     const int gtid = threadIdx.x - 192;
+    {  // zero this CTA's slice of the accumulator, then count the CTA on sync[0]
+      const int per = (nacc + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+      const int lo = static_cast<int>(blockIdx.x) * per;
+      const int hi = min(nacc, lo + per);
+      for (int e = lo + gtid; e < hi; e += 128) args.acc[e] = 0.0f;
+      gather_sync();
+      if (gtid == 0) ptx::red_release_gpu_add(args.sync, 1);
+    }
+    constexpr int kRowsPerThread = TOK / 16;
     const int chunk = gtid & 7;
     const int r0 = gtid >> 3;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < total_tiles; u += gridDim.x) {
-      const Tile t = fused_tile(u, n1_tiles, n_wt1, n_wt2, routed_blocks);
-      const uint16_t* src[kRowsPerThread];
-      uint32_t nbytes[kRowsPerThread];
-      int K;
-      if (t.phase == 1) {
-        K = args.d;
+    auto acquire = [&]() {
+      if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+        fail();
+        ok = false;
+      }
+      return ok;
+    };
+    auto advance = [&]() {
+      if (++stage == C::kStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    };
+    for (int i = 0; ok && i <= n_my; ++i) {
+      if (i < n_my) {
+        const TileInfo t = tile_of(i);
+        const uint16_t* src[kRowsPerThread];
+        uint32_t nbytes[kRowsPerThread];
 #pragma unroll
-        for (int i = 0; i < kRowsPerThread; ++i) {
-          const int r = r0 + 16 * i;
+        for (int r = 0; r < kRowsPerThread; ++r) {
+          const int row = r0 + 16 * r;
           int tok = 0;
           bool valid;
           if (!t.shared_blk) {
-            const int slot = args.sorted_ids[t.blk * args.block_m + r];
+            const int slot = args.sorted_ids[t.blk * args.block_m + row];
             valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
             if (valid) tok = slot / args.k;
           } else {
-            tok = (t.blk - routed_blocks) * args.block_m + r;
+            tok = (t.blk - routed_blocks) * args.block_m + row;
             valid = tok < args.T;
             if (!valid) tok = 0;
           }
-          src[i] = args.x + static_cast<size_t>(tok) * K + chunk * 8;
-          nbytes[i] = valid ? 16u : 0u;
+          src[r] = args.x + static_cast<size_t>(tok) * args.d + chunk * 8;
+          nbytes[r] = valid ? 16u : 0u;
         }
-      } else {
-        K = args.F;
-        // wait until every gate/up tile of this block has published its h
-        // (this thread holds no unsignalled stage while it waits)
-        const uint64_t t0 = ptx::globaltimer_ns();
-        while (ptx::ld_acquire_gpu(args.ready + t.blk) < n_wt1) {
-          if (*abort_flag || ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
-            fail();
-            ok = false;
-            break;
-          }
-          __nanosleep(128);
-        }
-        if (!ok) break;
+        for (int s = 0; s < nk1 && acquire(); ++s) {
+          const uint32_t sX = ptx::smem_u32(smem + stage * C::kStageBytes + C::kWBytes);
 #pragma unroll
-        for (int i = 0; i < kRowsPerThread; ++i) {
-          const int r = r0 + 16 * i;
-          src[i] = args.h + static_cast<size_t>(t.blk * args.block_m + r) * K + chunk * 8;
-          nbytes[i] = 16u;
+          for (int r = 0; r < kRowsPerThread; ++r) {
+            const int row = r0 + 16 * r;
+            const uint32_t dst = sX + (row >> 3) * 1024 + (row & 7) * 128 + ((chunk ^ (row & 7)) << 4);
+            ptx::cp_async_16(dst, src[r] + s * 64, nbytes[r]);
+          }
+          ptx::cp_async_arrive_noinc(&full[stage]);
+          advance();
         }
       }
-      const int nk = K / 64;
-      for (int kb = 0; kb < nk; ++kb) {
-        if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
-          fail();
-          ok = false;
-          break;
-        }
-        const uint32_t sX = ptx::smem_u32(smem + stage * C::kStageBytes + C::kWBytes);
-#pragma unroll
-        for (int i = 0; i < kRowsPerThread; ++i) {
-          const int r = r0 + 16 * i;
-          const uint32_t dst = sX + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4);
-          ptx::cp_async_16(dst, src[i] + kb * 64, nbytes[i]);
-        }
-        ptx::cp_async_arrive_noinc(&full[stage]);
-        if (++stage == C::kStages) {
-          stage = 0;
-          phase ^= 1u;
+      if (ok && i >= 1) {
+        for (int s = 0; s < nk2 && acquire(); ++s) {
+          ptx::mbar_arrive(&full[stage]);  // down-GEMM stages carry weights only
+          advance();
         }
       }
     }
+    cp_async_wait_all();
   }
 
   // every warp reconverges (the idle lanes of the producer and MMA warps
@@ -495,17 +639,39 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
   __syncthreads();
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, C::kTmemCols);
+    ptx::tmem_dealloc(tmem_base, 512);
   }
-  // Check out; the last CTA returns every counter to zero for the next
-  // launch (no other CTA touches them any more).
-  if (threadIdx.x == 0)
-    *last_flag = ptx::atom_acq_rel_gpu_add(args.finished, 1) == static_cast<int>(gridDim.x) - 1 ? 1 : 0;
+  // ---- grid end: all reductions issued -> convert the accumulator to bf16
+  if (threadIdx.x == 0) {
+    ptx::atom_acq_rel_gpu_add(args.sync + 1, 1);  // releases this CTA's reductions
+    const bool all = spin_until(args.sync + 1, static_cast<int>(gridDim.x), abort_flag);
+    if (!all) fail();
+    *flag = all ? 1 : 0;
+  }
   __syncthreads();
-  if (*last_flag) {
-    for (int i = threadIdx.x; i < total_blocks; i += blockDim.x) args.ready[i] = 0;
-    for (int i = threadIdx.x; i < n_wt2; i += blockDim.x) args.done[i] = 0;
-    if (threadIdx.x == 0) *args.finished = 0;
+  if (*flag) {
+    const int per = ((nacc + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x) + 3) & ~3;
+    const int lo = static_cast<int>(blockIdx.x) * per;
+    const int hi = min(nacc, lo + per);
+    const bool vec = (reinterpret_cast<uintptr_t>(args.out) & 7) == 0;
+    for (int e = lo + 4 * static_cast<int>(threadIdx.x); e < hi; e += 4 * C::kNumThreads) {
+      if (vec && e + 4 <= hi) {
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(args.acc + e));
+        uint2 o;
+        o.x = pack_bf16x2(a.x, a.y);
+        o.y = pack_bf16x2(a.z, a.w);
+        *reinterpret_cast<uint2*>(args.out + e) = o;
+      } else {
+        for (int m = e; m < min(hi, e + 4); ++m) args.out[m] = float_to_bf16_bits(__ldcg(args.acc + m));
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && ptx::atom_acq_rel_gpu_add(args.sync + 2, 1) == static_cast<int>(gridDim.x) - 1) {
+    // every CTA has passed both waits: return the counters to zero
+    args.sync[0] = 0;
+    args.sync[1] = 0;
+    args.sync[2] = 0;
   }
 }
 
@@ -530,20 +696,25 @@ cudaError_t launch_fused_variant(const FusedArgs& args, int grid, cudaStream_t s
 
 bool fused_expert_supported(int block_m) { return block_m == 16 || block_m == 32 || block_m == 64; }
 
-bool fused_expert_combines(int T, int k, int n_shared) {
-  return n_shared == 0 && static_cast<int64_t>(T) * k <= kCombineMaxSlots;
+int64_t fused_expert_max_tiles(int act_epi, int total_blocks_max, int F) {
+  const int h = act_epi == kEpiSwiGLU ? 64 : 128;
+  return static_cast<int64_t>(total_blocks_max) * ((F + h - 1) / h);
 }
 
 cudaError_t launch_fused_expert(int act_epi, int block_m, const FusedArgs& args, int grid, cudaStream_t stream) {
   const bool gated = act_epi == kEpiSwiGLU;
   switch (block_m) {
-    case 16: return gated ? launch_fused_variant<kEpiSwiGLU, 16>(args, grid, stream)
-                          : launch_fused_variant<kEpiRelu2, 16>(args, grid, stream);
-    case 32: return gated ? launch_fused_variant<kEpiSwiGLU, 32>(args, grid, stream)
-                          : launch_fused_variant<kEpiRelu2, 32>(args, grid, stream);
-    case 64: return gated ? launch_fused_variant<kEpiSwiGLU, 64>(args, grid, stream)
-                          : launch_fused_variant<kEpiRelu2, 64>(args, grid, stream);
-    default: return cudaErrorInvalidValue;
+    case 16:
+      return gated ? launch_fused_variant<kEpiSwiGLU, 16>(args, grid, stream)
+                   : launch_fused_variant<kEpiRelu2, 16>(args, grid, stream);
+    case 32:
+      return gated ? launch_fused_variant<kEpiSwiGLU, 32>(args, grid, stream)
+                   : launch_fused_variant<kEpiRelu2, 32>(args, grid, stream);
+    case 64:
+      return gated ? launch_fused_variant<kEpiSwiGLU, 64>(args, grid, stream)
+                   : launch_fused_variant<kEpiRelu2, 64>(args, grid, stream);
+    default:
+      return cudaErrorInvalidValue;
   }
 }
 

@@ -105,7 +105,8 @@ MOE_API size_t moe_align_workspace_size(int T, int k, int E);
 
 /* Bytes of device scratch moe_forward needs: a 64 KiB block of int32
  * counters, then the activation h [P_total, F] in bf16 and the scaled expert
- * outputs y [P_total, d] in fp32, where
+ * outputs y [P_total, d] in fp32 (block_m <= 64 uses its first T*d floats as
+ * the output accumulator), where
  * P_total = P_max + n_shared * ceil(T / block_m) * block_m.
  * The counter block (the first 64 KiB after rounding ws up to 256 bytes)
  * must be zero before the first moe_forward on a workspace (allocate it
@@ -174,8 +175,13 @@ MOE_API moe_status moe_align(const int32_t* topk_ids, int T, int k, int E, int b
  *                out[t] = sum_j topk_weights[t,j] * W2_e (act(W13_e x[t]))
  *                         (+ shared(x[t]) with weight 1),
  *                with fp32 accumulation; h is rounded to bf16 (it feeds the
- *                bf16 down GEMM), the per-slot scaled outputs stay fp32 and
- *                the k-sum is fp32 in slot order, rounded once to bf16.
+ *                bf16 down GEMM) and the weighted sum is fp32, rounded once
+ *                to bf16.  block_m = 128: the per-slot scaled outputs are
+ *                summed in slot order, so repeated calls agree bit for bit.
+ *                block_m <= 64 (one fused kernel split along F): partial
+ *                sums are added into an fp32 accumulator with atomics in an
+ *                order that depends on timing, so repeated calls agree to
+ *                fp32 rounding of that sum (at most 1 bf16 ulp in out).
  *   ws, ws_bytes scratch of moe_workspace_size bytes (its counter block zero,
  *                see moe_workspace_size); calls sharing a workspace must not
  *                overlap on the GPU.

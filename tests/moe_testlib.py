@@ -104,6 +104,22 @@ def compare_out(gpu_bits: np.ndarray, ref: np.ndarray, label: str = ""):
     return max_abs / rms, excess / rms, rel_l2
 
 
+def bf16_order_key(bits: np.ndarray) -> np.ndarray:
+    """Map bf16 bit patterns to integers whose difference counts ulps
+    (monotone in the value; +0 and -0 both map to 0)."""
+    b = bits.astype(np.int64)
+    mag = b & 0x7FFF
+    return np.where(b & 0x8000, -mag, mag)
+
+
+def assert_within_ulp(a_bits: np.ndarray, b_bits: np.ndarray, max_ulp: int = 1, label: str = ""):
+    """Two bf16 outputs agree to max_ulp units in the last place everywhere."""
+    assert a_bits.shape == b_bits.shape, label
+    gap = np.abs(bf16_order_key(a_bits) - bf16_order_key(b_bits))
+    worst = int(gap.max()) if gap.size else 0
+    assert worst <= max_ulp, f"{label}: outputs differ by {worst} bf16 ulp"
+
+
 def compare_route(ids_gpu, w_gpu, ids_ref, w_ref, label=""):
     assert np.array_equal(ids_gpu, ids_ref), f"{label}: topk_ids differ at {np.argwhere(ids_gpu != ids_ref)[:5]}"
     tol = WEIGHT_TOL * np.maximum(1.0, np.abs(w_ref))

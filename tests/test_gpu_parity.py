@@ -12,8 +12,8 @@ import torch
 import oracle
 from grouped_gemm_gating_b200 import moe as M
 from grouped_gemm_gating_b200 import workloads as W
-from moe_testlib import (DeviceLayer, compare_align, compare_out, compare_route, oracle_route,
-                         route_kwargs)
+from moe_testlib import (DeviceLayer, assert_within_ulp, compare_align, compare_out, compare_route,
+                         oracle_route, route_kwargs)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,8 +37,7 @@ SMALL = {
                                      seed=2008),
     "one_expert_hot": CFG["tiny"].with_(name="one_expert_hot", T=700, d=128, F=128, E=4, k=1, block_m=128,
                                         seed=2009, logits_kind="decode_hot"),
-    # fused expert kernel (block_m <= 64) with a shared expert, with the
-    # in-kernel combine (T <= 64) and with the separate combine (T > 64)
+    # fused expert kernel (block_m <= 64) with a shared expert
     "shared_bm16_fused_combine": CFG["dsv3"].with_(name="shared_bm16_fused_combine", T=40, d=256, F=192,
                                                    block_m=16, seed=2010),
     "shared_bm32_sep_combine": CFG["dsv3"].with_(name="shared_bm32_sep_combine", T=100, d=320, F=128,
@@ -262,7 +261,8 @@ def test_cuda_graph_replay_matches_eager():
     torch.cuda.synchronize()
     replayed = M_bits(lay.buf.out).copy()
     eager = M_bits(lay.run()).copy()
-    assert np.array_equal(replayed, eager)
+    # block_m <= 64 sums partials with fp32 atomics: equal up to 1 bf16 ulp
+    assert_within_ulp(replayed, eager, 1)
     ids, w = oracle_route(inp2)
     ref = oracle.forward(inp2.x, inp.w13, inp.w2, ids, w, cfg.act)
     compare_out(replayed, ref, "graph replay")
@@ -326,9 +326,9 @@ def test_fused_counters_return_to_zero_and_workspace_is_shareable():
     ref_a = M_bits(lay_a.run()).copy()
     ref_b = M_bits(lay_b.run()).copy()
     for _ in range(2):
-        assert np.array_equal(M_bits(lay_a.run()), ref_a)
+        assert_within_ulp(M_bits(lay_a.run()), ref_a, 1)
         torch.cuda.synchronize()
         base = (shared_ws.data_ptr() + 255) // 256 * 256 - shared_ws.data_ptr()
         assert int(shared_ws[base: base + 65536].count_nonzero()) == 0
-        assert np.array_equal(M_bits(lay_b.run()), ref_b)
+        assert_within_ulp(M_bits(lay_b.run()), ref_b, 1)
     assert lay_a.status() == 0 and lay_b.status() == 0
