@@ -38,6 +38,14 @@ import numpy as np  # noqa: E402
 from grouped_gemm_gating_b200 import workloads as W  # noqa: E402
 
 METRIC = "MoE layer TFLOPS and tokens/s on 1 B200; % of bf16 tensor peak / HBM roofline"
+
+# DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
+# capture of that kernel on that workload (bench.py --workload <w> --steps 3
+# --warmup 3 --no-cpu-baseline under ncu --set full -k <kernel> -c 1).  An
+# entry is removed whenever the kernel changes after its capture.
+NCU_TRAFFIC = {
+    ("decode", "fused_expert"): 202_747_904,
+}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -370,9 +378,12 @@ def run_ours(args):
         achieved = by / per_launch_s / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "unit": "GB/s"}
+    traffic = NCU_TRAFFIC.get((cfg.name, dom))
     roof.update({"kernel": dom, "achieved": round(achieved, 2), "peak": peak,
                  "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
-                 "frac": round(achieved / peak, 4), "traffic": None,
+                 "frac": round(achieved / peak, 4),
+                 "traffic": traffic,
+                 "traffic_vs_algorithmic": None if traffic is None else round(traffic / by, 3),
                  "per_launch_us": round(per_launch_s * 1e6, 2),
                  "algorithmic_flops": fl, "algorithmic_bytes": by})
 
