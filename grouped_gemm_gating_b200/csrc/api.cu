@@ -154,7 +154,7 @@ constexpr size_t kWsAlign = 256;
 // The forward workspace starts with a fixed block of int32 counters that the
 // fused expert kernel keeps at zero between calls (the last CTA of every
 // launch resets them; it uses the first three as grid counters, the rest is
-// reserved).  h and y follow it.
+// reserved).  h (block_m = 128) and the fp32 accumulator follow it.
 constexpr size_t kCounterInts = 16384;
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -234,9 +234,9 @@ size_t moe_workspace_size(int T, int d, int F, int E, int k, int block_m, moe_ac
   if (check_dims(T, d, F, E, k) != MOE_OK || !valid_block_m(block_m)) return 0;
   if ((act != MOE_ACT_SWIGLU && act != MOE_ACT_RELU2) || (n_shared != 0 && n_shared != 1)) return 0;
   const int64_t P = padded_total(T, k, E, block_m, n_shared);
-  const size_t h = round_up(static_cast<size_t>(P) * F * 2, kWsAlign);
-  const size_t y = round_up(static_cast<size_t>(P) * d * 4, kWsAlign);
-  return kCounterInts * 4 + h + y + kWsAlign;
+  const size_t h = block_m == 128 ? round_up(static_cast<size_t>(P) * F * 2, kWsAlign) : 0;
+  const size_t acc = round_up(static_cast<size_t>(T) * d * 4, kWsAlign);
+  return kCounterInts * 4 + h + acc + kWsAlign;
 }
 
 moe_status moe_route(const float* logits, int T, int E, int k, int n_group, int topk_group,
@@ -320,8 +320,7 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   if (n_shared != 0 && n_shared != 1) return MOE_ERR_UNSUPPORTED;
   if (n_shared && (!w13_shared || !w2_shared)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return finish(cudaSuccess, 0);
-  if (!x || !w13 || !w2 || !topk_weights || !sorted_token_ids || !expert_ids || !num_tokens_post_padded ||
-      !inv_pos || !out)
+  if (!x || !w13 || !w2 || !topk_weights || !sorted_token_ids || !expert_ids || !num_tokens_post_padded || !out)
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w13) || !aligned16(w2) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
   if (n_shared && (!aligned16(w13_shared) || !aligned16(w2_shared))) return MOE_ERR_INVALID_ARG;
@@ -335,9 +334,10 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   const int max_routed_blocks = static_cast<int>(P_max / bm);
   uint8_t* wsb = reinterpret_cast<uint8_t*>(round_up(reinterpret_cast<uintptr_t>(ws), kWsAlign));
   int32_t* counters = reinterpret_cast<int32_t*>(wsb);
+  // workspace: counters, then h (block_m = 128 only), then the fp32 [T, d] accumulator
   uint16_t* h = reinterpret_cast<uint16_t*>(wsb + kCounterInts * 4);
-  float* y =
-      reinterpret_cast<float*>(wsb + kCounterInts * 4 + round_up(static_cast<size_t>(P_total) * F * 2, kWsAlign));
+  const size_t h_bytes = bm == 128 ? round_up(static_cast<size_t>(P_total) * F * 2, kWsAlign) : 0;
+  float* y = reinterpret_cast<float*>(wsb + kCounterInts * 4 + h_bytes);
   const int n1 = act == MOE_ACT_SWIGLU ? 2 * F : F;
   const int num_sms = num_sms_current_device();
   if (num_sms <= 0) return MOE_ERR_CUDA;
@@ -396,7 +396,7 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   moe::GemmArgs a1;
   std::memset(&a1, 0, sizeof(a1));
   const int epi1 = act == MOE_ACT_SWIGLU ? moe::kEpiSwiGLU : moe::kEpiRelu2;
-  const uint32_t box1 = static_cast<uint32_t>(moe::gemm_box_rows(epi1, bm));
+  const uint32_t box1 = static_cast<uint32_t>(moe::gemm_box_rows(epi1));
   if (!encode_3d(&a1.tm_w, w13, d, n1, E, box1)) return MOE_ERR_CUDA;
   if (n_shared) {
     if (!encode_3d(&a1.tm_ws, w13_shared, d, n1, 1, box1)) return MOE_ERR_CUDA;
@@ -410,6 +410,8 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   a1.ntpp = num_tokens_post_padded;
   a1.topk_w = topk_weights;
   a1.out = h;
+  a1.acc = y;  // zeroed on the side for the down GEMM
+  a1.acc_elems = static_cast<int64_t>(T) * d;
   a1.status = dev_status;
   a1.T = T;
   a1.k = k;
@@ -421,21 +423,21 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   a1.block_m = bm;
   a1.max_routed_blocks = max_routed_blocks;
   a1.n_shared_blocks = n_shared_blocks;
-  int64_t tiles = moe::gemm_max_tiles(epi1, bm, max_routed_blocks, n_shared_blocks, F);
+  int64_t tiles = moe::gemm_max_tiles(epi1, max_routed_blocks, n_shared_blocks, F);
   int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
   if (grid < 1) grid = 1;
   cudaError_t err;
   {
     StageScope scope(2, s);
-    err = moe::launch_grouped_gemm(epi1, bm, a1, grid, s);
+    err = moe::launch_grouped_gemm(epi1, a1, grid, s);
   }
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   ++launches;
 
-  // down GEMM with the top-k weight epilogue: y [P_total, d] fp32
+  // down GEMM whose epilogue adds topk_weight * row into acc [T, d] fp32
   moe::GemmArgs a2;
   std::memset(&a2, 0, sizeof(a2));
-  const uint32_t box2 = static_cast<uint32_t>(moe::gemm_box_rows(moe::kEpiScale, bm));
+  const uint32_t box2 = static_cast<uint32_t>(moe::gemm_box_rows(moe::kEpiScale));
   if (!encode_3d(&a2.tm_w, w2, F, d, E, box2)) return MOE_ERR_CUDA;
   if (n_shared) {
     if (!encode_3d(&a2.tm_ws, w2_shared, F, d, 1, box2)) return MOE_ERR_CUDA;
@@ -448,7 +450,9 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   a2.expert_ids = expert_ids;
   a2.ntpp = num_tokens_post_padded;
   a2.topk_w = topk_weights;
-  a2.out = y;
+  a2.out = nullptr;
+  a2.acc = y;
+  a2.acc_elems = static_cast<int64_t>(T) * d;
   a2.status = dev_status;
   a2.T = T;
   a2.k = k;
@@ -460,19 +464,27 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   a2.block_m = bm;
   a2.max_routed_blocks = max_routed_blocks;
   a2.n_shared_blocks = n_shared_blocks;
-  tiles = moe::gemm_max_tiles(moe::kEpiScale, bm, max_routed_blocks, n_shared_blocks, d);
+  {
+    // column passes: keep each pass's slice of the accumulator within ~48 MB of L2
+    const int64_t acc_bytes = static_cast<int64_t>(T) * d * 4;
+    const int64_t budget = int64_t(48) << 20;
+    const int n_wt = (d + static_cast<int>(box2) - 1) / static_cast<int>(box2);
+    const int passes = static_cast<int>((acc_bytes + budget - 1) / budget);
+    a2.pass_cols = passes <= 1 ? 0 : (n_wt + passes - 1) / passes;
+  }
+  tiles = moe::gemm_max_tiles(moe::kEpiScale, max_routed_blocks, n_shared_blocks, d);
   grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
   if (grid < 1) grid = 1;
   {
     StageScope scope(3, s);
-    err = moe::launch_grouped_gemm(moe::kEpiScale, bm, a2, grid, s);
+    err = moe::launch_grouped_gemm(moe::kEpiScale, a2, grid, s);
   }
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   ++launches;
 
   {
     StageScope scope(4, s);
-    err = moe::launch_combine(y, inv_pos, num_tokens_post_padded, T, k, d, n_shared, out, s, &launches);
+    err = moe::launch_convert(y, static_cast<int64_t>(T) * d, out, num_sms, s, &launches);
   }
   return finish(err, launches);
 }

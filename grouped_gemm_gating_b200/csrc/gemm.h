@@ -9,10 +9,11 @@ namespace moe {
 enum EpiKind : int {
   kEpiSwiGLU = 0,  // gate/up GEMM, h = silu(gate) * up
   kEpiRelu2 = 1,   // fc1 GEMM, h = max(a, 0)^2
-  kEpiScale = 2    // down GEMM, y = topk_weight(row) * acc, stored fp32
+  kEpiScale = 2    // down GEMM, acc[token] += topk_weight(row) * row result (fp32)
 };
 
-// Arguments of one grouped GEMM launch.  Rows of the token operand are the
+// Arguments of one grouped GEMM launch (token-major tiles, block_m = 128).
+// Rows of the token operand are the
 // padded positions p = blk * block_m + r of the expert-sorted layout; block
 // blk < routed_blocks belongs to expert expert_ids[blk], blocks after that
 // (n_shared_blocks of them) to the shared expert, whose token is
@@ -26,7 +27,9 @@ struct GemmArgs {
   const int32_t* expert_ids;
   const int32_t* ntpp;
   const float* topk_w;  // [T * k], indexed by slot
-  void* out;            // [P_total, n_out]: bf16 h (gate/up GEMM) or fp32 y (down GEMM)
+  void* out;            // gate/up GEMM: bf16 h [P_total, n_out]
+  float* acc;           // fp32 [T, d] accumulator: zeroed by the gate/up GEMM, reduced into by the down GEMM
+  int64_t acc_elems;    // T * d
   int32_t* status;
   int T, k, S, E;
   int K;                // reduction length (multiple of 64)
@@ -35,14 +38,13 @@ struct GemmArgs {
   int block_m;
   int max_routed_blocks;
   int n_shared_blocks;
+  int pass_cols;        // output-column tiles per pass of the tile walk (0: one pass)
 };
 
-// Rows of one weight TMA box and output columns of one tile for a variant.
-int gemm_box_rows(int epi, int block_m);
-// Token rows per tile (== block_m).
-int gemm_token_rows(int block_m);
+// Rows of one weight TMA box (= output columns of one tile) for an epilogue.
+int gemm_box_rows(int epi);
 // Upper bound on tiles of one launch, for grid sizing.
-int64_t gemm_max_tiles(int epi, int block_m, int max_routed_blocks, int n_shared_blocks, int n_out);
-cudaError_t launch_grouped_gemm(int epi, int block_m, const GemmArgs& args, int grid, cudaStream_t stream);
+int64_t gemm_max_tiles(int epi, int max_routed_blocks, int n_shared_blocks, int n_out);
+cudaError_t launch_grouped_gemm(int epi, const GemmArgs& args, int grid, cudaStream_t stream);
 
 }  // namespace moe

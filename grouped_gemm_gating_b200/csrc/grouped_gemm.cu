@@ -13,13 +13,14 @@
 // epilogue; the down projection applies the top-k weight of each row in its
 // epilogue ("Common Pitfalls" 4: routed weights on the right rows).
 //
-// Two tile forms share this template:
-//  * token-major (block_m = 128): MMA M = 128 token rows, N = 256 weight rows
-//    (SwiGLU: 128 gate rows followed by the matching 128 up rows, so one
-//    thread holds both halves of its h columns).
-//  * weight-major "swap-AB" (block_m = 16..64, few tokens per expert): MMA
-//    M = 128 weight rows, N = block_m token rows; SwiGLU issues one MMA for
-//    the gate rows and one for the up rows into adjacent TMEM columns.
+// Tiles are token-major (block_m = 128): MMA M = 128 token rows, N = 256
+// weight rows (SwiGLU: 128 gate rows followed by the matching 128 up rows, so
+// one thread holds both halves of its h columns).  The down GEMM's epilogue
+// is the scatter-reduce: each row's top-k-weighted output is added into an
+// fp32 [T, d] accumulator at its token's row (red.global.add.v4.f32), so the
+// per-slot outputs never travel through HBM; the gate/up GEMM zeroes that
+// accumulator on the side (a warp of its own) and a small
+// kernel converts it to bf16 afterwards.
 //
 // Warp roles (one CTA per SM, persistent over a static tile stride):
 //   warp 0       TMA producer: weight tiles (and h tiles for the down GEMM)
@@ -29,6 +30,7 @@
 //                with 16-byte cp.async into the 128B-swizzled layout (padding
 //                rows zero-filled); each thread's copies of a stage arrive on
 //                the stage's full barrier by cp.async.mbarrier.arrive.noinc
+//   warp 10      gate/up GEMM only: zeroes the down GEMM's accumulator
 // Shared-memory stages are guarded by full/empty mbarriers (TMA operands
 // complete transaction bytes on the full barrier, gathered rows arrive on it
 // when their copies land; the MMA thread fences the generic and async
@@ -42,11 +44,12 @@
 
 namespace moe {
 
-template <bool SWAP, int EPI, int TOK>
+template <int EPI>
 struct GemmCfg {
+  static constexpr int TOK = 128;  // token rows per tile
   static constexpr bool kGated = (EPI == kEpiSwiGLU);
   static constexpr bool kGather = (EPI != kEpiScale);
-  static constexpr int kBoxRows = (!SWAP && !kGated) ? 256 : 128;
+  static constexpr int kBoxRows = kGated ? 128 : 256;
   static constexpr int kBoxes = kGated ? 2 : 1;
   static constexpr int kWRows = kBoxRows * kBoxes;
   static constexpr int kOutCols = kBoxRows;
@@ -55,23 +58,21 @@ struct GemmCfg {
   static constexpr int kStageBytes = kWBytes + kXBytes;
   static constexpr int kStagesRaw = (225 * 1024) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
-  static constexpr int kAccCols = SWAP ? (kGated ? 2 * TOK : TOK) : 256;
-  static constexpr int kTmemNeed = 2 * kAccCols;
-  static constexpr int kTmemCols = kTmemNeed <= 32    ? 32
-                                   : kTmemNeed <= 64  ? 64
-                                   : kTmemNeed <= 128 ? 128
-                                   : kTmemNeed <= 256 ? 256
-                                                      : 512;
-  static constexpr int kNumThreads = kGather ? 320 : 192;
+  static constexpr int kAccCols = 256;
+  static constexpr int kTmemCols = 512;
+  // gate/up: warps 6-9 gather token rows, warp 10 zeroes the accumulator
+  static constexpr int kNumThreads = kGather ? 352 : 192;
   static constexpr uint32_t kTxBytes = kWBytes + (kGather ? 0 : kXBytes);
   static constexpr int kBarrierBytes = 256;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes;
-  static constexpr uint32_t kIdesc = SWAP ? ptx::idesc_bf16_f32(128, TOK) : ptx::idesc_bf16_f32(128, 256);
+  // down GEMM: per epilogue warp a 32 x 33 fp32 transpose buffer, so the
+  // reduction is issued as full 128-byte row segments
+  static constexpr int kRedStride = 33;
+  static constexpr int kRedBytes = kGather ? 0 : 4 * 32 * kRedStride * 4;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes + kRedBytes;
+  static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(128, 256);
 
-  static_assert(TOK % 16 == 0 && TOK >= 16 && TOK <= 128, "token rows per tile");
-  static_assert(SWAP || TOK == 128, "token-major tiles hold 128 token rows");
   static_assert(kStages >= 3, "pipeline depth");
-  static_assert(kAccCols * 2 <= 512, "two accumulator buffers must fit TMEM");
+  static_assert(kAccCols * 2 <= kTmemCols, "two accumulator buffers must fit TMEM");
   static_assert((2 * kStages + 4) * 8 + 8 <= kBarrierBytes, "barrier area");
   static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
@@ -81,20 +82,37 @@ struct TileCoord {
   bool shared_blk;
 };
 
-__device__ __forceinline__ TileCoord tile_coord(int tile, int n_wt, int routed_blocks) {
+// Tiles are walked in column passes of pass_w output-column tiles: all
+// blocks for the first pass_w column tiles, then all blocks for the next
+// ones.  Within a pass, tiles are block-major, so CTAs working together
+// share an expert's weights in L2; the down GEMM picks pass_w so that one
+// pass's slice of the [T, d] accumulator stays resident in L2 while it is
+// being reduced into (a single pass when the whole accumulator fits).
+__device__ __forceinline__ TileCoord tile_coord(int tile, int n_wt, int pass_w, int total_blocks,
+                                                int routed_blocks) {
+  const int per_pass = total_blocks * pass_w;
+  const int pass = tile / per_pass;
+  const int w0 = pass * pass_w;
+  const int width = n_wt - w0 < pass_w ? n_wt - w0 : pass_w;
+  const int r = tile - pass * per_pass;
   TileCoord c;
-  c.blk = tile / n_wt;
-  c.wt = tile - c.blk * n_wt;
+  c.blk = r / width;
+  c.wt = w0 + (r - c.blk * width);
   c.shared_blk = c.blk >= routed_blocks;
   return c;
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
-template <bool SWAP, int EPI, int TOK>
-__global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
+__device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
-  using C = GemmCfg<SWAP, EPI, TOK>;
+  using C = GemmCfg<EPI>;
+  constexpr int TOK = C::TOK;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
@@ -142,6 +160,7 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
   if (routed_blocks > args.max_routed_blocks) routed_blocks = args.max_routed_blocks;
   const int total_blocks = routed_blocks + args.n_shared_blocks;
   const int n_wt = (args.n_out + C::kOutCols - 1) / C::kOutCols;
+  const int pass_w = args.pass_cols > 0 && args.pass_cols < n_wt ? args.pass_cols : n_wt;
   const int total_tiles = total_blocks * n_wt;
   const int nk = args.K / 64;
 
@@ -157,7 +176,7 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        const TileCoord tc = tile_coord(tile, n_wt, routed_blocks);
+        const TileCoord tc = tile_coord(tile, n_wt, pass_w, total_blocks, routed_blocks);
         const CUtensorMap* tm = tc.shared_blk ? &args.tm_ws : &args.tm_w;
         int e = 0;
         if (!tc.shared_blk) {
@@ -212,17 +231,8 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
-            const uint64_t dw = ptx::sw128_kmajor_desc(sW + kk * 32);
-            const uint64_t dx = ptx::sw128_kmajor_desc(sX + kk * 32);
-            if (!SWAP) {
-              ptx::mma_bf16(d_tmem, dx, dw, C::kIdesc, acc);
-            } else {
-              ptx::mma_bf16(d_tmem, dw, dx, C::kIdesc, acc);
-              if (C::kGated) {
-                const uint64_t du = ptx::sw128_kmajor_desc(sW + C::kBoxRows * 128 + kk * 32);
-                ptx::mma_bf16(d_tmem + TOK, du, dx, C::kIdesc, acc);
-              }
-            }
+            ptx::mma_bf16(d_tmem, ptx::sw128_kmajor_desc(sX + kk * 32), ptx::sw128_kmajor_desc(sW + kk * 32),
+                          C::kIdesc, acc);
           }
           ptx::mma_commit(&empty[stage]);
           if (++stage == C::kStages) {
@@ -245,7 +255,7 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
     int abuf = 0;
     uint32_t aphase = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      const TileCoord tc = tile_coord(tile, n_wt, routed_blocks);
+      const TileCoord tc = tile_coord(tile, n_wt, pass_w, total_blocks, routed_blocks);
       if (!ptx::mbar_wait_bounded(&tfull[abuf], aphase, abort_flag, kWaitLimitNs)) {
         fail();
         break;
@@ -253,116 +263,96 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
       ptx::tc_fence_after();
       const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(abuf * C::kAccCols);
       const int pos0 = tc.blk * args.block_m;
-      if (!SWAP) {
-        // thread = token row `row` of the tile, columns = weight rows
-        const int p = pos0 + row;
+      // thread = token row `row` of the tile, registers = output columns
+      const int p = pos0 + row;
+      if (EPI == kEpiSwiGLU) {
+        uint16_t* orow = static_cast<uint16_t*>(args.out) + static_cast<size_t>(p) * args.n_out;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 16) {
+          uint32_t g[16], u[16];
+          ptx::tmem_ld16(t_acc + c0, g);
+          ptx::tmem_ld16(t_acc + 128 + c0, u);
+          ptx::tmem_wait_ld();
+          const int col = tc.wt * 128 + c0;
+          if (col < args.n_out) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float h0 = silu_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+              const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+              pk[i] = pack_bf16x2(h0, h1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(orow + col);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      } else if (EPI == kEpiRelu2) {
+        uint16_t* orow = static_cast<uint16_t*>(args.out) + static_cast<size_t>(p) * args.n_out;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 256; c0 += 16) {
+          uint32_t a[16];
+          ptx::tmem_ld16(t_acc + c0, a);
+          ptx::tmem_wait_ld();
+          const int col = tc.wt * 256 + c0;
+          if (col < args.n_out) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float v0 = fmaxf(__uint_as_float(a[2 * i]), 0.0f);
+              const float v1 = fmaxf(__uint_as_float(a[2 * i + 1]), 0.0f);
+              pk[i] = pack_bf16x2(v0 * v0, v1 * v1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(orow + col);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      } else {
+        // scatter-reduce: acc[token] += topk_weight * row (shared expert: weight 1)
         bool valid;
+        int tok;
         float wrow = 1.0f;
         if (!tc.shared_blk) {
           const int slot = args.sorted_ids[p];
           valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
-          if (EPI == kEpiScale && valid) wrow = args.topk_w[slot];
+          tok = valid ? slot / args.k : 0;
+          if (valid) wrow = args.topk_w[slot];
         } else {
-          valid = (tc.blk - routed_blocks) * args.block_m + row < args.T;
+          tok = (tc.blk - routed_blocks) * args.block_m + row;
+          valid = tok < args.T;
         }
-        if (EPI != kEpiScale) valid = true;  // h rows are always written (padding rows are zero)
-        if (EPI == kEpiSwiGLU) {
-          uint16_t* orow = static_cast<uint16_t*>(args.out) + static_cast<size_t>(p) * args.n_out;
+        // 32 columns at a time: each lane parks its row's 32 values in the
+        // warp's transpose buffer, then 8 lanes cover one row's 128 bytes and
+        // one red.v4 instruction adds 4 whole row segments
+        float* stg = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + C::kBarrierBytes) +
+                     q * 32 * C::kRedStride;
+        const int rr = lane >> 3;        // row within a group of 4
+        const int cc = (lane & 7) * 4;   // column within the 32-column chunk
 #pragma unroll 1
-          for (int c0 = 0; c0 < 128; c0 += 16) {
-            uint32_t g[16], u[16];
-            ptx::tmem_ld16(t_acc + c0, g);
-            ptx::tmem_ld16(t_acc + 128 + c0, u);
-            ptx::tmem_wait_ld();
-            const int col = tc.wt * 128 + c0;
-            if (col < args.n_out) {
-              uint32_t pk[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float h0 = silu_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
-                const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
-                pk[i] = pack_bf16x2(h0, h1);
-              }
-              uint4* dst = reinterpret_cast<uint4*>(orow + col);
-              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            }
-          }
-        } else if (EPI == kEpiRelu2) {
-          uint16_t* orow = static_cast<uint16_t*>(args.out) + static_cast<size_t>(p) * args.n_out;
-#pragma unroll 1
-          for (int c0 = 0; c0 < 256; c0 += 16) {
-            uint32_t a[16];
-            ptx::tmem_ld16(t_acc + c0, a);
-            ptx::tmem_wait_ld();
-            const int col = tc.wt * 256 + c0;
-            if (col < args.n_out) {
-              uint32_t pk[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float v0 = fmaxf(__uint_as_float(a[2 * i]), 0.0f);
-                const float v1 = fmaxf(__uint_as_float(a[2 * i + 1]), 0.0f);
-                pk[i] = pack_bf16x2(v0 * v0, v1 * v1);
-              }
-              uint4* dst = reinterpret_cast<uint4*>(orow + col);
-              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            }
-          }
-        } else {
-          float* orow = static_cast<float*>(args.out) + static_cast<size_t>(p) * args.n_out;
-#pragma unroll 1
-          for (int c0 = 0; c0 < 256; c0 += 16) {
-            uint32_t a[16];
-            ptx::tmem_ld16(t_acc + c0, a);
-            ptx::tmem_wait_ld();
-            const int col = tc.wt * 256 + c0;
-            if (col < args.n_out && valid) {
-              float4* dst = reinterpret_cast<float4*>(orow + col);
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                dst[i] = make_float4(__uint_as_float(a[4 * i]) * wrow, __uint_as_float(a[4 * i + 1]) * wrow,
-                                     __uint_as_float(a[4 * i + 2]) * wrow, __uint_as_float(a[4 * i + 3]) * wrow);
-            }
-          }
-        }
-      } else {
-        // thread = weight row `row` (output column), columns = token rows
-        const int col = tc.wt * 128 + row;
-        const bool col_ok = col < args.n_out;
-#pragma unroll 1
-        for (int j0 = 0; j0 < TOK; j0 += 16) {
-          uint32_t a[16], u[16];
-          ptx::tmem_ld16(t_acc + j0, a);
-          if (EPI == kEpiSwiGLU) ptx::tmem_ld16(t_acc + TOK + j0, u);
+        for (int c0 = 0; c0 < 256; c0 += 32) {
+          uint32_t a[32];
+          ptx::tmem_ld16(t_acc + c0, *reinterpret_cast<uint32_t(*)[16]>(&a[0]));
+          ptx::tmem_ld16(t_acc + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&a[16]));
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int p = pos0 + j0 + jj;
-            float v = __uint_as_float(a[jj]);
-            bool valid = true;
-            if (EPI == kEpiSwiGLU) {
-              v = silu_f(v) * __uint_as_float(u[jj]);
-            } else if (EPI == kEpiRelu2) {
-              v = fmaxf(v, 0.0f);
-              v *= v;
-            } else {
-              if (!tc.shared_blk) {
-                const int slot = args.sorted_ids[p];
-                valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
-                v *= valid ? args.topk_w[slot] : 0.0f;
-              } else {
-                valid = (tc.blk - routed_blocks) * args.block_m + j0 + jj < args.T;
-              }
-            }
-            if (col_ok && valid) {
-              const size_t idx = static_cast<size_t>(p) * args.n_out + col;
-              if (EPI == kEpiScale)
-                static_cast<float*>(args.out)[idx] = v;
-              else
-                static_cast<uint16_t*>(args.out)[idx] = float_to_bf16_bits(v);
-            }
+          for (int j = 0; j < 32; ++j) asm volatile("" : "+r"(a[j]));  // uses stay after the wait
+          const int col = tc.wt * 256 + c0;
+          if (col >= args.n_out) break;  // uniform across the warp
+#pragma unroll
+          for (int j = 0; j < 32; ++j) stg[lane * C::kRedStride + j] = __uint_as_float(a[j]) * wrow;
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + rr;
+            const int tk = __shfl_sync(0xffffffffu, tok, r);
+            const int ok = __shfl_sync(0xffffffffu, valid ? 1 : 0, r);
+            const float* src = stg + r * C::kRedStride + cc;
+            if (ok)
+              red_add_v4_f32(args.acc + static_cast<size_t>(tk) * args.n_out + col + cc, src[0], src[1], src[2],
+                             src[3]);
           }
+          __syncwarp();
         }
       }
       ptx::tc_fence_before();
@@ -371,6 +361,20 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
       if (++abuf == 2) {
         abuf = 0;
         aphase ^= 1u;
+      }
+    }
+  } else if (C::kGather && warp == 10) {
+    // ------------------------------------------------ zero this CTA's share of the down GEMM's accumulator
+    if (args.acc != nullptr) {
+      const int64_t n = args.acc_elems;
+      const int64_t per = ((n + gridDim.x - 1) / gridDim.x + 3) & ~int64_t(3);
+      const int64_t lo = static_cast<int64_t>(blockIdx.x) * per;
+      const int64_t hi = lo + per < n ? lo + per : n;
+      for (int64_t i = lo + 4 * lane; i < hi; i += 4 * kWarp) {
+        if (i + 4 <= hi)
+          *reinterpret_cast<float4*>(args.acc + i) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        else
+          for (int64_t m = i; m < hi; ++m) args.acc[m] = 0.0f;
       }
     }
   } else if (C::kGather) {
@@ -383,7 +387,7 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
     uint32_t phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-      const TileCoord tc = tile_coord(tile, n_wt, routed_blocks);
+      const TileCoord tc = tile_coord(tile, n_wt, pass_w, total_blocks, routed_blocks);
       const uint16_t* src[kRowsPerThread];
       uint32_t nbytes[kRowsPerThread];
 #pragma unroll
@@ -440,10 +444,10 @@ __global__ void __launch_bounds__(GemmCfg<SWAP, EPI, TOK>::kNumThreads, 1)
 
 namespace {
 
-template <bool SWAP, int EPI, int TOK>
+template <int EPI>
 cudaError_t launch_variant(const GemmArgs& args, int grid, cudaStream_t stream) {
-  using C = GemmCfg<SWAP, EPI, TOK>;
-  auto kern = grouped_gemm_kernel<SWAP, EPI, TOK>;
+  using C = GemmCfg<EPI>;
+  auto kern = grouped_gemm_kernel<EPI>;
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -457,38 +461,22 @@ cudaError_t launch_variant(const GemmArgs& args, int grid, cudaStream_t stream) 
   return launch_pdl(kern, dim3(grid), dim3(C::kNumThreads), C::kSmemBytes, stream, args);
 }
 
-template <bool SWAP, int TOK>
-cudaError_t launch_epi(int epi, const GemmArgs& a, int grid, cudaStream_t s) {
-  switch (epi) {
-    case kEpiSwiGLU: return launch_variant<SWAP, kEpiSwiGLU, TOK>(a, grid, s);
-    case kEpiRelu2: return launch_variant<SWAP, kEpiRelu2, TOK>(a, grid, s);
-    case kEpiScale: return launch_variant<SWAP, kEpiScale, TOK>(a, grid, s);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
 }  // namespace
 
-int gemm_token_rows(int block_m) { return block_m; }
+int gemm_box_rows(int epi) { return epi == kEpiSwiGLU ? 128 : 256; }
 
-int gemm_box_rows(int epi, int block_m) {
-  const bool swap = block_m < 128;
-  const bool gated = epi == kEpiSwiGLU;
-  return (!swap && !gated) ? 256 : 128;
-}
-
-int64_t gemm_max_tiles(int epi, int block_m, int max_routed_blocks, int n_shared_blocks, int n_out) {
-  const int cols = gemm_box_rows(epi, block_m);
+int64_t gemm_max_tiles(int epi, int max_routed_blocks, int n_shared_blocks, int n_out) {
+  const int cols = gemm_box_rows(epi);
   const int64_t n_wt = (n_out + cols - 1) / cols;
   return static_cast<int64_t>(max_routed_blocks + n_shared_blocks) * n_wt;
 }
 
-cudaError_t launch_grouped_gemm(int epi, int block_m, const GemmArgs& a, int grid, cudaStream_t s) {
-  switch (block_m) {
-    case 16: return launch_epi<true, 16>(epi, a, grid, s);
-    case 32: return launch_epi<true, 32>(epi, a, grid, s);
-    case 64: return launch_epi<true, 64>(epi, a, grid, s);
-    case 128: return launch_epi<false, 128>(epi, a, grid, s);
+cudaError_t launch_grouped_gemm(int epi, const GemmArgs& a, int grid, cudaStream_t s) {
+  if (a.block_m != 128) return cudaErrorInvalidValue;
+  switch (epi) {
+    case kEpiSwiGLU: return launch_variant<kEpiSwiGLU>(a, grid, s);
+    case kEpiRelu2: return launch_variant<kEpiRelu2>(a, grid, s);
+    case kEpiScale: return launch_variant<kEpiScale>(a, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -104,9 +104,8 @@ MOE_API int64_t moe_max_padded(int T, int k, int E, int block_m);
 MOE_API size_t moe_align_workspace_size(int T, int k, int E);
 
 /* Bytes of device scratch moe_forward needs: a 64 KiB block of int32
- * counters, then the activation h [P_total, F] in bf16 and the scaled expert
- * outputs y [P_total, d] in fp32 (block_m <= 64 uses its first T*d floats as
- * the output accumulator), where
+ * counters, then (block_m = 128 only) the activation h [P_total, F] in bf16,
+ * then the fp32 output accumulator [T, d], where
  * P_total = P_max + n_shared * ceil(T / block_m) * block_m.
  * The counter block (the first 64 KiB after rounding ws up to 256 bytes)
  * must be zero before the first moe_forward on a workspace (allocate it
@@ -176,12 +175,13 @@ MOE_API moe_status moe_align(const int32_t* topk_ids, int T, int k, int E, int b
  *                         (+ shared(x[t]) with weight 1),
  *                with fp32 accumulation; h is rounded to bf16 (it feeds the
  *                bf16 down GEMM) and the weighted sum is fp32, rounded once
- *                to bf16.  block_m = 128: the per-slot scaled outputs are
- *                summed in slot order, so repeated calls agree bit for bit.
- *                block_m <= 64 (one fused kernel split along F): partial
- *                sums are added into an fp32 accumulator with atomics in an
- *                order that depends on timing, so repeated calls agree to
- *                fp32 rounding of that sum (at most 1 bf16 ulp in out).
+ *                to bf16.  The per-slot (block_m = 128) or per-h-slice
+ *                (block_m <= 64) partial results are added into the fp32
+ *                accumulator with atomics, in an order that depends on
+ *                timing, so repeated calls agree up to the fp32 rounding
+ *                of that sum (one bf16 ulp of a result, a little more where
+ *                the k terms cancel).  inv_pos is accepted for
+ *                interface stability and not read (it may be NULL).
  *   ws, ws_bytes scratch of moe_workspace_size bytes (its counter block zero,
  *                see moe_workspace_size); calls sharing a workspace must not
  *                overlap on the GPU.

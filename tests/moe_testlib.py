@@ -104,20 +104,21 @@ def compare_out(gpu_bits: np.ndarray, ref: np.ndarray, label: str = ""):
     return max_abs / rms, excess / rms, rel_l2
 
 
-def bf16_order_key(bits: np.ndarray) -> np.ndarray:
-    """Map bf16 bit patterns to integers whose difference counts ulps
-    (monotone in the value; +0 and -0 both map to 0)."""
-    b = bits.astype(np.int64)
-    mag = b & 0x7FFF
-    return np.where(b & 0x8000, -mag, mag)
-
-
 def assert_within_ulp(a_bits: np.ndarray, b_bits: np.ndarray, max_ulp: int = 1, label: str = ""):
-    """Two bf16 outputs agree to max_ulp units in the last place everywhere."""
+    """Two bf16 outputs of the same inputs agree up to the reordering of an
+    fp32 sum: max_ulp bf16 ulps of the result, plus 1e-4 rms for terms that
+    cancel (the reordering error scales with the terms, not with their sum;
+    a k-term fp32 sum moves by ~k * 2^-24 of the terms' magnitude)."""
     assert a_bits.shape == b_bits.shape, label
-    gap = np.abs(bf16_order_key(a_bits) - bf16_order_key(b_bits))
-    worst = int(gap.max()) if gap.size else 0
-    assert worst <= max_ulp, f"{label}: outputs differ by {worst} bf16 ulp"
+    a = W.bf16_bits_to_f32(a_bits).astype(np.float64)
+    b = W.bf16_bits_to_f32(b_bits).astype(np.float64)
+    if a.size == 0:
+        return
+    rms = float(np.sqrt((a ** 2).mean()))
+    ulp = np.maximum(np.abs(a), np.abs(b)) * 2.0 ** -7
+    bound = max_ulp * ulp + 1e-4 * rms
+    worst = float((np.abs(a - b) - bound).max())
+    assert worst <= 0.0, f"{label}: outputs differ beyond reordering ({worst:.3g} over the bound)"
 
 
 def compare_route(ids_gpu, w_gpu, ids_ref, w_ref, label=""):

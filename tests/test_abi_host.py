@@ -52,8 +52,12 @@ def test_workspace_sizes(lib):
     P = oracle.max_padded(T, k, E, bm) + T  # shared rows (T is a multiple of bm)
     size = M.moe_workspace_size(T, d, F, E, k, bm, M.ACT_SWIGLU, 1)
     counters = 65536
-    assert size >= P * (2 * F + 4 * d) + counters
-    assert size <= P * (2 * F + 4 * d) + counters + 1024
+    # counters, h [P_total, F] bf16, fp32 accumulator [T, d]
+    assert size >= P * 2 * F + T * 4 * d + counters
+    assert size <= P * 2 * F + T * 4 * d + counters + 1024
+    # block_m <= 64 keeps h in shared memory: counters and the accumulator only
+    small = M.moe_workspace_size(3, 2048, 768, 128, 8, 16, M.ACT_SWIGLU, 0)
+    assert 3 * 4 * 2048 + counters <= small <= 3 * 4 * 2048 + counters + 1024
     assert M.moe_workspace_size(T, d + 32, F, E, k, bm, M.ACT_SWIGLU, 0) == 0   # d % 64
     assert M.moe_workspace_size(T, d, F, 300, k, bm, M.ACT_SWIGLU, 0) == 0      # E > 256
     assert M.moe_align_workspace_size(3, 8, 128) == 0                           # single block

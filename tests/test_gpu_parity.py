@@ -224,13 +224,18 @@ def test_layer_full_size_sampled(name):
         assert (counts == 0).sum() == 8
 
 
-def test_repeated_calls_are_deterministic():
-    cfg = SMALL["zipf_small"]
-    lay = DeviceLayer(W.make_inputs(cfg))
-    a = M_bits(lay.run()).copy()
-    for _ in range(3):
-        b = M_bits(lay.run())
-        assert np.array_equal(a, b)
+def test_repeated_calls_agree_up_to_sum_order():
+    """Both paths add partial sums with fp32 atomics in a timing-dependent
+    order: repeated calls agree up to that reordering (a bf16 ulp of the
+    result, 1e-4 rms where terms cancel); routing / align outputs are
+    bit-identical."""
+    for name in ("zipf_small", "decode_d512"):
+        lay = DeviceLayer(W.make_inputs(SMALL[name]))
+        a = M_bits(lay.run()).copy()
+        ids = lay.buf.sorted_token_ids.clone()
+        for _ in range(3):
+            assert_within_ulp(M_bits(lay.run()), a, 1, name)
+            assert torch.equal(lay.buf.sorted_token_ids, ids)
 
 
 def test_forward_zero_tokens_is_noop():
@@ -261,7 +266,7 @@ def test_cuda_graph_replay_matches_eager():
     torch.cuda.synchronize()
     replayed = M_bits(lay.buf.out).copy()
     eager = M_bits(lay.run()).copy()
-    # block_m <= 64 sums partials with fp32 atomics: equal up to 1 bf16 ulp
+    # partial sums are added with fp32 atomics: equal up to their reordering
     assert_within_ulp(replayed, eager, 1)
     ids, w = oracle_route(inp2)
     ref = oracle.forward(inp2.x, inp.w13, inp.w2, ids, w, cfg.act)
