@@ -307,26 +307,20 @@ moe_status moe_align(const int32_t* topk_ids, int T, int k, int E, int block_m, 
   return finish(err, launches);
 }
 
-moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, const uint16_t* w2, int E, int F,
-                       const uint16_t* w13_shared, const uint16_t* w2_shared, int n_shared,
-                       const float* topk_weights, int k, const int32_t* sorted_token_ids,
-                       const int32_t* expert_ids, const int32_t* num_tokens_post_padded, const int32_t* inv_pos,
-                       int block_m, moe_act act, uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
-                       moe_stream_t stream) {
-  moe_status st = check_dims(T, d, F, E, k);
-  if (st != MOE_OK) return st;
-  if (!valid_block_m(block_m)) return MOE_ERR_UNSUPPORTED;
-  if (act != MOE_ACT_SWIGLU && act != MOE_ACT_RELU2) return MOE_ERR_INVALID_ARG;
-  if (n_shared != 0 && n_shared != 1) return MOE_ERR_UNSUPPORTED;
-  if (n_shared && (!w13_shared || !w2_shared)) return MOE_ERR_INVALID_ARG;
-  if (T == 0) return finish(cudaSuccess, 0);
-  if (!x || !w13 || !w2 || !topk_weights || !sorted_token_ids || !expert_ids || !num_tokens_post_padded || !out)
-    return MOE_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(w13) || !aligned16(w2) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-  if (n_shared && (!aligned16(w13_shared) || !aligned16(w2_shared))) return MOE_ERR_INVALID_ARG;
-  const size_t need = moe_workspace_size(T, d, F, E, k, block_m, act, n_shared);
-  if (ws == nullptr || ws_bytes < need) return MOE_ERR_WORKSPACE;
+}  // extern "C"
 
+namespace {
+
+// The forward after its argument checks.  route != nullptr: the fused kernel
+// also routes and aligns (the caller checked fused_routing_supported), and
+// topk_weights / sorted_token_ids / expert_ids / num_tokens_post_padded are
+// written by it instead of read.
+moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, const uint16_t* w2, int E, int F,
+                        const uint16_t* w13_shared, const uint16_t* w2_shared, int n_shared,
+                        const float* topk_weights, int k, const int32_t* sorted_token_ids,
+                        const int32_t* expert_ids, const int32_t* num_tokens_post_padded, int block_m, moe_act act,
+                        uint16_t* out, void* ws, int32_t* dev_status, cudaStream_t s, int* launches_io,
+                        const moe::FusedRoute* route) {
   const int bm = block_m;
   const int64_t P_max = moe_max_padded(T, k, E, bm);
   const int64_t P_total = padded_total(T, k, E, bm, n_shared);
@@ -341,8 +335,7 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
   const int n1 = act == MOE_ACT_SWIGLU ? 2 * F : F;
   const int num_sms = num_sms_current_device();
   if (num_sms <= 0) return MOE_ERR_CUDA;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  int launches = 0;
+  int& launches = *launches_io;
   const int total_blocks_max = static_cast<int>(P_total / bm);
 
   if (moe::fused_expert_supported(bm)) {
@@ -382,10 +375,11 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
     const int epi = act == MOE_ACT_SWIGLU ? moe::kEpiSwiGLU : moe::kEpiRelu2;
     const int64_t tiles = moe::fused_expert_max_tiles(epi, total_blocks_max, F);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+    if (route != nullptr) fa.route = *route;
     cudaError_t err;
     {
       StageScope scope(6, s);
-      err = moe::launch_fused_expert(epi, bm, fa, grid < 1 ? 1 : grid, s);
+      err = moe::launch_fused_expert(epi, bm, route != nullptr, fa, grid < 1 ? 1 : grid, s);
     }
     if (err != cudaSuccess) return MOE_ERR_CUDA;
     ++launches;
@@ -487,6 +481,111 @@ moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, con
     err = moe::launch_convert(y, static_cast<int64_t>(T) * d, out, num_sms, s, &launches);
   }
   return finish(err, launches);
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, const uint16_t* w2, int E, int F,
+                       const uint16_t* w13_shared, const uint16_t* w2_shared, int n_shared,
+                       const float* topk_weights, int k, const int32_t* sorted_token_ids,
+                       const int32_t* expert_ids, const int32_t* num_tokens_post_padded, const int32_t* inv_pos,
+                       int block_m, moe_act act, uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
+                       moe_stream_t stream) {
+  moe_status st = check_dims(T, d, F, E, k);
+  if (st != MOE_OK) return st;
+  if (!valid_block_m(block_m)) return MOE_ERR_UNSUPPORTED;
+  if (act != MOE_ACT_SWIGLU && act != MOE_ACT_RELU2) return MOE_ERR_INVALID_ARG;
+  if (n_shared != 0 && n_shared != 1) return MOE_ERR_UNSUPPORTED;
+  if (n_shared && (!w13_shared || !w2_shared)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return finish(cudaSuccess, 0);
+  if (!x || !w13 || !w2 || !topk_weights || !sorted_token_ids || !expert_ids || !num_tokens_post_padded || !out)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w13) || !aligned16(w2) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (n_shared && (!aligned16(w13_shared) || !aligned16(w2_shared))) return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_workspace_size(T, d, F, E, k, block_m, act, n_shared);
+  if (ws == nullptr || ws_bytes < need) return MOE_ERR_WORKSPACE;
+
+  int launches = 0;
+  return forward_impl(x, T, d, w13, w2, E, F, w13_shared, w2_shared, n_shared, topk_weights, k, sorted_token_ids,
+                      expert_ids, num_tokens_post_padded, block_m, act, out, ws, dev_status,
+                      reinterpret_cast<cudaStream_t>(stream), &launches, nullptr);
+}
+
+moe_status moe_layer(const float* logits, int T, int E, int k, int n_group, int topk_group,
+                     moe_group_score group_score, int renormalize, float routed_scaling, const uint16_t* x, int d,
+                     const uint16_t* w13, const uint16_t* w2, int F, const uint16_t* w13_shared,
+                     const uint16_t* w2_shared, int n_shared, int block_m, moe_act act, int32_t* topk_ids,
+                     float* topk_weights, int32_t* sorted_token_ids, int32_t* expert_ids,
+                     int32_t* num_tokens_post_padded, int32_t* inv_pos, uint16_t* out, void* ws, size_t ws_bytes,
+                     int32_t* dev_status, moe_stream_t stream) {
+  moe_status st = check_route_args(T, E, k, n_group, topk_group, group_score, routed_scaling);
+  if (st != MOE_OK) return st;
+  st = check_dims(T, d, F, E, k);
+  if (st != MOE_OK) return st;
+  if (!valid_block_m(block_m)) return MOE_ERR_UNSUPPORTED;
+  if (act != MOE_ACT_SWIGLU && act != MOE_ACT_RELU2) return MOE_ERR_INVALID_ARG;
+  if (n_shared != 0 && n_shared != 1) return MOE_ERR_UNSUPPORTED;
+  if (n_shared && (!w13_shared || !w2_shared)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return finish(cudaSuccess, 0);
+  if (!logits || !x || !w13 || !w2 || !topk_ids || !topk_weights || !sorted_token_ids || !expert_ids ||
+      !num_tokens_post_padded || !inv_pos || !out)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w13) || !aligned16(w2) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (n_shared && (!aligned16(w13_shared) || !aligned16(w2_shared))) return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_workspace_size(T, d, F, E, k, block_m, act, n_shared);
+  if (ws == nullptr || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int launches = 0;
+  if (moe::fused_expert_supported(block_m) && moe::fused_routing_supported(T, k, E, n_group, block_m)) {
+    moe::FusedRoute r;
+    r.logits = logits;
+    r.n_group = n_group;
+    r.topk_group = topk_group;
+    r.group_score = static_cast<int>(group_score);
+    r.renormalize = renormalize ? 1 : 0;
+    r.routed_scaling = routed_scaling;
+    r.topk_ids = topk_ids;
+    r.topk_w = topk_weights;
+    r.sorted_ids = sorted_token_ids;
+    r.expert_ids = expert_ids;
+    r.ntpp = num_tokens_post_padded;
+    r.inv_pos = inv_pos;
+    r.P_max = static_cast<int>(moe_max_padded(T, k, E, block_m));
+    return forward_impl(x, T, d, w13, w2, E, F, w13_shared, w2_shared, n_shared, topk_weights, k, sorted_token_ids,
+                        expert_ids, num_tokens_post_padded, block_m, act, out, ws, dev_status, s, &launches, &r);
+  }
+  // separate launches: routing and align (fused when the batch is small),
+  // then the forward; the align scratch borrows the forward's accumulator
+  // region, which the forward only touches after the align has finished
+  const int P_max = static_cast<int>(moe_max_padded(T, k, E, block_m));
+  cudaError_t err;
+  if (moe::route_align_fusable(T, k, n_group)) {
+    StageScope scope(5, s);
+    err = moe::launch_route_align(logits, T, E, k, n_group, topk_group, static_cast<int>(group_score),
+                                  renormalize ? 1 : 0, routed_scaling, topk_ids, topk_weights, block_m, P_max,
+                                  sorted_token_ids, expert_ids, num_tokens_post_padded, inv_pos, dev_status, s,
+                                  &launches);
+  } else {
+    {
+      StageScope scope(0, s);
+      err = moe::launch_route(logits, T, E, k, n_group, topk_group, static_cast<int>(group_score),
+                              renormalize ? 1 : 0, routed_scaling, topk_ids, topk_weights, dev_status, s, &launches);
+    }
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    const size_t align_need = moe_align_workspace_size(T, k, E);
+    uint8_t* wsb = reinterpret_cast<uint8_t*>(round_up(reinterpret_cast<uintptr_t>(ws), kWsAlign));
+    const size_t acc_off = need - kWsAlign - round_up(static_cast<size_t>(T) * d * 4, kWsAlign);
+    if (align_need > round_up(static_cast<size_t>(T) * d * 4, kWsAlign)) return MOE_ERR_WORKSPACE;
+    StageScope scope(1, s);
+    err = moe::launch_align(topk_ids, T * k, E, block_m, P_max, sorted_token_ids, expert_ids,
+                            num_tokens_post_padded, inv_pos, reinterpret_cast<int32_t*>(wsb + acc_off), dev_status, s,
+                            &launches);
+  }
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  return forward_impl(x, T, d, w13, w2, E, F, w13_shared, w2_shared, n_shared, topk_weights, k, sorted_token_ids,
+                      expert_ids, num_tokens_post_padded, block_m, act, out, ws, dev_status, s, &launches, nullptr);
 }
 
 moe_status moe_read_status(const int32_t* dev_status, moe_stream_t stream) {

@@ -8,6 +8,22 @@
 
 namespace moe {
 
+// Routing done inside the fused kernel (small batches): every CTA routes all
+// tokens and sorts their slots in shared memory; CTA 0 also writes the
+// results to these outputs, which then equal moe_route + moe_align's.
+struct FusedRoute {
+  const float* logits;  // [T, E] fp32
+  int n_group, topk_group, group_score, renormalize;
+  float routed_scaling;
+  int32_t* topk_ids;    // [T, k] out
+  float* topk_w;        // [T, k] out
+  int32_t* sorted_ids;  // [P_max] out
+  int32_t* expert_ids;  // [P_max / block_m] out
+  int32_t* ntpp;        // [1] out
+  int32_t* inv_pos;     // [T * k] out
+  int P_max;
+};
+
 struct FusedArgs {
   CUtensorMap tm_w13;   // routed gate/up (or fc1) weights, 3-D {d, N1, E}; boxes of 64 x 64 rows
                         // (SwiGLU: 64 gate rows, then the matching 64 up rows) or 64 x 128 (relu^2)
@@ -27,11 +43,15 @@ struct FusedArgs {
   int block_m;
   int max_routed_blocks;
   int n_shared_blocks;
+  FusedRoute route;     // used by the launch with in-kernel routing only
 };
 
 bool fused_expert_supported(int block_m);
+// In-kernel routing covers block_m = 16, T*k <= 256, n_group <= 64.
+bool fused_routing_supported(int T, int k, int E, int n_group, int block_m);
 // Upper bound on the fused kernel's tiles, for grid sizing.
 int64_t fused_expert_max_tiles(int act_epi, int total_blocks_max, int F);
-cudaError_t launch_fused_expert(int act_epi, int block_m, const FusedArgs& args, int grid, cudaStream_t stream);
+cudaError_t launch_fused_expert(int act_epi, int block_m, bool route, const FusedArgs& args, int grid,
+                                cudaStream_t stream);
 
 }  // namespace moe

@@ -46,16 +46,23 @@
 // two gate/up accumulators of block_m columns, then a ring of down-GEMM
 // accumulators (groups of 64 columns).  Every wait is bounded in time; on expiry the kernel records
 // MOE_ERR_DEVICE_TIMEOUT and all roles leave.
+#include "align_impl.cuh"
 #include "common.cuh"
 #include "fused.h"
 #include "gemm.h"
 #include "ptx.cuh"
+#include "route_impl.cuh"
 
 namespace moe {
 
 namespace {
 
-template <int EPI1, int TOK>
+// In-kernel routing limits (block_m = 16 only): T*k <= 256 slots, hence
+// P_max <= 256 + 256 * 15 = 4096 padded rows.
+constexpr int kRouteMaxS = 256;
+constexpr int kRouteMaxP = 4096;
+
+template <int EPI1, int TOK, bool ROUTE>
 struct FusedCfg {
   static constexpr bool kGated = (EPI1 == kEpiSwiGLU);
   static constexpr int kH = kGated ? 64 : 128;  // h columns per tile
@@ -67,7 +74,10 @@ struct FusedCfg {
   static constexpr int kXbufBytes = kGated ? 64 * TOK * 4 : 0;  // up half handed to the gate half
   static constexpr int kTokBytes = 2 * 2 * 64 * 4;              // token id and weight per row, two tiles
   static constexpr int kBarrierBytes = 1024;
-  static constexpr int kFixedBytes = 2 * kHBufBytes + kXbufBytes + kTokBytes + kBarrierBytes + 1024;
+  // routing results kept for the whole kernel: padded rows, block experts,
+  // slot weights, slot ids, inverse positions, padded total
+  static constexpr int kRouteBytes = ROUTE ? (kRouteMaxP + kRouteMaxP / 16 + 3 * kRouteMaxS + 8) * 4 : 0;
+  static constexpr int kFixedBytes = 2 * kHBufBytes + kXbufBytes + kTokBytes + kBarrierBytes + kRouteBytes + 1024;
   static constexpr int kStagesRaw = (227 * 1024 - kFixedBytes) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
   // Down-GEMM accumulators: groups of kGroup d tiles (64 TMEM columns) form
@@ -156,10 +166,10 @@ __device__ __forceinline__ bool spin_until(const int32_t* p, int target, volatil
   return true;
 }
 
-template <int EPI1, int TOK>
-__global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
+template <int EPI1, int TOK, bool ROUTE>
+__global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
     fused_expert_kernel(const __grid_constant__ FusedArgs args) {
-  using C = FusedCfg<EPI1, TOK>;
+  using C = FusedCfg<EPI1, TOK, ROUTE>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* hbuf = smem + C::kStages * C::kStageBytes;                // [2][kHk][TOK rows x 128 B]
@@ -219,7 +229,59 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
 
   pdl_wait();
   pdl_launch_dependents();
-  int routed_blocks = *args.ntpp / args.block_m;
+  const int32_t* sorted_ids = args.sorted_ids;
+  const int32_t* expert_ids = args.expert_ids;
+  const float* topk_w = args.topk_w;
+  int ntpp_v;
+  if constexpr (ROUTE) {
+    // ---- routing and align of all tokens, redundantly in every CTA, before
+    // any weight streams.  Results live after the barriers; the per-warp
+    // group scratch and the counting-sort scratch borrow the stage ring,
+    // which is idle until the producer starts.
+    int* r_sorted = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::kBarrierBytes);
+    int* r_eid = r_sorted + kRouteMaxP;
+    float* r_w = reinterpret_cast<float*>(r_eid + kRouteMaxP / 16);
+    int* r_ids = reinterpret_cast<int*>(r_w + kRouteMaxS);
+    int* r_inv = r_ids + kRouteMaxS;
+    int* r_ntpp = r_inv + kRouteMaxS;
+    constexpr int kWarps = C::kNumThreads / kWarp;
+    float* gscore = reinterpret_cast<float*>(smem);  // [kWarps][64]
+    unsigned char* gkeep = reinterpret_cast<unsigned char*>(gscore + kWarps * 64);  // [kWarps][64]
+    int* cnt = reinterpret_cast<int*>(smem + 8192);
+    int* off = cnt + MOE_MAX_EXPERTS;
+    int* run = off + MOE_MAX_EXPERTS + 1;
+    int* tot = run + MOE_MAX_EXPERTS;
+    int(*wcnt)[MOE_MAX_EXPERTS] = reinterpret_cast<int(*)[MOE_MAX_EXPERTS]>(tot + MOE_MAX_EXPERTS + 3);
+    const FusedRoute& R = args.route;
+    for (int t = warp; t < args.T; t += kWarps)
+      route_one_token<8>(R.logits + static_cast<size_t>(t) * args.E, args.E, args.k, R.n_group, R.topk_group,
+                         R.group_score, R.renormalize, R.routed_scaling, gscore + warp * 64, gkeep + warp * 64,
+                         r_ids + t * args.k, r_w + t * args.k, args.status, lane);
+    for (int i = threadIdx.x; i < kWarps * MOE_MAX_EXPERTS; i += C::kNumThreads) (&wcnt[0][0])[i] = 0;
+    __syncthreads();
+    auto get_expert = [&](int s, bool) { return r_ids[s]; };
+    align_detail::align_one_block<kWarps>(get_expert, args.S, args.E, args.block_m, R.P_max, r_sorted, r_eid, r_ntpp,
+                                          r_inv, cnt, off, run, tot, wcnt);
+    __syncthreads();
+    if (blockIdx.x == 0) {  // the same results as the separate routing and align calls
+      for (int i = threadIdx.x; i < args.S; i += C::kNumThreads) {
+        R.topk_ids[i] = r_ids[i];
+        R.topk_w[i] = r_w[i];
+        R.inv_pos[i] = r_inv[i];
+      }
+      for (int i = threadIdx.x; i < R.P_max; i += C::kNumThreads) R.sorted_ids[i] = r_sorted[i];
+      for (int i = threadIdx.x; i < R.P_max / args.block_m; i += C::kNumThreads) R.expert_ids[i] = r_eid[i];
+      if (threadIdx.x == 0) *R.ntpp = *r_ntpp;
+    }
+    sorted_ids = r_sorted;
+    expert_ids = r_eid;
+    topk_w = r_w;
+    ntpp_v = *r_ntpp;
+    __syncthreads();  // the scratch on the stage ring is free again
+  } else {
+    ntpp_v = *args.ntpp;
+  }
+  int routed_blocks = ntpp_v / args.block_m;
   if (routed_blocks < 0) routed_blocks = 0;
   if (routed_blocks > args.max_routed_blocks) routed_blocks = args.max_routed_blocks;
   const int total_blocks = routed_blocks + args.n_shared_blocks;
@@ -252,7 +314,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
       bool ok = true;
       auto expert_of = [&](const TileInfo& t) {
         if (t.shared_blk) return 0;
-        const int e = args.expert_ids[t.blk];
+        const int e = expert_ids[t.blk];
         if (e < 0 || e >= args.E) set_status(args.status, MOE_ERR_BAD_EXPERT_ID);  // TMA fills zeros
         return e;
       };
@@ -408,10 +470,10 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
           int tok = -1;
           float wj = 0.0f;
           if (!t.shared_blk) {
-            const int slot = args.sorted_ids[t.blk * args.block_m + j];
+            const int slot = sorted_ids[t.blk * args.block_m + j];
             if (static_cast<unsigned>(slot) < static_cast<unsigned>(args.S)) {
               tok = slot / args.k;
-              wj = args.topk_w[slot];
+              wj = topk_w[slot];
             }
           } else {
             const int tk = (t.blk - routed_blocks) * args.block_m + j;
@@ -599,7 +661,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
           int tok = 0;
           bool valid;
           if (!t.shared_blk) {
-            const int slot = args.sorted_ids[t.blk * args.block_m + row];
+            const int slot = sorted_ids[t.blk * args.block_m + row];
             valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
             if (valid) tok = slot / args.k;
           } else {
@@ -675,10 +737,10 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK>::kNumThreads, 1)
   }
 }
 
-template <int EPI1, int TOK>
+template <int EPI1, int TOK, bool ROUTE>
 cudaError_t launch_fused_variant(const FusedArgs& args, int grid, cudaStream_t stream) {
-  using C = FusedCfg<EPI1, TOK>;
-  auto kern = fused_expert_kernel<EPI1, TOK>;
+  using C = FusedCfg<EPI1, TOK, ROUTE>;
+  auto kern = fused_expert_kernel<EPI1, TOK, ROUTE>;
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -701,18 +763,28 @@ int64_t fused_expert_max_tiles(int act_epi, int total_blocks_max, int F) {
   return static_cast<int64_t>(total_blocks_max) * ((F + h - 1) / h);
 }
 
-cudaError_t launch_fused_expert(int act_epi, int block_m, const FusedArgs& args, int grid, cudaStream_t stream) {
+bool fused_routing_supported(int T, int k, int E, int n_group, int block_m) {
+  return block_m == 16 && static_cast<int64_t>(T) * k <= kRouteMaxS && E <= MOE_MAX_EXPERTS && n_group <= 64;
+}
+
+cudaError_t launch_fused_expert(int act_epi, int block_m, bool route, const FusedArgs& args, int grid,
+                                cudaStream_t stream) {
   const bool gated = act_epi == kEpiSwiGLU;
+  if (route) {
+    if (block_m != 16) return cudaErrorInvalidValue;
+    return gated ? launch_fused_variant<kEpiSwiGLU, 16, true>(args, grid, stream)
+                 : launch_fused_variant<kEpiRelu2, 16, true>(args, grid, stream);
+  }
   switch (block_m) {
     case 16:
-      return gated ? launch_fused_variant<kEpiSwiGLU, 16>(args, grid, stream)
-                   : launch_fused_variant<kEpiRelu2, 16>(args, grid, stream);
+      return gated ? launch_fused_variant<kEpiSwiGLU, 16, false>(args, grid, stream)
+                   : launch_fused_variant<kEpiRelu2, 16, false>(args, grid, stream);
     case 32:
-      return gated ? launch_fused_variant<kEpiSwiGLU, 32>(args, grid, stream)
-                   : launch_fused_variant<kEpiRelu2, 32>(args, grid, stream);
+      return gated ? launch_fused_variant<kEpiSwiGLU, 32, false>(args, grid, stream)
+                   : launch_fused_variant<kEpiRelu2, 32, false>(args, grid, stream);
     case 64:
-      return gated ? launch_fused_variant<kEpiSwiGLU, 64>(args, grid, stream)
-                   : launch_fused_variant<kEpiRelu2, 64>(args, grid, stream);
+      return gated ? launch_fused_variant<kEpiSwiGLU, 64, false>(args, grid, stream)
+                   : launch_fused_variant<kEpiRelu2, 64, false>(args, grid, stream);
     default:
       return cudaErrorInvalidValue;
   }

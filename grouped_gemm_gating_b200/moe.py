@@ -43,6 +43,8 @@ _SIG = {
                              ctypes.c_size_t, _P, _P]),
     "moe_forward": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _P, _I, _P, _I, _P, _P, _P, _P, _I, _I,
                          _P, _P, ctypes.c_size_t, _P, _P]),
+    "moe_layer": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _I, _P, _P, _I, _P, _P, _I, _I, _I,
+                       _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
     "moe_read_status": (_I, [_P, _P]),
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_last_launch_count": (_I, []),
@@ -230,6 +232,25 @@ def moe_forward(x, w13, w2, topk_weights, sorted_token_ids, expert_ids, num_toke
     _check("moe_forward", code)
 
 
+def moe_layer(logits, x, w13, w2, k, block_m, act, topk_ids, topk_weights, sorted_token_ids, expert_ids,
+              num_tokens_post_padded, inv_pos, out, ws, w13_shared=None, w2_shared=None, n_group=1, topk_group=1,
+              group_score=GROUP_MAX, renormalize=True, routed_scaling=1.0, dev_status=None):
+    """Route, align and forward in one call (one kernel for decode batches)."""
+    T, E = logits.shape
+    d = x.shape[1]
+    F = w2.shape[2]
+    if logits.dtype != torch.float32 or topk_weights.dtype != torch.float32:
+        raise ValueError("moe_layer: logits/weights fp32")
+    n_shared = 0 if w13_shared is None else 1
+    code = load_library().moe_layer(
+        _ptr(logits), T, E, k, n_group, topk_group, group_score, 1 if renormalize else 0, float(routed_scaling),
+        _ptr(_bits(x)), d, _ptr(_bits(w13)), _ptr(_bits(w2)), F, _ptr(_bits(w13_shared)), _ptr(_bits(w2_shared)),
+        n_shared, block_m, act, _ptr(topk_ids), _ptr(topk_weights), _ptr(sorted_token_ids), _ptr(expert_ids),
+        _ptr(num_tokens_post_padded), _ptr(inv_pos), _ptr(_bits(out)), _ptr(ws), ws.numel() * ws.element_size(),
+        _ptr(dev_status), _stream(x.device))
+    _check("moe_layer", code)
+
+
 def moe_read_status(dev_status) -> int:
     """Synchronise the current stream and return the device status code."""
     return int(load_library().moe_read_status(_ptr(dev_status), _stream(dev_status.device)))
@@ -288,6 +309,13 @@ class MoEBuffers:
         moe_route_align(logits, self.k, self.block_m, self.topk_ids, self.topk_weights, self.sorted_token_ids,
                         self.expert_ids, self.ntpp, self.inv_pos, self.align_ws, n_group, topk_group, group_score,
                         renormalize, routed_scaling, self.status)
+
+    def layer(self, logits, x, w13, w2, w13_shared=None, w2_shared=None, n_group=1, topk_group=1,
+              group_score=GROUP_MAX, renormalize=True, routed_scaling=1.0):
+        moe_layer(logits, x, w13, w2, self.k, self.block_m, self.act, self.topk_ids, self.topk_weights,
+                  self.sorted_token_ids, self.expert_ids, self.ntpp, self.inv_pos, self.out, self.ws, w13_shared,
+                  w2_shared, n_group, topk_group, group_score, renormalize, routed_scaling, self.status)
+        return self.out
 
     def forward(self, x, w13, w2, w13_shared=None, w2_shared=None):
         moe_forward(x, w13, w2, self.topk_weights, self.sorted_token_ids, self.expert_ids, self.ntpp,

@@ -240,6 +240,36 @@ MOE_API moe_status moe_route_align(const float* logits, int T, int E, int k,
                            void* ws, size_t ws_bytes,
                            int32_t* dev_status, moe_stream_t stream);
 
+/*
+ * moe_layer — the whole layer in one call: moe_route, moe_align and
+ * moe_forward on the same arguments, with the same outputs (topk_ids,
+ * topk_weights, sorted_token_ids, expert_ids, num_tokens_post_padded and
+ * inv_pos are written as by moe_route_align; out as by moe_forward) and the
+ * same errors.  No passage of the source pages has this entry point: it is
+ * the three calls of "Token-Expert Routing" and "Grouped GEMM Structure"
+ * chained, for callers that hold only the router logits.  With block_m = 16,
+ * T*k <= 256 and n_group <= 64 (decode / verifier batches) it is one kernel
+ * launch: every CTA of the fused expert kernel routes and sorts all tokens
+ * in shared memory before streaming weights, and one CTA also writes the
+ * routing and align outputs.  Otherwise the routing / align kernels and the
+ * forward kernels run back to back.
+ *   ws, ws_bytes  scratch of moe_workspace_size(T, d, F, E, k, block_m, act,
+ *                 n_shared) bytes (its counter block zero, as for
+ *                 moe_forward); the align scratch, when one is needed, is
+ *                 carved from it.
+ */
+MOE_API moe_status moe_layer(const float* logits, int T, int E, int k,
+                     int n_group, int topk_group, moe_group_score group_score,
+                     int renormalize, float routed_scaling,
+                     const uint16_t* x, int d, const uint16_t* w13, const uint16_t* w2, int F,
+                     const uint16_t* w13_shared, const uint16_t* w2_shared, int n_shared,
+                     int block_m, moe_act act,
+                     int32_t* topk_ids, float* topk_weights,
+                     int32_t* sorted_token_ids, int32_t* expert_ids,
+                     int32_t* num_tokens_post_padded, int32_t* inv_pos,
+                     uint16_t* out, void* ws, size_t ws_bytes,
+                     int32_t* dev_status, moe_stream_t stream);
+
 /* Synchronises `stream`, then returns the code stored in dev_status (MOE_OK
  * when 0), or MOE_ERR_CUDA if the synchronisation or the copy failed. */
 MOE_API moe_status moe_read_status(const int32_t* dev_status, moe_stream_t stream);
@@ -256,10 +286,11 @@ MOE_API int moe_last_launch_count(void);
  * around each of its kernels (events come from a pool the library owns; the
  * calls may be captured into a CUDA graph, where the records become event
  * nodes that are re-recorded at every replay).
- * Stages: 0 route, 1 align, 2 gate/up (fc1) GEMM, 3 down GEMM, 4 combine,
- * 5 fused route+align (moe_route_align on a small batch), 6 fused expert
- * kernel (moe_forward with block_m <= 64: both GEMMs, and the combine when
- * T*k <= 64 without a shared expert).
+ * Stages: 0 route, 1 align, 2 gate/up (fc1) GEMM, 3 down GEMM, 4 combine
+ * (the accumulator's conversion to bf16), 5 fused route+align
+ * (moe_route_align on a small batch), 6 fused expert kernel (moe_forward
+ * with block_m <= 64: both GEMMs and the scatter-reduce; under moe_layer on
+ * a small batch also the routing and align).
  * moe_profile_enable(1) starts a fresh record (and primes the event pool),
  * (0) stops recording and keeps what was recorded.  moe_profile_collect waits for the recorded events,
  * writes into stage_ms[i] (i < n_stages) the summed milliseconds of stage i

@@ -115,6 +115,30 @@ def test_forward_host_checks(lib):
     assert f(*args(T=0, x=NULL)) == 0          # T == 0: no-op
 
 
+def test_layer_host_checks(lib):
+    f = lib.moe_layer
+    p = ctypes.c_void_p(256)
+    odd = ctypes.c_void_p(258)
+
+    def args(**kw):
+        return [kw.get("logits", p), kw.get("T", 4), kw.get("E", 8), kw.get("k", 2), kw.get("ng", 1), kw.get("tg", 1),
+                0, 1, kw.get("scale", 1.0), kw.get("x", p), kw.get("d", 128), p, p, kw.get("F", 128), NULL, NULL,
+                kw.get("ns", 0), kw.get("bm", 16), kw.get("act", 0), p, p, p, p, p, kw.get("inv", p), p,
+                kw.get("ws", p), kw.get("wsb", 1 << 40), NULL, NULL]
+    assert f(*args(k=9)) == 1                  # k > E
+    assert f(*args(ng=3)) == 1                 # E % n_group
+    assert f(*args(scale=0.0)) == 1            # routed_scaling <= 0
+    assert f(*args(d=96)) == 2                 # d % 64
+    assert f(*args(bm=8)) == 2                 # block_m
+    assert f(*args(act=3)) == 1                # activation
+    assert f(*args(ns=1)) == 1                 # shared expert weights missing
+    assert f(*args(x=odd)) == 1                # misaligned
+    assert f(*args(logits=NULL)) == 1          # null logits
+    assert f(*args(inv=NULL)) == 1             # inv_pos is an output here
+    assert f(*args(wsb=16)) == 3               # workspace too small
+    assert f(*args(T=0, x=NULL, logits=NULL)) == 0  # T == 0: no-op
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(M, "_lib", None)
     monkeypatch.setattr(M, "library_path", lambda: str(tmp_path / "nope.so"))

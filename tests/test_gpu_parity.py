@@ -318,6 +318,60 @@ def test_route_align_matches_separate_calls(name, T):
     compare_route(b.buf.topk_ids.cpu().numpy(), b.buf.topk_weights.cpu().numpy(), ids, w, name)
 
 
+@pytest.mark.parametrize("name,one_launch", [("decode", True), ("tiny", True), ("shared_bm16_fused_combine", True),
+                                             ("decode_d512", True), ("relu2_small", False), ("dsv3_small", False),
+                                             ("swap_bm32", False)])
+def test_layer_entry_matches_separate_calls(name, one_launch):
+    """moe_layer writes the same routing / align outputs as moe_route_align
+    (bit for bit) and the same output as moe_forward (up to the reordering
+    of fp32 sums); small decode batches take one launch."""
+    cfg = SMALL[name]
+    inp = W.make_inputs(cfg)
+    a = DeviceLayer(inp)
+    b = DeviceLayer(inp)
+    ref_out = M_bits(a.run(fused_route_align=True)).copy()
+    rk = route_kwargs(cfg)
+    b.buf.layer(b.logits, b.x, b.w13, b.w2, b.w13s, b.w2s, **rk)
+    torch.cuda.synchronize()
+    if one_launch:
+        assert M.moe_last_launch_count() == 1
+    assert b.status() == 0, M.status_name(b.status())
+    S = cfg.T * cfg.k
+    for attr in ("topk_ids", "topk_weights", "sorted_token_ids", "expert_ids", "ntpp"):
+        x, y = getattr(a.buf, attr), getattr(b.buf, attr)
+        assert torch.equal(x.view(torch.int32), y.view(torch.int32)), attr
+    assert torch.equal(a.buf.inv_pos[:S], b.buf.inv_pos[:S])
+    got = M_bits(b.buf.out).copy()
+    assert_within_ulp(got, ref_out, 1, name)
+    ids, w = oracle_route(inp)
+    ref = oracle.forward(inp.x, inp.w13, inp.w2, ids, w, cfg.act, inp.w13_shared, inp.w2_shared)
+    compare_out(got, ref, name + " (moe_layer)")
+
+
+def test_layer_entry_graph_replay():
+    """The one-launch layer captures into a CUDA graph and replays on new
+    logits and activations."""
+    cfg = SMALL["decode_d512"]
+    inp = W.make_inputs(cfg)
+    lay = DeviceLayer(inp)
+    lay.buf.layer(lay.logits, lay.x, lay.w13, lay.w2)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        lay.buf.layer(lay.logits, lay.x, lay.w13, lay.w2)
+    inp2 = W.make_inputs(cfg.with_(seed=cfg.seed + 7))
+    lay.x.copy_(torch.from_numpy(inp2.x.view(np.int16)).cuda().view(torch.bfloat16))
+    lay.logits.copy_(torch.from_numpy(inp2.logits).cuda())
+    g.replay()
+    torch.cuda.synchronize()
+    assert lay.status() == 0
+    ids, w = oracle_route(inp2)
+    compare_route(lay.buf.topk_ids.cpu().numpy(), lay.buf.topk_weights.cpu().numpy(), ids, w, "layer replay")
+    compare_align(lay.buf, oracle.align(ids, cfg.E, cfg.block_m), "layer replay")
+    ref = oracle.forward(inp2.x, inp.w13, inp.w2, ids, w, cfg.act)
+    compare_out(M_bits(lay.buf.out), ref, "layer replay")
+
+
 def test_fused_counters_return_to_zero_and_workspace_is_shareable():
     """The fused kernel's counter block is zero after every call, so one
     workspace serves calls of different shapes in turn."""
