@@ -431,7 +431,11 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
   // down GEMM whose epilogue adds topk_weight * row into acc [T, d] fp32
   moe::GemmArgs a2;
   std::memset(&a2, 0, sizeof(a2));
-  const uint32_t box2 = static_cast<uint32_t>(moe::gemm_box_rows(moe::kEpiScale));
+  // CTA pairs share each 256-row W2 tile (128 rows per CTA).  Worth it when
+  // the K loop is long (d_ff >= 1024); with a short one the epilogue's
+  // reductions bound the kernel and unpaired blocks would only add work.
+  const bool pair2 = F >= 1024 && moe::down_gemm_pair_supported(bm, total_blocks_max);
+  const uint32_t box2 = pair2 ? 128u : static_cast<uint32_t>(moe::gemm_box_rows(moe::kEpiScale));
   if (!encode_3d(&a2.tm_w, w2, F, d, E, box2)) return MOE_ERR_CUDA;
   if (n_shared) {
     if (!encode_3d(&a2.tm_ws, w2_shared, F, d, 1, box2)) return MOE_ERR_CUDA;
@@ -462,7 +466,7 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
     // column passes: keep each pass's slice of the accumulator within ~48 MB of L2
     const int64_t acc_bytes = static_cast<int64_t>(T) * d * 4;
     const int64_t budget = int64_t(48) << 20;
-    const int n_wt = (d + static_cast<int>(box2) - 1) / static_cast<int>(box2);
+    const int n_wt = (d + 255) / 256;
     const int passes = static_cast<int>((acc_bytes + budget - 1) / budget);
     a2.pass_cols = passes <= 1 ? 0 : (n_wt + passes - 1) / passes;
   }
@@ -471,7 +475,10 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
   if (grid < 1) grid = 1;
   {
     StageScope scope(3, s);
-    err = moe::launch_grouped_gemm(moe::kEpiScale, a2, grid, s);
+    if (pair2)
+      err = moe::launch_down_gemm_pair(a2, num_sms & ~1, s);
+    else
+      err = moe::launch_grouped_gemm(moe::kEpiScale, a2, grid, s);
   }
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   ++launches;

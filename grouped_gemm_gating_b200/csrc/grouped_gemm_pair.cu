@@ -1,0 +1,361 @@
+// Down GEMM of the token-major path on CTA pairs (tcgen05 cta_group::2).
+//
+// Same computation as the down GEMM of grouped_gemm.cu -- the "Grouped GEMM
+// Structure" of the fused-moe-kernel page ("Fused MoE Kernel Optimization",
+// skillmd zjli2013) with the top-k weight of each row applied and the result
+// added into the fp32 [T, d] accumulator at the row's token ("Common
+// Pitfalls" 4; the weighted sum of the axolotl `_moe_triton_forward`,
+// src/axolotl/monkeypatch/deepseek_v3/__init__.py) -- with a 256 x 256 tile
+// per pair of SMs instead of 128 x 256 per SM.
+//
+// A cluster of two CTAs works on a "pair unit": two consecutive 128-row
+// blocks of the same expert (the last block of an expert with an odd count
+// is paired with nothing; the odd CTA then computes rows it discards).  Each
+// CTA loads its own block's h rows (A) and half of the 256 W2 rows of the
+// tile (B) by TMA; the transaction bytes of both CTAs complete on the even
+// CTA's full barrier, where its single MMA thread issues M = 256, N = 256
+// MMAs that read A and B from both CTAs' shared memory.  Commits go to both
+// CTAs (empty stages, full accumulators).  Each CTA's epilogue drains its own
+// TMEM half (its 128 rows) and signals the even CTA that the accumulator is
+// free.  Per SM and 64-wide K step the pair moves 32 KB of operands instead
+// of 48 KB, so the same shared memory holds six stages instead of four.
+//
+// Every mbarrier wait is bounded; on expiry the CTA records
+// MOE_ERR_DEVICE_TIMEOUT and its roles leave their loops.  Both CTAs always
+// reach the closing cluster barrier, which orders the peer's last remote
+// arrivals before either CTA frees its TMEM and exits.
+#include "common.cuh"
+#include "gemm.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+struct PairCfg {
+  static constexpr int kABytes = 128 * 128;  // 128 h rows x 64 bf16
+  static constexpr int kBBytes = 128 * 128;  // 128 W2 rows x 64 bf16 (this CTA's half of N = 256)
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = 6;
+  static constexpr int kAccCols = 256;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kNumThreads = 192;  // producer, MMA, 4 epilogue warps
+  static constexpr int kBarrierBytes = 256;
+  static constexpr int kRedStride = 33;
+  static constexpr int kRedBytes = 4 * 32 * kRedStride * 4;
+  static constexpr int kMaxUnits = 2048;  // pair units of one launch
+  static constexpr int kUnitBytes = kMaxUnits * 4;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + kRedBytes + kUnitBytes + 1024;
+  static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(256, 256);
+  static_assert((2 * kStages + 4) * 8 + 8 <= kBarrierBytes, "barrier area");
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+};
+
+__device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
+struct PairTile {
+  int b0;      // first block of the unit
+  int nb;      // blocks in the unit (1 or 2)
+  int wt;      // 256-wide output column tile
+  bool shared_blk;
+};
+
+__global__ void __launch_bounds__(PairCfg::kNumThreads, 1)
+    down_gemm_pair_kernel(const __grid_constant__ GemmArgs args) {
+  using C = PairCfg;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  float* red_buf = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + C::kBarrierBytes);
+  int* unit_b0 = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(red_buf) + C::kRedBytes);
+
+  const int warp = threadIdx.x / kWarp;
+  const int lane = threadIdx.x % kWarp;
+  const uint32_t rank = ptx::cluster_ctarank();  // 0: issues the pair's MMAs
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      ptx::mbar_init(&full[s], 1);   // even CTA: its producer's arrive + both CTAs' bytes
+      ptx::mbar_init(&empty[s], 1);  // one commit of the pair's MMA
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&tfull[b], 1);
+      ptx::mbar_init(&tempty[b], 8);  // even CTA: four epilogue warps of each CTA
+    }
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&args.tm_w);
+    if (args.n_shared_blocks) ptx::prefetch_tmap(&args.tm_ws);
+    ptx::prefetch_tmap(&args.tm_x);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(tmem_holder, C::kTmemCols);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // both CTAs' barriers exist before any remote arrival
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  pdl_wait();
+  pdl_launch_dependents();
+  int routed_blocks = *args.ntpp / args.block_m;
+  if (routed_blocks < 0) routed_blocks = 0;
+  if (routed_blocks > args.max_routed_blocks) routed_blocks = args.max_routed_blocks;
+  const int total_blocks = routed_blocks + args.n_shared_blocks;
+
+  // ---- pair units: a unit starts at the first block of an expert's run and
+  // at every second block after it (the shared expert's blocks are one run)
+  if (warp == 0) {
+    int seg_start = 0, n_units = 0, prev_e = -2;
+    for (int base = 0; base < total_blocks; base += kWarp) {
+      const int b = base + lane;
+      int e = -3;
+      if (b < total_blocks) e = b < routed_blocks ? args.expert_ids[b] : -1;
+      const int pe = __shfl_up_sync(0xffffffffu, e, 1);
+      const int left = lane == 0 ? prev_e : pe;
+      const bool new_seg = b < total_blocks && (b == 0 || e != left);
+      const unsigned segs = __ballot_sync(0xffffffffu, new_seg);
+      const unsigned upto = segs & (0xffffffffu >> (31 - lane));
+      const int my_seg = upto ? base + (31 - __clz(upto)) : seg_start;
+      const bool start = b < total_blocks && ((b - my_seg) & 1) == 0;
+      const unsigned starts = __ballot_sync(0xffffffffu, start);
+      const int idx = n_units + __popc(starts & ((1u << lane) - 1u));
+      if (start && idx < C::kMaxUnits) unit_b0[idx] = b;
+      n_units += __popc(starts);
+      seg_start = __shfl_sync(0xffffffffu, my_seg, 31);
+      prev_e = __shfl_sync(0xffffffffu, e, 31);
+    }
+    if (lane == 0) tmem_holder[2] = static_cast<uint32_t>(n_units < C::kMaxUnits ? n_units : C::kMaxUnits);
+  }
+  __syncthreads();
+  const int n_units = static_cast<int>(tmem_holder[2]);
+  const int n_wt = (args.n_out + 255) / 256;
+  const int pass_w = args.pass_cols > 0 && args.pass_cols < n_wt ? args.pass_cols : n_wt;
+  const int total_tiles = n_units * n_wt;
+  const int nk = args.K / 64;
+
+  auto tile_of = [&](int tile) {
+    const int per_pass = n_units * pass_w;
+    const int ps = tile / per_pass;
+    const int w0 = ps * pass_w;
+    const int width = n_wt - w0 < pass_w ? n_wt - w0 : pass_w;
+    const int r = tile - ps * per_pass;
+    const int u = r / width;
+    PairTile t;
+    t.b0 = unit_b0[u];
+    const int next = u + 1 < n_units ? unit_b0[u + 1] : total_blocks;
+    t.nb = next - t.b0 >= 2 ? 2 : 1;
+    t.wt = w0 + (r - u * width);
+    t.shared_blk = t.b0 >= routed_blocks;
+    return t;
+  };
+  auto fail = [&]() {
+    *abort_flag = 1;
+    set_status(args.status, MOE_ERR_DEVICE_TIMEOUT);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+        const PairTile t = tile_of(tile);
+        const CUtensorMap* tm = t.shared_blk ? &args.tm_ws : &args.tm_w;
+        int e = 0;
+        if (!t.shared_blk) {
+          e = args.expert_ids[t.b0];
+          if (e < 0 || e >= args.E) set_status(args.status, MOE_ERR_BAD_EXPERT_ID);
+        }
+        // this CTA's block (the odd CTA of a one-block unit loads the even
+        // CTA's rows again and discards its result)
+        const int blk = t.b0 + (static_cast<int>(rank) < t.nb ? static_cast<int>(rank) : 0);
+        const int wrow = t.wt * 256 + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait_cluster_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+            fail();
+            ok = false;
+            break;
+          }
+          uint8_t* sA = smem + stage * C::kStageBytes;
+          if (rank == 0) ptx::mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
+          ptx::tma_load_2d_pair(sA, &args.tm_x, &full[stage], kb * 64, blk * args.block_m);
+          ptx::tma_load_3d_pair(sA + C::kABytes, tm, &full[stage], kb * 64, wrow, e);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int abuf = 0;
+      uint32_t aphase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+        if (!ptx::mbar_wait_cluster_bounded(&tempty[abuf], aphase ^ 1u, abort_flag, kWaitLimitNs)) {
+          fail();
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * C::kAccCols);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait_cluster_bounded(&full[stage], phase, abort_flag, kWaitLimitNs)) {
+            fail();
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sA = ptx::smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t sB = sA + C::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::mma_bf16_pair(d_tmem, ptx::sw128_kmajor_desc(sA + kk * 32), ptx::sw128_kmajor_desc(sB + kk * 32),
+                               C::kIdesc, (kb | kk) != 0 ? 1u : 0u);
+          ptx::mma_commit_pair(&empty[stage]);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        ptx::mma_commit_pair(&tfull[abuf]);
+        if (++abuf == 2) {
+          abuf = 0;
+          aphase ^= 1u;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (both CTAs, own TMEM half)
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    float* stg = red_buf + q * 32 * C::kRedStride;
+    const int rr = lane >> 3;
+    const int cc = (lane & 7) * 4;
+    int abuf = 0;
+    uint32_t aphase = 0;
+    for (int tile = pair; tile < total_tiles; tile += n_pairs) {
+      const PairTile t = tile_of(tile);
+      if (!ptx::mbar_wait_cluster_bounded(&tfull[abuf], aphase, abort_flag, kWaitLimitNs)) {
+        fail();
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t t_acc =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(abuf * C::kAccCols);
+      if (static_cast<int>(rank) < t.nb) {
+        const int blk = t.b0 + static_cast<int>(rank);
+        const int p = blk * args.block_m + row;
+        bool valid;
+        int tok;
+        float wrow = 1.0f;
+        if (blk < routed_blocks) {
+          const int slot = args.sorted_ids[p];
+          valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
+          tok = valid ? slot / args.k : 0;
+          if (valid) wrow = args.topk_w[slot];
+        } else {
+          tok = (blk - routed_blocks) * args.block_m + row;
+          valid = tok < args.T;
+        }
+#pragma unroll 1
+        for (int c0 = 0; c0 < 256; c0 += 32) {
+          uint32_t a[32];
+          ptx::tmem_ld16(t_acc + c0, *reinterpret_cast<uint32_t(*)[16]>(&a[0]));
+          ptx::tmem_ld16(t_acc + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&a[16]));
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) asm volatile("" : "+r"(a[j]));  // uses stay after the wait
+          const int col = t.wt * 256 + c0;
+          if (col >= args.n_out) break;  // uniform across the warp
+#pragma unroll
+          for (int j = 0; j < 32; ++j) stg[lane * C::kRedStride + j] = __uint_as_float(a[j]) * wrow;
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + rr;
+            const int tk = __shfl_sync(0xffffffffu, tok, r);
+            const int ok = __shfl_sync(0xffffffffu, valid ? 1 : 0, r);
+            const float* src = stg + r * C::kRedStride + cc;
+            if (ok)
+              red_add_v4_f32(args.acc + static_cast<size_t>(tk) * args.n_out + col + cc, src[0], src[1], src[2],
+                             src[3]);
+          }
+          __syncwarp();
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_leader(&tempty[abuf]);
+      if (++abuf == 2) {
+        abuf = 0;
+        aphase ^= 1u;
+      }
+    }
+  }
+
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // the peer's last arrivals and reads are done
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem_base, C::kTmemCols);
+  }
+}
+
+}  // namespace
+
+bool down_gemm_pair_supported(int block_m, int total_blocks_max) {
+  return block_m == 128 && total_blocks_max <= PairCfg::kMaxUnits;
+}
+
+cudaError_t launch_down_gemm_pair(const GemmArgs& args, int grid, cudaStream_t stream) {
+  using C = PairCfg;
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_done[dev]) {
+    err = cudaFuncSetAttribute(down_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (err != cudaSuccess) return err;
+    attr_done[dev] = true;
+  }
+  grid &= ~1;
+  if (grid < 2) grid = 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::kNumThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, down_gemm_pair_kernel, args);
+}
+
+}  // namespace moe
