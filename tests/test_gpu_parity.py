@@ -37,6 +37,11 @@ SMALL = {
                                      seed=2008),
     "one_expert_hot": CFG["tiny"].with_(name="one_expert_hot", T=700, d=128, F=128, E=4, k=1, block_m=128,
                                         seed=2009, logits_kind="decode_hot"),
+    # token-major GEMMs on CTA pairs (d, d_ff >= 1024), odd and even block
+    # runs per expert, a shared expert, and the relu^2 variant
+    "pair_dsv3": CFG["dsv3"].with_(name="pair_dsv3", T=600, d=1024, F=1024, seed=2012),
+    "pair_relu2": CFG["relu2"].with_(name="pair_relu2", T=400, d=1024, F=1088, E=6, k=2, block_m=128,
+                                     seed=2013),
     # fused expert kernel (block_m <= 64) with a shared expert
     "shared_bm16_fused_combine": CFG["dsv3"].with_(name="shared_bm16_fused_combine", T=40, d=256, F=192,
                                                    block_m=16, seed=2010),
