@@ -159,6 +159,17 @@ constexpr size_t kCounterInts = 16384;
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// The token-major GEMMs run on CTA pairs when the layer is wide enough for
+// the K loops to dominate a tile: d_ff >= 1024 for both GEMMs (and d >= 1024
+// for the gate/up GEMM, whose token rows are first copied into the
+// expert-sorted order so that it can read them by TMA).  With a narrow d_ff
+// the down GEMM's epilogue bounds it, blocks left unpaired only add work,
+// and the copy of x outgrows what the gathered rows cost from L2.
+bool uses_pair_gate_up(int block_m, int d, int F, int64_t P_total) {
+  return block_m == 128 && d >= 1024 && F >= 1024 &&
+         moe::gemm_pair_supported(block_m, static_cast<int>(P_total / block_m));
+}
+
 int64_t padded_total(int T, int k, int E, int bm, int n_shared) {
   const int64_t pmax = moe_max_padded(T, k, E, bm);
   if (pmax < 0) return -1;
@@ -236,7 +247,9 @@ size_t moe_workspace_size(int T, int d, int F, int E, int k, int block_m, moe_ac
   const int64_t P = padded_total(T, k, E, block_m, n_shared);
   const size_t h = block_m == 128 ? round_up(static_cast<size_t>(P) * F * 2, kWsAlign) : 0;
   const size_t acc = round_up(static_cast<size_t>(T) * d * 4, kWsAlign);
-  return kCounterInts * 4 + h + acc + kWsAlign;
+  // permuted x for the paired gate/up GEMM
+  const size_t xs = uses_pair_gate_up(block_m, d, F, P) ? round_up(static_cast<size_t>(P) * d * 2, kWsAlign) : 0;
+  return kCounterInts * 4 + h + acc + xs + kWsAlign;
 }
 
 moe_status moe_route(const float* logits, int T, int E, int k, int n_group, int topk_group,
@@ -332,6 +345,8 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
   uint16_t* h = reinterpret_cast<uint16_t*>(wsb + kCounterInts * 4);
   const size_t h_bytes = bm == 128 ? round_up(static_cast<size_t>(P_total) * F * 2, kWsAlign) : 0;
   float* y = reinterpret_cast<float*>(wsb + kCounterInts * 4 + h_bytes);
+  uint16_t* x_sorted = reinterpret_cast<uint16_t*>(wsb + kCounterInts * 4 + h_bytes +
+                                                   round_up(static_cast<size_t>(T) * d * 4, kWsAlign));
   const int n1 = act == MOE_ACT_SWIGLU ? 2 * F : F;
   const int num_sms = num_sms_current_device();
   if (num_sms <= 0) return MOE_ERR_CUDA;
@@ -390,14 +405,20 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
   moe::GemmArgs a1;
   std::memset(&a1, 0, sizeof(a1));
   const int epi1 = act == MOE_ACT_SWIGLU ? moe::kEpiSwiGLU : moe::kEpiRelu2;
-  const uint32_t box1 = static_cast<uint32_t>(moe::gemm_box_rows(epi1));
+  const bool pair1 = uses_pair_gate_up(bm, d, F, P_total);
+  const uint32_t box1 = pair1 ? 128u : static_cast<uint32_t>(moe::gemm_box_rows(epi1));
   if (!encode_3d(&a1.tm_w, w13, d, n1, E, box1)) return MOE_ERR_CUDA;
   if (n_shared) {
     if (!encode_3d(&a1.tm_ws, w13_shared, d, n1, 1, box1)) return MOE_ERR_CUDA;
   } else {
     a1.tm_ws = a1.tm_w;
   }
-  a1.tm_x = a1.tm_w;  // unused by the gate/up GEMM (rows are gathered with cp.async)
+  if (pair1) {
+    // token rows by TMA from x permuted into the expert-sorted order
+    if (!encode_2d(&a1.tm_x, x_sorted, d, static_cast<uint64_t>(P_total), 128)) return MOE_ERR_CUDA;
+  } else {
+    a1.tm_x = a1.tm_w;  // unused: the single-CTA kernel gathers rows with cp.async
+  }
   a1.x = x;
   a1.sorted_ids = sorted_token_ids;
   a1.expert_ids = expert_ids;
@@ -423,7 +444,16 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
   cudaError_t err;
   {
     StageScope scope(2, s);
-    err = moe::launch_grouped_gemm(epi1, a1, grid, s);
+    if (pair1) {
+      {
+        StageScope pscope(7, s);
+        err = moe::launch_permute_rows(x, sorted_token_ids, num_tokens_post_padded, T, k, d, static_cast<int>(P_max),
+                                       n_shared_blocks * bm, x_sorted, num_sms, s, &launches);
+      }
+      if (err == cudaSuccess) err = moe::launch_grouped_gemm_pair(epi1, a1, num_sms & ~1, s);
+    } else {
+      err = moe::launch_grouped_gemm(epi1, a1, grid, s);
+    }
   }
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   ++launches;
@@ -434,7 +464,7 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
   // CTA pairs share each 256-row W2 tile (128 rows per CTA).  Worth it when
   // the K loop is long (d_ff >= 1024); with a short one the epilogue's
   // reductions bound the kernel and unpaired blocks would only add work.
-  const bool pair2 = F >= 1024 && moe::down_gemm_pair_supported(bm, total_blocks_max);
+  const bool pair2 = F >= 1024 && moe::gemm_pair_supported(bm, total_blocks_max);
   const uint32_t box2 = pair2 ? 128u : static_cast<uint32_t>(moe::gemm_box_rows(moe::kEpiScale));
   if (!encode_3d(&a2.tm_w, w2, F, d, E, box2)) return MOE_ERR_CUDA;
   if (n_shared) {
@@ -476,7 +506,7 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
   {
     StageScope scope(3, s);
     if (pair2)
-      err = moe::launch_down_gemm_pair(a2, num_sms & ~1, s);
+      err = moe::launch_grouped_gemm_pair(moe::kEpiScale, a2, num_sms & ~1, s);
     else
       err = moe::launch_grouped_gemm(moe::kEpiScale, a2, grid, s);
   }

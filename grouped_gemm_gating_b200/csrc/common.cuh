@@ -77,6 +77,12 @@ cudaError_t launch_route_align(const float* logits, int T, int E, int k, int n_g
                                float* topk_weights, int block_m, int P_max, int32_t* sorted_ids, int32_t* expert_ids,
                                int32_t* ntpp, int32_t* inv_pos, int32_t* status, cudaStream_t stream, int* launches);
 
+// x_sorted[p] = x[sorted_ids[p] / k] for live rows p < ntpp, x_sorted[ntpp + t]
+// = x[t] for t < min(T, n_shared_rows).
+cudaError_t launch_permute_rows(const uint16_t* x, const int32_t* sorted_ids, const int32_t* ntpp, int T, int k,
+                                int d, int P_max, int n_shared_rows, uint16_t* x_sorted, int num_sms,
+                                cudaStream_t stream, int* launches);
+
 // out = bf16(acc) over n = T * d elements (the scatter-reduce's last step).
 cudaError_t launch_convert(const float* acc, int64_t n, uint16_t* out, int num_sms, cudaStream_t stream,
                            int* launches);

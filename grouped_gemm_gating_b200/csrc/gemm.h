@@ -47,9 +47,11 @@ int gemm_box_rows(int epi);
 int64_t gemm_max_tiles(int epi, int max_routed_blocks, int n_shared_blocks, int n_out);
 cudaError_t launch_grouped_gemm(int epi, const GemmArgs& args, int grid, cudaStream_t stream);
 
-// Down GEMM on CTA pairs (cluster of two, tcgen05 cta_group::2): args as for
-// the kEpiScale launch, except that tm_w / tm_ws must use 128-row boxes.
-bool down_gemm_pair_supported(int block_m, int total_blocks_max);
-cudaError_t launch_down_gemm_pair(const GemmArgs& args, int grid, cudaStream_t stream);
+// The same GEMMs on CTA pairs (cluster of two, tcgen05 cta_group::2): args
+// as for launch_grouped_gemm, except that tm_w / tm_ws use 128-row boxes and
+// the gate/up GEMM reads its token rows through tm_x (permuted x, 2-D
+// {K, P_total}, 64 x 128 boxes) instead of gathering them.
+bool gemm_pair_supported(int block_m, int total_blocks_max);
+cudaError_t launch_grouped_gemm_pair(int epi, const GemmArgs& args, int grid, cudaStream_t stream);
 
 }  // namespace moe

@@ -1,18 +1,22 @@
-// Down GEMM of the token-major path on CTA pairs (tcgen05 cta_group::2).
+// Token-major grouped GEMMs on CTA pairs (tcgen05 cta_group::2).
 //
-// Same computation as the down GEMM of grouped_gemm.cu -- the "Grouped GEMM
-// Structure" of the fused-moe-kernel page ("Fused MoE Kernel Optimization",
-// skillmd zjli2013) with the top-k weight of each row applied and the result
-// added into the fp32 [T, d] accumulator at the row's token ("Common
-// Pitfalls" 4; the weighted sum of the axolotl `_moe_triton_forward`,
-// src/axolotl/monkeypatch/deepseek_v3/__init__.py) -- with a 256 x 256 tile
-// per pair of SMs instead of 128 x 256 per SM.
+// The same computations as grouped_gemm.cu -- the "Grouped GEMM Structure"
+// of the fused-moe-kernel page ("Fused MoE Kernel Optimization", skillmd
+// zjli2013): the gate/up GEMM with `act_fn(gate) * up` (or the relu^2 fc1 of
+// the mlxcel PR) written as h, and the down GEMM whose rows, scaled by their
+// top-k weight, are added into the fp32 [T, d] accumulator at their token
+// ("Common Pitfalls" 4; the weighted sum of the axolotl
+// `_moe_triton_forward`, src/axolotl/monkeypatch/deepseek_v3/__init__.py) --
+// with a 256 x 256 tile per pair of SMs instead of 128 x 256 per SM.  Both
+// operands arrive by TMA: the gate/up GEMM reads its token rows from a copy
+// of x already permuted into the expert-sorted row order (permute.cu).
 //
 // A cluster of two CTAs works on a "pair unit": two consecutive 128-row
 // blocks of the same expert (the last block of an expert with an odd count
 // is paired with nothing; the odd CTA then computes rows it discards).  Each
-// CTA loads its own block's h rows (A) and half of the 256 W2 rows of the
-// tile (B) by TMA; the transaction bytes of both CTAs complete on the even
+// CTA loads its own block's token rows (A: permuted x or h) and half of the
+// 256 weight rows of the tile (B; SwiGLU: the even CTA the 128 gate rows,
+// the odd CTA the matching 128 up rows) by TMA; the transaction bytes of both CTAs complete on the even
 // CTA's full barrier, where its single MMA thread issues M = 256, N = 256
 // MMAs that read A and B from both CTAs' shared memory.  Commits go to both
 // CTAs (empty stages, full accumulators).  Each CTA's epilogue drains its own
@@ -32,17 +36,21 @@ namespace moe {
 
 namespace {
 
+template <int EPI>
 struct PairCfg {
-  static constexpr int kABytes = 128 * 128;  // 128 h rows x 64 bf16
-  static constexpr int kBBytes = 128 * 128;  // 128 W2 rows x 64 bf16 (this CTA's half of N = 256)
+  static constexpr bool kGated = EPI == kEpiSwiGLU;
+  static constexpr bool kZero = EPI != kEpiScale;  // gate/up: a warp zeroes the down GEMM's accumulator
+  static constexpr int kOutCols = kGated ? 128 : 256;  // output columns of a tile
+  static constexpr int kABytes = 128 * 128;  // 128 token rows x 64 bf16
+  static constexpr int kBBytes = 128 * 128;  // 128 weight rows x 64 bf16 (this CTA's half of N = 256)
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = 6;
   static constexpr int kAccCols = 256;
   static constexpr int kTmemCols = 512;
-  static constexpr int kNumThreads = 192;  // producer, MMA, 4 epilogue warps
+  static constexpr int kNumThreads = kZero ? 224 : 192;  // producer, MMA, 4 epilogue warps (+ zeroing)
   static constexpr int kBarrierBytes = 256;
   static constexpr int kRedStride = 33;
-  static constexpr int kRedBytes = 4 * 32 * kRedStride * 4;
+  static constexpr int kRedBytes = kZero ? 0 : 4 * 32 * kRedStride * 4;
   static constexpr int kMaxUnits = 2048;  // pair units of one launch
   static constexpr int kUnitBytes = kMaxUnits * 4;
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + kRedBytes + kUnitBytes + 1024;
@@ -50,6 +58,8 @@ struct PairCfg {
   static_assert((2 * kStages + 4) * 8 + 8 <= kBarrierBytes, "barrier area");
   static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
 __device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
@@ -62,9 +72,10 @@ struct PairTile {
   bool shared_blk;
 };
 
-__global__ void __launch_bounds__(PairCfg::kNumThreads, 1)
-    down_gemm_pair_kernel(const __grid_constant__ GemmArgs args) {
-  using C = PairCfg;
+template <int EPI>
+__global__ void __launch_bounds__(PairCfg<EPI>::kNumThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ GemmArgs args) {
+  using C = PairCfg<EPI>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
@@ -140,7 +151,7 @@ __global__ void __launch_bounds__(PairCfg::kNumThreads, 1)
   }
   __syncthreads();
   const int n_units = static_cast<int>(tmem_holder[2]);
-  const int n_wt = (args.n_out + 255) / 256;
+  const int n_wt = (args.n_out + C::kOutCols - 1) / C::kOutCols;
   const int pass_w = args.pass_cols > 0 && args.pass_cols < n_wt ? args.pass_cols : n_wt;
   const int total_tiles = n_units * n_wt;
   const int nk = args.K / 64;
@@ -182,7 +193,8 @@ __global__ void __launch_bounds__(PairCfg::kNumThreads, 1)
         // this CTA's block (the odd CTA of a one-block unit loads the even
         // CTA's rows again and discards its result)
         const int blk = t.b0 + (static_cast<int>(rank) < t.nb ? static_cast<int>(rank) : 0);
-        const int wrow = t.wt * 256 + static_cast<int>(rank) * 128;
+        const int wrow = C::kGated ? t.wt * 128 + (rank ? args.up_row_offset : 0)
+                                   : t.wt * 256 + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < nk; ++kb) {
           if (!ptx::mbar_wait_cluster_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
             fail();
@@ -242,7 +254,7 @@ __global__ void __launch_bounds__(PairCfg::kNumThreads, 1)
         }
       }
     }
-  } else {
+  } else if (warp < 6) {
     // ------------------------------------------------ epilogue (both CTAs, own TMEM half)
     const int q = warp & 3;
     const int row = q * 32 + lane;
@@ -260,7 +272,52 @@ __global__ void __launch_bounds__(PairCfg::kNumThreads, 1)
       ptx::tc_fence_after();
       const uint32_t t_acc =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(abuf * C::kAccCols);
-      if (static_cast<int>(rank) < t.nb) {
+      if (static_cast<int>(rank) < t.nb && EPI == kEpiSwiGLU) {
+        const int p = (t.b0 + static_cast<int>(rank)) * args.block_m + row;
+        uint16_t* orow = static_cast<uint16_t*>(args.out) + static_cast<size_t>(p) * args.n_out;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 16) {
+          uint32_t g[16], u[16];
+          ptx::tmem_ld16(t_acc + c0, g);
+          ptx::tmem_ld16(t_acc + 128 + c0, u);
+          ptx::tmem_wait_ld();
+          const int col = t.wt * 128 + c0;
+          if (col < args.n_out) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float h0 = silu_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+              const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+              pk[i] = pack_bf16x2(h0, h1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(orow + col);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      } else if (static_cast<int>(rank) < t.nb && EPI == kEpiRelu2) {
+        const int p = (t.b0 + static_cast<int>(rank)) * args.block_m + row;
+        uint16_t* orow = static_cast<uint16_t*>(args.out) + static_cast<size_t>(p) * args.n_out;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 256; c0 += 16) {
+          uint32_t a[16];
+          ptx::tmem_ld16(t_acc + c0, a);
+          ptx::tmem_wait_ld();
+          const int col = t.wt * 256 + c0;
+          if (col < args.n_out) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float v0 = fmaxf(__uint_as_float(a[2 * i]), 0.0f);
+              const float v1 = fmaxf(__uint_as_float(a[2 * i + 1]), 0.0f);
+              pk[i] = pack_bf16x2(v0 * v0, v1 * v1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(orow + col);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      } else if (static_cast<int>(rank) < t.nb) {
         const int blk = t.b0 + static_cast<int>(rank);
         const int p = blk * args.block_m + row;
         bool valid;
@@ -309,6 +366,20 @@ __global__ void __launch_bounds__(PairCfg::kNumThreads, 1)
         aphase ^= 1u;
       }
     }
+  } else if (C::kZero) {
+    // ------------------------------------------------ zero this CTA's share of the down GEMM's accumulator
+    if (args.acc != nullptr) {
+      const int64_t n = args.acc_elems;
+      const int64_t per = ((n + gridDim.x - 1) / gridDim.x + 3) & ~int64_t(3);
+      const int64_t lo = static_cast<int64_t>(blockIdx.x) * per;
+      const int64_t hi = lo + per < n ? lo + per : n;
+      for (int64_t i = lo + 4 * lane; i < hi; i += 4 * kWarp) {
+        if (i + 4 <= hi)
+          *reinterpret_cast<float4*>(args.acc + i) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        else
+          for (int64_t m = i; m < hi; ++m) args.acc[m] = 0.0f;
+      }
+    }
   }
 
   __syncwarp();
@@ -321,21 +392,17 @@ __global__ void __launch_bounds__(PairCfg::kNumThreads, 1)
   }
 }
 
-}  // namespace
-
-bool down_gemm_pair_supported(int block_m, int total_blocks_max) {
-  return block_m == 128 && total_blocks_max <= PairCfg::kMaxUnits;
-}
-
-cudaError_t launch_down_gemm_pair(const GemmArgs& args, int grid, cudaStream_t stream) {
-  using C = PairCfg;
+template <int EPI>
+cudaError_t launch_pair_variant(const GemmArgs& args, int grid, cudaStream_t stream) {
+  using C = PairCfg<EPI>;
+  auto kern = grouped_gemm_pair_kernel<EPI>;
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_done[dev]) {
-    err = cudaFuncSetAttribute(down_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
     attr_done[dev] = true;
   }
@@ -355,7 +422,23 @@ cudaError_t launch_down_gemm_pair(const GemmArgs& args, int grid, cudaStream_t s
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, down_gemm_pair_kernel, args);
+  return cudaLaunchKernelEx(&cfg, kern, args);
+}
+
+}  // namespace
+
+bool gemm_pair_supported(int block_m, int total_blocks_max) {
+  return block_m == 128 && total_blocks_max <= PairCfg<kEpiScale>::kMaxUnits;
+}
+
+cudaError_t launch_grouped_gemm_pair(int epi, const GemmArgs& args, int grid, cudaStream_t stream) {
+  if (args.block_m != 128) return cudaErrorInvalidValue;
+  switch (epi) {
+    case kEpiSwiGLU: return launch_pair_variant<kEpiSwiGLU>(args, grid, stream);
+    case kEpiRelu2: return launch_pair_variant<kEpiRelu2>(args, grid, stream);
+    case kEpiScale: return launch_pair_variant<kEpiScale>(args, grid, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace moe

@@ -52,7 +52,7 @@ _SIG = {
     "moe_profile_collect": (_I, [_P, _P, _I, _I]),
 }
 
-STAGES = ("route", "align", "gate_up_gemm", "down_gemm", "combine", "route_align", "fused_expert")
+STAGES = ("route", "align", "gate_up_gemm", "down_gemm", "combine", "route_align", "fused_expert", "permute")
 
 _lib = None
 _lock = threading.Lock()

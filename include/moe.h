@@ -105,7 +105,8 @@ MOE_API size_t moe_align_workspace_size(int T, int k, int E);
 
 /* Bytes of device scratch moe_forward needs: a 64 KiB block of int32
  * counters, then (block_m = 128 only) the activation h [P_total, F] in bf16,
- * then the fp32 output accumulator [T, d], where
+ * then the fp32 output accumulator [T, d], then (block_m = 128, d >= 1024 and
+ * F >= 1024) the token rows in expert-sorted order [P_total, d] in bf16, where
  * P_total = P_max + n_shared * ceil(T / block_m) * block_m.
  * The counter block (the first 64 KiB after rounding ws up to 256 bytes)
  * must be zero before the first moe_forward on a workspace (allocate it
@@ -290,7 +291,8 @@ MOE_API int moe_last_launch_count(void);
  * (the accumulator's conversion to bf16), 5 fused route+align
  * (moe_route_align on a small batch), 6 fused expert kernel (moe_forward
  * with block_m <= 64: both GEMMs and the scatter-reduce; under moe_layer on
- * a small batch also the routing and align).
+ * a small batch also the routing and align), 7 permute (x rows copied into
+ * the expert-sorted order for the gate/up GEMM on CTA pairs).
  * moe_profile_enable(1) starts a fresh record (and primes the event pool),
  * (0) stops recording and keeps what was recorded.  moe_profile_collect waits for the recorded events,
  * writes into stage_ms[i] (i < n_stages) the summed milliseconds of stage i
@@ -298,7 +300,7 @@ MOE_API int moe_last_launch_count(void);
  * release != 0 it then returns the events to the pool and clears the record
  * (release == 0 keeps them, e.g. to read a graph's events after each
  * replay).  MOE_ERR_CUDA if an event call failed. */
-#define MOE_NUM_STAGES 7
+#define MOE_NUM_STAGES 8
 MOE_API moe_status moe_profile_enable(int on);
 MOE_API moe_status moe_profile_collect(double* stage_ms, int* stage_calls, int n_stages, int release);
 

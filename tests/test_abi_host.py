@@ -52,9 +52,13 @@ def test_workspace_sizes(lib):
     P = oracle.max_padded(T, k, E, bm) + T  # shared rows (T is a multiple of bm)
     size = M.moe_workspace_size(T, d, F, E, k, bm, M.ACT_SWIGLU, 1)
     counters = 65536
-    # counters, h [P_total, F] bf16, fp32 accumulator [T, d]
-    assert size >= P * 2 * F + T * 4 * d + counters
-    assert size <= P * 2 * F + T * 4 * d + counters + 1024
+    # counters, h [P_total, F] bf16, fp32 accumulator [T, d], and (d, F >= 1024)
+    # the token rows in expert-sorted order [P_total, d] bf16
+    assert size >= P * 2 * F + T * 4 * d + P * 2 * d + counters
+    assert size <= P * 2 * F + T * 4 * d + P * 2 * d + counters + 1280
+    d_small = 512
+    size = M.moe_workspace_size(T, d_small, F, E, k, bm, M.ACT_SWIGLU, 1)
+    assert P * 2 * F + T * 4 * d_small + counters <= size <= P * 2 * F + T * 4 * d_small + counters + 1024
     # block_m <= 64 keeps h in shared memory: counters and the accumulator only
     small = M.moe_workspace_size(3, 2048, 768, 128, 8, 16, M.ACT_SWIGLU, 0)
     assert 3 * 4 * 2048 + counters <= small <= 3 * 4 * 2048 + counters + 1024
