@@ -44,6 +44,8 @@ METRIC = "MoE layer TFLOPS and tokens/s on 1 B200; % of bf16 tensor peak / HBM r
 # --warmup 3 --no-cpu-baseline under ncu --set full -k <kernel> -c 1).  An
 # entry is removed whenever the kernel changes after its capture.
 NCU_TRAFFIC = {
+    ("decode", "fused_expert"): 201_991_936,
+    ("dsv3", "gate_up_gemm"): 1_165_228_280,
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
