@@ -57,10 +57,8 @@ namespace moe {
 
 namespace {
 
-// In-kernel routing limits (block_m = 16 only): T*k <= 256 slots, hence
-// P_max <= 256 + 256 * 15 = 4096 padded rows.
+// In-kernel routing limit (block_m = 16 only): T*k <= 256 slots.
 constexpr int kRouteMaxS = 256;
-constexpr int kRouteMaxP = 4096;
 
 template <int EPI1, int TOK, bool ROUTE>
 struct FusedCfg {
@@ -74,9 +72,10 @@ struct FusedCfg {
   static constexpr int kXbufBytes = kGated ? 64 * TOK * 4 : 0;  // up half handed to the gate half
   static constexpr int kTokBytes = 2 * 2 * 64 * 4;              // token id and weight per row, two tiles
   static constexpr int kBarrierBytes = 1024;
-  // routing results kept for the whole kernel: padded rows, block experts,
-  // slot weights, slot ids, inverse positions, padded total
-  static constexpr int kRouteBytes = ROUTE ? (kRouteMaxP + kRouteMaxP / 16 + 3 * kRouteMaxS + 8) * 4 : 0;
+  // routing results kept for the whole kernel: expert and weight of every
+  // slot, its rank among its expert's slots, the slots in expert order, and
+  // per expert its slot count and padded / unpadded offsets
+  static constexpr int kRouteBytes = ROUTE ? (4 * kRouteMaxS + 3 * (MOE_MAX_EXPERTS + 1) + 5) * 4 : 0;
   static constexpr int kFixedBytes = 2 * kHBufBytes + kXbufBytes + kTokBytes + kBarrierBytes + kRouteBytes + 1024;
   static constexpr int kStagesRaw = (227 * 1024 - kFixedBytes) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
@@ -229,58 +228,85 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
 
   pdl_wait();
   pdl_launch_dependents();
-  const int32_t* sorted_ids = args.sorted_ids;
-  const int32_t* expert_ids = args.expert_ids;
-  const float* topk_w = args.topk_w;
+  // routing results in shared memory (in-kernel routing only)
+  int* r_ids = nullptr;      // [S] expert of each slot
+  float* r_w = nullptr;      // [S] its weight
+  int* r_rank = nullptr;     // [S] rank of the slot among its expert's slots
+  int* r_compact = nullptr;  // [S] slots in (expert, slot) order
+  int* r_cnt = nullptr;      // [E] slots per expert
+  int* r_off = nullptr;      // [E + 1] padded offsets (r_off[E] = padded total)
+  int* r_coff = nullptr;     // [E + 1] unpadded offsets
   int ntpp_v;
   if constexpr (ROUTE) {
-    // ---- routing and align of all tokens, redundantly in every CTA, before
-    // any weight streams.  Results live after the barriers; the per-warp
-    // group scratch and the counting-sort scratch borrow the stage ring,
-    // which is idle until the producer starts.
-    int* r_sorted = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::kBarrierBytes);
-    int* r_eid = r_sorted + kRouteMaxP;
-    float* r_w = reinterpret_cast<float*>(r_eid + kRouteMaxP / 16);
-    int* r_ids = reinterpret_cast<int*>(r_w + kRouteMaxS);
-    int* r_inv = r_ids + kRouteMaxS;
-    int* r_ntpp = r_inv + kRouteMaxS;
+    // ---- routing of all tokens and their per-expert order, redundantly in
+    // every CTA, before any weight streams: counts, two scans and a rank per
+    // slot are all the kernel needs (a block's expert and a row's slot are
+    // looked up from them); the padded sort itself is only written out, by
+    // CTA 0's epilogue warps while the first weights stream.
+    r_ids = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::kBarrierBytes);
+    r_w = reinterpret_cast<float*>(r_ids + kRouteMaxS);
+    r_rank = reinterpret_cast<int*>(r_w + kRouteMaxS);
+    r_compact = r_rank + kRouteMaxS;
+    r_cnt = r_compact + kRouteMaxS;
+    r_off = r_cnt + MOE_MAX_EXPERTS + 1;
+    r_coff = r_off + MOE_MAX_EXPERTS + 1;
     constexpr int kWarps = C::kNumThreads / kWarp;
-    float* gscore = reinterpret_cast<float*>(smem);  // [kWarps][64]
+    float* gscore = reinterpret_cast<float*>(smem);  // [kWarps][64] on the idle stage ring
     unsigned char* gkeep = reinterpret_cast<unsigned char*>(gscore + kWarps * 64);  // [kWarps][64]
-    int* cnt = reinterpret_cast<int*>(smem + 8192);
-    int* off = cnt + MOE_MAX_EXPERTS;
-    int* run = off + MOE_MAX_EXPERTS + 1;
-    int* tot = run + MOE_MAX_EXPERTS;
-    int(*wcnt)[MOE_MAX_EXPERTS] = reinterpret_cast<int(*)[MOE_MAX_EXPERTS]>(tot + MOE_MAX_EXPERTS + 3);
     const FusedRoute& R = args.route;
-    for (int t = warp; t < args.T; t += kWarps)
-      route_one_token<8>(R.logits + static_cast<size_t>(t) * args.E, args.E, args.k, R.n_group, R.topk_group,
-                         R.group_score, R.renormalize, R.routed_scaling, gscore + warp * 64, gkeep + warp * 64,
-                         r_ids + t * args.k, r_w + t * args.k, args.status, lane);
-    for (int i = threadIdx.x; i < kWarps * MOE_MAX_EXPERTS; i += C::kNumThreads) (&wcnt[0][0])[i] = 0;
-    __syncthreads();
-    auto get_expert = [&](int s, bool) { return r_ids[s]; };
-    align_detail::align_one_block<kWarps>(get_expert, args.S, args.E, args.block_m, R.P_max, r_sorted, r_eid, r_ntpp,
-                                          r_inv, cnt, off, run, tot, wcnt);
-    __syncthreads();
-    if (blockIdx.x == 0) {  // the same results as the separate routing and align calls
-      for (int i = threadIdx.x; i < args.S; i += C::kNumThreads) {
-        R.topk_ids[i] = r_ids[i];
-        R.topk_w[i] = r_w[i];
-        R.inv_pos[i] = r_inv[i];
-      }
-      for (int i = threadIdx.x; i < R.P_max; i += C::kNumThreads) R.sorted_ids[i] = r_sorted[i];
-      for (int i = threadIdx.x; i < R.P_max / args.block_m; i += C::kNumThreads) R.expert_ids[i] = r_eid[i];
-      if (threadIdx.x == 0) *R.ntpp = *r_ntpp;
+    for (int i = threadIdx.x; i < args.E; i += C::kNumThreads) r_cnt[i] = 0;
+    for (int t = warp; t < args.T; t += kWarps) {
+      const float* row = R.logits + static_cast<size_t>(t) * args.E;
+      if (args.E <= 128)
+        route_one_token<4>(row, args.E, args.k, R.n_group, R.topk_group, R.group_score, R.renormalize,
+                           R.routed_scaling, gscore + warp * 64, gkeep + warp * 64, r_ids + t * args.k,
+                           r_w + t * args.k, args.status, lane);
+      else
+        route_one_token<8>(row, args.E, args.k, R.n_group, R.topk_group, R.group_score, R.renormalize,
+                           R.routed_scaling, gscore + warp * 64, gkeep + warp * 64, r_ids + t * args.k,
+                           r_w + t * args.k, args.status, lane);
     }
-    sorted_ids = r_sorted;
-    expert_ids = r_eid;
-    topk_w = r_w;
-    ntpp_v = *r_ntpp;
-    __syncthreads();  // the scratch on the stage ring is free again
+    __syncthreads();
+    for (int i = threadIdx.x; i < args.S; i += C::kNumThreads) atomicAdd(&r_cnt[r_ids[i]], 1);
+    __syncthreads();
+    if (warp == 0) align_detail::warp_padded_scan(r_cnt, r_off, args.E, args.block_m, lane);
+    if (warp == 1) align_detail::warp_padded_scan(r_cnt, r_coff, args.E, 1, lane);
+    __syncthreads();
+    for (int i = threadIdx.x; i < args.S; i += C::kNumThreads) {
+      const int e = r_ids[i];
+      int rank = 0;
+      for (int j = 0; j < i; ++j) rank += r_ids[j] == e ? 1 : 0;
+      r_rank[i] = rank;
+      r_compact[r_coff[e] + rank] = i;
+    }
+    __syncthreads();  // the stage ring is free again
+    ntpp_v = r_off[args.E];
   } else {
     ntpp_v = *args.ntpp;
   }
+  // expert of routed block `blk`, and the slot of row j of it (S: padding)
+  auto block_exp = [&](int blk) -> int {
+    if constexpr (ROUTE) {
+      return align_detail::block_expert(r_off, args.E, blk * args.block_m);
+    } else {
+      return args.expert_ids[blk];
+    }
+  };
+  auto row_slot = [&](int blk, int e, int j) -> int {
+    if constexpr (ROUTE) {
+      const int i = blk * args.block_m + j - r_off[e];
+      return i < r_cnt[e] ? r_compact[r_coff[e] + i] : args.S;
+    } else {
+      return args.sorted_ids[blk * args.block_m + j];
+    }
+  };
+  auto slot_weight = [&](int slot) -> float {
+    if constexpr (ROUTE) {
+      return r_w[slot];
+    } else {
+      return args.topk_w[slot];
+    }
+  };
   int routed_blocks = ntpp_v / args.block_m;
   if (routed_blocks < 0) routed_blocks = 0;
   if (routed_blocks > args.max_routed_blocks) routed_blocks = args.max_routed_blocks;
@@ -314,7 +340,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
       bool ok = true;
       auto expert_of = [&](const TileInfo& t) {
         if (t.shared_blk) return 0;
-        const int e = expert_ids[t.blk];
+        const int e = block_exp(t.blk);
         if (e < 0 || e >= args.E) set_status(args.status, MOE_ERR_BAD_EXPERT_ID);  // TMA fills zeros
         return e;
       };
@@ -453,6 +479,28 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
     const int q = warp & 3;         // TMEM lane quadrant this warp may access
     const int row = q * 32 + lane;  // accumulator row: weight row / d row within the tile
     const int etid = threadIdx.x - 64;
+    if constexpr (ROUTE) {
+      if (blockIdx.x == 0) {  // the outputs of the separate routing and align calls
+        const FusedRoute& R = args.route;
+        for (int i = etid; i < args.S; i += 128) {
+          R.topk_ids[i] = r_ids[i];
+          R.topk_w[i] = r_w[i];
+          R.inv_pos[i] = r_off[r_ids[i]] + r_rank[i];
+        }
+        for (int p = etid; p < R.P_max; p += 128) {
+          int v = args.S;
+          if (p < ntpp_v) {
+            const int e = align_detail::block_expert(r_off, args.E, p);
+            const int i = p - r_off[e];
+            if (i < r_cnt[e]) v = r_compact[r_coff[e] + i];
+          }
+          R.sorted_ids[p] = v;
+        }
+        for (int b = etid; b < R.P_max / args.block_m; b += 128)
+          R.expert_ids[b] = align_detail::block_expert(r_off, args.E, b * args.block_m);
+        if (etid == 0) *R.ntpp = ntpp_v;
+      }
+    }
     bool zero_seen = false;
     int d2c = 0;
     // Same order as the MMA: the gate/up accumulator of tile i is turned
@@ -470,10 +518,10 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
           int tok = -1;
           float wj = 0.0f;
           if (!t.shared_blk) {
-            const int slot = sorted_ids[t.blk * args.block_m + j];
+            const int slot = row_slot(t.blk, block_exp(t.blk), j);
             if (static_cast<unsigned>(slot) < static_cast<unsigned>(args.S)) {
               tok = slot / args.k;
-              wj = topk_w[slot];
+              wj = slot_weight(slot);
             }
           } else {
             const int tk = (t.blk - routed_blocks) * args.block_m + j;
@@ -653,6 +701,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
     for (int i = 0; ok && i <= n_my; ++i) {
       if (i < n_my) {
         const TileInfo t = tile_of(i);
+        const int e_blk = t.shared_blk ? 0 : block_exp(t.blk);
         const uint16_t* src[kRowsPerThread];
         uint32_t nbytes[kRowsPerThread];
 #pragma unroll
@@ -661,7 +710,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
           int tok = 0;
           bool valid;
           if (!t.shared_blk) {
-            const int slot = sorted_ids[t.blk * args.block_m + row];
+            const int slot = row_slot(t.blk, e_blk, row);
             valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
             if (valid) tok = slot / args.k;
           } else {
