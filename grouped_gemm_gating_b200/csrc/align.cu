@@ -31,7 +31,8 @@ using namespace align_detail;
 constexpr int kSingleBlockMax = 8192;
 constexpr int kSmallThreads = 1024;
 constexpr int kChunk = 2048;        // slots per chunk on the multi-block path
-constexpr int kChunkThreads = 256;  // threads per chunk block
+constexpr int kChunkThreads = 256;  // threads per chunk block (count)
+constexpr int kScatterThreads = 1024;  // threads per chunk block (scatter: two rounds of 1024 slots)
 
 __global__ void __launch_bounds__(kSmallThreads)
     align_single_kernel(const int32_t* __restrict__ ids, int S, int E, int bm, int P_max,
@@ -75,48 +76,65 @@ __global__ void __launch_bounds__(1024)
     align_scan_kernel(const int32_t* __restrict__ counts, int nchunks, int S, int E, int bm, int P_max,
                       int32_t* __restrict__ bases, int32_t* __restrict__ sorted_ids,
                       int32_t* __restrict__ expert_ids, int32_t* ntpp) {
+  constexpr int kSlices = 1024 / MOE_MAX_EXPERTS;  // contiguous chunk ranges per expert
+  __shared__ int part[kSlices][MOE_MAX_EXPERTS];
   __shared__ int cnt[MOE_MAX_EXPERTS];
   __shared__ int off[MOE_MAX_EXPERTS + 1];
   const int tid = threadIdx.x;
+  const int e = tid % MOE_MAX_EXPERTS, slice = tid / MOE_MAX_EXPERTS;
+  const int per = (nchunks + kSlices - 1) / kSlices;
+  const int c_lo = slice * per, c_hi = min(nchunks, c_lo + per);
   pdl_wait();
   pdl_launch_dependents();
+  // threads over experts (coalesced loads), each summing one chunk range
+  int sum = 0;
+  if (e < E) {
+#pragma unroll 8
+    for (int c = c_lo; c < c_hi; ++c) sum += counts[static_cast<size_t>(c) * E + e];
+  }
+  part[slice][e] = sum;
+  __syncthreads();
   if (tid < E) {
     int total = 0;
-    for (int c = 0; c < nchunks; ++c) total += counts[static_cast<size_t>(c) * E + tid];
+#pragma unroll
+    for (int s2 = 0; s2 < kSlices; ++s2) total += part[s2][tid];
     cnt[tid] = total;
   }
   __syncthreads();
   if (tid < 32) warp_padded_scan(cnt, off, E, bm, tid);
   __syncthreads();
-  if (tid < E) {
-    int run = off[tid];
-    for (int c = 0; c < nchunks; ++c) {
-      bases[static_cast<size_t>(c) * E + tid] = run;
-      run += counts[static_cast<size_t>(c) * E + tid];
+  // chunk bases: the expert's offset, the earlier slices, then this range
+  if (e < E) {
+    int run = off[e];
+    for (int s2 = 0; s2 < slice; ++s2) run += part[s2][e];
+#pragma unroll 8
+    for (int c = c_lo; c < c_hi; ++c) {
+      bases[static_cast<size_t>(c) * E + e] = run;
+      run += counts[static_cast<size_t>(c) * E + e];
     }
-    // padding inside this expert's last block
-    for (int p = off[tid] + cnt[tid]; p < off[tid + 1]; ++p) sorted_ids[p] = S;
+    // padding inside this expert's last block, split over the slices
+    for (int p = off[e] + cnt[e] + slice; p < off[e + 1]; p += kSlices) sorted_ids[p] = S;
   }
   if (tid == 0) *ntpp = off[E];
   for (int p = off[E] + tid; p < P_max; p += blockDim.x) sorted_ids[p] = S;
   for (int b = tid; b < P_max / bm; b += blockDim.x) expert_ids[b] = block_expert(off, E, b * bm);
 }
 
-__global__ void __launch_bounds__(kChunkThreads)
+__global__ void __launch_bounds__(kScatterThreads)
     align_scatter_kernel(const int32_t* __restrict__ ids, int S, int E, const int32_t* __restrict__ bases,
                          int32_t* __restrict__ sorted_ids, int32_t* __restrict__ inv_pos) {
-  constexpr int kWarps = kChunkThreads / 32;
+  constexpr int kWarps = kScatterThreads / 32;
   __shared__ int run[MOE_MAX_EXPERTS];
   __shared__ int tot[MOE_MAX_EXPERTS];
   __shared__ int wcnt[kWarps][MOE_MAX_EXPERTS];
   const int c = blockIdx.x;
   pdl_wait();
   pdl_launch_dependents();
-  for (int i = threadIdx.x; i < E; i += kChunkThreads) run[i] = bases[static_cast<size_t>(c) * E + i];
-  for (int i = threadIdx.x; i < kWarps * MOE_MAX_EXPERTS; i += kChunkThreads) (&wcnt[0][0])[i] = 0;
+  for (int i = threadIdx.x; i < E; i += kScatterThreads) run[i] = bases[static_cast<size_t>(c) * E + i];
+  for (int i = threadIdx.x; i < kWarps * MOE_MAX_EXPERTS; i += kScatterThreads) (&wcnt[0][0])[i] = 0;
   __syncthreads();
   const int end = min(S, (c + 1) * kChunk);
-  for (int base = c * kChunk; base < end; base += kChunkThreads) {
+  for (int base = c * kChunk; base < end; base += kScatterThreads) {
     const int s = base + threadIdx.x;
     const int e = s < end ? load_expert(ids, s, S, E, nullptr) : -1;
     scatter_round<kWarps>(e, s, wcnt, run, tot, E, sorted_ids, inv_pos);
@@ -146,7 +164,7 @@ cudaError_t launch_align(const int32_t* topk_ids, int S, int E, int block_m, int
   err = launch_pdl(align_scan_kernel, dim3(1), dim3(1024), 0, stream, static_cast<const int32_t*>(counts), nchunks,
                    S, E, block_m, P_max, bases, sorted_ids, expert_ids, ntpp);
   if (err != cudaSuccess) return err;
-  err = launch_pdl(align_scatter_kernel, dim3(nchunks), dim3(kChunkThreads), 0, stream, topk_ids, S, E,
+  err = launch_pdl(align_scatter_kernel, dim3(nchunks), dim3(kScatterThreads), 0, stream, topk_ids, S, E,
                    static_cast<const int32_t*>(bases), sorted_ids, inv_pos);
   *launches += 3;
   return err;

@@ -8,25 +8,17 @@
 namespace moe {
 namespace route_detail {
 
-struct Cand {
-  float v;
-  int i;
-};
-
-// true if a is selected before b
-__device__ __forceinline__ bool beats(const Cand& a, const Cand& b) {
-  return a.v > b.v || (a.v == b.v && a.i < b.i);
+// Unsigned key with the order of the fp32 values (-0 taken as +0, so the
+// two zeros tie as they do in a float comparison); 0 is below every value
+// and marks an excluded expert.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  uint32_t u = __float_as_uint(v);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ Cand warp_best(Cand c) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    Cand o;
-    o.v = __shfl_xor_sync(0xffffffffu, c.v, off);
-    o.i = __shfl_xor_sync(0xffffffffu, c.i, off);
-    if (beats(o, c)) c = o;
-  }
-  return c;
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -115,23 +107,34 @@ __device__ __forceinline__ int route_one_token(const float* __restrict__ row, in
     }
   }
 
-  // k rounds of warp arg-max over the remaining allowed experts
+  // k rounds of warp arg-max over the remaining allowed experts, on
+  // order-preserving integer keys: one warp max of the lanes' best keys,
+  // then one warp min of the expert ids that hold it (ties -> lowest id).
+  uint32_t key[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) key[i] = allowed[i] ? order_key(v[i]) : 0u;
   int my_id = 0;
   float my_val = 0.0f;
   for (int j = 0; j < k; ++j) {
-    Cand best{-INFINITY, 0x7fffffff};
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const Cand c{v[i], lane + 32 * i};
-      if (allowed[i] && (best.i == 0x7fffffff || beats(c, best))) best = c;
-    }
-    best = warp_best(best);
+    uint32_t hk = 0u;
+    int hi = 0;
 #pragma unroll
     for (int i = 0; i < VPL; ++i)
-      if (lane + 32 * i == best.i) allowed[i] = false;
+      if (key[i] > hk) {  // strict: the lowest id of this lane among equal keys
+        hk = key[i];
+        hi = i;
+      }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, hk);
+    const uint32_t cand = (hk == m && hk != 0u) ? static_cast<uint32_t>(lane + 32 * hi) : 0xffffffffu;
+    const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+    if (static_cast<int>(win & 31u) == lane) {
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (i == static_cast<int>(win >> 5)) key[i] = 0u;
+    }
     if (lane == j) {
-      my_id = best.i;
-      my_val = best.v;
+      my_id = static_cast<int>(win);
+      my_val = key_value(m);
     }
   }
 
