@@ -314,10 +314,16 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
   const int n_h = (args.F + C::kH - 1) / C::kH;
   const int n_d = (args.d + 127) / 128;
   const int total_tiles = total_blocks * n_h;
-  // tiles of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
-  const int n_my = static_cast<int>(blockIdx.x) < total_tiles
-                       ? (total_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
-                             static_cast<int>(gridDim.x)
+  // Tiles are dealt to the fewest CTAs that can each take the per-CTA
+  // maximum: with 252 tiles on 148 CTAs, 126 CTAs take two tiles each
+  // instead of 104 taking two and 44 taking one.  Every CTA streams the same
+  // bytes and gets a larger share of HBM while it streams.  The other CTAs
+  // only zero and convert their share of the accumulator.
+  // Tiles of this CTA: blockIdx.x, blockIdx.x + tile_stride, ...
+  const int tiles_per_cta = (total_tiles + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+  const int tile_stride = tiles_per_cta > 0 ? (total_tiles + tiles_per_cta - 1) / tiles_per_cta : 1;
+  const int n_my = static_cast<int>(blockIdx.x) < tile_stride
+                       ? (total_tiles - static_cast<int>(blockIdx.x) + tile_stride - 1) / tile_stride
                        : 0;
   const int nk1 = args.d / 64;
   const int nk2 = n_d * C::kHk;  // down-GEMM stages per tile
@@ -327,7 +333,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
     *abort_flag = 1;
     set_status(args.status, MOE_ERR_DEVICE_TIMEOUT);
   };
-  auto tile_of = [&](int i) { return tile_info(static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x), n_h, routed_blocks); };
+  auto tile_of = [&](int i) { return tile_info(static_cast<int>(blockIdx.x) + i * tile_stride, n_h, routed_blocks); };
 
   // Stage order of every role: gate/up of tile 0; then for i >= 1 gate/up of
   // tile i followed by the down GEMM of tile i-1; last the down GEMM of the
@@ -380,7 +386,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
           const TileInfo t = tile_of(i - 1);
           const int e = expert_of(t);
           const CUtensorMap* tm = t.shared_blk ? &args.tm_w2s : &args.tm_w2;
-          const int rot = d_rotation(static_cast<int>(blockIdx.x) + (i - 1) * static_cast<int>(gridDim.x), n_d);
+          const int rot = d_rotation(static_cast<int>(blockIdx.x) + (i - 1) * tile_stride, n_d);
           for (int s = 0; s < nk2 && acquire(); ++s) {
             const int dk = s / C::kHk, kk = s - dk * C::kHk;
             const int di = d_tile(dk, rot, n_d);
@@ -609,7 +615,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
           zero_seen = true;
         }
         // ---- down-GEMM partial of every d tile -> fp32 accumulator
-        const int rot = d_rotation(static_cast<int>(blockIdx.x) + p * static_cast<int>(gridDim.x), n_d);
+        const int rot = d_rotation(static_cast<int>(blockIdx.x) + p * tile_stride, n_d);
         const int* tk = tok_s + b * 64;
         const float* wk = w_s + b * 64;
         // valid rows of a block come first (an expert's padding ends its
