@@ -318,16 +318,20 @@ def run_ours(args):
             g.replay()
     torch.cuda.synchronize(dev)
 
-    def timed(runs, n):
-        """Device time of n steps (step i runs runs[i % len(runs)]), max over ranks."""
+    def timed(runs, n, whole=None):
+        """Device time of n steps (step i runs runs[i % len(runs)], or one
+        call of `whole` runs all n), max over ranks."""
         barrier(pg)
         torch.cuda.synchronize(dev)
         if rotate:
             start = torch.cuda.Event(enable_timing=True)
             end = torch.cuda.Event(enable_timing=True)
             start.record(stream)
-            for i in range(n):
-                runs[i % len(runs)]()
+            if whole is not None:
+                whole()
+            else:
+                for i in range(n):
+                    runs[i % len(runs)]()
             end.record(stream)
             torch.cuda.synchronize(dev)
             ms = start.elapsed_time(end)
@@ -344,8 +348,17 @@ def run_ours(args):
         barrier(pg)
         return max_over_ranks(pg, ms)
 
+    # Back to back, the K timed steps are one graph (as in a captured model
+    # forward): consecutive steps' kernels are chained by programmatic
+    # dependent launch instead of paying a graph launch each.
+    g_steps = None
+    if rotate:
+        g_steps = capture(lambda: [step(sets[i % n_copies]) for i in range(args.steps)])
+        g_steps.replay()
+        torch.cuda.synchronize(dev)
+
     # ---- device-timed region: inputs resident in HBM ----
-    total_ms = timed([g.replay for g in g_main], args.steps)
+    total_ms = timed([g.replay for g in g_main], args.steps, g_steps.replay if g_steps is not None else None)
     launches = launches_per_step * args.steps
     assert M.moe_read_status(buf.status) == 0, "device status set during the timed region"
 
@@ -383,9 +396,14 @@ def run_ours(args):
     e2e_step(sets[0])
     torch.cuda.synchronize(dev)
     g_e2e = [capture(lambda st=st: e2e_step(st)) for st in sets]
-    e2e_ms = timed([g.replay for g in g_e2e], args.steps)
+    g_e2e_steps = None
+    if rotate:
+        g_e2e_steps = capture(lambda: [e2e_step(sets[i % n_copies]) for i in range(args.steps)])
+        g_e2e_steps.replay()
+        torch.cuda.synchronize(dev)
+    e2e_ms = timed([g.replay for g in g_e2e], args.steps, g_e2e_steps.replay if g_e2e_steps is not None else None)
     assert torch.equal(out_h.view(torch.int16), buf.out.cpu().view(torch.int16))
-    del g_main, g_prof, g_e2e
+    del g_main, g_prof, g_e2e, g_steps, g_e2e_steps
 
     alg = algorithmic(cfg, topk_ids)
     sec_per_step = total_ms / args.steps / 1e3
@@ -438,7 +456,9 @@ def run_ours(args):
                           f"x, logits and the expert weights ({touched / 1e6:.0f} MB of weights read per step; "
                           f"a copy is reused after >= 2x L2 of other data)") if rotate else
                          "flushed before every timed step (write of 2x L2), outside the step's events",
-                   "launch": "CUDA graph of the step, kernels chained by programmatic dependent launch",
+                   "launch": ("one CUDA graph of the K timed steps, kernels chained by programmatic dependent "
+                              "launch") if rotate else
+                             "CUDA graph of the step, kernels chained by programmatic dependent launch",
                    "experts_hit": alg["U"], "flops_per_step": alg["flops_total"],
                    "flops_routed_per_step": alg["flops_routed"]},
         "ms_per_step_eager": round(eager_ms / args.steps, 5),

@@ -18,16 +18,19 @@ __device__ __forceinline__ int load_expert(const int32_t* ids, int s, int S, int
 }
 
 // Exclusive prefix of padded counts over experts, by one warp.  off[E] is
-// the padded total.
+// the padded total.  bm is a power of two (block_m, or 1 for no padding), so
+// rounding up is a mask: a runtime integer division per expert made this
+// scan cost more than a microsecond.
 __device__ __forceinline__ void warp_padded_scan(const int* cnt, int* off, int E, int bm, int lane) {
   constexpr int kPer = MOE_MAX_EXPERTS / 32;
   int local[kPer];
   int sum = 0;
+  const int mask = -bm;
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int e = lane * kPer + i;
     const int c = e < E ? cnt[e] : 0;
-    local[i] = (c + bm - 1) / bm * bm;
+    local[i] = (c + bm - 1) & mask;
     sum += local[i];
   }
   int incl = sum;

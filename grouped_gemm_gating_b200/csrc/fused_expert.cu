@@ -36,9 +36,11 @@
 //   start: the gather warps zero this CTA's slice of the accumulator and
 //          count the CTA on sync[0]; the epilogue waits for all CTAs there
 //          before its first reduction (the weight stream does not wait).
-//   end:   every CTA counts itself on sync[1] once its reductions are issued,
-//          waits for all, converts its slice of the accumulator to bf16 and
-//          counts itself on sync[2]; the last one resets the counters.
+//   end:   every CTA counts itself on sync[1] once its reductions are issued;
+//          the last to arrive zeroes sync[0..1] and stores -(G-1) in sync[2],
+//          which releases the others; each of them adds 1 back to sync[2]
+//          (so every counter is zero when the kernel ends), and every CTA
+//          converts its slice of the accumulator to bf16.
 //
 // Warp roles: warp 0 TMA producer (weights), warp 1 TMEM allocator + MMA
 // issuer, warps 2-5 epilogue, warps 6-9 token-row gather (cp.async; each
@@ -153,6 +155,16 @@ __device__ __forceinline__ bool epilogue_any(bool v) {
       : "r"(v ? 1u : 0u)
       : "memory");
   return r != 0;
+}
+
+// Bounded spin until *p != 0 (acquire).  False on timeout or abort.
+__device__ __forceinline__ bool spin_until_nonzero(const int32_t* p, volatile int* abort_flag) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (ptx::ld_acquire_gpu(p) == 0) {
+    if (*abort_flag || ptx::globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    __nanosleep(64);
+  }
+  return true;
 }
 
 // Bounded spin until *p >= target (acquire).  False on timeout or abort.
@@ -758,10 +770,23 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, 512);
   }
-  // ---- grid end: all reductions issued -> convert the accumulator to bf16
+  // ---- grid end: all reductions issued -> convert the accumulator to bf16.
+  // sync[1] counts the CTAs that have issued all their reductions.  The last
+  // one to arrive returns sync[0] and sync[1] to zero and releases the others
+  // by storing -(G-1) in sync[2]; each released CTA adds 1 to sync[2] as it
+  // goes (fire-and-forget), so all three counters are zero again when the
+  // kernel completes and no CTA waits on another round of atomics to exit.
   if (threadIdx.x == 0) {
-    ptx::atom_acq_rel_gpu_add(args.sync + 1, 1);  // releases this CTA's reductions
-    const bool all = spin_until(args.sync + 1, static_cast<int>(gridDim.x), abort_flag);
+    const int G = static_cast<int>(gridDim.x);
+    bool all = true;
+    if (ptx::atom_acq_rel_gpu_add(args.sync + 1, 1) == G - 1) {  // releases this CTA's reductions
+      args.sync[0] = 0;
+      args.sync[1] = 0;
+      ptx::st_release_gpu(args.sync + 2, -(G - 1));
+    } else {
+      all = spin_until_nonzero(args.sync + 2, abort_flag);
+      if (all) ptx::red_relaxed_gpu_add(args.sync + 2, 1);
+    }
     if (!all) fail();
     *flag = all ? 1 : 0;
   }
@@ -782,13 +807,6 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
         for (int m = e; m < min(hi, e + 4); ++m) args.out[m] = float_to_bf16_bits(__ldcg(args.acc + m));
       }
     }
-  }
-  __syncthreads();
-  if (threadIdx.x == 0 && ptx::atom_acq_rel_gpu_add(args.sync + 2, 1) == static_cast<int>(gridDim.x) - 1) {
-    // every CTA has passed both waits: return the counters to zero
-    args.sync[0] = 0;
-    args.sync[1] = 0;
-    args.sync[2] = 0;
   }
 }
 
