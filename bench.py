@@ -66,6 +66,9 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="decode", choices=sorted(W.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--single-copy", action="store_true",
+                    help="one copy of the inputs and an L2 flush before every step (small device footprint, "
+                         "e.g. for profiler captures)")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -125,7 +128,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={CLOCK_QUERY}", "--format=csv,noheader,nounits", "-lms", "100",
+                ["nvidia-smi", f"--query-gpu={CLOCK_QUERY}", "--format=csv,noheader,nounits", "-lms", "20",
                  "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -284,7 +287,7 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     topk_ids = buf.topk_ids.cpu().numpy()
     touched = algorithmic(cfg, topk_ids)["weight_bytes"]
-    rotate = touched * 2 >= l2
+    rotate = touched * 2 >= l2 and not args.single_copy
     n_copies = 1 + -(-2 * l2 // touched) if rotate else 1
     sets += [input_set() for _ in range(n_copies - 1)]
     flush = None if rotate else torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
@@ -427,17 +430,27 @@ def run_ours(args):
     else:
         fl, by = alg[dom]
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    src = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
     if fl / by >= ridge:
         achieved = fl / per_launch_s / 1e12
-        peak = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "unit": "TFLOP/s"}
+        if rotate:
+            # back-to-back steps run under the 1 kW power cap within tens of
+            # milliseconds: the kernel is timed inside a long run, so its
+            # denominator is the sustained (power-capped) cuBLAS figure
+            peak = peaks["bf16_tflops_sustained"]
+            src += ", sustained bf16 (timed inside back-to-back steps)"
+            roof["frac_of_burst_peak"] = round(achieved / peaks["bf16_tflops"], 4)
+        else:
+            peak = peaks["bf16_tflops"]
+            src += ", burst bf16"
     else:
         achieved = by / per_launch_s / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "unit": "GB/s"}
+        src += ", HBM copy"
     traffic = NCU_TRAFFIC.get((cfg.name, dom))
-    roof.update({"kernel": dom, "achieved": round(achieved, 2), "peak": peak,
-                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
+    roof.update({"kernel": dom, "achieved": round(achieved, 2), "peak": peak, "peak_source": src,
                  "frac": round(achieved / peak, 4),
                  "traffic": traffic,
                  "traffic_vs_algorithmic": None if traffic is None else round(traffic / by, 3),

@@ -59,7 +59,9 @@ struct PairCfg {
   static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+// silu(g) = g * sigmoid(g), with the fast approximate divide: h is rounded
+// to bf16 right after, far coarser than the divide's error.
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
@@ -275,24 +277,30 @@ __global__ void __launch_bounds__(PairCfg<EPI>::kNumThreads, 1)
       if (static_cast<int>(rank) < t.nb && EPI == kEpiSwiGLU) {
         const int p = (t.b0 + static_cast<int>(rank)) * args.block_m + row;
         uint16_t* orow = static_cast<uint16_t*>(args.out) + static_cast<size_t>(p) * args.n_out;
+        // 32 h columns per TMEM wait (F is a multiple of 64, so a chunk is
+        // either wholly inside the layer or wholly past it)
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 16) {
-          uint32_t g[16], u[16];
-          ptx::tmem_ld16(t_acc + c0, g);
-          ptx::tmem_ld16(t_acc + 128 + c0, u);
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t g[32], u[32];
+          ptx::tmem_ld16(t_acc + c0, *reinterpret_cast<uint32_t(*)[16]>(&g[0]));
+          ptx::tmem_ld16(t_acc + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&g[16]));
+          ptx::tmem_ld16(t_acc + 128 + c0, *reinterpret_cast<uint32_t(*)[16]>(&u[0]));
+          ptx::tmem_ld16(t_acc + 128 + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&u[16]));
           ptx::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) asm volatile("" : "+r"(g[j]), "+r"(u[j]));  // uses stay after the wait
           const int col = t.wt * 128 + c0;
           if (col < args.n_out) {
-            uint32_t pk[8];
+            uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < 16; ++i) {
               const float h0 = silu_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
               const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
               pk[i] = pack_bf16x2(h0, h1);
             }
             uint4* dst = reinterpret_cast<uint4*>(orow + col);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           }
         }
       } else if (static_cast<int>(rank) < t.nb && EPI == kEpiRelu2) {
