@@ -44,10 +44,11 @@ METRIC = "MoE layer TFLOPS and tokens/s on 1 B200; % of bf16 tensor peak / HBM r
 
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
 # capture of that kernel on that workload (bench.py --workload <w> --steps 3
-# --warmup 3 --no-cpu-baseline under ncu --set full -k <kernel> -c 1).  An
+# --warmup 3 --no-cpu-baseline --single-copy under ncu -k <kernel>).  An
 # entry is removed whenever the kernel changes after its capture.
 NCU_TRAFFIC = {
-    ("dsv3", "gate_up_gemm"): 1_165_228_280,
+    ("decode", "fused_expert"): 201_664_000,
+    ("zipf", "gate_up_gemm"): 1_501_903_864,
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
