@@ -359,11 +359,13 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
     // counters are zero on entry and are returned to zero by its last CTA
     moe::FusedArgs fa;
     std::memset(&fa, 0, sizeof(fa));
-    // gate/up boxes: 64 gate rows + 64 up rows per tile (SwiGLU) or 128 fc1 rows
-    const uint32_t box13 = act == MOE_ACT_SWIGLU ? 64 : 128;
-    if (!encode_3d(&fa.tm_w13, w13, d, n1, E, box13) || !encode_3d(&fa.tm_w2, w2, F, d, E, 128)) return MOE_ERR_CUDA;
+    // gate/up tiles: 64 gate rows + 64 up rows (SwiGLU) or 128 fc1 rows,
+    // loaded in boxes of the kernel's box height; W2 tiles: 128 d rows
+    const uint32_t box13 = act == MOE_ACT_SWIGLU ? moe::kFusedBoxRowsGated : moe::kFusedBoxRowsRelu2;
+    const uint32_t box2 = moe::kFusedBoxRowsW2;
+    if (!encode_3d(&fa.tm_w13, w13, d, n1, E, box13) || !encode_3d(&fa.tm_w2, w2, F, d, E, box2)) return MOE_ERR_CUDA;
     if (n_shared) {
-      if (!encode_3d(&fa.tm_w13s, w13_shared, d, n1, 1, box13) || !encode_3d(&fa.tm_w2s, w2_shared, F, d, 1, 128))
+      if (!encode_3d(&fa.tm_w13s, w13_shared, d, n1, 1, box13) || !encode_3d(&fa.tm_w2s, w2_shared, F, d, 1, box2))
         return MOE_ERR_CUDA;
     } else {
       fa.tm_w13s = fa.tm_w13;

@@ -37,10 +37,12 @@
 //          count the CTA on sync[0]; the epilogue waits for all CTAs there
 //          before its first reduction (the weight stream does not wait).
 //   end:   every CTA counts itself on sync[1] once its reductions are issued;
-//          the last to arrive zeroes sync[0..1] and stores -(G-1) in sync[2],
-//          which releases the others; each of them adds 1 back to sync[2]
-//          (so every counter is zero when the kernel ends), and every CTA
-//          converts its slice of the accumulator to bf16.
+//          the last to arrive zeroes sync[0..1].  For a small output (T*d <=
+//          16384) that CTA converts the whole accumulator to bf16 and the
+//          others have already left.  Otherwise it stores -(G-1) in sync[2],
+//          which releases the others; each of them adds 1 back to sync[2] (so
+//          every counter is zero when the kernel ends), and every CTA
+//          converts its slice of the accumulator.
 //
 // Warp roles: warp 0 TMA producer (weights), warp 1 TMEM allocator + MMA
 // issuer, warps 2-5 epilogue, warps 6-9 token-row gather (cp.async; each
@@ -61,6 +63,9 @@ namespace {
 
 // In-kernel routing limit (block_m = 16 only): T*k <= 256 slots.
 constexpr int kRouteMaxS = 256;
+// Outputs of at most this many elements (T * d) are converted to bf16 by the
+// last CTA to finish, alone: the others leave without waiting for a release.
+constexpr int kLastCtaConvertMax = 16384;
 
 template <int EPI1, int TOK, bool ROUTE>
 struct FusedCfg {
@@ -92,6 +97,10 @@ struct FusedCfg {
   static_assert(TOK == 16 || TOK == 32 || TOK == 64, "token rows per tile");
   static_assert(kStageBytes % 1024 == 0 && kHBufBytes % 1024 == 0, "1024-byte aligned operand tiles");
   static_assert(kStages >= 3, "pipeline depth");
+  // every box starts on a 1024-byte swizzle atom (8 rows of 128 B) of the operand
+  static_assert(64 % kFusedBoxRowsGated == 0 && 128 % kFusedBoxRowsRelu2 == 0 && 128 % kFusedBoxRowsW2 == 0 &&
+                    kFusedBoxRowsGated % 8 == 0 && kFusedBoxRowsRelu2 % 8 == 0 && kFusedBoxRowsW2 % 8 == 0,
+                "weight boxes tile the 128-row operand on swizzle-atom boundaries");
   static_assert((2 * kStages + 9 + 2 * kD2Slots) * 8 + 16 <= kBarrierBytes, "barrier area");
   static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
@@ -283,15 +292,22 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
     __syncthreads();
     if (warp == 0) align_detail::warp_padded_scan(r_cnt, r_off, args.E, args.block_m, lane);
     if (warp == 1) align_detail::warp_padded_scan(r_cnt, r_coff, args.E, 1, lane);
-    __syncthreads();
-    for (int i = threadIdx.x; i < args.S; i += C::kNumThreads) {
-      const int e = r_ids[i];
-      int rank = 0;
-      for (int j = 0; j < i; ++j) rank += r_ids[j] == e ? 1 : 0;
-      r_rank[i] = rank;
-      r_compact[r_coff[e] + rank] = i;
-    }
     __syncthreads();  // the stage ring is free again
+    // The weight producer and the MMA issuer need only the counts and the
+    // padded offsets: they start streaming now, while the epilogue and
+    // gather warps rank the slots (for row -> slot lookups) and meet at
+    // named barrier 3.
+    if (warp >= 2) {
+      for (int i = static_cast<int>(threadIdx.x) - 64; i < args.S; i += C::kNumThreads - 64) {
+        const int e = r_ids[i];
+        int rank = 0;
+        for (int j = 0; j < i; ++j) rank += r_ids[j] == e ? 1 : 0;
+        r_rank[i] = rank;
+        r_compact[r_coff[e] + rank] = i;
+      }
+      __syncwarp();
+      asm volatile("bar.sync 3, %0;" ::"r"(C::kNumThreads - 64) : "memory");
+    }
     ntpp_v = r_off[args.E];
   } else {
     ntpp_v = *args.ntpp;
@@ -386,10 +402,17 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
             uint8_t* sW = smem + stage * C::kStageBytes;
             ptx::mbar_arrive_expect_tx(&full[stage], C::kWBytes);
             if (C::kGated) {
-              ptx::tma_load_3d_hint(sW, tm, &full[stage], s * 64, t.wt * 64, e, evict_first);
-              ptx::tma_load_3d_hint(sW + 64 * 128, tm, &full[stage], s * 64, args.F + t.wt * 64, e, evict_first);
+              // 64 gate rows into operand rows 0-63, the matching up rows into 64-127
+#pragma unroll
+              for (int r = 0; r < 64; r += kFusedBoxRowsGated) {
+                ptx::tma_load_3d_hint(sW + r * 128, tm, &full[stage], s * 64, t.wt * 64 + r, e, evict_first);
+                ptx::tma_load_3d_hint(sW + (64 + r) * 128, tm, &full[stage], s * 64, args.F + t.wt * 64 + r, e,
+                                      evict_first);
+              }
             } else {
-              ptx::tma_load_3d_hint(sW, tm, &full[stage], s * 64, t.wt * 128, e, evict_first);
+#pragma unroll
+              for (int r = 0; r < 128; r += kFusedBoxRowsRelu2)
+                ptx::tma_load_3d_hint(sW + r * 128, tm, &full[stage], s * 64, t.wt * 128 + r, e, evict_first);
             }
             advance();
           }
@@ -404,7 +427,10 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
             const int di = d_tile(dk, rot, n_d);
             uint8_t* sW = smem + stage * C::kStageBytes;
             ptx::mbar_arrive_expect_tx(&full[stage], C::kWBytes);
-            ptx::tma_load_3d_hint(sW, tm, &full[stage], t.wt * C::kH + kk * 64, di * 128, e, evict_first);
+#pragma unroll
+            for (int r = 0; r < 128; r += kFusedBoxRowsW2)
+              ptx::tma_load_3d_hint(sW + r * 128, tm, &full[stage], t.wt * C::kH + kk * 64, di * 128 + r, e,
+                                    evict_first);
             advance();
           }
         }
@@ -766,36 +792,47 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
   __syncwarp();
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
-    ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, 512);
-  }
   // ---- grid end: all reductions issued -> convert the accumulator to bf16.
-  // sync[1] counts the CTAs that have issued all their reductions.  The last
-  // one to arrive returns sync[0] and sync[1] to zero and releases the others
-  // by storing -(G-1) in sync[2]; each released CTA adds 1 to sync[2] as it
-  // goes (fire-and-forget), so all three counters are zero again when the
-  // kernel completes and no CTA waits on another round of atomics to exit.
+  // sync[1] counts the CTAs that have issued all their reductions; the last
+  // one to arrive returns sync[0] and sync[1] to zero.  A small output is
+  // then converted by that CTA alone while the others leave.  Otherwise the
+  // last CTA releases the others by storing -(G-1) in sync[2]; each released
+  // CTA adds 1 to sync[2] as it goes (fire-and-forget) and converts its slice,
+  // so all three counters are zero again when the kernel completes and no CTA
+  // waits on another round of atomics to exit.
+  const bool last_converts = nacc <= kLastCtaConvertMax;
   if (threadIdx.x == 0) {
     const int G = static_cast<int>(gridDim.x);
     bool all = true;
+    int mode = 0;  // 0: leave, 1: convert this CTA's slice, 2: convert everything
     if (ptx::atom_acq_rel_gpu_add(args.sync + 1, 1) == G - 1) {  // releases this CTA's reductions
       args.sync[0] = 0;
       args.sync[1] = 0;
-      ptx::st_release_gpu(args.sync + 2, -(G - 1));
-    } else {
+      if (last_converts) {
+        mode = 2;
+      } else {
+        ptx::st_release_gpu(args.sync + 2, -(G - 1));
+        mode = 1;
+      }
+    } else if (!last_converts) {
       all = spin_until_nonzero(args.sync + 2, abort_flag);
       if (all) ptx::red_relaxed_gpu_add(args.sync + 2, 1);
+      mode = all ? 1 : 0;
     }
     if (!all) fail();
-    *flag = all ? 1 : 0;
+    *flag = mode;
+  }
+  if (warp == 1) {  // TMEM is freed while thread 0 waits at the grid barrier
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, 512);
   }
   __syncthreads();
   if (*flag) {
     const int per = ((nacc + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x) + 3) & ~3;
-    const int lo = static_cast<int>(blockIdx.x) * per;
-    const int hi = min(nacc, lo + per);
+    const int lo = *flag == 2 ? 0 : static_cast<int>(blockIdx.x) * per;
+    const int hi = *flag == 2 ? nacc : min(nacc, lo + per);
     const bool vec = (reinterpret_cast<uintptr_t>(args.out) & 7) == 0;
+#pragma unroll 4
     for (int e = lo + 4 * static_cast<int>(threadIdx.x); e < hi; e += 4 * C::kNumThreads) {
       if (vec && e + 4 <= hi) {
         const float4 a = __ldcg(reinterpret_cast<const float4*>(args.acc + e));
