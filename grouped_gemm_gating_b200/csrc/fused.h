@@ -47,10 +47,9 @@ struct FusedArgs {
 };
 
 // Rows per TMA box of the fused kernel's weight tensor maps.  A stage of 128
-// weight rows is filled by several boxes: 32-row boxes for the gate/up rows
-// of SwiGLU (64 gate rows then the matching 64 up rows), 64-row boxes for
-// relu^2 fc1 rows and for W2 rows.  Shorter boxes stream faster on the decode
-// shape (measured: 43.7 -> 43.2 us per step); 16-row boxes are far slower.
+// weight rows (gate, up or fc1 rows of one 64-wide K block, or W2 rows) is
+// filled by several boxes.  Boxes shorter than a stage streamed faster on the
+// decode shape; 16-row boxes were far slower.
 constexpr int kFusedBoxRowsGated = 32;
 constexpr int kFusedBoxRowsRelu2 = 64;
 constexpr int kFusedBoxRowsW2 = 64;

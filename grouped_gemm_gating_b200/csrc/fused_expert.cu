@@ -12,14 +12,14 @@
 // anything that stalls that stream.
 //
 // Split along d_ff.  A tile is (block of block_m token rows, one slice of
-// the hidden dimension: 64 h columns for SwiGLU, 128 for relu^2).  A CTA
+// 128 h columns).  A CTA
 //   1. computes the slice's pre-activations with the weights as the MMA's
-//      M = 128 rows (SwiGLU stacks 64 gate rows on the matching 64 up rows;
-//      the epilogue hands the up half to the gate half through shared
-//      memory),
+//      M = 128 rows (SwiGLU: the 128 gate rows and the matching 128 up rows
+//      of each K block are two stages, multiplied into two accumulators),
 //   2. writes h = act(...) for the slice into shared memory, already in the
 //      K-major 128-byte-swizzled layout the tensor core reads,
-//   3. streams the matching columns of W2 for every 128-row d tile and
+//   3. streams the matching columns of W2 (256 contiguous bytes of every
+//      row, as two 64-column K blocks) for every 128-row d tile and
 //      multiplies them by that h slice,
 //   4. adds topk_weight * partial into an fp32 [T, d] accumulator with
 //      red.global.add (fire-and-forget).
@@ -70,26 +70,30 @@ constexpr int kLastCtaConvertMax = 16384;
 template <int EPI1, int TOK, bool ROUTE>
 struct FusedCfg {
   static constexpr bool kGated = (EPI1 == kEpiSwiGLU);
-  static constexpr int kH = kGated ? 64 : 128;  // h columns per tile
+  static constexpr int kH = 128;                // h columns per tile
   static constexpr int kHk = kH / 64;           // 64-wide K blocks of the down GEMM per tile
+  // gate/up stages per 64-wide K block: SwiGLU loads the slice's 128 gate
+  // rows and then its 128 up rows, each multiplied into its own accumulator
+  static constexpr int kGU = kGated ? 2 : 1;
+  static constexpr int kAcc1 = kGU * TOK;       // TMEM columns of one tile's gate/up accumulator(s)
+  static constexpr int kBoxRows = kGated ? kFusedBoxRowsGated : kFusedBoxRowsRelu2;
   static constexpr int kWBytes = 128 * 128;     // 128 weight rows x 64 bf16 per stage
   static constexpr int kXBytes = TOK * 128;     // token rows x 64 bf16 per stage
   static constexpr int kStageBytes = kWBytes + kXBytes;
   static constexpr int kHBufBytes = kHk * TOK * 128;            // one h slice (B operand of the down GEMM)
-  static constexpr int kXbufBytes = kGated ? 64 * TOK * 4 : 0;  // up half handed to the gate half
   static constexpr int kTokBytes = 2 * 2 * 64 * 4;              // token id and weight per row, two tiles
   static constexpr int kBarrierBytes = 1024;
   // routing results kept for the whole kernel: expert and weight of every
   // slot, its rank among its expert's slots, the slots in expert order, and
   // per expert its slot count and padded / unpadded offsets
   static constexpr int kRouteBytes = ROUTE ? (4 * kRouteMaxS + 3 * (MOE_MAX_EXPERTS + 1) + 5) * 4 : 0;
-  static constexpr int kFixedBytes = 2 * kHBufBytes + kXbufBytes + kTokBytes + kBarrierBytes + kRouteBytes + 1024;
+  static constexpr int kFixedBytes = 2 * kHBufBytes + kTokBytes + kBarrierBytes + kRouteBytes + 1024;
   static constexpr int kStagesRaw = (227 * 1024 - kFixedBytes) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
   // Down-GEMM accumulators: groups of kGroup d tiles (64 TMEM columns) form
   // one slot of a TMEM ring, so the epilogue synchronises once per group.
   static constexpr int kGroup = 64 / TOK;
-  static constexpr int kD2Raw = (512 - 2 * TOK) / 64;
+  static constexpr int kD2Raw = (512 - 2 * kAcc1) / 64;
   static constexpr int kD2Slots = kD2Raw > 8 ? 8 : kD2Raw;
   static constexpr int kNumThreads = 320;
   static constexpr int kSmemBytes = kStages * kStageBytes + kFixedBytes;
@@ -98,7 +102,7 @@ struct FusedCfg {
   static_assert(kStageBytes % 1024 == 0 && kHBufBytes % 1024 == 0, "1024-byte aligned operand tiles");
   static_assert(kStages >= 3, "pipeline depth");
   // every box starts on a 1024-byte swizzle atom (8 rows of 128 B) of the operand
-  static_assert(64 % kFusedBoxRowsGated == 0 && 128 % kFusedBoxRowsRelu2 == 0 && 128 % kFusedBoxRowsW2 == 0 &&
+  static_assert(128 % kFusedBoxRowsGated == 0 && 128 % kFusedBoxRowsRelu2 == 0 && 128 % kFusedBoxRowsW2 == 0 &&
                     kFusedBoxRowsGated % 8 == 0 && kFusedBoxRowsRelu2 % 8 == 0 && kFusedBoxRowsW2 % 8 == 0,
                 "weight boxes tile the 128-row operand on swizzle-atom boundaries");
   static_assert((2 * kStages + 9 + 2 * kD2Slots) * 8 + 16 <= kBarrierBytes, "barrier area");
@@ -192,9 +196,8 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
   using C = FusedCfg<EPI1, TOK, ROUTE>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* hbuf = smem + C::kStages * C::kStageBytes;                // [2][kHk][TOK rows x 128 B]
-  float* xbuf = reinterpret_cast<float*>(hbuf + 2 * C::kHBufBytes);  // [TOK][64]
-  int* tok_s = reinterpret_cast<int*>(hbuf + 2 * C::kHBufBytes + C::kXbufBytes);  // [2][64]
+  uint8_t* hbuf = smem + C::kStages * C::kStageBytes;        // [2][kHk][TOK rows x 128 B]
+  int* tok_s = reinterpret_cast<int*>(hbuf + 2 * C::kHBufBytes);  // [2][64]
   float* w_s = reinterpret_cast<float*>(tok_s + 2 * 64);                           // [2][64]
   uint64_t* full = reinterpret_cast<uint64_t*>(w_s + 2 * 64);
   uint64_t* empty = full + C::kStages;
@@ -355,6 +358,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
                        : 0;
   const int nk1 = args.d / 64;
   const int nk2 = n_d * C::kHk;  // down-GEMM stages per tile
+  const int ng = nk1 * C::kGU;   // gate/up stages per tile
   const int nacc = args.T * args.d;
 
   auto fail = [&]() {
@@ -398,22 +402,15 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
           const TileInfo t = tile_of(i);
           const int e = expert_of(t);
           const CUtensorMap* tm = t.shared_blk ? &args.tm_w13s : &args.tm_w13;
-          for (int s = 0; s < nk1 && acquire(); ++s) {
+          for (int s = 0; s < ng && acquire(); ++s) {
+            // K block s / kGU; SwiGLU: gate rows [wt*128, +128), then up rows [F + wt*128, +128)
+            const int kb = s / C::kGU;
+            const int row0 = (C::kGated && s != kb * C::kGU ? args.F : 0) + t.wt * C::kH;
             uint8_t* sW = smem + stage * C::kStageBytes;
             ptx::mbar_arrive_expect_tx(&full[stage], C::kWBytes);
-            if (C::kGated) {
-              // 64 gate rows into operand rows 0-63, the matching up rows into 64-127
 #pragma unroll
-              for (int r = 0; r < 64; r += kFusedBoxRowsGated) {
-                ptx::tma_load_3d_hint(sW + r * 128, tm, &full[stage], s * 64, t.wt * 64 + r, e, evict_first);
-                ptx::tma_load_3d_hint(sW + (64 + r) * 128, tm, &full[stage], s * 64, args.F + t.wt * 64 + r, e,
-                                      evict_first);
-              }
-            } else {
-#pragma unroll
-              for (int r = 0; r < 128; r += kFusedBoxRowsRelu2)
-                ptx::tma_load_3d_hint(sW + r * 128, tm, &full[stage], s * 64, t.wt * 128 + r, e, evict_first);
-            }
+            for (int r = 0; r < 128; r += C::kBoxRows)
+              ptx::tma_load_3d_hint(sW + r * 128, tm, &full[stage], kb * 64, row0 + r, e, evict_first);
             advance();
           }
         }
@@ -456,16 +453,18 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
           const uint32_t bph = static_cast<uint32_t>((i >> 1) & 1);
           if (!wait(&d1_empty[b], bph ^ 1u)) break;
           ptx::tc_fence_after();
-          const uint32_t d1 = tmem_base + static_cast<uint32_t>(b * TOK);
-          for (int kb = 0; kb < nk1; ++kb) {
+          const uint32_t d1 = tmem_base + static_cast<uint32_t>(b * C::kAcc1);
+          for (int s = 0; s < ng; ++s) {
             if (!wait(&full[stage], phase)) break;
             ptx::tc_fence_after();
             ptx::fence_proxy_async_smem();  // token rows were written by cp.async
+            const int kb = s / C::kGU;
+            const uint32_t acc = d1 + static_cast<uint32_t>((s - kb * C::kGU) * TOK);  // gate or up accumulator
             const uint32_t sW = ptx::smem_u32(smem + stage * C::kStageBytes);
             const uint32_t sX = sW + C::kWBytes;
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              ptx::mma_bf16(d1, ptx::sw128_kmajor_desc(sW + q * 32), ptx::sw128_kmajor_desc(sX + q * 32), C::kIdesc,
+              ptx::mma_bf16(acc, ptx::sw128_kmajor_desc(sW + q * 32), ptx::sw128_kmajor_desc(sX + q * 32), C::kIdesc,
                             (kb | q) != 0 ? 1u : 0u);
             ptx::mma_commit(&empty[stage]);
             if (++stage == C::kStages) {
@@ -489,7 +488,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
             if (!wait(&d2_empty[slot], sph ^ 1u)) break;
             ptx::tc_fence_after();
             for (int w = 0; ok && w < C::kGroup && g * C::kGroup + w < n_d; ++w) {
-              const uint32_t d2 = tmem_base + static_cast<uint32_t>(2 * TOK + slot * 64 + w * TOK);
+              const uint32_t d2 = tmem_base + static_cast<uint32_t>(2 * C::kAcc1 + slot * 64 + w * TOK);
               for (int kk = 0; kk < C::kHk; ++kk) {
                 if (!wait(&full[stage], phase)) break;
                 ptx::tc_fence_after();
@@ -584,49 +583,40 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
           break;
         }
         ptx::tc_fence_after();
-        // ---- gate/up accumulator -> h slice in shared memory (MMA operand layout)
-        const uint32_t t1 = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * TOK);
+        // ---- gate/up accumulator(s) -> h slice in shared memory (MMA operand
+        // layout).  Thread `row` owns h column row of the slice: the gate (or
+        // fc1) row `row` and, for SwiGLU, the matching up row are its TMEM lane
+        // in the two accumulators.
+        const uint32_t t1 =
+            tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * C::kAcc1);
         uint8_t* hb = hbuf + b * C::kHBufBytes;
-        if (C::kGated) {
-          float gate[TOK];
+        {
+          const int c = row & 63, kk = row >> 6;  // h column within its 64-wide K block
+          // a slice past d_ff (the last slice when F % 128 == 64) reads other
+          // rows or zeros there: its h columns are set to zero
+          const bool live = t.wt * C::kH + row < args.F;
 #pragma unroll
           for (int j0 = 0; j0 < TOK; j0 += 16) {
-            uint32_t a[16];
+            uint32_t a[16], u[16];
             ptx::tmem_ld16(t1 + j0, a);
+            if (C::kGated) ptx::tmem_ld16(t1 + TOK + j0, u);
             ptx::tmem_wait_ld();
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
-              if (q >= 2)
-                xbuf[(j0 + jj) * 64 + (row - 64)] = __uint_as_float(a[jj]);
-              else
-                gate[j0 + jj] = __uint_as_float(a[jj]);
+              asm volatile("" : "+r"(a[jj]));  // uses stay after the wait
+              if (C::kGated) asm volatile("" : "+r"(u[jj]));
             }
-          }
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&d1_empty[b]);
-          epilogue_sync();
-          if (q < 2) {
-            const int c = row;  // h column within the slice (0..63)
-#pragma unroll
-            for (int j = 0; j < TOK; ++j) {
-              const float hv = silu_fast(gate[j]) * xbuf[j * 64 + c];
-              const uint32_t off = (j >> 3) * 1024 + (j & 7) * 128 + (((c >> 3) ^ (j & 7)) << 4) + (c & 7) * 2;
-              *reinterpret_cast<uint16_t*>(hb + off) = float_to_bf16_bits(hv);
-            }
-          }
-        } else {
-          const int c = row & 63, kk = row >> 6;  // h column within its 64-wide K block
-#pragma unroll
-          for (int j0 = 0; j0 < TOK; j0 += 16) {
-            uint32_t a[16];
-            ptx::tmem_ld16(t1 + j0, a);
-            ptx::tmem_wait_ld();
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
               const int j = j0 + jj;
-              float v = fmaxf(__uint_as_float(a[jj]), 0.0f);
-              v *= v;
+              float v;
+              if (C::kGated) {
+                v = silu_fast(__uint_as_float(a[jj])) * __uint_as_float(u[jj]);
+              } else {
+                v = fmaxf(__uint_as_float(a[jj]), 0.0f);
+                v *= v;
+              }
+              if (!live) v = 0.0f;
               const uint32_t off =
                   kk * TOK * 128 + (j >> 3) * 1024 + (j & 7) * 128 + (((c >> 3) ^ (j & 7)) << 4) + (c & 7) * 2;
               *reinterpret_cast<uint16_t*>(hb + off) = float_to_bf16_bits(v);
@@ -677,7 +667,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
           ptx::tc_fence_after();
           const int n_w = min(C::kGroup, n_d - g * C::kGroup);
           const uint32_t t2 =
-              tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(2 * TOK + slot * 64);
+              tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(2 * C::kAcc1 + slot * 64);
           uint32_t a[C::kGroup][TOK];
 #pragma unroll
           for (int w = 0; w < C::kGroup; ++w) {
@@ -765,13 +755,14 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
           src[r] = args.x + static_cast<size_t>(tok) * args.d + chunk * 8;
           nbytes[r] = valid ? 16u : 0u;
         }
-        for (int s = 0; s < nk1 && acquire(); ++s) {
+        for (int s = 0; s < ng && acquire(); ++s) {
+          const int kb = s / C::kGU;  // SwiGLU: the gate and the up stage of a K block carry the same rows
           const uint32_t sX = ptx::smem_u32(smem + stage * C::kStageBytes + C::kWBytes);
 #pragma unroll
           for (int r = 0; r < kRowsPerThread; ++r) {
             const int row = r0 + 16 * r;
             const uint32_t dst = sX + (row >> 3) * 1024 + (row & 7) * 128 + ((chunk ^ (row & 7)) << 4);
-            ptx::cp_async_16(dst, src[r] + s * 64, nbytes[r]);
+            ptx::cp_async_16(dst, src[r] + kb * 64, nbytes[r]);
           }
           ptx::cp_async_arrive_noinc(&full[stage]);
           advance();
@@ -869,8 +860,8 @@ cudaError_t launch_fused_variant(const FusedArgs& args, int grid, cudaStream_t s
 bool fused_expert_supported(int block_m) { return block_m == 16 || block_m == 32 || block_m == 64; }
 
 int64_t fused_expert_max_tiles(int act_epi, int total_blocks_max, int F) {
-  const int h = act_epi == kEpiSwiGLU ? 64 : 128;
-  return static_cast<int64_t>(total_blocks_max) * ((F + h - 1) / h);
+  (void)act_epi;  // 128 h columns per tile for both activations
+  return static_cast<int64_t>(total_blocks_max) * ((F + 127) / 128);
 }
 
 bool fused_routing_supported(int T, int k, int E, int n_group, int block_m) {
