@@ -47,7 +47,6 @@ METRIC = "MoE layer TFLOPS and tokens/s on 1 B200; % of bf16 tensor peak / HBM r
 # --warmup 3 --no-cpu-baseline --single-copy under ncu -k <kernel>).  An
 # entry is removed whenever the kernel changes after its capture.
 NCU_TRAFFIC = {
-    ("decode", "fused_expert"): 201_664_000,
     ("zipf", "gate_up_gemm"): 1_501_903_864,
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
