@@ -26,6 +26,8 @@
 //   warp 0       TMA producer: weight tiles (and h tiles for the down GEMM)
 //   warp 1       TMEM allocator and MMA issuer (one thread)
 //   warps 2..5   epilogue: TMEM -> registers -> activation -> bf16 -> global
+//                (down GEMM: warps 2..9, two per TMEM lane quadrant, each on
+//                half of the tile's 256 columns)
 //   warps 6..9   gate/up GEMM only: row gather of x through sorted_token_ids
 //                with 16-byte cp.async into the 128B-swizzled layout (padding
 //                rows zero-filled); each thread's copies of a stage arrive on
@@ -61,13 +63,16 @@ struct GemmCfg {
   static constexpr int kAccCols = 256;
   static constexpr int kTmemCols = 512;
   // gate/up: warps 6-9 gather token rows, warp 10 zeroes the accumulator
-  static constexpr int kNumThreads = kGather ? 352 : 192;
+  // epilogue warps: the down GEMM's scatter-reduce bounds that kernel, so it
+  // runs two warps per TMEM lane quadrant, each on half of the tile's columns
+  static constexpr int kEpiWarps = kGather ? 4 : 8;
+  static constexpr int kNumThreads = kGather ? 352 : 64 + 32 * kEpiWarps;
   static constexpr uint32_t kTxBytes = kWBytes + (kGather ? 0 : kXBytes);
   static constexpr int kBarrierBytes = 256;
   // down GEMM: per epilogue warp a 32 x 33 fp32 transpose buffer, so the
   // reduction is issued as full 128-byte row segments
   static constexpr int kRedStride = 33;
-  static constexpr int kRedBytes = kGather ? 0 : 4 * 32 * kRedStride * 4;
+  static constexpr int kRedBytes = kGather ? 0 : kEpiWarps * 32 * kRedStride * 4;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes + kRedBytes;
   static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(128, 256);
 
@@ -134,7 +139,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&tfull[b], 1);
-      ptx::mbar_init(&tempty[b], 4);
+      ptx::mbar_init(&tempty[b], C::kEpiWarps);
     }
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -250,7 +255,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
         }
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + C::kEpiWarps) {
     // ------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int row = q * 32 + lane;
@@ -334,11 +339,13 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
         // warp's transpose buffer, then 8 lanes cover one row's 128 bytes and
         // one red.v4 instruction adds 4 whole row segments
         float* stg = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + C::kBarrierBytes) +
-                     q * 32 * C::kRedStride;
+                     (warp - 2) * 32 * C::kRedStride;
         const int rr = lane >> 3;        // row within a group of 4
         const int cc = (lane & 7) * 4;   // column within the 32-column chunk
+        // columns of this warp: all 256, or its half when two warps share a quadrant
+        const int c_lo = C::kEpiWarps == 8 ? ((warp - 2) >> 2) * 128 : 0;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 256; c0 += 32) {
+        for (int c0 = c_lo; c0 < c_lo + 256 * 4 / C::kEpiWarps; c0 += 32) {
           uint32_t a[32];
           ptx::tmem_ld16(t_acc + c0, *reinterpret_cast<uint32_t(*)[16]>(&a[0]));
           ptx::tmem_ld16(t_acc + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&a[16]));
