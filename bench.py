@@ -47,7 +47,8 @@ METRIC = "MoE layer TFLOPS and tokens/s on 1 B200; % of bf16 tensor peak / HBM r
 # --warmup 3 --no-cpu-baseline --single-copy under ncu -k <kernel>).  An
 # entry is removed whenever the kernel changes after its capture.
 NCU_TRAFFIC = {
-    ("zipf", "gate_up_gemm"): 1_501_903_864,
+    ("decode", "fused_expert"): 202_819_328,
+    ("zipf", "gate_up_gemm"): 1_496_556_680,
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
