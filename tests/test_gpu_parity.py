@@ -47,6 +47,13 @@ SMALL = {
                                                    block_m=16, seed=2010),
     "shared_bm32_sep_combine": CFG["dsv3"].with_(name="shared_bm32_sep_combine", T=100, d=320, F=128,
                                                  block_m=32, seed=2011),
+    # the header's limits: E = 256 experts, top_k = 16, T*k = 256 slots (the
+    # largest one-launch moe_layer), grouped routing, a last h slice past d_ff
+    "limits_e256_k16": CFG["decode"].with_(name="limits_e256_k16", T=16, d=256, F=192, E=256, k=16, n_group=8,
+                                           topk_group=4, seed=2014, logits_kind="normal"),
+    # SwiGLU in the fused kernel with 64-token blocks and a half-empty last slice
+    "swap_bm64_swiglu": CFG["tiny"].with_(name="swap_bm64_swiglu", T=150, d=192, F=320, E=6, k=2, block_m=64,
+                                          seed=2015, logits_kind="normal"),
 }
 
 
@@ -324,8 +331,8 @@ def test_route_align_matches_separate_calls(name, T):
 
 
 @pytest.mark.parametrize("name,one_launch", [("decode", True), ("tiny", True), ("shared_bm16_fused_combine", True),
-                                             ("decode_d512", True), ("relu2_small", False), ("dsv3_small", False),
-                                             ("swap_bm32", False)])
+                                             ("decode_d512", True), ("limits_e256_k16", True), ("relu2_small", False),
+                                             ("dsv3_small", False), ("swap_bm32", False)])
 def test_layer_entry_matches_separate_calls(name, one_launch):
     """moe_layer writes the same routing / align outputs as moe_route_align
     (bit for bit) and the same output as moe_forward (up to the reordering
