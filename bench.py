@@ -48,6 +48,8 @@ METRIC = "MoE layer TFLOPS and tokens/s on 1 B200; % of bf16 tensor peak / HBM r
 # entry is removed whenever the kernel changes after its capture.
 NCU_TRAFFIC = {
     ("decode", "fused_expert"): 202_819_328,
+    ("relu2", "fused_expert"): 2_642_480_832,
+    ("dsv3", "gate_up_gemm"): 1_020_184_832,
     ("zipf", "gate_up_gemm"): 1_496_556_680,
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
