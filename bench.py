@@ -211,7 +211,9 @@ def time_oracle(inp: W.MoEInputs, steps: int, warmup: int, min_seconds: float = 
 
 # --------------------------------------------------------------------------
 
-def dist_setup(gpus: int):
+def dist_setup(gpus: int, backend: str = "nccl"):
+    """Rank plumbing for one process per GPU (torchrun env).  "nccl" binds
+    the process to its GPU; "gloo" runs the same host logic on the CPU."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -223,11 +225,14 @@ def dist_setup(gpus: int):
         import datetime
 
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
         pg = dist
-    else:
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return world, rank, local, pg
 
@@ -237,13 +242,21 @@ def barrier(pg):
         pg.barrier()
 
 
-def max_over_ranks(pg, value: float) -> float:
+def max_over_ranks(pg, value: float, device: str = "cuda") -> float:
+    """The slowest rank's time: every rank runs the same steps, the job
+    takes as long as its slowest replica."""
     if pg is None:
         return value
     import torch
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=device)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_step: float, ms_total: float, steps: int) -> float:
+    """Throughput of all replicas together: world x the per-replica FLOPs of
+    a step over the (max-over-ranks) time of one step."""
+    return world * flops_per_step / (ms_total / steps / 1e3) / 1e12
 
 
 def run_ours(args):
@@ -429,8 +442,8 @@ def run_ours(args):
 
     alg = algorithmic(cfg, topk_ids)
     sec_per_step = total_ms / args.steps / 1e3
-    value = world * alg["flops_total"] / sec_per_step / 1e12
-    e2e_value = world * alg["flops_total"] / (e2e_ms / args.steps / 1e3) / 1e12
+    value = whole_job_tflops(world, alg["flops_total"], total_ms, args.steps)
+    e2e_value = whole_job_tflops(world, alg["flops_total"], e2e_ms, args.steps)
 
     # ---- roofline of the dominant kernel ----
     peaks, peak_src = load_peaks()

@@ -1,0 +1,64 @@
+"""Multi-process host logic of bench.py on CPU (gloo, world size 2).
+
+The layer does not shard: under torchrun every rank runs an independent
+replica, the ranks meet at barriers, the reported time is the slowest
+rank's and the throughput counts every replica's work.  These checks run
+that plumbing with the gloo backend, without a GPU.
+"""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    w, r, local, pg = bench.dist_setup(world, backend="gloo")
+    assert (w, r, local) == (world, rank, rank) and pg is not None
+    bench.barrier(pg)
+    # rank r took (r + 1) ms per step: the job's time is the slowest rank's
+    slowest = bench.max_over_ranks(pg, float(rank + 1), device="cpu")
+    value = bench.whole_job_tflops(w, 2.0e12, slowest * 10, 10)
+    bench.barrier(pg)
+    pg.destroy_process_group()
+    with open(os.path.join(out_dir, f"rank{rank}.txt"), "w") as f:
+        f.write(f"{slowest} {value}\n")
+
+
+def test_two_gloo_ranks_take_the_slowest_time_and_sum_the_work(tmp_path):
+    world = 2
+    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    for rank in range(world):
+        slowest, value = map(float, (tmp_path / f"rank{rank}.txt").read_text().split())
+        assert slowest == pytest.approx(2.0)               # max over ranks of 1 and 2 ms
+        assert value == pytest.approx(2 * 2.0e12 / 2e-3 / 1e12)  # both replicas' FLOPs over 2 ms
+
+
+def test_single_process_needs_no_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(None, 3.5) == 3.5
+    assert bench.whole_job_tflops(1, 1e12, 10.0, 10) == pytest.approx(1000.0)
+
+
+def test_reference_arm_prints_on_rank_zero_only(monkeypatch, capsys):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    bench.main(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3", "--workload", "tiny"])
+    assert capsys.readouterr().out == ""
