@@ -526,6 +526,62 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
 
 extern "C" {
 
+moe_status moe_router(const uint16_t* x, int T, int d, const uint16_t* w_gate, int E, int k, int n_group,
+                      int topk_group, moe_group_score group_score, int renormalize, float routed_scaling,
+                      float* logits, int32_t* topk_ids, float* topk_weights, int32_t* dev_status,
+                      moe_stream_t stream) {
+  moe_status st = check_route_args(T, E, k, n_group, topk_group, group_score, routed_scaling);
+  if (st != MOE_OK) return st;
+  if (d < 64 || d % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  if (E > moe::kRouterMaxE || k > moe::kRouterMaxK) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return finish(cudaSuccess, 0);
+  if (!x || !w_gate || !logits || !topk_ids || !topk_weights) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate) || (reinterpret_cast<uintptr_t>(logits) & 3u) != 0)
+    return MOE_ERR_INVALID_ARG;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int num_sms = num_sms_current_device();
+  if (num_sms <= 0) return MOE_ERR_CUDA;
+  moe::GemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  // W_g as the single weight matrix {K = d, rows = E, 1} with 256-row boxes
+  // (rows past E read as zeros); x rows by 2-D TMA, 128 tokens per block
+  if (!encode_3d(&a.tm_ws, w_gate, d, static_cast<uint64_t>(E), 1, moe::kRouterMaxE)) return MOE_ERR_CUDA;
+  a.tm_w = a.tm_ws;
+  if (!encode_2d(&a.tm_x, x, d, static_cast<uint64_t>(T), 128)) return MOE_ERR_CUDA;
+  a.status = dev_status;
+  a.T = T;
+  a.k = k;
+  a.S = T * k;
+  a.E = E;
+  a.K = d;
+  a.n_out = E;
+  a.block_m = 128;
+  a.max_routed_blocks = 0;
+  a.n_shared_blocks = (T + 127) / 128;
+  a.logits = logits;
+  // grouped selection runs in the routing kernel on the written logits
+  const bool fused_topk = n_group == 1;
+  a.r_ids = fused_topk ? topk_ids : nullptr;
+  a.r_w = topk_weights;
+  a.r_renorm = renormalize ? 1 : 0;
+  a.r_scaling = routed_scaling;
+  const int grid = a.n_shared_blocks < num_sms ? a.n_shared_blocks : num_sms;
+  int launches = 0;
+  cudaError_t err;
+  {
+    StageScope scope(8, s);
+    err = moe::launch_grouped_gemm(moe::kEpiRouter, a, grid, s);
+  }
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  ++launches;
+  if (!fused_topk) {
+    StageScope scope(0, s);
+    err = moe::launch_route(logits, T, E, k, n_group, topk_group, static_cast<int>(group_score),
+                            renormalize ? 1 : 0, routed_scaling, topk_ids, topk_weights, dev_status, s, &launches);
+  }
+  return finish(err, launches);
+}
+
 moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, const uint16_t* w2, int E, int F,
                        const uint16_t* w13_shared, const uint16_t* w2_shared, int n_shared,
                        const float* topk_weights, int k, const int32_t* sorted_token_ids,

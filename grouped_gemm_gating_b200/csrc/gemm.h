@@ -9,7 +9,8 @@ namespace moe {
 enum EpiKind : int {
   kEpiSwiGLU = 0,  // gate/up GEMM, h = silu(gate) * up
   kEpiRelu2 = 1,   // fc1 GEMM, h = max(a, 0)^2
-  kEpiScale = 2    // down GEMM, acc[token] += topk_weight(row) * row result (fp32)
+  kEpiScale = 2,   // down GEMM, acc[token] += topk_weight(row) * row result (fp32)
+  kEpiRouter = 3   // router GEMM, logits = x . W_g^T (fp32), top-k gating of each row
 };
 
 // Arguments of one grouped GEMM launch (token-major tiles, block_m = 128).
@@ -39,6 +40,15 @@ struct GemmArgs {
   int max_routed_blocks;
   int n_shared_blocks;
   int pass_cols;        // output-column tiles per pass of the tile walk (0: one pass)
+  // router GEMM only: fp32 logits [T, E]; when r_ids is set, the top-k of
+  // every row (ids [T, k], weights [T, k]) with the routing kernel's order
+  // (logit desc, id asc) and weights (softmax over the chosen k when
+  // r_renorm, else the full softmax at the chosen ids) x r_scaling
+  float* logits;
+  int32_t* r_ids;
+  float* r_w;
+  int r_renorm;
+  float r_scaling;
 };
 
 // Rows of one weight TMA box (= output columns of one tile) for an epilogue.
@@ -46,6 +56,10 @@ int gemm_box_rows(int epi);
 // Upper bound on tiles of one launch, for grid sizing.
 int64_t gemm_max_tiles(int epi, int max_routed_blocks, int n_shared_blocks, int n_out);
 cudaError_t launch_grouped_gemm(int epi, const GemmArgs& args, int grid, cudaStream_t stream);
+// Router GEMM: x [T, K] (tm_x, 2-D {K, T}, 64 x 128 boxes) times W_g [E, K]
+// (tm_ws, 3-D {K, E, 1}, 256-row boxes), E <= 256, top-k k <= 16.
+constexpr int kRouterMaxE = 256;
+constexpr int kRouterMaxK = 16;
 
 // The same GEMMs on CTA pairs (cluster of two, tcgen05 cta_group::2): args
 // as for launch_grouped_gemm, except that tm_w / tm_ws use 128-row boxes and

@@ -40,6 +40,8 @@
 // tmem-full/tmem-empty mbarriers.  Every wait is
 // bounded in time; on expiry the kernel records MOE_ERR_DEVICE_TIMEOUT and
 // all roles leave their loops so the CTA frees its TMEM and exits.
+#include <cmath>
+
 #include "common.cuh"
 #include "gemm.h"
 #include "ptx.cuh"
@@ -50,7 +52,7 @@ template <int EPI>
 struct GemmCfg {
   static constexpr int TOK = 128;  // token rows per tile
   static constexpr bool kGated = (EPI == kEpiSwiGLU);
-  static constexpr bool kGather = (EPI != kEpiScale);
+  static constexpr bool kGather = (EPI == kEpiSwiGLU || EPI == kEpiRelu2);
   static constexpr int kBoxRows = kGated ? 128 : 256;
   static constexpr int kBoxes = kGated ? 2 : 1;
   static constexpr int kWRows = kBoxRows * kBoxes;
@@ -65,14 +67,14 @@ struct GemmCfg {
   // gate/up: warps 6-9 gather token rows, warp 10 zeroes the accumulator
   // epilogue warps: the down GEMM's scatter-reduce bounds that kernel, so it
   // runs two warps per TMEM lane quadrant, each on half of the tile's columns
-  static constexpr int kEpiWarps = kGather ? 4 : 8;
+  static constexpr int kEpiWarps = EPI == kEpiScale ? 8 : 4;
   static constexpr int kNumThreads = kGather ? 352 : 64 + 32 * kEpiWarps;
   static constexpr uint32_t kTxBytes = kWBytes + (kGather ? 0 : kXBytes);
   static constexpr int kBarrierBytes = 256;
   // down GEMM: per epilogue warp a 32 x 33 fp32 transpose buffer, so the
   // reduction is issued as full 128-byte row segments
   static constexpr int kRedStride = 33;
-  static constexpr int kRedBytes = kGather ? 0 : kEpiWarps * 32 * kRedStride * 4;
+  static constexpr int kRedBytes = EPI == kEpiScale ? kEpiWarps * 32 * kRedStride * 4 : 0;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes + kRedBytes;
   static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(128, 256);
 
@@ -161,7 +163,9 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
   // everything above overlaps the previous kernel; global reads start here
   pdl_wait();
   pdl_launch_dependents();
-  int ntpp = *args.ntpp;
+  // the router GEMM has no routed blocks: its token blocks are the
+  // "shared" blocks (rows blk * 128 + r of x, the single weight matrix)
+  int ntpp = EPI == kEpiRouter ? 0 : *args.ntpp;
   int routed_blocks = ntpp / args.block_m;
   if (routed_blocks < 0) routed_blocks = 0;
   if (routed_blocks > args.max_routed_blocks) routed_blocks = args.max_routed_blocks;
@@ -319,6 +323,92 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
             uint4* dst = reinterpret_cast<uint4*>(orow + col);
             dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      } else if (EPI == kEpiRouter) {
+        // thread = token row of the tile, TMEM columns 0..E-1 = its logits.
+        // Top-k over columns in increasing id order into a list sorted by
+        // logit (desc): a value enters only if it beats the current k-th (or
+        // the list is short), and goes after every entry it does not beat,
+        // so equal logits keep the lower id first, as the routing kernel.
+        const int t = (tc.blk - routed_blocks) * args.block_m + row;
+        const bool valid = t < args.T;
+        const int E = args.E, kk = args.k;
+        float kv[kRouterMaxK];
+        int ki[kRouterMaxK];
+#pragma unroll
+        for (int j = 0; j < kRouterMaxK; ++j) {
+          kv[j] = -INFINITY;
+          ki[j] = 0;
+        }
+        int n_in = 0;
+        float kth = -INFINITY;
+        float run_max = -INFINITY, run_sum = 0.0f;  // full softmax, online (no renormalisation)
+        bool finite = true;
+        float* lrow = args.logits + static_cast<size_t>(valid ? t : 0) * E;
+#pragma unroll 1
+        for (int c0 = 0; c0 < E; c0 += 16) {
+          uint32_t a[16];
+          ptx::tmem_ld16(t_acc + c0, a);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) asm volatile("" : "+r"(a[jj]));  // uses stay after the wait
+          if (!valid) continue;
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int e = c0 + jj;
+            if (e >= E) continue;
+            const float v = __uint_as_float(a[jj]);
+            lrow[e] = v;
+            if (!isfinite(v)) finite = false;
+            if (!args.r_renorm) {
+              if (v > run_max) {
+                run_sum = run_sum * expf(run_max - v) + 1.0f;
+                run_max = v;
+              } else {
+                run_sum += expf(v - run_max);
+              }
+            }
+            if (n_in < kk || v > kth) {
+              int pos = 0;
+#pragma unroll
+              for (int j = 0; j < kRouterMaxK; ++j) pos += (j < n_in && kv[j] >= v) ? 1 : 0;
+#pragma unroll
+              for (int j = kRouterMaxK - 1; j > 0; --j)
+                if (j > pos) {
+                  kv[j] = kv[j - 1];
+                  ki[j] = ki[j - 1];
+                }
+#pragma unroll
+              for (int j = 0; j < kRouterMaxK; ++j)
+                if (j == pos) {
+                  kv[j] = v;
+                  ki[j] = e;
+                }
+              if (n_in < kk) ++n_in;
+              if (n_in == kk) {
+#pragma unroll
+                for (int j = 0; j < kRouterMaxK; ++j)
+                  if (j == kk - 1) kth = kv[j];
+              }
+            }
+          }
+        }
+        if (valid && !finite) set_status(args.status, MOE_ERR_NONFINITE);
+        if (valid && args.r_ids != nullptr) {
+          // weights: softmax over the chosen k (the first is the largest), or
+          // the full softmax taken at the chosen ids; then x routed_scaling
+          float z = 0.0f;
+#pragma unroll
+          for (int j = 0; j < kRouterMaxK; ++j)
+            if (j < kk) z += expf(kv[j] - kv[0]);
+#pragma unroll
+          for (int j = 0; j < kRouterMaxK; ++j) {
+            if (j < kk) {
+              const float w = args.r_renorm ? expf(kv[j] - kv[0]) / z : expf(kv[j] - run_max) / run_sum;
+              args.r_ids[static_cast<size_t>(t) * kk + j] = ki[j];
+              args.r_w[static_cast<size_t>(t) * kk + j] = w * args.r_scaling;
+            }
           }
         }
       } else {
@@ -492,6 +582,7 @@ cudaError_t launch_grouped_gemm(int epi, const GemmArgs& a, int grid, cudaStream
     case kEpiSwiGLU: return launch_variant<kEpiSwiGLU>(a, grid, s);
     case kEpiRelu2: return launch_variant<kEpiRelu2>(a, grid, s);
     case kEpiScale: return launch_variant<kEpiScale>(a, grid, s);
+    case kEpiRouter: return launch_variant<kEpiRouter>(a, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -37,6 +37,7 @@ _SIG = {
     "moe_align_workspace_size": (ctypes.c_size_t, [_I, _I, _I]),
     "moe_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "moe_route": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _P, _P]),
+    "moe_router": (_I, [_P, _I, _I, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _P, _P, _P]),
     "moe_align": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
     "moe_align_noalloc": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "moe_route_align": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P, _P, _P, _P, _P, _P, _P,
@@ -52,7 +53,8 @@ _SIG = {
     "moe_profile_collect": (_I, [_P, _P, _I, _I]),
 }
 
-STAGES = ("route", "align", "gate_up_gemm", "down_gemm", "combine", "route_align", "fused_expert", "permute")
+STAGES = ("route", "align", "gate_up_gemm", "down_gemm", "combine", "route_align", "fused_expert", "permute",
+          "router")
 
 _lib = None
 _lock = threading.Lock()
@@ -163,6 +165,21 @@ def moe_route(logits, k, topk_ids, topk_weights, n_group=1, topk_group=1, group_
                                     _ptr(topk_ids), _ptr(topk_weights), _ptr(dev_status),
                                     _stream(logits.device))
     _check("moe_route", code)
+
+
+def moe_router(x, w_gate, k, logits, topk_ids, topk_weights, n_group=1, topk_group=1, group_score=GROUP_MAX,
+               renormalize=True, routed_scaling=1.0, dev_status=None):
+    """Router projection x . W_g^T (fp32 logits [T, E]) and top-k gating in one call."""
+    T, d = x.shape
+    E = w_gate.shape[0]
+    if w_gate.shape[1] != d:
+        raise ValueError("moe_router: w_gate must be [E, d]")
+    if logits.dtype != torch.float32 or topk_weights.dtype != torch.float32 or topk_ids.dtype != torch.int32:
+        raise ValueError("moe_router: logits/weights fp32, ids int32")
+    code = load_library().moe_router(_ptr(_bits(x)), T, d, _ptr(_bits(w_gate)), E, k, n_group, topk_group,
+                                     group_score, 1 if renormalize else 0, float(routed_scaling), _ptr(logits),
+                                     _ptr(topk_ids), _ptr(topk_weights), _ptr(dev_status), _stream(x.device))
+    _check("moe_router", code)
 
 
 def moe_align(topk_ids, E, block_m, sorted_token_ids, expert_ids, num_tokens_post_padded, inv_pos,

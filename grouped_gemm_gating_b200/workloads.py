@@ -194,6 +194,16 @@ def make_inputs(cfg: MoEConfig, threads: int = 8) -> MoEInputs:
     return MoEInputs(cfg, x, logits, w13, w2, w13s, w2s, router_w)
 
 
+def router_inputs(T: int, d: int, E: int, seed: int, zero_rows=()):
+    """Seeded router-projection inputs: x ~ N(0, 1) and W_g ~ N(0, 0.02),
+    both bf16 bits ([T, d] and [E, d]); the listed token rows are zero."""
+    ss = np.random.SeedSequence(seed).spawn(2)
+    x = _normal_bf16(ss[0], (T, d), 1.0)
+    for t in zero_rows:
+        x[t] = 0
+    return x, _normal_bf16(ss[1], (E, d), 0.02)
+
+
 def tie_logits(T: int, E: int, seed: int, levels: int = 3) -> np.ndarray:
     """Logits drawn from a handful of values so that ties are everywhere."""
     rng = np.random.Generator(np.random.PCG64(seed))

@@ -139,6 +139,34 @@ MOE_API moe_status moe_route(const float* logits, int T, int E, int k,
                      int32_t* dev_status, moe_stream_t stream);
 
 /*
+ * moe_router — the gate of the MoE block in one call: router projection
+ * logits = x . W_g^T (W_g [E, d_model]) and top-k gating.  In the axolotl
+ * DeepSeek-V3 benchmark (scripts/benchmarks/deepseek_v3_moe.py,
+ * timed_forward) the block's gate maps the flattened hidden states to their
+ * top-k expert ids and weights; "Fused MoE Kernel Optimization" (overview:
+ * top-k gating fusion; "Token-Expert Routing" step 1) gates on those
+ * logits.  Here the product runs on the tensor cores and each token's gating
+ * runs in the GEMM's epilogue.
+ *   x             [T, d] bf16, device, row-major; d a multiple of 64.
+ *   w_gate        [E, d] bf16, device, row-major (K = d contiguous); E <= 256.
+ *   k, n_group, topk_group, group_score, renormalize, routed_scaling:
+ *                 as for moe_route; k <= 16.
+ *   logits        [T, E] fp32 out, device (4-byte aligned): x . W_g^T with
+ *                 fp32 accumulation of the exact bf16 products.
+ *   topk_ids, topk_weights: [T, k] out, device: the same values moe_route
+ *                 writes for these logits (ids bit for bit, weights up to
+ *                 the rounding of the softmax sum).
+ * n_group == 1: one launch (the gating runs in the GEMM epilogue); otherwise
+ * the routing kernel runs on the written logits (two launches).  T == 0 is a
+ * no-op.  Errors as for moe_route; x and w_gate must be 16-byte aligned.
+ */
+MOE_API moe_status moe_router(const uint16_t* x, int T, int d, const uint16_t* w_gate, int E, int k,
+                     int n_group, int topk_group, moe_group_score group_score,
+                     int renormalize, float routed_scaling,
+                     float* logits, int32_t* topk_ids, float* topk_weights,
+                     int32_t* dev_status, moe_stream_t stream);
+
+/*
  * moe_align — sort token-slots by expert and pad to block_m ("Token-Expert
  * Routing" steps 2-3, "Grouped GEMM Structure", "Common Pitfalls" 1-2).
  *   topk_ids               [T, k] int32, device, values in [0, E).

@@ -5,4 +5,4 @@ leg may import this package; the product path never does.
 """
 from .moe_oracle import (ACT_RELU2, ACT_SWIGLU, GROUP_MAX, GROUP_TOP2SUM,  # noqa: F401
                          align, bf16_to_f64, expert_hidden, expert_mlp, forward, group_scores,
-                         max_padded, route, silu)
+                         max_padded, route, router_logits, silu)

@@ -27,6 +27,9 @@ Sources (web pages on fused MoE kernels):
   and one shared expert.
 * mlxcel PR "perf(moe): preserve squared-ReLU fused MoE kernel behind a
   dedicated flag", Summary: fc1 -> relu^2 -> fc2 experts with no gate.
+* the same axolotl diff, scripts/benchmarks/deepseek_v3_moe.py
+  ``timed_forward``: the block's gate maps the flattened hidden states to the
+  top-k expert ids and weights (router projection, then gating).
 
 Readings where the pages are silent (each is also listed in the design notes):
 
@@ -65,6 +68,12 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
 # --------------------------------------------------------------------------
 # Route
 # --------------------------------------------------------------------------
+
+def router_logits(x_bits: np.ndarray, w_gate_bits: np.ndarray) -> np.ndarray:
+    """Router projection of the gate: logits[t, e] = sum_i x[t, i] * W_g[e, i]
+    over the exact bf16 values, in fp64 (x [T, d], W_g [E, d], bf16 bits)."""
+    return bf16_to_f64(x_bits) @ bf16_to_f64(w_gate_bits).T
+
 
 def _order_desc(values: np.ndarray) -> np.ndarray:
     """Indices ordered by (value descending, index ascending)."""

@@ -89,6 +89,18 @@ def test_route_host_checks(lib):
     assert r(NULL, 0, 8, 2, 1, 1, 0, 1, 1.0, NULL, NULL, NULL, NULL) == 0      # T == 0: no-op
 
 
+def test_router_host_checks(lib):
+    r = lib.moe_router
+    #        x     T  d    w_g   E    k  ng tg gs rn scale logits ids   wts   status stream
+    assert r(NULL, 4, 128, NULL, 300, 2, 1, 1, 0, 1, 1.0, NULL, NULL, NULL, NULL, NULL) == 2    # E > 256
+    assert r(NULL, 4, 128, NULL, 64, 17, 1, 1, 0, 1, 1.0, NULL, NULL, NULL, NULL, NULL) == 2    # k > 16
+    assert r(NULL, 4, 96, NULL, 8, 2, 1, 1, 0, 1, 1.0, NULL, NULL, NULL, NULL, NULL) == 2      # d % 64
+    assert r(NULL, 4, 128, NULL, 8, 9, 1, 1, 0, 1, 1.0, NULL, NULL, NULL, NULL, NULL) == 1     # k > E
+    assert r(NULL, 4, 128, NULL, 18, 4, 4, 2, 0, 1, 1.0, NULL, NULL, NULL, NULL, NULL) == 1    # E % n_group
+    assert r(NULL, 4, 128, NULL, 8, 2, 1, 1, 0, 1, 1.0, NULL, NULL, NULL, NULL, NULL) == 1     # null pointers
+    assert r(NULL, 0, 128, NULL, 8, 2, 1, 1, 0, 1, 1.0, NULL, NULL, NULL, NULL, NULL) == 0     # T == 0: no-op
+
+
 def test_align_host_checks(lib):
     a = lib.moe_align
     p = ctypes.c_void_p(16)

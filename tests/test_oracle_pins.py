@@ -356,3 +356,40 @@ def test_workload_tiny_route_and_forward_are_sane():
     out = oracle.forward(inp.x, inp.w13, inp.w2, ids, w, c.act)
     rms = float(np.sqrt((out ** 2).mean()))
     assert 1e-3 < rms < 10.0
+
+
+# ------------------------------------------------------------ router -----
+
+def test_router_one_hot_tokens_read_out_weight_columns():
+    """A token that is the i-th unit vector scores expert e with W_g[e, i]."""
+    rng = np.random.default_rng(31)
+    E, d = 5, 64
+    w = _bits(rng.normal(0.0, 0.5, (E, d)))
+    x = np.zeros((d, d), np.float32)
+    np.fill_diagonal(x, 1.0)
+    got = oracle.router_logits(_bits(x), w)
+    assert np.array_equal(got, oracle.bf16_to_f64(w).T)
+
+
+def test_router_matches_python_loops():
+    rng = np.random.default_rng(32)
+    T, E, d = 3, 4, 8
+    x, w = _bits(rng.normal(0, 1, (T, d))), _bits(rng.normal(0, 1, (E, d)))
+    xf, wf = oracle.bf16_to_f64(x), oracle.bf16_to_f64(w)
+    got = oracle.router_logits(x, w)
+    for t in range(T):
+        for e in range(E):
+            ref = math.fsum(float(xf[t, i]) * float(wf[e, i]) for i in range(d))
+            assert got[t, e] == pytest.approx(ref, rel=1e-14, abs=1e-14)
+
+
+def test_router_permuting_experts_permutes_columns_and_scaling_is_exact():
+    rng = np.random.default_rng(33)
+    T, E, d = 6, 7, 64
+    x, w = _bits(rng.normal(0, 1, (T, d))), _bits(rng.normal(0, 0.1, (E, d)))
+    base = oracle.router_logits(x, w)
+    perm = rng.permutation(E)
+    assert np.array_equal(oracle.router_logits(x, w[perm]), base[:, perm])
+    # doubling x doubles every logit exactly (a power of two, no rounding)
+    x2 = _bits(oracle.bf16_to_f64(x) * 2.0)
+    assert np.array_equal(oracle.router_logits(x2, w), 2.0 * base)
