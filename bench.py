@@ -440,6 +440,29 @@ def run_ours(args):
     assert torch.equal(out_h.view(torch.int16), buf.out.cpu().view(torch.int16))
     del g_main, g_prof, g_e2e, g_steps, g_e2e_steps
 
+    # ---- the gate before the layer (moe_router: x . W_g^T + top-k), on its
+    # own: same x copies, a seeded W_g ~ N(0, 0.02), the same timing rule ----
+    wg = to_dev(W.router_inputs(1, cfg.d, cfg.E, seed=cfg.seed + 7)[1])
+    r_logits = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=dev)
+    r_ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
+    r_w = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
+
+    def router_call(st):
+        M.moe_router(st["x"], wg, cfg.k, r_logits, r_ids, r_w, **rk)
+        return M.moe_last_launch_count()
+
+    r_launches = router_call(sets[0])
+    torch.cuda.synchronize(dev)
+    g_router = [capture(lambda st=st: router_call(st)) for st in sets]
+    g_router_steps = None
+    if rotate:
+        g_router_steps = capture(lambda: [router_call(sets[i % n_copies]) for i in range(args.steps)])
+        g_router_steps.replay()
+        torch.cuda.synchronize(dev)
+    router_ms = timed([g.replay for g in g_router], args.steps,
+                      g_router_steps.replay if g_router_steps is not None else None)
+    del g_router, g_router_steps
+
     alg = algorithmic(cfg, topk_ids)
     sec_per_step = total_ms / args.steps / 1e3
     value = whole_job_tflops(world, alg["flops_total"], total_ms, args.steps)
@@ -489,6 +512,17 @@ def run_ours(args):
                  "per_launch_us": round(per_launch_s * 1e6, 2), "per_launch_source": per_launch_src,
                  "algorithmic_flops": fl, "algorithmic_bytes": by})
 
+    r_s = router_ms / args.steps / 1e3
+    r_flops = 2.0 * cfg.T * cfg.E * cfg.d
+    r_bytes = cfg.T * cfg.d * 2 + cfg.E * cfg.d * 2 + cfg.T * cfg.E * 4 + cfg.T * cfg.k * 8
+    r_t_min = max(r_flops / (peaks["bf16_tflops"] * 1e12), r_bytes / (peaks["hbm_gbs"] * 1e9))
+    router = {"us_per_call": round(r_s * 1e6, 2), "launches": int(r_launches),
+              "tflops": round(r_flops / r_s / 1e12, 3), "gbs": round(r_bytes / r_s / 1e9, 1),
+              "algorithmic_flops": int(r_flops), "algorithmic_bytes": int(r_bytes),
+              "roofline_frac": round(r_t_min / r_s, 4),
+              "roofline_note": "time at the slower of FLOPs / burst bf16 peak and bytes / HBM copy bandwidth, "
+                               "over the measured time"}
+
     line = {
         "metric": METRIC, "value": round(value, 4), "unit": "TFLOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
@@ -510,6 +544,7 @@ def run_ours(args):
         "stages_us": {k: round(v[0] / max(v[1], 1) * 1e3, 2) for k, v in stages.items()},
         "stages_source": stage_source,
         "roofline": roof,
+        "router": router,
         "e2e": {"value": round(e2e_value, 4), "unit": "TFLOPS", "ms_per_step": round(e2e_ms / args.steps, 5),
                 "h2d_bytes_per_step": int(io_bytes),
                 "d2h_bytes_per_step": int(cfg.T * cfg.d * 2)},

@@ -328,9 +328,11 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
       } else if (EPI == kEpiRouter) {
         // thread = token row of the tile, TMEM columns 0..E-1 = its logits.
         // Top-k over columns in increasing id order into a list sorted by
-        // logit (desc): a value enters only if it beats the current k-th (or
-        // the list is short), and goes after every entry it does not beat,
-        // so equal logits keep the lower id first, as the routing kernel.
+        // logit (desc): a value enters only if it beats the current k-th,
+        // walks down the list past every entry it does not beat (so equal
+        // logits keep the lower id first, as the routing kernel), and every
+        // entry after it shifts down by one; one unrolled pass of selects
+        // keeps the list in registers.
         const int t = (tc.blk - routed_blocks) * args.block_m + row;
         const bool valid = t < args.T;
         const int E = args.E, kk = args.k;
@@ -341,8 +343,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
           kv[j] = -INFINITY;
           ki[j] = 0;
         }
-        int n_in = 0;
-        float kth = -INFINITY;
+        float kth = -INFINITY;  // current k-th largest (-inf until k values are in)
         float run_max = -INFINITY, run_sum = 0.0f;  // full softmax, online (no renormalisation)
         bool finite = true;
         float* lrow = args.logits + static_cast<size_t>(valid ? t : 0) * E;
@@ -354,43 +355,56 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) asm volatile("" : "+r"(a[jj]));  // uses stay after the wait
           if (!valid) continue;
+          // one cheap unrolled pass stores the logits and marks the columns
+          // that beat the k-th at the chunk's start; the insertion (one
+          // copy of its code) then runs over the marked columns only
+          uint32_t cand = 0;
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
             const int e = c0 + jj;
-            if (e >= E) continue;
             const float v = __uint_as_float(a[jj]);
-            lrow[e] = v;
-            if (!isfinite(v)) finite = false;
-            if (!args.r_renorm) {
-              if (v > run_max) {
-                run_sum = run_sum * expf(run_max - v) + 1.0f;
-                run_max = v;
-              } else {
-                run_sum += expf(v - run_max);
+            if (e < E) {
+              lrow[e] = v;
+              if (!isfinite(v)) finite = false;
+              if (!args.r_renorm) {
+                if (v > run_max) {
+                  run_sum = run_sum * expf(run_max - v) + 1.0f;
+                  run_max = v;
+                } else {
+                  run_sum += expf(v - run_max);
+                }
               }
+              if (v > kth) cand |= 1u << jj;
             }
-            if (n_in < kk || v > kth) {
-              int pos = 0;
+          }
+          while (cand != 0) {
+            const int jj = __ffs(cand) - 1;
+            cand &= cand - 1;
+            float v = 0.0f;
 #pragma unroll
-              for (int j = 0; j < kRouterMaxK; ++j) pos += (j < n_in && kv[j] >= v) ? 1 : 0;
+            for (int q = 0; q < 16; ++q)
+              if (q == jj) v = __uint_as_float(a[q]);
+            if (v > kth) {  // the k-th may have risen since the chunk started
+              float cv = v;
+              int ci = c0 + jj;
+              bool placed = false;
 #pragma unroll
-              for (int j = kRouterMaxK - 1; j > 0; --j)
-                if (j > pos) {
-                  kv[j] = kv[j - 1];
-                  ki[j] = ki[j - 1];
-                }
-#pragma unroll
-              for (int j = 0; j < kRouterMaxK; ++j)
-                if (j == pos) {
-                  kv[j] = v;
-                  ki[j] = e;
-                }
-              if (n_in < kk) ++n_in;
-              if (n_in == kk) {
-#pragma unroll
-                for (int j = 0; j < kRouterMaxK; ++j)
-                  if (j == kk - 1) kth = kv[j];
+              for (int j = 0; j < kRouterMaxK; ++j) {
+                const bool take = j < kk && (placed || cv > kv[j]);
+                const float tv = kv[j];
+                const int ti = ki[j];
+                kv[j] = take ? cv : tv;
+                ki[j] = take ? ci : ti;
+                cv = take ? tv : cv;
+                ci = take ? ti : ci;
+                placed = placed || take;
               }
+              // the list is sorted, so its k-th entry is its minimum (written as a
+              // min: a select on j == kk - 1 becomes a runtime-indexed load)
+              kth = kv[0];
+#pragma unroll
+              for (int j = 1; j < kRouterMaxK; ++j)
+                if (j < kk) kth = fminf(kth, kv[j]);
             }
           }
         }
