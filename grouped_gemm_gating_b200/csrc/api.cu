@@ -539,6 +539,22 @@ moe_status moe_router(const uint16_t* x, int T, int d, const uint16_t* w_gate, i
   if (!aligned16(x) || !aligned16(w_gate) || (reinterpret_cast<uintptr_t>(logits) & 3u) != 0)
     return MOE_ERR_INVALID_ARG;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int launches = 0;
+  if (T <= moe::kRouterGemvMaxT && static_cast<int64_t>(T) * d * 2 <= 160 * 1024) {
+    // a few tokens: a matrix-vector product bound by reading W_g once, spread
+    // over E warps on the CUDA cores; then the routing kernel gates
+    cudaError_t err;
+    {
+      StageScope scope(8, s);
+      err = moe::launch_router_gemv(x, w_gate, T, d, E, logits, s, &launches);
+    }
+    if (err == cudaSuccess) {
+      StageScope scope(0, s);
+      err = moe::launch_route(logits, T, E, k, n_group, topk_group, static_cast<int>(group_score),
+                              renormalize ? 1 : 0, routed_scaling, topk_ids, topk_weights, dev_status, s, &launches);
+    }
+    return finish(err, launches);
+  }
   const int num_sms = num_sms_current_device();
   if (num_sms <= 0) return MOE_ERR_CUDA;
   moe::GemmArgs a;
@@ -566,7 +582,6 @@ moe_status moe_router(const uint16_t* x, int T, int d, const uint16_t* w_gate, i
   a.r_renorm = renormalize ? 1 : 0;
   a.r_scaling = routed_scaling;
   const int grid = a.n_shared_blocks < num_sms ? a.n_shared_blocks : num_sms;
-  int launches = 0;
   cudaError_t err;
   {
     StageScope scope(8, s);

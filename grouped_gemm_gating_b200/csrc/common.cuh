@@ -83,6 +83,12 @@ cudaError_t launch_permute_rows(const uint16_t* x, const int32_t* sorted_ids, co
                                 int d, int P_max, int n_shared_rows, uint16_t* x_sorted, int num_sms,
                                 cudaStream_t stream, int* launches);
 
+// Router projection on the CUDA cores for T <= kRouterGemvMaxT tokens:
+// logits [T, E] fp32 = x [T, d] . W_g [E, d]^T (d a multiple of 8).
+constexpr int kRouterGemvMaxT = 16;
+cudaError_t launch_router_gemv(const uint16_t* x, const uint16_t* w_gate, int T, int d, int E, float* logits,
+                               cudaStream_t stream, int* launches);
+
 // out = bf16(acc) over n = T * d elements (the scatter-reduce's last step).
 cudaError_t launch_convert(const float* acc, int64_t n, uint16_t* out, int num_sms, cudaStream_t stream,
                            int* launches);

@@ -47,8 +47,10 @@ def _run(T, d, E, k, n_group=1, topk_group=1, score=0, renorm=True, scale=1.0, s
 
 
 @pytest.mark.parametrize("T,d,E,k", [
-    (32, 128, 8, 2),      # the tiny layer's router shape
-    (3, 2048, 128, 8),    # decode batch
+    (32, 128, 8, 2),      # the tiny layer's router shape (tensor cores)
+    (3, 2048, 128, 8),    # decode batch (CUDA-core product for <= 16 tokens)
+    (16, 2688, 128, 6),   # the largest small batch
+    (17, 256, 40, 3),     # the smallest tensor-core batch
     (300, 512, 18, 4),    # E not a multiple of 16, several token blocks, a ragged last block
     (130, 256, 256, 16),  # the limits: E = 256, k = 16
     (1, 64, 1, 1),
