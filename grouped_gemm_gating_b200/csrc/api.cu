@@ -540,9 +540,10 @@ moe_status moe_router(const uint16_t* x, int T, int d, const uint16_t* w_gate, i
     return MOE_ERR_INVALID_ARG;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int launches = 0;
-  if (T <= moe::kRouterGemvMaxT && static_cast<int64_t>(T) * d * 2 <= 160 * 1024) {
-    // a few tokens: a matrix-vector product bound by reading W_g once, spread
-    // over E warps on the CUDA cores; then the routing kernel gates
+  if (T <= moe::kRouterGemvTokens && static_cast<int64_t>(moe::kRouterGemvMaxT) * d * 2 <= 160 * 1024) {
+    // up to a thousand tokens: the product spread over (E / 8) x (T / 16)
+    // CTAs on the CUDA cores (one tensor-core tile per 128 tokens would
+    // leave most SMs idle); then the routing kernel gates
     cudaError_t err;
     {
       StageScope scope(8, s);

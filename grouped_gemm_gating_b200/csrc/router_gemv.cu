@@ -1,11 +1,12 @@
-// Router projection for small token batches: logits[t, e] = x[t] . W_g[e]
-// on the CUDA cores.  The gate of the MoE block (axolotl DeepSeek-V3
+// Router projection for small and mid-size token batches: logits[t, e] =
+// x[t] . W_g[e] on the CUDA cores.  The gate of the MoE block (axolotl DeepSeek-V3
 // benchmark, scripts/benchmarks/deepseek_v3_moe.py, timed_forward: the gate
 // maps the flattened hidden states to their top-k experts) starts with this
 // product; with a handful of tokens it is a matrix-vector product bound by
 // reading W_g once, which one tensor-core tile per 128 tokens would stream
-// through a single SM.  Here every warp owns one expert row of W_g (16-byte
-// loads, one pass) and the CTA's tokens sit in shared memory; products of the
+// through a single SM.  Here a CTA takes 8 experts x 16 tokens: every warp
+// owns one expert row of W_g (16-byte loads, one pass; the other token
+// chunks read it from L2) and the CTA's tokens sit in shared memory; products of the
 // bf16 values are exact in fp32 and summed in fp32 (per-lane partial sums,
 // then a warp tree), within the same d * 2^-24 * sum|x w| bound as the
 // tensor-core path.  The top-k gating then runs in the routing kernel.
@@ -18,11 +19,16 @@ namespace {
 constexpr int kGemvWarps = 8;  // experts per CTA
 
 __global__ void __launch_bounds__(kGemvWarps * 32)
-    router_gemv_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ w_gate, int T, int d, int E,
+    router_gemv_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ w_gate, int T_all, int d, int E,
                        float* __restrict__ logits) {
-  extern __shared__ __align__(16) uint16_t xs[];  // [T][d]
+  extern __shared__ __align__(16) uint16_t xs[];  // [chunk tokens][d]
   pdl_wait();
   pdl_launch_dependents();
+  // this CTA's token chunk: rows t0 .. t0 + T - 1
+  const int t0 = blockIdx.y * kRouterGemvMaxT;
+  const int T = min(kRouterGemvMaxT, T_all - t0);
+  x += static_cast<size_t>(t0) * d;
+  logits += static_cast<size_t>(t0) * E;
   // stage the tokens (T * d bf16, 16 bytes per thread per step)
   const int n16 = T * d / 8;
   for (int i = threadIdx.x; i < n16; i += blockDim.x)
@@ -68,16 +74,17 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
 
 cudaError_t launch_router_gemv(const uint16_t* x, const uint16_t* w_gate, int T, int d, int E, float* logits,
                                cudaStream_t stream, int* launches) {
-  if (T < 1 || T > kRouterGemvMaxT || d % 8 != 0) return cudaErrorInvalidValue;
-  const size_t smem = static_cast<size_t>(T) * d * 2;
+  if (T < 1 || d % 8 != 0) return cudaErrorInvalidValue;
+  const int chunk = T < kRouterGemvMaxT ? T : kRouterGemvMaxT;
+  const size_t smem = static_cast<size_t>(chunk) * d * 2;
   if (smem > 48 * 1024) {
     cudaError_t err = cudaFuncSetAttribute(router_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
   }
-  const int grid = (E + kGemvWarps - 1) / kGemvWarps;
-  cudaError_t err = launch_pdl(router_gemv_kernel, dim3(grid), dim3(kGemvWarps * 32), smem, stream, x, w_gate, T, d,
-                               E, logits);
+  const dim3 grid((E + kGemvWarps - 1) / kGemvWarps, (T + kRouterGemvMaxT - 1) / kRouterGemvMaxT);
+  cudaError_t err = launch_pdl(router_gemv_kernel, grid, dim3(kGemvWarps * 32), smem, stream, x, w_gate, T, d, E,
+                               logits);
   if (err == cudaSuccess && launches) ++*launches;
   return err;
 }

@@ -156,13 +156,12 @@ MOE_API moe_status moe_route(const float* logits, int T, int E, int k,
  *   topk_ids, topk_weights: [T, k] out, device: the same values moe_route
  *                 writes for these logits (ids bit for bit, weights up to
  *                 the rounding of the softmax sum).
- * Batches of more than 16 tokens: with n_group == 1 one launch (the gating
- * runs in the GEMM epilogue), otherwise the routing kernel runs on the
- * written logits (two launches).  Up to 16 tokens (and T*d*2 <= 160 KiB) the
- * product is a matrix-vector product bound by reading W_g: it runs on the
- * CUDA cores, one warp per expert row, and the routing kernel gates (two
- * launches).  T == 0 is a no-op.  Errors as for moe_route; x and w_gate must
- * be 16-byte aligned.
+ * Up to 1024 tokens (and d <= 5120) the product runs on the CUDA cores, in
+ * CTAs of 8 expert rows x 16 tokens, and the routing kernel gates (two
+ * launches).  Larger batches run on the tensor cores: with n_group == 1 in
+ * one launch (the gating runs in the GEMM epilogue), otherwise the routing
+ * kernel runs on the written logits (two launches).  T == 0 is a no-op.
+ * Errors as for moe_route; x and w_gate must be 16-byte aligned.
  */
 MOE_API moe_status moe_router(const uint16_t* x, int T, int d, const uint16_t* w_gate, int E, int k,
                      int n_group, int topk_group, moe_group_score group_score,

@@ -47,29 +47,34 @@ def _run(T, d, E, k, n_group=1, topk_group=1, score=0, renorm=True, scale=1.0, s
 
 
 @pytest.mark.parametrize("T,d,E,k", [
-    (32, 128, 8, 2),      # the tiny layer's router shape (tensor cores)
-    (3, 2048, 128, 8),    # decode batch (CUDA-core product for <= 16 tokens)
-    (16, 2688, 128, 6),   # the largest small batch
-    (17, 256, 40, 3),     # the smallest tensor-core batch
-    (300, 512, 18, 4),    # E not a multiple of 16, several token blocks, a ragged last block
+    (32, 128, 8, 2),      # the tiny layer's router shape (CUDA-core product, two token chunks)
+    (3, 2048, 128, 8),    # decode batch
+    (16, 2688, 128, 6),   # one full chunk of 16 tokens, d = 2688
+    (300, 512, 18, 4),    # E not a multiple of 8, a ragged last chunk
     (130, 256, 256, 16),  # the limits: E = 256, k = 16
     (1, 64, 1, 1),
+    (1024, 256, 40, 3),   # the largest CUDA-core batch
+    (1025, 256, 40, 3),   # the smallest tensor-core batch, a ragged last tile
+    (5000, 512, 18, 4),   # tensor cores, E not a multiple of 16
 ])
 def test_router_parity(T, d, E, k):
     _run(T, d, E, k, seed=T * 7 + E)
 
 
-def test_router_full_softmax_and_scaling():
-    _run(200, 256, 64, 6, renorm=False, scale=2.5, seed=5)
+@pytest.mark.parametrize("T", [200, 4200])
+def test_router_full_softmax_and_scaling(T):
+    _run(T, 256, 64, 6, renorm=False, scale=2.5, seed=5)
 
 
-def test_router_grouped_runs_the_routing_kernel_on_its_logits():
-    _run(257, 384, 18, 4, n_group=6, topk_group=4, score=1, seed=6)
+@pytest.mark.parametrize("T", [257, 4500])
+def test_router_grouped_runs_the_routing_kernel_on_its_logits(T):
+    _run(T, 384, 18, 4, n_group=6, topk_group=4, score=1, seed=6)
 
 
-def test_router_zero_token_ties_to_lowest_ids():
+@pytest.mark.parametrize("T", [40, 4100])
+def test_router_zero_token_ties_to_lowest_ids(T):
     # a zero token scores every expert 0: the gating keeps experts 0..k-1
-    lg = _run(40, 128, 32, 5, seed=7, zero_rows=(0, 17, 39))
+    lg = _run(T, 128, 32, 5, seed=7, zero_rows=(0, 17, 39))
     assert (lg[[0, 17, 39]] == 0).all()
 
 
