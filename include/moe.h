@@ -72,7 +72,7 @@ typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1,    /* shape, pointer, alignment or range check failed */
-  MOE_ERR_UNSUPPORTED = 2,    /* valid arguments outside this build's limits */
+  MOE_ERR_UNSUPPORTED = 2,    /* valid arguments outside the library's limits */
   MOE_ERR_WORKSPACE = 3,      /* workspace pointer missing or too small */
   MOE_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed (launch, attribute, tensor map) */
   MOE_ERR_NONFINITE = 5,      /* device: a router logit was NaN or infinite */
@@ -87,7 +87,7 @@ typedef enum {
   MOE_GROUP_TOP2SUM = 1  /* group score = fp32 sum of the two largest logits in the group */
 } moe_group_score;
 
-/* Limits of this build (checked; MOE_ERR_UNSUPPORTED beyond them):
+/* Limits of the library (checked; MOE_ERR_UNSUPPORTED beyond them):
  *   1 <= E <= 256, 1 <= k <= min(E, 16), d and F multiples of 64 with
  *   64 <= d, F <= 16384, block_m in {16, 32, 64, 128}, n_shared in {0, 1},
  *   T * k < 2^30. */
