@@ -6,6 +6,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -109,15 +110,15 @@ EncodeTiledFn encode_fn() {
 }
 
 int num_sms_current_device() {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];  // per device; concurrent first calls store the same value
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 // bf16 tensor [depth, rows, K] (K innermost) as a 3-D map with 64 x box_rows

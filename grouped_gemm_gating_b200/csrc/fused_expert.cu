@@ -50,6 +50,7 @@
 // two gate/up accumulators of block_m columns, then a ring of down-GEMM
 // accumulators (groups of 64 columns).  Every wait is bounded in time; on expiry the kernel records
 // MOE_ERR_DEVICE_TIMEOUT and all roles leave.
+#include <atomic>
 #include "align_impl.cuh"
 #include "common.cuh"
 #include "fused.h"
@@ -842,15 +843,16 @@ template <int EPI1, int TOK, bool ROUTE>
 cudaError_t launch_fused_variant(const FusedArgs& args, int grid, cudaStream_t stream) {
   using C = FusedCfg<EPI1, TOK, ROUTE>;
   auto kern = fused_expert_kernel<EPI1, TOK, ROUTE>;
-  static bool attr_done[64] = {false};
+  // per device, set once; concurrent first calls may both set it (idempotent)
+  static std::atomic<bool> attr_done[64];
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_done[dev]) {
+  if (!attr_done[dev].load(std::memory_order_acquire)) {
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
-    attr_done[dev] = true;
+    attr_done[dev].store(true, std::memory_order_release);
   }
   return launch_pdl(kern, dim3(grid), dim3(C::kNumThreads), C::kSmemBytes, stream, args);
 }

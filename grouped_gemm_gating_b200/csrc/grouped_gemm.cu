@@ -40,6 +40,7 @@
 // tmem-full/tmem-empty mbarriers.  Every wait is
 // bounded in time; on expiry the kernel records MOE_ERR_DEVICE_TIMEOUT and
 // all roles leave their loops so the CTA frees its TMEM and exits.
+#include <atomic>
 #include <cmath>
 
 #include "common.cuh"
@@ -567,15 +568,16 @@ template <int EPI>
 cudaError_t launch_variant(const GemmArgs& args, int grid, cudaStream_t stream) {
   using C = GemmCfg<EPI>;
   auto kern = grouped_gemm_kernel<EPI>;
-  static bool attr_done[64] = {false};
+  // per device, set once; concurrent first calls may both set it (idempotent)
+  static std::atomic<bool> attr_done[64];
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_done[dev]) {
+  if (!attr_done[dev].load(std::memory_order_acquire)) {
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
-    attr_done[dev] = true;
+    attr_done[dev].store(true, std::memory_order_release);
   }
   return launch_pdl(kern, dim3(grid), dim3(C::kNumThreads), C::kSmemBytes, stream, args);
 }

@@ -28,6 +28,7 @@
 // MOE_ERR_DEVICE_TIMEOUT and its roles leave their loops.  Both CTAs always
 // reach the closing cluster barrier, which orders the peer's last remote
 // arrivals before either CTA frees its TMEM and exits.
+#include <atomic>
 #include "common.cuh"
 #include "gemm.h"
 #include "ptx.cuh"
@@ -404,15 +405,16 @@ template <int EPI>
 cudaError_t launch_pair_variant(const GemmArgs& args, int grid, cudaStream_t stream) {
   using C = PairCfg<EPI>;
   auto kern = grouped_gemm_pair_kernel<EPI>;
-  static bool attr_done[64] = {false};
+  // per device, set once; concurrent first calls may both set it (idempotent)
+  static std::atomic<bool> attr_done[64];
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_done[dev]) {
+  if (!attr_done[dev].load(std::memory_order_acquire)) {
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
-    attr_done[dev] = true;
+    attr_done[dev].store(true, std::memory_order_release);
   }
   grid &= ~1;
   if (grid < 2) grid = 2;
