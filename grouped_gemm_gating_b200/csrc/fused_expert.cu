@@ -44,13 +44,19 @@
 //          every counter is zero when the kernel ends), and every CTA
 //          converts its slice of the accumulator.
 //
+// Tiles are dealt to the fewest CTAs that can take equal shares; the other
+// CTAs only zero and convert their slice of the accumulator.
+//
 // Warp roles: warp 0 TMA producer (weights), warp 1 TMEM allocator + MMA
 // issuer, warps 2-5 epilogue, warps 6-9 token-row gather (cp.async; each
 // thread's copies arrive on the stage's full barrier when they land).  TMEM:
-// two gate/up accumulators of block_m columns, then a ring of down-GEMM
-// accumulators (groups of 64 columns).  Every wait is bounded in time; on expiry the kernel records
-// MOE_ERR_DEVICE_TIMEOUT and all roles leave.
+// the gate/up accumulators of two tiles in flight (block_m columns each;
+// SwiGLU has a gate and an up accumulator per tile), then a ring of
+// down-GEMM accumulators (groups of 64 columns).  Every wait is bounded in
+// time; on expiry the kernel records MOE_ERR_DEVICE_TIMEOUT and all roles
+// leave.
 #include <atomic>
+
 #include "align_impl.cuh"
 #include "common.cuh"
 #include "fused.h"
