@@ -113,10 +113,10 @@ def algorithmic(cfg: W.MoEConfig, topk_ids: np.ndarray):
     g2_flops = 2 * rows * cfg.d * cfg.F
     g1_bytes = n_w * n1 * cfg.d * 2 + cfg.T * cfg.d * 2 + rows * cfg.F * 2
     g2_bytes = n_w * cfg.d * cfg.F * 2 + rows * cfg.F * 2 + rows * cfg.d * 4
-    # fused kernel: both weight sets, x in, h out and back in, y, out (combine
-    # fused for small T)
-    fused_bytes = n_w * (n1 * cfg.d + cfg.d * cfg.F) * 2 + cfg.T * cfg.d * 2 + 2 * rows * cfg.F * 2 + \
-        rows * cfg.d * 4 + cfg.T * cfg.d * 2
+    # fused kernel (block_m <= 64): both weight sets of every hit expert, x
+    # in, out; h stays in shared memory and the per-slot products are fp32
+    # reductions into an L2-resident accumulator, not DRAM traffic
+    fused_bytes = n_w * (n1 * cfg.d + cfg.d * cfg.F) * 2 + cfg.T * cfg.d * 2 + cfg.T * cfg.d * 2
     return dict(S=S, U=U, flops_routed=cfg.flops_routed(), flops_total=cfg.flops_total(),
                 gate_up_gemm=(g1_flops, g1_bytes), down_gemm=(g2_flops, g2_bytes), fused_bytes=fused_bytes,
                 weight_bytes=n_w * (n1 * cfg.d + cfg.d * cfg.F) * 2)

@@ -62,3 +62,35 @@ def test_reference_arm_prints_on_rank_zero_only(monkeypatch, capsys):
     monkeypatch.setenv("WORLD_SIZE", "2")
     bench.main(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3", "--workload", "tiny"])
     assert capsys.readouterr().out == ""
+
+
+def test_algorithmic_work_of_the_decode_step():
+    """Roofline numerators: 21 hit experts of the decode shape stream their
+    gate/up ([2*768, 2048]) and down ([2048, 768]) bf16 weights once."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+
+    import bench
+    from grouped_gemm_gating_b200 import workloads as W
+    cfg = W.CONFIGS["decode"]
+    ids = (np.arange(cfg.T * cfg.k, dtype=np.int32) % 21).reshape(cfg.T, cfg.k)   # 21 distinct experts
+    a = bench.algorithmic(cfg, ids)
+    per_expert = (2 * 768 * 2048 + 2048 * 768) * 2
+    assert a["U"] == 21 and a["weight_bytes"] == 21 * per_expert
+    assert a["fused_bytes"] == 21 * per_expert + 2 * 3 * 2048 * 2          # + x in, out
+    assert a["flops_routed"] == 2 * 3 * 8 * 3 * 2048 * 768                  # 2*T*k*3*d*F (SwiGLU)
+    gu, dn = a["gate_up_gemm"][0], a["down_gemm"][0]
+    assert gu + dn == a["flops_routed"]
+
+
+def test_algorithmic_counts_the_shared_expert():
+    sys.path.insert(0, ROOT)
+    import numpy as np
+
+    import bench
+    from grouped_gemm_gating_b200 import workloads as W
+    cfg = W.CONFIGS["dsv3"]
+    ids = (np.arange(cfg.T * cfg.k, dtype=np.int32) % cfg.E).reshape(cfg.T, cfg.k)
+    a = bench.algorithmic(cfg, ids)
+    assert a["flops_total"] == a["flops_routed"] + 2 * cfg.T * 3 * cfg.d * cfg.F
+    assert a["weight_bytes"] == (cfg.E + 1) * (2 * cfg.F * cfg.d + cfg.d * cfg.F) * 2
