@@ -393,3 +393,38 @@ def test_router_permuting_experts_permutes_columns_and_scaling_is_exact():
     # doubling x doubles every logit exactly (a power of two, no rounding)
     x2 = _bits(oracle.bf16_to_f64(x) * 2.0)
     assert np.array_equal(oracle.router_logits(x2, w), 2.0 * base)
+
+
+# ------------------------------------------------- randomised properties --
+
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.integers(1, 6), st.integers(1, 7), st.data())
+def test_route_selection_is_the_unique_bruteforce_subset(T, E, data):
+    """Any logits (ties included, drawn from a few levels): the chosen set is
+    the one k-subset whose members all beat every other expert, listed in
+    selection order."""
+    k = data.draw(st.integers(1, E))
+    levels = data.draw(st.lists(st.sampled_from([-1.5, -0.0, 0.0, 0.25, 2.0]), min_size=T * E, max_size=T * E))
+    lg = np.array(levels, np.float32).reshape(T, E)
+    ids, w = oracle.route(lg, k)
+    for t in range(T):
+        assert set(ids[t].tolist()) == _brute_topk(lg[t].astype(np.float64), list(range(E)), k)
+        _check_selection_order(lg[t].astype(np.float64), ids[t])
+        assert abs(w[t].sum() - 1.0) <= 1e-12
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.integers(0, 40), st.integers(1, 9), st.sampled_from([16, 32, 64, 128]), st.data())
+def test_align_invariants_on_random_ids(T, E, bm, data):
+    k = data.draw(st.integers(1, E))
+    flat = data.draw(st.lists(st.integers(0, E - 1), min_size=T * k, max_size=T * k))
+    ids = np.array(flat, np.int32).reshape(T, k)
+    st_, ex, n, inv = oracle.align(ids, E, bm)
+    _check_align_invariants(ids, E, bm, st_, ex, n, inv)
+    # the sort is stable: within an expert's run the slots ascend
+    order = [int(s) for s in st_[:n] if s < T * k]
+    assert order == sorted(range(T * k), key=lambda s: (int(ids.reshape(-1)[s]), s))
