@@ -19,6 +19,13 @@ Multi-GPU (torchrun, one process per GPU): the layer does not shard, so each
 rank runs an independent replica of the workload ("scaling": "weak"); ranks
 meet at barriers and the slowest rank's time is reported.
 
+The line also carries, measured in the same run: the end-to-end step through
+the public API with host buffers (one host-to-device copy of x and logits,
+one device-to-host copy of out per step), the dominant kernel's roofline,
+the clocks seen, the CPU oracle on a bounded token sample, and the router
+(moe_router: x . W_g^T and top-k gating, the step before the layer) on its
+own with a seeded W_g.
+
 --impl reference times the CPU fp64 oracle (test infrastructure) on the host
 cores on a bounded sample of the same workload; rank 0 only.
 """
