@@ -1,7 +1,13 @@
 #!/usr/bin/env python
 """Benchmark of the B200 fused MoE expert layer.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload all|NAME] [--impl ours|reference]
+
+By default every workload is measured in one run: the line's headline
+(metric, value, roofline, e2e, cpu_baseline) is the largest, the zipf
+training-forward prefill (T=16384, 1.24 TFLOP per step), and a `workloads`
+object carries the same figures for each of tiny, decode, dsv3, relu2 and
+zipf.  --workload NAME measures one workload only.
 
 A step is one pass of the whole layer over one batch of the workload:
 route (top-k gating) -> align (sort/pad by expert) -> gate/up GEMM with the
@@ -19,7 +25,7 @@ Multi-GPU (torchrun, one process per GPU): the layer does not shard, so each
 rank runs an independent replica of the workload ("scaling": "weak"); ranks
 meet at barriers and the slowest rank's time is reported.
 
-The line also carries, measured in the same run: the end-to-end step through
+Each workload also carries, measured in the same run: the end-to-end step through
 the public API with host buffers (one host-to-device copy of x and logits,
 one device-to-host copy of out per step), the dominant kernel's roofline,
 the clocks seen, the CPU oracle on a bounded token sample, and the router
@@ -73,9 +79,9 @@ CPU_SAMPLE_TOKENS = {"tiny": 32, "decode": 1, "relu2": 2, "dsv3": 8, "zipf": 8}
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="decode", choices=sorted(W.CONFIGS))
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="all", choices=["all"] + sorted(W.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--single-copy", action="store_true",
@@ -173,7 +179,21 @@ class ClockSampler:
                 "reasons": sorted(active), "samples": len(sm)}
 
 
-def cpu_threads():
+def cpu_info():
+    """Host cores and CPU model of the machine the oracle is timed on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count() or 1, "model": model}
+
+
+def blas_threads():
     try:
         from threadpoolctl import threadpool_info
         n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
@@ -193,29 +213,54 @@ def oracle_step(inp: W.MoEInputs, tokens: np.ndarray):
     return oracle.forward(inp.x[tokens], inp.w13, inp.w2, ids, w, c.act, inp.w13_shared, inp.w2_shared)
 
 
-def time_oracle(inp: W.MoEInputs, steps: int, warmup: int, min_seconds: float = 0.0):
-    """Time the oracle on seeded token samples: at least `steps` steps, and
-    more (up to 10x) until `min_seconds` of CPU work has been measured."""
+def time_oracle(inp: W.MoEInputs, steps: int, warmup: int, min_seconds: float = 0.0, max_steps: int = 0,
+                threads: int | None = None):
+    """Time the oracle on seeded token samples: `warmup` untimed steps, then
+    at least `steps` timed steps, and more (up to max_steps, default 10x
+    steps) until `min_seconds` of CPU work has been measured.  threads=1
+    limits the BLAS pool to one thread."""
+    import contextlib
     c = inp.cfg
     n = min(c.T, CPU_SAMPLE_TOKENS.get(c.name, 8))
     rng = np.random.default_rng(c.seed)
+    limit = contextlib.nullcontext()
+    if threads is not None:
+        try:
+            from threadpoolctl import threadpool_limits
+            limit = threadpool_limits(limits=threads)
+        except Exception:
+            pass
+    cap = max_steps or 10 * steps
     times = []
-    i = 0
-    while True:
-        tokens = np.sort(rng.choice(c.T, size=n, replace=False))
-        t0 = time.perf_counter()
-        oracle_step(inp, tokens)
-        if i >= warmup:
-            times.append(time.perf_counter() - t0)
-        i += 1
-        if len(times) >= steps and (sum(times) >= min_seconds or len(times) >= 10 * steps):
-            break
+    with limit:
+        cores = blas_threads()
+        i = 0
+        while True:
+            tokens = np.sort(rng.choice(c.T, size=n, replace=False))
+            t0 = time.perf_counter()
+            oracle_step(inp, tokens)
+            if i >= warmup:
+                times.append(time.perf_counter() - t0)
+            i += 1
+            if len(times) >= steps and (sum(times) >= min_seconds or len(times) >= cap):
+                break
     sec = float(np.mean(times))
     flops = c.flops_total() * n / c.T
-    return {"value": flops / sec / 1e12, "unit": "TFLOPS", "tokens_per_s": n / sec, "cores": cpu_threads(),
-            "kind": "oracle", "steps": len(times),
+    return {"value": flops / sec / 1e12, "unit": "TFLOPS", "tokens_per_s": n / sec, "cores": cores,
+            "kind": "oracle", "steps": len(times), "ms_per_step": sec * 1e3, "tokens": n,
             "sample": f"{n} of {c.T} tokens per step (seeded), {len(times)} steps after {warmup} warm-up "
-                      f"({sum(times):.1f} s); route+align+forward in fp64 numpy"}
+                      f"({sum(times):.1f} s); route+align+forward in fp64 numpy, {cores} BLAS thread(s)"}
+
+
+def cpu_baseline(inp: W.MoEInputs, seconds: float):
+    """The oracle on the host cores (all BLAS threads) plus a single-thread
+    run, each on a bounded token sample of the workload."""
+    cb = time_oracle(inp, steps=2, warmup=1, min_seconds=seconds)
+    one = time_oracle(inp, steps=1, warmup=0, min_seconds=seconds / 3, threads=1)
+    info = cpu_info()
+    return {"value": cb["value"], "unit": "TFLOPS", "cores": cb["cores"], "kind": "oracle",
+            "sample": cb["sample"], "host_nproc": info["nproc"], "cpu_model": info["model"],
+            "single_thread_value": one["value"], "single_thread_sample": one["sample"]}
 
 
 # --------------------------------------------------------------------------
@@ -268,17 +313,72 @@ def whole_job_tflops(world: int, flops_per_step: float, ms_total: float, steps: 
     return world * flops_per_step / (ms_total / steps / 1e3) / 1e12
 
 
-def run_ours(args):
+# Headline workload when every workload is measured: the largest (1.24
+# TFLOP per step), the tensor-bound training-forward prefill.
+HEADLINE = "zipf"
+# measurement order: the headline first, while the GPU is cool
+ORDER = ("zipf", "dsv3", "relu2", "decode", "tiny")
+NOMINAL_HBM_GBS = 8000.0
+
+
+def job_config(cfg: W.MoEConfig, world: int, experts_hit: int) -> dict:
+    """The `config` object of a line: the workload only (the same on both arms)."""
+    return {"workload": workload_desc(cfg), "global_batch": world * cfg.T,
+            "parallelism": f"replicas x{world}", "experts_hit": experts_hit,
+            "flops_per_step": cfg.flops_total(), "flops_routed_per_step": cfg.flops_routed()}
+
+
+def roofline(cfg, alg, stages, total_ms, steps, launches_per_step, rotate, peaks, peak_src):
+    """Roofline of the dominant kernel: algorithmic FLOPs (or bytes) of one
+    launch over its average launch duration, against the measured peak."""
+    dom = max(("gate_up_gemm", "down_gemm", "fused_expert"), key=lambda s: stages[s][0])
+    dom_ms, dom_calls = stages[dom]
+    per_launch_s = dom_ms / max(dom_calls, 1) / 1e3
+    per_launch_src = "CUDA events around the kernel (profiled graphs)"
+    if rotate and launches_per_step == 1:
+        # the step is this one kernel: its back-to-back step time is its
+        # average launch duration, without the events' own launch gap
+        per_launch_s = total_ms / steps / 1e3
+        per_launch_src = "CUDA events around the back-to-back timed steps (the step is this one kernel)"
+    if dom == "fused_expert":   # both GEMMs (and the combine) in one kernel
+        fl = alg["gate_up_gemm"][0] + alg["down_gemm"][0]
+        by = alg["fused_bytes"]
+    else:
+        fl, by = alg[dom]
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    src = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    if fl / by >= ridge:
+        achieved = fl / per_launch_s / 1e12
+        # the timed region is tens of milliseconds: the burst (not the
+        # power-capped sustained) cuBLAS figure is the denominator
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "unit": "TFLOP/s",
+                "frac_of_sustained_peak": round(achieved / peaks["bf16_tflops_sustained"], 4)}
+        src += ", burst bf16"
+    else:
+        achieved = by / per_launch_s / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "unit": "GB/s", "frac_of_nominal_hbm": round(achieved / NOMINAL_HBM_GBS, 4)}
+        src += ", HBM copy"
+    traffic = NCU_TRAFFIC.get((cfg.name, dom))
+    roof.update({"kernel": dom, "achieved": round(achieved, 2), "peak": peak, "peak_source": src,
+                 "frac": round(achieved / peak, 4),
+                 "traffic": traffic,
+                 "traffic_vs_algorithmic": None if traffic is None else round(traffic / by, 3),
+                 "per_launch_us": round(per_launch_s * 1e6, 2), "per_launch_source": per_launch_src,
+                 "algorithmic_flops": fl, "algorithmic_bytes": by})
+    return roof
+
+
+def measure_workload(name, args, dev, pg, world, rank, cpu_seconds):
+    """Every figure of one workload: device-timed steps, per-kernel times,
+    roofline, the end-to-end step, the router and the CPU oracle."""
     import torch
 
     from grouped_gemm_gating_b200 import moe as M
 
-    world, rank, local, pg = dist_setup(args.gpus)
-    dev = torch.device("cuda", local if world > 1 else 0)
-    M.load_library()
-    cfg = W.CONFIGS[args.workload]
+    cfg = W.CONFIGS[name]
     inp = W.make_inputs(cfg)
-
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
 
     def to_dev(bits):
@@ -326,7 +426,8 @@ def run_ours(args):
     step(sets[0])
     torch.cuda.synchronize(dev)
     topk_ids = buf.topk_ids.cpu().numpy()
-    touched = algorithmic(cfg, topk_ids)["weight_bytes"]
+    alg = algorithmic(cfg, topk_ids)
+    touched = alg["weight_bytes"]
     n_copies = 1 + -(-2 * l2 // touched)
     rotate = n_copies <= MAX_INPUT_COPIES and not args.single_copy
     if not rotate:
@@ -335,8 +436,6 @@ def run_ours(args):
     flush = None if rotate else torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
 
     stream = torch.cuda.current_stream(dev)
-    clocks = ClockSampler(dev.index if dev.index is not None else 0)
-    clocks.start()
     launches_per_step = 0
     for i in range(args.warmup):
         launches_per_step = step(sets[i % n_copies])
@@ -344,24 +443,11 @@ def run_ours(args):
     assert M.moe_read_status(buf.status) == 0, "device status set during warm-up"
     assert np.array_equal(buf.topk_ids.cpu().numpy(), topk_ids)
 
-    # The step's launches are replayed from CUDA graphs (kernels chained by
-    # programmatic dependent launch), one graph per input copy.  A second set
-    # of graphs carries library-recorded events around every kernel; it is
-    # replayed over the same number of steps to time each kernel.
     def capture(fn):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             fn()
         return g
-
-    g_main = [capture(lambda st=st: step(st)) for st in sets]
-    M.moe_profile_enable(True)
-    g_prof = [capture(lambda st=st: step(st)) for st in sets]
-    M.moe_profile_enable(False)
-    for _ in range(3):
-        for g in g_main + g_prof:
-            g.replay()
-    torch.cuda.synchronize(dev)
 
     def timed(runs, n, whole=None):
         """Device time of n steps (step i runs runs[i % len(runs)], or one
@@ -393,21 +479,37 @@ def run_ours(args):
         barrier(pg)
         return max_over_ranks(pg, ms)
 
-    # Back to back, the K timed steps are one graph (as in a captured model
-    # forward): consecutive steps' kernels are chained by programmatic
-    # dependent launch instead of paying a graph launch each.
+    # The step's launches are replayed from CUDA graphs (kernels chained by
+    # programmatic dependent launch), one graph per input copy; back to back,
+    # the K timed steps are one graph (as in a captured model forward).
+    g_main = [capture(lambda st=st: step(st)) for st in sets]
     g_steps = None
     if rotate:
         g_steps = capture(lambda: [step(sets[i % n_copies]) for i in range(args.steps)])
+    for g in g_main:
+        g.replay()
+    if g_steps is not None:
         g_steps.replay()
-        torch.cuda.synchronize(dev)
+    torch.cuda.synchronize(dev)
 
     # ---- device-timed region: inputs resident in HBM ----
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks.start()
+    time.sleep(0.1)  # the sampler is running before the timed region starts
     total_ms = timed([g.replay for g in g_main], args.steps, g_steps.replay if g_steps is not None else None)
+    clk = clocks.stop()
     launches = launches_per_step * args.steps
     assert M.moe_read_status(buf.status) == 0, "device status set during the timed region"
 
-    # ---- per-kernel durations: the profiled graphs over the same steps ----
+    # ---- per-kernel durations: a second set of graphs carries
+    # library-recorded events around every kernel, replayed over the same
+    # number of steps ----
+    M.moe_profile_enable(True)
+    g_prof = [capture(lambda st=st: step(st)) for st in sets]
+    M.moe_profile_enable(False)
+    for g in g_prof:
+        g.replay()
+    torch.cuda.synchronize(dev)
     stages = {k_: [0.0, 0] for k_ in M.STAGES}
     for _ in range(-(-args.steps // n_copies)):
         # every graph is replayed once per round: each graph's events hold
@@ -421,8 +523,6 @@ def run_ours(args):
             stages[k_][0] += ms
             stages[k_][1] += c
     M.moe_profile_collect(release=True)
-    stage_source = "CUDA events around each kernel in replayed graphs of the step"
-    clk = clocks.stop()
 
     # ---- the same steps enqueued eagerly from Python (no graph), for context ----
     eager_ms = timed([lambda st=st: step(st) for st in sets], args.steps)
@@ -474,54 +574,11 @@ def run_ours(args):
                       g_router_steps.replay if g_router_steps is not None else None)
     del g_router, g_router_steps
 
-    alg = algorithmic(cfg, topk_ids)
     sec_per_step = total_ms / args.steps / 1e3
     value = whole_job_tflops(world, alg["flops_total"], total_ms, args.steps)
     e2e_value = whole_job_tflops(world, alg["flops_total"], e2e_ms, args.steps)
-
-    # ---- roofline of the dominant kernel ----
     peaks, peak_src = load_peaks()
-    dom = max(("gate_up_gemm", "down_gemm", "fused_expert"), key=lambda s: stages[s][0])
-    dom_ms, dom_calls = stages[dom]
-    per_launch_s = dom_ms / max(dom_calls, 1) / 1e3
-    per_launch_src = "CUDA events around the kernel (profiled graphs)"
-    if rotate and launches_per_step == 1:
-        # the step is this one kernel: its back-to-back step time is its
-        # average launch duration, without the events' own launch gap
-        per_launch_s = total_ms / args.steps / 1e3
-        per_launch_src = "CUDA events around the back-to-back timed steps (the step is this one kernel)"
-    if dom == "fused_expert":   # both GEMMs (and the combine) in one kernel
-        fl = alg["gate_up_gemm"][0] + alg["down_gemm"][0]
-        by = alg["fused_bytes"]
-    else:
-        fl, by = alg[dom]
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    src = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
-    if fl / by >= ridge:
-        achieved = fl / per_launch_s / 1e12
-        roof = {"bound": "tensor", "unit": "TFLOP/s"}
-        if rotate:
-            # back-to-back steps run under the 1 kW power cap within tens of
-            # milliseconds: the kernel is timed inside a long run, so its
-            # denominator is the sustained (power-capped) cuBLAS figure
-            peak = peaks["bf16_tflops_sustained"]
-            src += ", sustained bf16 (timed inside back-to-back steps)"
-            roof["frac_of_burst_peak"] = round(achieved / peaks["bf16_tflops"], 4)
-        else:
-            peak = peaks["bf16_tflops"]
-            src += ", burst bf16"
-    else:
-        achieved = by / per_launch_s / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "unit": "GB/s"}
-        src += ", HBM copy"
-    traffic = NCU_TRAFFIC.get((cfg.name, dom))
-    roof.update({"kernel": dom, "achieved": round(achieved, 2), "peak": peak, "peak_source": src,
-                 "frac": round(achieved / peak, 4),
-                 "traffic": traffic,
-                 "traffic_vs_algorithmic": None if traffic is None else round(traffic / by, 3),
-                 "per_launch_us": round(per_launch_s * 1e6, 2), "per_launch_source": per_launch_src,
-                 "algorithmic_flops": fl, "algorithmic_bytes": by})
+    roof = roofline(cfg, alg, stages, total_ms, args.steps, launches_per_step, rotate, peaks, peak_src)
 
     r_s = router_ms / args.steps / 1e3
     r_flops = 2.0 * cfg.T * cfg.E * cfg.d
@@ -534,37 +591,74 @@ def run_ours(args):
               "roofline_note": "time at the slower of FLOPs / burst bf16 peak and bytes / HBM copy bandwidth, "
                                "over the measured time"}
 
-    line = {
-        "metric": METRIC, "value": round(value, 4), "unit": "TFLOPS", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
+    res = {
+        "value": round(value, 4), "unit": "TFLOPS", "ms_per_step": round(total_ms / args.steps, 5),
         "tokens_per_s": round(world * cfg.T / sec_per_step, 1),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded; random-init expert weights ~N(0,0.02))",
-        "config": {"workload": workload_desc(cfg), "global_batch": world * cfg.T,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": (f"inputs larger than L2: steps run back to back, each on one of {n_copies} copies of "
+        "config": job_config(cfg, world, alg["U"]),
+        "timing": {"l2": (f"inputs larger than L2: steps run back to back, each on one of {n_copies} copies of "
                           f"x, logits and the expert weights ({touched / 1e6:.1f} MB of weights read per step; "
                           f"a copy is reused after >= 2x L2 of other data)") if rotate else
                          "flushed before every timed step (write of 2x L2), outside the step's events",
                    "launch": ("one CUDA graph of the K timed steps, kernels chained by programmatic dependent "
                               "launch") if rotate else
-                             "CUDA graph of the step, kernels chained by programmatic dependent launch",
-                   "experts_hit": alg["U"], "flops_per_step": alg["flops_total"],
-                   "flops_routed_per_step": alg["flops_routed"]},
+                             "CUDA graph of the step, kernels chained by programmatic dependent launch"},
         "ms_per_step_eager": round(eager_ms / args.steps, 5),
-        "stages_us": {k: round(v[0] / max(v[1], 1) * 1e3, 2) for k, v in stages.items()},
-        "stages_source": stage_source,
+        "stages_us": {k: round(v[0] / max(v[1], 1) * 1e3, 2) for k, v in stages.items() if v[1]},
+        "stages_source": "CUDA events around each kernel in replayed graphs of the step",
         "roofline": roof,
         "router": router,
         "e2e": {"value": round(e2e_value, 4), "unit": "TFLOPS", "ms_per_step": round(e2e_ms / args.steps, 5),
                 "h2d_bytes_per_step": int(io_bytes),
                 "d2h_bytes_per_step": int(cfg.T * cfg.d * 2)},
         "gpu_launches": int(launches),
+        "launches_per_step": int(launches_per_step),
         "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = time_oracle(inp, steps=2, warmup=1, min_seconds=10.0)
-        line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    # free this workload's device memory before the next one
+    del sets, buf, wg, r_logits, r_ids, r_w, flush
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and cpu_seconds > 0:
+        res["cpu_baseline"] = cpu_baseline(inp, cpu_seconds)
+    return res
+
+
+def run_ours(args):
+    import torch
+
+    from grouped_gemm_gating_b200 import moe as M
+
+    world, rank, local, pg = dist_setup(args.gpus)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    M.load_library()
+    names = ORDER if args.workload == "all" else (args.workload,)
+    head = HEADLINE if args.workload == "all" else args.workload
+    results = {}
+    for name in names:
+        cpu_s = 0.0 if args.no_cpu_baseline else (10.0 if name == head else 3.0)
+        results[name] = measure_workload(name, args, dev, pg, world, rank, cpu_s)
+    h = results[head]
+    line = {
+        "metric": METRIC, "value": h["value"], "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": h["ms_per_step"],
+        "tokens_per_s": h["tokens_per_s"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random-init expert weights ~N(0,0.02))",
+        "config": h["config"],
+        "timing": h["timing"],
+        "ms_per_step_eager": h["ms_per_step_eager"],
+        "stages_us": h["stages_us"],
+        "stages_source": h["stages_source"],
+        "roofline": h["roofline"],
+        "router": h["router"],
+        "e2e": h["e2e"],
+        "gpu_launches": h["gpu_launches"],
+        "clocks": h["clocks"],
+    }
+    if "cpu_baseline" in h:
+        line["cpu_baseline"] = h["cpu_baseline"]
+    if len(names) > 1:
+        line["workloads"] = {n: results[n] for n in names}
     if pg is not None:
         pg.destroy_process_group()
     if rank == 0:
@@ -572,26 +666,32 @@ def run_ours(args):
 
 
 def run_reference(args):
+    """The CPU oracle, as it stands, on the host cores: the headline
+    workload's config, metric and unit, the same K steps after the same W
+    warm-up steps, each step a bounded token sample of the workload."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    cfg = W.CONFIGS[args.workload]
+    name = HEADLINE if args.workload == "all" else args.workload
+    cfg = W.CONFIGS[name]
     inp = W.make_inputs(cfg)
-    steps = min(args.steps, 20)
-    warm = min(args.warmup, 3)
-    cb = time_oracle(inp, steps=steps, warmup=warm)
-    steps = cb["steps"]
-    n = min(cfg.T, CPU_SAMPLE_TOKENS.get(cfg.name, 8))
+    import oracle
+    ids, _ = oracle.route(inp.logits, cfg.k, cfg.n_group, cfg.topk_group, cfg.group_score,
+                          bool(cfg.renormalize), cfg.routed_scaling)
+    experts_hit = int(np.unique(ids).size)
+    cb = time_oracle(inp, steps=args.steps, warmup=args.warmup, max_steps=args.steps)
+    info = cpu_info()
     line = {
         "impl": "reference", "metric": METRIC, "value": round(cb["value"], 6), "unit": "TFLOPS",
-        "n_gpus": world, "steps": steps, "warmup": warm,
-        "ms_per_step": round(n / cb["tokens_per_s"] * 1e3, 3), "tokens_per_s": round(cb["tokens_per_s"], 3),
+        "n_gpus": world, "steps": cb["steps"], "warmup": args.warmup,
+        "ms_per_step": round(cb["ms_per_step"], 3), "tokens_per_s": round(cb["tokens_per_s"], 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)",
-        "config": {"workload": workload_desc(cfg), "global_batch": cfg.T, "parallelism": "host CPU"},
+        "config": job_config(cfg, world, experts_hit),
         "cpu_baseline": {"value": round(cb["value"], 6), "unit": "TFLOPS", "cores": cb["cores"],
-                         "kind": "oracle", "sample": cb["sample"]},
+                         "kind": "oracle", "sample": cb["sample"], "host_nproc": info["nproc"],
+                         "cpu_model": info["model"]},
         "e2e": {"value": round(cb["value"], 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

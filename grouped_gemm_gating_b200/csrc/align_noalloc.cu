@@ -11,6 +11,8 @@
 // The multi-block align path needs per-chunk expert counts and bases; here
 // they live in a file-scope static __device__ array of fixed size, which
 // every GPU that loads this library holds until the process exits.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -28,9 +30,28 @@ static __device__ __align__(256) int32_t g_align_scratch[kScratchInts];
 
 // In host code g_align_scratch is only a host-side stand-in for the device
 // array, so its address must not be handed to a kernel.  The device address
-// is looked up once per device, with that device current, and cached.
+// is looked up with cudaGetSymbolAddress, with that device current, the first
+// time a device's context is seen, and cached next to that context: a new
+// context on the same device (after cudaDeviceReset, say) holds the array at
+// a new address, so a change of context makes the next call look it up again.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
 int32_t* scratch_on_current_device(cudaError_t* err) {
   static int32_t* cache[64] = {nullptr};
+  static CUcontext cache_ctx[64] = {nullptr};
   static std::mutex mu;
   int dev = 0;
   *err = cudaGetDevice(&dev);
@@ -39,12 +60,24 @@ int32_t* scratch_on_current_device(cudaError_t* err) {
     *err = cudaErrorInvalidDevice;
     return nullptr;
   }
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  CUcontext ctx = nullptr;
+  if (get_ctx == nullptr || get_ctx(&ctx) != CUDA_SUCCESS) {
+    *err = cudaErrorInitializationError;
+    return nullptr;
+  }
   std::lock_guard<std::mutex> lock(mu);
-  if (cache[dev] == nullptr) {
+  if (ctx == nullptr || cache[dev] == nullptr || cache_ctx[dev] != ctx) {
     void* p = nullptr;
+    // also makes the device's context current if no call has done so yet
     *err = cudaGetSymbolAddress(&p, g_align_scratch);
     if (*err != cudaSuccess) return nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) {
+      *err = cudaErrorInitializationError;
+      return nullptr;
+    }
     cache[dev] = static_cast<int32_t*>(p);
+    cache_ctx[dev] = ctx;
   }
   return cache[dev];
 }

@@ -223,6 +223,12 @@ moe_status check_align_args(const int32_t* topk_ids, int T, int k, int E, int bl
 
 namespace moe {
 void record_launches(int n) { g_last_launches = n; }
+
+// Set by moe_debug_timeouts; read when a launch's arguments are filled.
+std::atomic<uint64_t> g_wait_limit_ns{kWaitLimitNs};
+std::atomic<int> g_unreachable{0};
+uint64_t launch_wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+int launch_unreachable_arrivals() { return g_unreachable.load(std::memory_order_relaxed); }
 }  // namespace moe
 
 extern "C" {
@@ -381,6 +387,8 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
     fa.topk_w = topk_weights;
     fa.sync = counters;
     fa.status = dev_status;
+    fa.wait_ns = moe::launch_wait_limit_ns();
+    fa.start_surplus = moe::launch_unreachable_arrivals();
     fa.T = T;
     fa.k = k;
     fa.S = T * k;
@@ -431,6 +439,8 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
   a1.acc = y;  // zeroed on the side for the down GEMM
   a1.acc_elems = static_cast<int64_t>(T) * d;
   a1.status = dev_status;
+  a1.wait_ns = moe::launch_wait_limit_ns();
+  a1.tfull_surplus = moe::launch_unreachable_arrivals();
   a1.T = T;
   a1.k = k;
   a1.S = T * k;
@@ -485,6 +495,8 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
   a2.acc = y;
   a2.acc_elems = static_cast<int64_t>(T) * d;
   a2.status = dev_status;
+  a2.wait_ns = moe::launch_wait_limit_ns();
+  a2.tfull_surplus = moe::launch_unreachable_arrivals();
   a2.T = T;
   a2.k = k;
   a2.S = T * k;
@@ -567,6 +579,8 @@ moe_status moe_router(const uint16_t* x, int T, int d, const uint16_t* w_gate, i
   a.tm_w = a.tm_ws;
   if (!encode_2d(&a.tm_x, x, d, static_cast<uint64_t>(T), 128)) return MOE_ERR_CUDA;
   a.status = dev_status;
+  a.wait_ns = moe::launch_wait_limit_ns();
+  a.tfull_surplus = moe::launch_unreachable_arrivals();
   a.T = T;
   a.k = k;
   a.S = T * k;
@@ -724,6 +738,13 @@ const char* moe_status_string(moe_status status) {
 }
 
 int moe_last_launch_count(void) { return g_last_launches; }
+
+moe_status moe_debug_timeouts(uint64_t wait_limit_ns, int unreachable_arrivals) {
+  if (unreachable_arrivals < 0 || unreachable_arrivals > 1024) return MOE_ERR_INVALID_ARG;
+  moe::g_wait_limit_ns.store(wait_limit_ns == 0 ? moe::kWaitLimitNs : wait_limit_ns, std::memory_order_relaxed);
+  moe::g_unreachable.store(unreachable_arrivals, std::memory_order_relaxed);
+  return MOE_OK;
+}
 
 moe_status moe_profile_enable(int on) {
   if (on) release_records();  // a fresh record; disabling keeps the records readable

@@ -10,9 +10,20 @@
 namespace moe {
 
 constexpr int kWarp = 32;
-// Pipeline waits inside a kernel give up after this much wall time, set an
-// error in the status word and let the kernel return (no trap, no hang).
+// Pipeline waits inside a kernel give up after a wall-time limit (a launch
+// argument: kWaitLimitNs unless moe_debug_timeouts lowered it), set an error
+// in the status word and let the kernel return (no trap, no hang).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// After giving up, a role waits for its own asynchronous operations still in
+// flight (TMA loads, MMAs) before the CTA frees TMEM and exits; those waits
+// have their own limit, which the debug hook does not lower: the operations
+// complete on their own within microseconds.
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
+
+// Wait limit and start-barrier surplus for the next launches (process-wide;
+// set by moe_debug_timeouts, read when a launch's arguments are filled).
+uint64_t launch_wait_limit_ns();
+int launch_unreachable_arrivals();
 
 // Programmatic dependent launch: every kernel of the layer is launched with
 // programmatic stream serialisation, so it may start (prologue: barrier

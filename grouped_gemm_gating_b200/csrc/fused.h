@@ -37,8 +37,11 @@ struct FusedArgs {
   const int32_t* expert_ids;
   const int32_t* ntpp;
   const float* topk_w;  // [T * k]
-  int32_t* sync;        // [3] grid counters (zeroed, finished, released); zero at rest
+  int32_t* sync;        // [3] grid counters: CTAs that zeroed their accumulator slice, CTAs
+                        // finished (both zero at rest), release generation (any value)
   int32_t* status;
+  uint64_t wait_ns;     // limit of every pipeline and grid wait (kWaitLimitNs unless lowered for a test)
+  int start_surplus;    // extra arrivals the start barrier waits for (0; > 0 only in the timeout test)
   int T, k, S, E, d, F;
   int block_m;
   int max_routed_blocks;

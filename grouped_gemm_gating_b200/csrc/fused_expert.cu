@@ -39,10 +39,12 @@
 //   end:   every CTA counts itself on sync[1] once its reductions are issued;
 //          the last to arrive zeroes sync[0..1].  For a small output (T*d <=
 //          16384) that CTA converts the whole accumulator to bf16 and the
-//          others have already left.  Otherwise it stores -(G-1) in sync[2],
-//          which releases the others; each of them adds 1 back to sync[2] (so
-//          every counter is zero when the kernel ends), and every CTA
-//          converts its slice of the accumulator.
+//          others have already left.  Otherwise it moves the generation in
+//          sync[2] on by one, which releases the others (each read it before
+//          counting itself), and every CTA converts its slice of the
+//          accumulator.  A CTA that gave up on a wait counts itself and
+//          leaves, so sync[0..1] are zero after every launch, timeouts
+//          included, and sync[2] only ever moves forward.
 //
 // Tiles are dealt to the fewest CTAs that can take equal shares; the other
 // CTAs only zero and convert their slice of the accumulator.
@@ -163,6 +165,12 @@ __device__ __forceinline__ void gather_sync() {
   asm volatile("bar.sync 2, 128;" ::: "memory");
 }
 
+// Named barrier 4 over the producer warp and the four gather warps, at exit.
+__device__ __forceinline__ void exit_handshake() {
+  __syncwarp();
+  asm volatile("bar.sync 4, 160;" ::: "memory");
+}
+
 __device__ __forceinline__ bool epilogue_any(bool v) {
   uint32_t r;
   __syncwarp();
@@ -177,21 +185,22 @@ __device__ __forceinline__ bool epilogue_any(bool v) {
   return r != 0;
 }
 
-// Bounded spin until *p != 0 (acquire).  False on timeout or abort.
-__device__ __forceinline__ bool spin_until_nonzero(const int32_t* p, volatile int* abort_flag) {
+// Bounded spin until *p != v (acquire).  False on timeout.
+__device__ __forceinline__ bool spin_until_changed(const int32_t* p, int v, uint64_t limit_ns) {
   const uint64_t t0 = ptx::globaltimer_ns();
-  while (ptx::ld_acquire_gpu(p) == 0) {
-    if (*abort_flag || ptx::globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  while (ptx::ld_acquire_gpu(p) == v) {
+    if (ptx::globaltimer_ns() - t0 > limit_ns) return false;
     __nanosleep(64);
   }
   return true;
 }
 
 // Bounded spin until *p >= target (acquire).  False on timeout or abort.
-__device__ __forceinline__ bool spin_until(const int32_t* p, int target, volatile int* abort_flag) {
+__device__ __forceinline__ bool spin_until(const int32_t* p, int target, volatile int* abort_flag,
+                                           uint64_t limit_ns) {
   const uint64_t t0 = ptx::globaltimer_ns();
   while (ptx::ld_acquire_gpu(p) < target) {
-    if (*abort_flag || ptx::globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (*abort_flag || ptx::globaltimer_ns() - t0 > limit_ns) return false;
     __nanosleep(64);
   }
   return true;
@@ -218,6 +227,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(d2_empty + C::kD2Slots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* flag = reinterpret_cast<volatile int*>(tmem_holder + 2);
+  volatile int* prod_issued = reinterpret_cast<volatile int*>(tmem_holder + 3);  // stages the producer filled
 
   const int warp = threadIdx.x / kWarp;
   const int lane = threadIdx.x % kWarp;
@@ -390,13 +400,15 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
         return e;
       };
       auto acquire = [&]() {
-        if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+        if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.wait_ns)) {
           fail();
           ok = false;
         }
         return ok;
       };
+      int issued = 0;  // stages filled so far
       auto advance = [&]() {
+        ++issued;
         if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;
@@ -439,6 +451,29 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
           }
         }
       }
+      *prod_issued = issued;
+    }
+    // The last load into every stage lands before the CTA's shared memory is
+    // released.  After an abort some were never consumed, and a stage's
+    // phase completes only with the gather warps' arrivals too: they add the
+    // ones they did not make (exit_handshake), then the producer waits for
+    // the last phase of every stage it filled (at once after a normal run,
+    // where the MMA has waited for all of them).
+    exit_handshake();
+    exit_handshake();
+    if (lane == 0) {
+      const int issued = *prod_issued;
+      int stage = issued % C::kStages;
+      uint32_t phase = static_cast<uint32_t>((issued / C::kStages) & 1);
+      for (int j = 1; j <= C::kStages && j <= issued; ++j) {
+        int st = stage - j;
+        uint32_t ph = phase;
+        if (st < 0) {
+          st += C::kStages;
+          ph ^= 1u;
+        }
+        ptx::mbar_wait_bounded(&full[st], ph, flag, kDrainLimitNs);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
@@ -448,7 +483,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
       int d2c = 0;
       bool ok = true;
       auto wait = [&](uint64_t* bar, uint32_t parity) {
-        if (!ptx::mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs)) {
+        if (!ptx::mbar_wait_bounded(bar, parity, abort_flag, args.wait_ns)) {
           fail();
           ok = false;
         }
@@ -522,7 +557,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
       // no MMA of this CTA may still run when TMEM is freed (this wait
       // ignores the abort flag; *flag stays zero until the block barrier)
       ptx::mma_commit(mma_done);
-      if (!ptx::mbar_wait_bounded(mma_done, 0u, flag, kWaitLimitNs)) fail();
+      if (!ptx::mbar_wait_bounded(mma_done, 0u, flag, kDrainLimitNs)) fail();
     }
   } else if (warp < 6) {
     // ------------------------------------------------ epilogue
@@ -583,8 +618,8 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
           tok_s[b * 64 + j] = tok;
           w_s[b * 64 + j] = wj;
         }
-        const bool got = ptx::mbar_wait_bounded(&d1_full[b], bph, abort_flag, kWaitLimitNs) &&
-                         ptx::mbar_wait_bounded(&hb_empty[b], bph ^ 1u, abort_flag, kWaitLimitNs);
+        const bool got = ptx::mbar_wait_bounded(&d1_full[b], bph, abort_flag, args.wait_ns) &&
+                         ptx::mbar_wait_bounded(&hb_empty[b], bph ^ 1u, abort_flag, args.wait_ns);
         if (epilogue_any(!got)) {
           if (!got) fail();
           break;
@@ -642,7 +677,8 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
         const int b = p & 1;
         // every CTA has zeroed its slice of the accumulator before anyone adds
         if (!zero_seen) {
-          const bool got = etid != 0 || spin_until(args.sync, static_cast<int>(gridDim.x), abort_flag);
+          const bool got = etid != 0 || spin_until(args.sync, static_cast<int>(gridDim.x) + args.start_surplus,
+                                                   abort_flag, args.wait_ns);
           if (epilogue_any(!got)) {
             if (!got) fail();
             break;
@@ -665,7 +701,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
         for (int g = 0; g < n_g; ++g, ++d2c) {
           const int slot = d2c % C::kD2Slots;
           const uint32_t sph = static_cast<uint32_t>((d2c / C::kD2Slots) & 1);
-          const bool got = ptx::mbar_wait_bounded(&d2_full[slot], sph, abort_flag, kWaitLimitNs);
+          const bool got = ptx::mbar_wait_bounded(&d2_full[slot], sph, abort_flag, args.wait_ns);
           if (epilogue_any(!got)) {
             if (!got) fail();
             left = true;
@@ -726,14 +762,16 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    int arrived = 0;  // stages this thread has arrived on
     auto acquire = [&]() {
-      if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+      if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.wait_ns)) {
         fail();
         ok = false;
       }
       return ok;
     };
     auto advance = [&]() {
+      ++arrived;
       if (++stage == C::kStages) {
         stage = 0;
         phase ^= 1u;
@@ -783,6 +821,14 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
       }
     }
     cp_async_wait_all();
+    // after an abort: arrive on every stage the producer filled and this
+    // thread did not, so that the producer can wait for its own loads
+    exit_handshake();
+    for (const int target = *prod_issued; arrived < target;) {
+      ptx::mbar_arrive(&full[stage]);
+      advance();
+    }
+    exit_handshake();
   }
 
   // every warp reconverges (the idle lanes of the producer and MMA warps
@@ -794,14 +840,17 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
   // sync[1] counts the CTAs that have issued all their reductions; the last
   // one to arrive returns sync[0] and sync[1] to zero.  A small output is
   // then converted by that CTA alone while the others leave.  Otherwise the
-  // last CTA releases the others by storing -(G-1) in sync[2]; each released
-  // CTA adds 1 to sync[2] as it goes (fire-and-forget) and converts its slice,
-  // so all three counters are zero again when the kernel completes and no CTA
-  // waits on another round of atomics to exit.
+  // last CTA releases the others by moving the generation in sync[2] on by
+  // one (each CTA read it before counting itself, and waits for it to
+  // change) and every CTA converts its slice.  A CTA that gave up (a wait
+  // ran out) counts itself and leaves; since nothing is handed back, the
+  // counters are consistent for the next launch whichever CTAs gave up.
   const bool last_converts = nacc <= kLastCtaConvertMax;
   if (threadIdx.x == 0) {
     const int G = static_cast<int>(gridDim.x);
-    bool all = true;
+    const bool aborted = *abort_flag != 0;  // final: every role has finished
+    // the last CTA moves the generation on only after this CTA's count below
+    const int gen = ptx::ld_acquire_gpu(args.sync + 2);
     int mode = 0;  // 0: leave, 1: convert this CTA's slice, 2: convert everything
     if (ptx::atom_acq_rel_gpu_add(args.sync + 1, 1) == G - 1) {  // releases this CTA's reductions
       args.sync[0] = 0;
@@ -809,15 +858,15 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
       if (last_converts) {
         mode = 2;
       } else {
-        ptx::st_release_gpu(args.sync + 2, -(G - 1));
+        ptx::st_release_gpu(args.sync + 2, static_cast<int>(static_cast<uint32_t>(gen) + 1u));
         mode = 1;
       }
-    } else if (!last_converts) {
-      all = spin_until_nonzero(args.sync + 2, abort_flag);
-      if (all) ptx::red_relaxed_gpu_add(args.sync + 2, 1);
-      mode = all ? 1 : 0;
+    } else if (!last_converts && !aborted) {
+      if (spin_until_changed(args.sync + 2, gen, args.wait_ns))
+        mode = 1;
+      else
+        fail();
     }
-    if (!all) fail();
     *flag = mode;
   }
   if (warp == 1) {  // TMEM is freed while thread 0 waits at the grid barrier

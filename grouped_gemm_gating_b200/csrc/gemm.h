@@ -32,6 +32,8 @@ struct GemmArgs {
   float* acc;           // fp32 [T, d] accumulator: zeroed by the gate/up GEMM, reduced into by the down GEMM
   int64_t acc_elems;    // T * d
   int32_t* status;
+  uint64_t wait_ns;     // limit of every pipeline wait (kWaitLimitNs unless lowered for a test)
+  int tfull_surplus;    // extra arrivals the accumulator-full barriers expect (0; > 0 only in the timeout test)
   int T, k, S, E;
   int K;                // reduction length (multiple of 64)
   int n_out;            // output columns (multiple of 16)

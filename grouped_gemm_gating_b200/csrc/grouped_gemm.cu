@@ -71,7 +71,7 @@ struct GemmCfg {
   static constexpr int kEpiWarps = EPI == kEpiScale ? 8 : 4;
   static constexpr int kNumThreads = kGather ? 352 : 64 + 32 * kEpiWarps;
   static constexpr uint32_t kTxBytes = kWBytes + (kGather ? 0 : kXBytes);
-  static constexpr int kBarrierBytes = 256;
+  static constexpr int kBarrierBytes = 512;
   // down GEMM: per epilogue warp a 32 x 33 fp32 transpose buffer, so the
   // reduction is issued as full 128-byte row segments
   static constexpr int kRedStride = 33;
@@ -81,7 +81,7 @@ struct GemmCfg {
 
   static_assert(kStages >= 3, "pipeline depth");
   static_assert(kAccCols * 2 <= kTmemCols, "two accumulator buffers must fit TMEM");
-  static_assert((2 * kStages + 4) * 8 + 8 <= kBarrierBytes, "barrier area");
+  static_assert((2 * kStages + 5) * 8 + 16 <= kBarrierBytes, "barrier area");
   static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
 
@@ -114,6 +114,12 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, int n_wt, int pass_w, 
 // to bf16 right after, far coarser than the divide's error.
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
+// Named barrier 4 over the producer warp and the four gather warps, at exit.
+__device__ __forceinline__ void exit_handshake() {
+  __syncwarp();
+  asm volatile("bar.sync 4, 160;" ::: "memory");
+}
+
 __device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
@@ -129,8 +135,11 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* mma_done = tempty + 2;       // the MMA issuer's last commit (drain before TMEM is freed)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* never = reinterpret_cast<volatile int*>(tmem_holder + 2);  // stays 0: drains ignore the abort
+  volatile int* prod_issued = reinterpret_cast<volatile int*>(tmem_holder + 3);  // stages the producer filled
 
   const int warp = threadIdx.x / kWarp;
   const int lane = threadIdx.x % kWarp;
@@ -141,10 +150,12 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
       ptx::mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(&tfull[b], 1);
+      ptx::mbar_init(&tfull[b], 1 + args.tfull_surplus);
       ptx::mbar_init(&tempty[b], C::kEpiWarps);
     }
+    ptx::mbar_init(mma_done, 1);
     *abort_flag = 0;
+    *never = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
@@ -187,6 +198,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      int issued = 0;  // stages filled so far
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
         const TileCoord tc = tile_coord(tile, n_wt, pass_w, total_blocks, routed_blocks);
         const CUtensorMap* tm = tc.shared_blk ? &args.tm_ws : &args.tm_w;
@@ -197,7 +209,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
         }
         const int row0 = tc.wt * C::kBoxRows;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+          if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.wait_ns)) {
             fail();
             ok = false;
             break;
@@ -208,11 +220,37 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
           if (C::kGated)
             ptx::tma_load_3d(sW + C::kBoxRows * 128, tm, &full[stage], kb * 64, args.up_row_offset + row0, e);
           if (!C::kGather) ptx::tma_load_2d(sW + C::kWBytes, &args.tm_x, &full[stage], kb * 64, tc.blk * args.block_m);
+          ++issued;
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
+      }
+      *prod_issued = issued;
+    }
+    // The last load into every stage lands before the CTA's shared memory is
+    // released.  After an abort some were never consumed; with gathered
+    // rows a stage's phase completes only with the gather warps' arrivals
+    // too, so they first add the ones they did not make (exit_handshake).
+    // Then the producer waits for the last phase of every stage it filled
+    // (at once after a normal run, where the MMA has waited for all of them).
+    if (C::kGather) {
+      exit_handshake();
+      exit_handshake();
+    }
+    if (lane == 0) {
+      const int issued = *prod_issued;
+      const int stage = issued % C::kStages;
+      const uint32_t phase = static_cast<uint32_t>((issued / C::kStages) & 1);
+      for (int j = 1; j <= C::kStages && j <= issued; ++j) {
+        int st = stage - j;
+        uint32_t ph = phase;
+        if (st < 0) {
+          st += C::kStages;
+          ph ^= 1u;
+        }
+        ptx::mbar_wait_bounded(&full[st], ph, never, kDrainLimitNs);
       }
     }
   } else if (warp == 1) {
@@ -224,14 +262,14 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
       uint32_t aphase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        if (!ptx::mbar_wait_bounded(&tempty[abuf], aphase ^ 1u, abort_flag, kWaitLimitNs)) {
+        if (!ptx::mbar_wait_bounded(&tempty[abuf], aphase ^ 1u, abort_flag, args.wait_ns)) {
           fail();
           break;
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * C::kAccCols);
         for (int kb = 0; kb < nk; ++kb) {
-          if (!ptx::mbar_wait_bounded(&full[stage], phase, abort_flag, kWaitLimitNs)) {
+          if (!ptx::mbar_wait_bounded(&full[stage], phase, abort_flag, args.wait_ns)) {
             fail();
             ok = false;
             break;
@@ -259,6 +297,9 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
           aphase ^= 1u;
         }
       }
+      // no MMA of this CTA may still run when TMEM is freed
+      ptx::mma_commit(mma_done);
+      if (!ptx::mbar_wait_bounded(mma_done, 0u, never, kDrainLimitNs)) fail();
     }
   } else if (warp < 2 + C::kEpiWarps) {
     // ------------------------------------------------ epilogue
@@ -268,7 +309,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
     uint32_t aphase = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       const TileCoord tc = tile_coord(tile, n_wt, pass_w, total_blocks, routed_blocks);
-      if (!ptx::mbar_wait_bounded(&tfull[abuf], aphase, abort_flag, kWaitLimitNs)) {
+      if (!ptx::mbar_wait_bounded(&tfull[abuf], aphase, abort_flag, args.wait_ns)) {
         fail();
         break;
       }
@@ -506,6 +547,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    int arrived = 0;  // stages this thread has arrived on
     for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
       const TileCoord tc = tile_coord(tile, n_wt, pass_w, total_blocks, routed_blocks);
       const uint16_t* src[kRowsPerThread];
@@ -528,7 +570,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
         nbytes[i] = valid ? 16u : 0u;
       }
       for (int kb = 0; kb < nk; ++kb) {
-        if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+        if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.wait_ns)) {
           fail();
           ok = false;
           break;
@@ -541,12 +583,25 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
           ptx::cp_async_16(dst, src[i] + kb * 64, nbytes[i]);
         }
         ptx::cp_async_arrive_noinc(&full[stage]);
+        ++arrived;
         if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's rows have landed
+    // after an abort: arrive on every stage the producer filled and this
+    // thread did not, so that the producer can wait for its own loads
+    exit_handshake();
+    for (const int target = *prod_issued; arrived < target; ++arrived) {
+      ptx::mbar_arrive(&full[stage]);
+      if (++stage == C::kStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    exit_handshake();
   }
 
   // every warp reconverges (the idle lanes of the producer and MMA warps

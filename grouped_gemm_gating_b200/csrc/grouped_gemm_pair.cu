@@ -25,9 +25,10 @@
 // of 48 KB, so the same shared memory holds six stages instead of four.
 //
 // Every mbarrier wait is bounded; on expiry the CTA records
-// MOE_ERR_DEVICE_TIMEOUT and its roles leave their loops.  Both CTAs always
-// reach the closing cluster barrier, which orders the peer's last remote
-// arrivals before either CTA frees its TMEM and exits.
+// MOE_ERR_DEVICE_TIMEOUT and its roles leave their loops; the even CTA then
+// waits for its MMAs and for its stages' loads still in flight.  Both CTAs
+// always reach the closing cluster barrier, which orders the peer's last
+// remote arrivals before either CTA frees its TMEM and exits.
 #include <atomic>
 #include "common.cuh"
 #include "gemm.h"
@@ -36,6 +37,10 @@
 namespace moe {
 
 namespace {
+
+// After an abort, the odd CTA's wait for its last loads to land (they
+// complete on the even CTA's barriers): far above a TMA load's latency.
+constexpr uint64_t kDrainGraceNs = 50000;
 
 template <int EPI>
 struct PairCfg {
@@ -56,7 +61,7 @@ struct PairCfg {
   static constexpr int kUnitBytes = kMaxUnits * 4;
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + kRedBytes + kUnitBytes + 1024;
   static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(256, 256);
-  static_assert((2 * kStages + 4) * 8 + 8 <= kBarrierBytes, "barrier area");
+  static_assert((2 * kStages + 5) * 8 + 16 <= kBarrierBytes, "barrier area");
   static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
 
@@ -85,8 +90,10 @@ __global__ void __launch_bounds__(PairCfg<EPI>::kNumThreads, 1)
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* mma_done = tempty + 2;  // even CTA: the MMA issuer's last commit (drain before TMEM is freed)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* never = reinterpret_cast<volatile int*>(tmem_holder + 3);  // stays 0: drains ignore the abort
   float* red_buf = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + C::kBarrierBytes);
   int* unit_b0 = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(red_buf) + C::kRedBytes);
 
@@ -102,10 +109,12 @@ __global__ void __launch_bounds__(PairCfg<EPI>::kNumThreads, 1)
       ptx::mbar_init(&empty[s], 1);  // one commit of the pair's MMA
     }
     for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(&tfull[b], 1);
+      ptx::mbar_init(&tfull[b], 1 + args.tfull_surplus);
       ptx::mbar_init(&tempty[b], 8);  // even CTA: four epilogue warps of each CTA
     }
+    ptx::mbar_init(mma_done, 1);
     *abort_flag = 0;
+    *never = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&args.tm_w);
     if (args.n_shared_blocks) ptx::prefetch_tmap(&args.tm_ws);
@@ -185,6 +194,7 @@ __global__ void __launch_bounds__(PairCfg<EPI>::kNumThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      int issued = 0;  // stages filled so far
       for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
         const PairTile t = tile_of(tile);
         const CUtensorMap* tm = t.shared_blk ? &args.tm_ws : &args.tm_w;
@@ -199,7 +209,7 @@ __global__ void __launch_bounds__(PairCfg<EPI>::kNumThreads, 1)
         const int wrow = C::kGated ? t.wt * 128 + (rank ? args.up_row_offset : 0)
                                    : t.wt * 256 + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!ptx::mbar_wait_cluster_bounded(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+          if (!ptx::mbar_wait_cluster_bounded(&empty[stage], phase ^ 1u, abort_flag, args.wait_ns)) {
             fail();
             ok = false;
             break;
@@ -208,10 +218,32 @@ __global__ void __launch_bounds__(PairCfg<EPI>::kNumThreads, 1)
           if (rank == 0) ptx::mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
           ptx::tma_load_2d_pair(sA, &args.tm_x, &full[stage], kb * 64, blk * args.block_m);
           ptx::tma_load_3d_pair(sA + C::kABytes, tm, &full[stage], kb * 64, wrow, e);
+          ++issued;
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1u;
           }
+        }
+      }
+      // The even CTA's full barriers count both CTAs' bytes: before the pair
+      // releases its shared memory, the even CTA waits for the last phase of
+      // every stage it filled (at once after a normal run).  The odd CTA's
+      // loads complete only on the even CTA's barriers, which it cannot wait
+      // on; after an abort it may have filled a phase the even CTA never
+      // did, so it then gives its last loads a fixed grace period to land.
+      if (rank != 0 && !ok) {
+        const uint64_t t0 = ptx::globaltimer_ns();
+        while (ptx::globaltimer_ns() - t0 < kDrainGraceNs) __nanosleep(256);
+      }
+      if (rank == 0) {
+        for (int j = 1; j <= C::kStages && j <= issued; ++j) {
+          int st = stage - j;
+          uint32_t ph = phase;
+          if (st < 0) {
+            st += C::kStages;
+            ph ^= 1u;
+          }
+          ptx::mbar_wait_cluster_bounded(&full[st], ph, never, kDrainLimitNs);
         }
       }
     }
@@ -224,14 +256,14 @@ __global__ void __launch_bounds__(PairCfg<EPI>::kNumThreads, 1)
       uint32_t aphase = 0;
       bool ok = true;
       for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
-        if (!ptx::mbar_wait_cluster_bounded(&tempty[abuf], aphase ^ 1u, abort_flag, kWaitLimitNs)) {
+        if (!ptx::mbar_wait_cluster_bounded(&tempty[abuf], aphase ^ 1u, abort_flag, args.wait_ns)) {
           fail();
           break;
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * C::kAccCols);
         for (int kb = 0; kb < nk; ++kb) {
-          if (!ptx::mbar_wait_cluster_bounded(&full[stage], phase, abort_flag, kWaitLimitNs)) {
+          if (!ptx::mbar_wait_cluster_bounded(&full[stage], phase, abort_flag, args.wait_ns)) {
             fail();
             ok = false;
             break;
@@ -256,6 +288,14 @@ __global__ void __launch_bounds__(PairCfg<EPI>::kNumThreads, 1)
           aphase ^= 1u;
         }
       }
+      // no MMA of the pair may still run when TMEM is freed: the last commit
+      // arrives on both CTAs' mma_done (every tcgen05 operation of the kernel
+      // is a cta_group::2 one)
+      ptx::mma_commit_pair(mma_done);
+      if (!ptx::mbar_wait_bounded(mma_done, 0u, never, kDrainLimitNs)) fail();
+    } else if (lane == 0) {
+      // odd CTA: the even CTA's final commit also arrives here
+      if (!ptx::mbar_wait_cluster_bounded(mma_done, 0u, never, kDrainLimitNs)) fail();
     }
   } else if (warp < 6) {
     // ------------------------------------------------ epilogue (both CTAs, own TMEM half)
@@ -268,7 +308,7 @@ __global__ void __launch_bounds__(PairCfg<EPI>::kNumThreads, 1)
     uint32_t aphase = 0;
     for (int tile = pair; tile < total_tiles; tile += n_pairs) {
       const PairTile t = tile_of(tile);
-      if (!ptx::mbar_wait_cluster_bounded(&tfull[abuf], aphase, abort_flag, kWaitLimitNs)) {
+      if (!ptx::mbar_wait_cluster_bounded(&tfull[abuf], aphase, abort_flag, args.wait_ns)) {
         fail();
         break;
       }

@@ -49,6 +49,7 @@ _SIG = {
     "moe_read_status": (_I, [_P, _P]),
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_last_launch_count": (_I, []),
+    "moe_debug_timeouts": (_I, [ctypes.c_uint64, _I]),
     "moe_profile_enable": (_I, [_I]),
     "moe_profile_collect": (_I, [_P, _P, _I, _I]),
 }
@@ -133,6 +134,13 @@ def moe_workspace_size(T, d, F, E, k, block_m, act, n_shared) -> int:
 
 def moe_last_launch_count() -> int:
     return int(load_library().moe_last_launch_count())
+
+
+def moe_debug_timeouts(wait_limit_ns: int = 0, unreachable_arrivals: int = 0) -> None:
+    """Test hook: the wait limit of kernels launched afterwards (0: the
+    default 2 s) and, when unreachable_arrivals > 0, a start barrier in the
+    fused expert kernel that waits for more CTAs than its grid has."""
+    _check("moe_debug_timeouts", load_library().moe_debug_timeouts(int(wait_limit_ns), int(unreachable_arrivals)))
 
 
 def moe_profile_enable(on: bool = True) -> None:

@@ -110,9 +110,13 @@ MOE_API size_t moe_align_workspace_size(int T, int k, int E);
  * P_total = P_max + n_shared * ceil(T / block_m) * block_m.
  * The counter block (the first 64 KiB after rounding ws up to 256 bytes)
  * must be zero before the first moe_forward on a workspace (allocate it
- * zero-filled or cudaMemset it once); every moe_forward leaves it at zero
- * again, so a workspace can be reused across calls and layer shapes as long
- * as nothing else writes that block.  Returns 0 on invalid arguments. */
+ * zero-filled or cudaMemset it once).  The kernels keep it consistent from
+ * one call to the next -- also after a call whose kernel gave up on a wait
+ * (MOE_ERR_DEVICE_TIMEOUT): every CTA counts itself out on every exit path,
+ * the last one returns the two grid counters to zero, and the third word is
+ * a release generation that only moves forward -- so a workspace can be
+ * reused across calls and layer shapes, errors included, as long as nothing
+ * else writes that block.  Returns 0 on invalid arguments. */
 MOE_API size_t moe_workspace_size(int T, int d, int F, int E, int k, int block_m,
                           moe_act act, int n_shared);
 
@@ -214,11 +218,12 @@ MOE_API moe_status moe_align(const int32_t* topk_ids, int T, int k, int E, int b
  *                of that sum (one bf16 ulp of a result, a little more where
  *                the k terms cancel).  inv_pos is accepted for
  *                interface stability and not read (it may be NULL).
- *   ws, ws_bytes scratch of moe_workspace_size bytes (its counter block zero,
- *                see moe_workspace_size); calls sharing a workspace must not
- *                overlap on the GPU.
+ *   ws, ws_bytes scratch of moe_workspace_size bytes (its counter block zero
+ *                before the first call, see moe_workspace_size); calls sharing
+ *                a workspace must not overlap on the GPU.
  * Errors: host checks as above; MOE_ERR_DEVICE_TIMEOUT in dev_status if a
- * pipeline wait inside a GEMM kernel exceeded its limit (out is then invalid).
+ * pipeline wait inside a GEMM kernel exceeded its limit (out is then invalid;
+ * the workspace stays usable for the next call).
  */
 MOE_API moe_status moe_forward(const uint16_t* x, int T, int d,
                        const uint16_t* w13, const uint16_t* w2, int E, int F,
@@ -243,8 +248,10 @@ MOE_API moe_status moe_forward(const uint16_t* x, int T, int d,
  *   larger problems return MOE_ERR_UNSUPPORTED and launch nothing.
  *   Every GPU that loads the library holds the 1 MiB until the process exits.
  *   The first call on a device looks up the array's device address (one
- *   cudaGetSymbolAddress, cached per device); make that first call before
- *   any stream capture.  It allocates nothing, ever.
+ *   cudaGetSymbolAddress, cached per device together with its context, and
+ *   looked up again when the device's context changes, e.g. after
+ *   cudaDeviceReset); make that first call, and the first after such a
+ *   change, before any stream capture.  It allocates nothing, ever.
  *   All calls share the one array and it keeps the last call's contents
  *   (nothing in it needs to start at zero); calls whose kernels overlap on
  *   the GPU (other streams, other host threads) race on it and must be
@@ -312,6 +319,29 @@ MOE_API const char* moe_status_string(moe_status status);
 /* Number of kernel launches the most recent successful call on this host
  * thread issued (for launch accounting in benchmarks). */
 MOE_API int moe_last_launch_count(void);
+
+/*
+ * moe_debug_timeouts -- test hook for the bounded waits; not for production.
+ * No passage of the source pages has a counterpart: it exists so that tests
+ * can drive the error path of the kernels' pipeline waits without faulting
+ * or hanging the GPU.  Every wait inside the library's kernels (mbarrier
+ * phases, grid counters) gives up after a time limit, records
+ * MOE_ERR_DEVICE_TIMEOUT in dev_status, waits for its own TMA loads and MMAs
+ * still in flight, frees its tensor memory and returns.
+ *   wait_limit_ns         limit for kernels launched afterwards, from any
+ *                         host thread (0 restores the default of 2 s).
+ *   unreachable_arrivals  > 0: kernels launched afterwards wait for that many
+ *                         more arrivals than ever come, so the wait runs out
+ *                         after the limit: the fused expert kernel (block_m
+ *                         <= 64) at its start barrier (more CTAs than its
+ *                         grid has), the grouped GEMM kernels (block_m = 128,
+ *                         the router's tensor-core path) at their first
+ *                         accumulator-full barrier (more commits than the
+ *                         MMA issuer makes); 0 restores normal launches.
+ * Process-wide; calls that overlap a launch in another thread race with it.
+ * MOE_ERR_INVALID_ARG for unreachable_arrivals outside [0, 1024].
+ */
+MOE_API moe_status moe_debug_timeouts(uint64_t wait_limit_ns, int unreachable_arrivals);
 
 /* Stage profiling (host-thread local).  While enabled, every moe_route,
  * moe_align and moe_forward call records a pair of CUDA events on its stream
