@@ -30,6 +30,12 @@ Sources (web pages on fused MoE kernels):
 * the same axolotl diff, scripts/benchmarks/deepseek_v3_moe.py
   ``timed_forward``: the block's gate maps the flattened hidden states to the
   top-k expert ids and weights (router projection, then gating).
+* backward: the same diff's grouped-GEMM backward kernels,
+  src/axolotl/kernels/moe/tt_cg_gemm/cg_backward.py (``_kernel_cg_backward_dx``:
+  the gradient of the token rows from dY and each expert's weights;
+  ``_kernel_cg_backward_dw``: each expert's weight gradient summed over the
+  rows routed to it) and the Gemma-4 MoE training note (the expert path of a
+  training step, forward and backward), restated as the chain rule.
 
 Readings where the pages are silent (each is also listed in the design notes):
 
@@ -193,7 +199,11 @@ def expert_hidden(x: np.ndarray, w13_e: np.ndarray, act: int) -> np.ndarray:
     projection; h = silu(gate) * up.  Squared ReLU: w13_e is fc1 [F, d] and
     h = max(fc1 x, 0)^2.
     """
-    W1 = bf16_to_f64(w13_e)
+    return hidden_values(x, bf16_to_f64(w13_e), act)
+
+
+def hidden_values(x: np.ndarray, W1: np.ndarray, act: int) -> np.ndarray:
+    """expert_hidden on an fp64 weight array W1 [n1, d] (any values)."""
     if act == ACT_SWIGLU:
         F = W1.shape[0] // 2
         g = x @ W1[:F].T
@@ -234,4 +244,122 @@ def forward(x_bits: np.ndarray, w13: np.ndarray, w2: np.ndarray,
     if w13_shared is not None:
         for s in range(w13_shared.shape[0]):
             out += expert_mlp(x, w13_shared[s], w2_shared[s], act)
+    return out
+
+
+# --------------------------------------------------------------------------
+# Backward
+# --------------------------------------------------------------------------
+#
+# The training pass of the same layer: given dL/dout, the gradients of the
+# loss with respect to the tokens, both expert weight stacks and the top-k
+# weights.  The pages motivate it by training (the Gemma-4 MoE note: the
+# Python-loop expert path dominates a training step; the axolotl diff's
+# grouped-GEMM backward kernels compute the gradient of the token rows, dX,
+# and of every expert's weights, dW, from the grouped layout).  Here it is
+# the chain rule through each expert's MLP, written out per expert over the
+# rows routed to it, with no blocking and nothing rounded.
+
+
+def silu_grad(z: np.ndarray) -> np.ndarray:
+    """Derivative of silu(z) = z * sigmoid(z): sigmoid(z) * (1 + z * (1 - sigmoid(z)))."""
+    sg = 1.0 / (1.0 + np.exp(-z))
+    return sg * (1.0 + z * (1.0 - sg))
+
+
+def expert_backward_values(x: np.ndarray, W13: np.ndarray, W2: np.ndarray, dy: np.ndarray, act: int):
+    """One expert y = W2 act(W13 x) on rows x [n, d], all fp64 arrays, with
+    dL/dy = dy [n, d].  Returns (dx [n, d], dW13 [n1, d], dW2 [d, F], y [n, d]).
+
+    SwiGLU: a = [g; u] = W13 x (gate rows first), h = silu(g) * u,
+    dh = W2^T dy, dg = dh * u * silu'(g), du = dh * silu(g).
+    Squared ReLU: a = W13 x, h = max(a, 0)^2, da = dh * 2 max(a, 0).
+    Then dx = W13^T da, dW13 = sum over rows of da x^T, dW2 = sum of dy h^T.
+    """
+    dh = dy @ W2                                   # [n, F]
+    if act == ACT_SWIGLU:
+        F = W13.shape[0] // 2
+        g = x @ W13[:F].T
+        u = x @ W13[F:].T
+        h = silu(g) * u
+        da = np.concatenate([dh * u * silu_grad(g), dh * silu(g)], axis=1)
+    elif act == ACT_RELU2:
+        a = x @ W13.T
+        h = np.maximum(a, 0.0) ** 2
+        da = dh * 2.0 * np.maximum(a, 0.0)
+    else:
+        raise ValueError("unknown activation")
+    return da @ W13, da.T @ x, dy.T @ h, h @ W2.T
+
+
+def backward_values(x: np.ndarray, W13: np.ndarray, W2: np.ndarray, topk_ids: np.ndarray,
+                    topk_weights: np.ndarray, act: int, dout: np.ndarray,
+                    W13_shared: np.ndarray | None = None, W2_shared: np.ndarray | None = None) -> dict:
+    """Gradients of out[t] = sum_j w[t,j] * expert_{ids[t,j]}(x[t]) (+ shared(x[t]))
+    for dL/dout = dout, on fp64 arrays: x [T, d], W13 [E, n1, d], W2 [E, d, F].
+
+    Per expert e and the rows (t, j) routed to it: the expert sees dL/dy =
+    w[t,j] * dout[t]; dL/dw[t,j] = dout[t] . y_e(x[t]).  Returns a dict with
+    dx [T, d], dw13 [E, n1, d], dw2 [E, d, F], dtopk_weights [T, k] and,
+    with a shared expert, dw13_shared / dw2_shared [n_shared, ...].
+    """
+    ids = np.asarray(topk_ids)
+    wts = np.asarray(topk_weights, dtype=np.float64)
+    T, d = x.shape
+    E = W13.shape[0]
+    dx = np.zeros((T, d), dtype=np.float64)
+    dw13 = np.zeros(W13.shape, dtype=np.float64)
+    dw2 = np.zeros(W2.shape, dtype=np.float64)
+    dtopk = np.zeros(ids.shape, dtype=np.float64)
+    for e in range(E):
+        t_idx, j_idx = np.nonzero(ids == e)
+        if t_idx.size == 0:
+            continue
+        w = wts[t_idx, j_idx][:, None]
+        gx, gw13, gw2, y = expert_backward_values(x[t_idx], W13[e], W2[e], w * dout[t_idx], act)
+        np.add.at(dx, t_idx, gx)
+        dw13[e] = gw13
+        dw2[e] = gw2
+        dtopk[t_idx, j_idx] = np.sum(dout[t_idx] * y, axis=1)
+    res = {"dx": dx, "dw13": dw13, "dw2": dw2, "dtopk_weights": dtopk}
+    if W13_shared is not None:
+        ns = W13_shared.shape[0]
+        res["dw13_shared"] = np.zeros(W13_shared.shape, dtype=np.float64)
+        res["dw2_shared"] = np.zeros(W2_shared.shape, dtype=np.float64)
+        for i in range(ns):
+            gx, gw13, gw2, _ = expert_backward_values(x, W13_shared[i], W2_shared[i], dout, act)
+            dx += gx
+            res["dw13_shared"][i] = gw13
+            res["dw2_shared"][i] = gw2
+    return res
+
+
+def backward(x_bits: np.ndarray, w13: np.ndarray, w2: np.ndarray, topk_ids: np.ndarray,
+             topk_weights: np.ndarray, act: int, dout_bits: np.ndarray,
+             w13_shared: np.ndarray | None = None, w2_shared: np.ndarray | None = None) -> dict:
+    """backward_values over the exact values of bf16 inputs (x, weights and
+    dL/dout as uint16 bit patterns; topk_weights as given)."""
+    return backward_values(bf16_to_f64(x_bits), bf16_to_f64(w13), bf16_to_f64(w2), topk_ids, topk_weights,
+                           act, bf16_to_f64(dout_bits),
+                           None if w13_shared is None else bf16_to_f64(w13_shared),
+                           None if w2_shared is None else bf16_to_f64(w2_shared))
+
+
+def forward_values(x: np.ndarray, W13: np.ndarray, W2: np.ndarray, topk_ids: np.ndarray,
+                   topk_weights: np.ndarray, act: int, W13_shared: np.ndarray | None = None,
+                   W2_shared: np.ndarray | None = None) -> np.ndarray:
+    """forward on fp64 arrays of any values (x [T, d], W13 [E, n1, d],
+    W2 [E, d, F]): sequential per-expert matmuls with top-k selection."""
+    ids = np.asarray(topk_ids)
+    wts = np.asarray(topk_weights, dtype=np.float64)
+    out = np.zeros(x.shape, dtype=np.float64)
+    for e in range(W13.shape[0]):
+        t_idx, j_idx = np.nonzero(ids == e)
+        if t_idx.size == 0:
+            continue
+        y = hidden_values(x[t_idx], W13[e], act) @ W2[e].T
+        np.add.at(out, t_idx, wts[t_idx, j_idx][:, None] * y)
+    if W13_shared is not None:
+        for i in range(W13_shared.shape[0]):
+            out += hidden_values(x, W13_shared[i], act) @ W2_shared[i].T
     return out
