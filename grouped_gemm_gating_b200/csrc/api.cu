@@ -219,6 +219,30 @@ moe_status check_align_args(const int32_t* topk_ids, int T, int k, int E, int bl
   return MOE_OK;
 }
 
+
+// Regions of the backward's workspace, each 256-byte aligned: the token rows
+// and the dL/dout rows in expert-sorted order, the fp32 pre-activations,
+// their gradient da (bf16), w * h, and the fp32 dx accumulator.
+struct BwdLayout {
+  int64_t P_total;
+  size_t xs, gs, pre, da, hw, acc, total;
+};
+
+BwdLayout bwd_layout(int T, int d, int F, int E, int k, moe_act act, int n_shared) {
+  BwdLayout L{};
+  L.P_total = padded_total(T, k, E, 128, n_shared);
+  const size_t P = static_cast<size_t>(L.P_total);
+  const size_t n1 = act == MOE_ACT_SWIGLU ? 2 * static_cast<size_t>(F) : static_cast<size_t>(F);
+  L.xs = 0;
+  L.gs = L.xs + round_up(P * d * 2, kWsAlign);
+  L.pre = L.gs + round_up(P * d * 2, kWsAlign);
+  L.da = L.pre + round_up(P * n1 * 4, kWsAlign);
+  L.hw = L.da + round_up(P * n1 * 2, kWsAlign);
+  L.acc = L.hw + round_up(P * F * 2, kWsAlign);
+  L.total = L.acc + round_up(static_cast<size_t>(T) * d * 4, kWsAlign);
+  return L;
+}
+
 }  // namespace
 
 namespace moe {
@@ -712,6 +736,223 @@ moe_status moe_layer(const float* logits, int T, int E, int k, int n_group, int 
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   return forward_impl(x, T, d, w13, w2, E, F, w13_shared, w2_shared, n_shared, topk_weights, k, sorted_token_ids,
                       expert_ids, num_tokens_post_padded, block_m, act, out, ws, dev_status, s, &launches, nullptr);
+}
+
+size_t moe_backward_workspace_size(int T, int d, int F, int E, int k, moe_act act, int n_shared) {
+  if (check_dims(T, d, F, E, k) != MOE_OK) return 0;
+  if ((act != MOE_ACT_SWIGLU && act != MOE_ACT_RELU2) || (n_shared != 0 && n_shared != 1)) return 0;
+  return bwd_layout(T, d, F, E, k, act, n_shared).total + kWsAlign;
+}
+
+moe_status moe_backward(const uint16_t* x, int T, int d, const uint16_t* w13, const uint16_t* w2, int E, int F,
+                        const uint16_t* w13_shared, const uint16_t* w2_shared, int n_shared,
+                        const float* topk_weights, int k, const int32_t* sorted_token_ids,
+                        const int32_t* expert_ids, const int32_t* num_tokens_post_padded, moe_act act,
+                        const uint16_t* dout, uint16_t* dx, uint16_t* dw13, uint16_t* dw2, uint16_t* dw13_shared,
+                        uint16_t* dw2_shared, float* dtopk_weights, void* ws, size_t ws_bytes, int32_t* dev_status,
+                        moe_stream_t stream) {
+  moe_status st = check_dims(T, d, F, E, k);
+  if (st != MOE_OK) return st;
+  if (act != MOE_ACT_SWIGLU && act != MOE_ACT_RELU2) return MOE_ERR_INVALID_ARG;
+  if (n_shared != 0 && n_shared != 1) return MOE_ERR_UNSUPPORTED;
+  if (n_shared && (!w13_shared || !w2_shared || !dw13_shared || !dw2_shared)) return MOE_ERR_INVALID_ARG;
+  if (!w13 || !w2 || !dw13 || !dw2) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w13) || !aligned16(w2) || !aligned16(dw13) || !aligned16(dw2)) return MOE_ERR_INVALID_ARG;
+  if (n_shared && (!aligned16(w13_shared) || !aligned16(w2_shared) || !aligned16(dw13_shared) ||
+                   !aligned16(dw2_shared)))
+    return MOE_ERR_INVALID_ARG;
+  if (T > 0) {
+    if (!x || !topk_weights || !sorted_token_ids || !expert_ids || !num_tokens_post_padded || !dout || !dx)
+      return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(dout) || !aligned16(dx)) return MOE_ERR_INVALID_ARG;
+    if (dtopk_weights && !aligned16(dtopk_weights)) return MOE_ERR_INVALID_ARG;
+  }
+  const size_t need = moe_backward_workspace_size(T, d, F, E, k, act, n_shared);
+  if (ws == nullptr || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int num_sms = num_sms_current_device();
+  if (num_sms <= 0) return MOE_ERR_CUDA;
+  const int bm = 128;
+  const int n1 = act == MOE_ACT_SWIGLU ? 2 * F : F;
+  const int64_t P_max = moe_max_padded(T, k, E, bm);
+  const BwdLayout L = bwd_layout(T, d, F, E, k, act, n_shared);
+  const int n_shared_blocks = n_shared ? (T + bm - 1) / bm : 0;
+  const int max_routed_blocks = static_cast<int>(P_max / bm);
+  uint8_t* wsb = reinterpret_cast<uint8_t*>(round_up(reinterpret_cast<uintptr_t>(ws), kWsAlign));
+  uint16_t* xs = reinterpret_cast<uint16_t*>(wsb + L.xs);
+  uint16_t* gs = reinterpret_cast<uint16_t*>(wsb + L.gs);
+  float* pre = reinterpret_cast<float*>(wsb + L.pre);
+  uint16_t* da = reinterpret_cast<uint16_t*>(wsb + L.da);
+  uint16_t* hw = reinterpret_cast<uint16_t*>(wsb + L.hw);
+  float* acc = reinterpret_cast<float*>(wsb + L.acc);
+  const uint64_t wait_ns = moe::launch_wait_limit_ns();
+  const int surplus = moe::launch_unreachable_arrivals();
+  int launches = 0;
+  cudaError_t err = cudaSuccess;
+  auto grid_for = [&](int64_t tiles) { return static_cast<int>(tiles < 1 ? 1 : (tiles < num_sms ? tiles : num_sms)); };
+
+  if (T == 0) {
+    // no rows: every weight gradient is zero
+    const size_t n13 = static_cast<size_t>(E) * n1 * d * 2, n2 = static_cast<size_t>(E) * d * F * 2;
+    if (cudaMemsetAsync(dw13, 0, n13, s) != cudaSuccess || cudaMemsetAsync(dw2, 0, n2, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (n_shared && (cudaMemsetAsync(dw13_shared, 0, n13 / E, s) != cudaSuccess ||
+                     cudaMemsetAsync(dw2_shared, 0, n2 / E, s) != cudaSuccess))
+      return MOE_ERR_CUDA;
+    return finish(cudaSuccess, 0);
+  }
+
+  // 1. token rows and dL/dout rows in the expert-sorted order, padding rows zero
+  {
+    StageScope scope(7, s);
+    err = moe::launch_permute_rows(x, sorted_token_ids, num_tokens_post_padded, T, k, d, static_cast<int>(P_max),
+                                   n_shared_blocks * bm, xs, num_sms, s, &launches, true);
+    if (err == cudaSuccess)
+      err = moe::launch_permute_rows(dout, sorted_token_ids, num_tokens_post_padded, T, k, d,
+                                     static_cast<int>(P_max), n_shared_blocks * bm, gs, num_sms, s, &launches, true);
+  }
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+
+  auto base_args = [&](moe::GemmArgs& a) {
+    std::memset(&a, 0, sizeof(a));
+    a.sorted_ids = sorted_token_ids;
+    a.expert_ids = expert_ids;
+    a.ntpp = num_tokens_post_padded;
+    a.topk_w = topk_weights;
+    a.status = dev_status;
+    a.wait_ns = wait_ns;
+    a.tfull_surplus = surplus;
+    a.T = T;
+    a.k = k;
+    a.S = T * k;
+    a.E = E;
+    a.block_m = bm;
+    a.max_routed_blocks = max_routed_blocks;
+    a.n_shared_blocks = n_shared_blocks;
+  };
+
+  // 2. gate/up (fc1) pre-activations recomputed from the sorted token rows;
+  //    a spare warp zeroes the dx accumulator and dL/d topk_weights
+  {
+    moe::GemmArgs a;
+    base_args(a);
+    const int epi = act == MOE_ACT_SWIGLU ? moe::kEpiPreSwiGLU : moe::kEpiPreRelu2;
+    const uint32_t box = static_cast<uint32_t>(moe::gemm_box_rows(epi));
+    if (!encode_3d(&a.tm_w, w13, d, n1, E, box)) return MOE_ERR_CUDA;
+    if (n_shared) {
+      if (!encode_3d(&a.tm_ws, w13_shared, d, n1, 1, box)) return MOE_ERR_CUDA;
+    } else {
+      a.tm_ws = a.tm_w;
+    }
+    if (!encode_2d(&a.tm_x, xs, d, static_cast<uint64_t>(L.P_total), bm)) return MOE_ERR_CUDA;
+    a.out = pre;
+    a.out_ld = n1;
+    a.K = d;
+    a.n_out = F;
+    a.up_row_offset = F;
+    a.acc = acc;
+    a.acc_elems = static_cast<int64_t>(T) * d;
+    a.zero2 = dtopk_weights;
+    a.zero2_elems = dtopk_weights ? static_cast<int64_t>(T) * k : 0;
+    StageScope scope(9, s);
+    err = moe::launch_grouped_gemm(epi, a, grid_for(moe::gemm_max_tiles(epi, max_routed_blocks, n_shared_blocks, F)),
+                                   s);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    ++launches;
+  }
+  // 3. dh = W2^T dout rows, and in its epilogue da (from the
+  //    pre-activations), w * h and dL/d topk_weights
+  {
+    moe::GemmArgs a;
+    base_args(a);
+    const int epi = act == MOE_ACT_SWIGLU ? moe::kEpiGradSwiGLU : moe::kEpiGradRelu2;
+    // W2 [E, d, F] read MN-major: {F (contiguous), d rows, E}, boxes of 64 x 64
+    if (!encode_3d(&a.tm_w, w2, F, d, E, 64)) return MOE_ERR_CUDA;
+    if (n_shared) {
+      if (!encode_3d(&a.tm_ws, w2_shared, F, d, 1, 64)) return MOE_ERR_CUDA;
+    } else {
+      a.tm_ws = a.tm_w;
+    }
+    if (!encode_2d(&a.tm_x, gs, d, static_cast<uint64_t>(L.P_total), bm)) return MOE_ERR_CUDA;
+    a.pre = pre;
+    a.out = da;
+    a.out_ld = n1;
+    a.hw = hw;
+    a.dtopk = dtopk_weights;
+    a.K = d;
+    a.n_out = F;
+    a.up_row_offset = F;
+    StageScope scope(10, s);
+    err = moe::launch_grouped_gemm(epi, a, grid_for(moe::gemm_max_tiles(epi, max_routed_blocks, n_shared_blocks, F)),
+                                   s);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    ++launches;
+  }
+  // 4. dx rows = W13^T da, added into the fp32 accumulator at their token;
+  //    then dx = bf16(accumulator)
+  {
+    moe::GemmArgs a;
+    base_args(a);
+    // W13 [E, n1, d] read MN-major: {d (contiguous), n1 rows, E}, boxes of 64 x 64
+    if (!encode_3d(&a.tm_w, w13, d, n1, E, 64)) return MOE_ERR_CUDA;
+    if (n_shared) {
+      if (!encode_3d(&a.tm_ws, w13_shared, d, n1, 1, 64)) return MOE_ERR_CUDA;
+    } else {
+      a.tm_ws = a.tm_w;
+    }
+    if (!encode_2d(&a.tm_x, da, n1, static_cast<uint64_t>(L.P_total), bm)) return MOE_ERR_CUDA;
+    a.acc = acc;
+    a.acc_elems = static_cast<int64_t>(T) * d;
+    a.K = n1;
+    a.n_out = d;
+    {
+      const int64_t acc_bytes = static_cast<int64_t>(T) * d * 4;
+      const int64_t budget = int64_t(48) << 20;
+      const int n_wt = (d + 255) / 256;
+      const int passes = static_cast<int>((acc_bytes + budget - 1) / budget);
+      a.pass_cols = passes <= 1 ? 0 : (n_wt + passes - 1) / passes;
+    }
+    StageScope scope(11, s);
+    err = moe::launch_grouped_gemm(moe::kEpiDx, a,
+                                   grid_for(moe::gemm_max_tiles(moe::kEpiDx, max_routed_blocks, n_shared_blocks, d)), s);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    ++launches;
+  }
+  {
+    StageScope scope(4, s);
+    err = moe::launch_convert(acc, static_cast<int64_t>(T) * d, dx, num_sms, s, &launches);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  // 5. weight gradients per expert: dW13_e = da_e^T x_e, dW2_e = dout_e^T (w h)_e
+  auto wgrad = [&](const uint16_t* A, int M, const uint16_t* B, int N, uint16_t* out, uint16_t* out_shared,
+                   int stage) -> moe_status {
+    moe::WgradArgs w;
+    std::memset(&w, 0, sizeof(w));
+    if (!encode_2d(&w.tm_a, A, M, static_cast<uint64_t>(L.P_total), 64)) return MOE_ERR_CUDA;
+    if (!encode_2d(&w.tm_b, B, N, static_cast<uint64_t>(L.P_total), 64)) return MOE_ERR_CUDA;
+    w.expert_ids = expert_ids;
+    w.ntpp = num_tokens_post_padded;
+    w.out = out;
+    w.out_shared = out_shared;
+    w.status = dev_status;
+    w.wait_ns = wait_ns;
+    w.E = E;
+    w.M = M;
+    w.N = N;
+    w.block_m = bm;
+    w.max_routed_blocks = max_routed_blocks;
+    w.n_shared_blocks = n_shared_blocks;
+    StageScope scope(stage, s);
+    if (moe::launch_wgrad(w, grid_for(moe::wgrad_max_tiles(E, n_shared, M, N)), s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    ++launches;
+    return MOE_OK;
+  };
+  st = wgrad(da, n1, xs, d, dw13, dw13_shared, 12);
+  if (st != MOE_OK) return st;
+  st = wgrad(gs, d, hw, F, dw2, dw2_shared, 13);
+  if (st != MOE_OK) return st;
+  return finish(cudaSuccess, launches);
 }
 
 moe_status moe_read_status(const int32_t* dev_status, moe_stream_t stream) {

@@ -89,10 +89,11 @@ cudaError_t launch_route_align(const float* logits, int T, int E, int k, int n_g
                                int32_t* ntpp, int32_t* inv_pos, int32_t* status, cudaStream_t stream, int* launches);
 
 // x_sorted[p] = x[sorted_ids[p] / k] for live rows p < ntpp, x_sorted[ntpp + t]
-// = x[t] for t < min(T, n_shared_rows).
+// = x[t] for t < min(T, n_shared_rows); with zero_pad, the other rows up to
+// ntpp + n_shared_rows are set to zero.
 cudaError_t launch_permute_rows(const uint16_t* x, const int32_t* sorted_ids, const int32_t* ntpp, int T, int k,
                                 int d, int P_max, int n_shared_rows, uint16_t* x_sorted, int num_sms,
-                                cudaStream_t stream, int* launches);
+                                cudaStream_t stream, int* launches, bool zero_pad = false);
 
 // Router projection on the CUDA cores: logits [T, E] fp32 = x [T, d] .
 // W_g [E, d]^T (d a multiple of 8), CTAs of 8 experts x kRouterGemvMaxT

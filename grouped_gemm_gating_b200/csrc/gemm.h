@@ -7,10 +7,17 @@
 namespace moe {
 
 enum EpiKind : int {
-  kEpiSwiGLU = 0,  // gate/up GEMM, h = silu(gate) * up
-  kEpiRelu2 = 1,   // fc1 GEMM, h = max(a, 0)^2
-  kEpiScale = 2,   // down GEMM, acc[token] += topk_weight(row) * row result (fp32)
-  kEpiRouter = 3   // router GEMM, logits = x . W_g^T (fp32), top-k gating of each row
+  kEpiSwiGLU = 0,      // gate/up GEMM, h = silu(gate) * up
+  kEpiRelu2 = 1,       // fc1 GEMM, h = max(a, 0)^2
+  kEpiScale = 2,       // down GEMM, acc[token] += topk_weight(row) * row result (fp32)
+  kEpiRouter = 3,      // router GEMM, logits = x . W_g^T (fp32), top-k gating of each row
+  // backward (token rows by TMA from the expert-sorted copies)
+  kEpiPreSwiGLU = 4,   // gate/up pre-activations [g | u] of every row, fp32
+  kEpiPreRelu2 = 5,    // fc1 pre-activations, fp32
+  kEpiGradSwiGLU = 6,  // dh = W2^T dout rows (W2 read MN-major); epilogue: [dg | du] from [g | u] (bf16),
+                       // w * h, and dL/dw of the row's slot
+  kEpiGradRelu2 = 7,   // the same for relu^2: da over a
+  kEpiDx = 8           // dx rows = da . W13 (W13 read MN-major), added into the fp32 accumulator
 };
 
 // Arguments of one grouped GEMM launch (token-major tiles, block_m = 128).
@@ -42,6 +49,13 @@ struct GemmArgs {
   int max_routed_blocks;
   int n_shared_blocks;
   int pass_cols;        // output-column tiles per pass of the tile walk (0: one pass)
+  // backward only
+  int out_ld;           // row stride (elements) of `out` and `pre` (pre / grad kinds: n1)
+  const float* pre;     // grad kinds: the fp32 pre-activations [P_total, n1] (`out` is then da, bf16)
+  uint16_t* hw;         // grad kinds: w * h [P_total, F] bf16
+  float* dtopk;         // grad kinds: dL/d topk_weights [T * k] (fp32 adds; zeroed by the pre kinds)
+  float* zero2;         // pre kinds: a second buffer their spare warp zeroes (dtopk), zero2_elems floats
+  int64_t zero2_elems;
   // router GEMM only: fp32 logits [T, E]; when r_ids is set, the top-k of
   // every row (ids [T, k], weights [T, k]) with the routing kernel's order
   // (logit desc, id asc) and weights (softmax over the chosen k when
@@ -69,5 +83,27 @@ constexpr int kRouterMaxK = 16;
 // {K, P_total}, 64 x 128 boxes) instead of gathering them.
 bool gemm_pair_supported(int block_m, int total_blocks_max);
 cudaError_t launch_grouped_gemm_pair(int epi, const GemmArgs& args, int grid, cudaStream_t stream);
+
+// Per-expert weight gradient (backward): for every expert e (and the shared
+// expert, when present), dW_e [M, N] = sum over the rows p of e's blocks of
+// A[p, :]^T B[p, :], with A [P_total, M] and B [P_total, N] in the
+// expert-sorted row order (padding rows zero), rounded to bf16.  Both
+// operands are read MN-major (their M / N index contiguous) by TMA.
+struct WgradArgs {
+  CUtensorMap tm_a;        // A, 2-D {M, P_total}, 64 x 64 boxes, 128B swizzle
+  CUtensorMap tm_b;        // B, 2-D {N, P_total}, 64 x 64 boxes, 128B swizzle
+  const int32_t* expert_ids;
+  const int32_t* ntpp;
+  uint16_t* out;           // [E, M, N] bf16
+  uint16_t* out_shared;    // [M, N] bf16 (the shared expert's rows follow the routed ones)
+  int32_t* status;
+  uint64_t wait_ns;
+  int E, M, N;
+  int block_m;             // 128
+  int max_routed_blocks;
+  int n_shared_blocks;
+};
+int64_t wgrad_max_tiles(int E, int n_shared, int M, int N);
+cudaError_t launch_wgrad(const WgradArgs& args, int grid, cudaStream_t stream);
 
 }  // namespace moe

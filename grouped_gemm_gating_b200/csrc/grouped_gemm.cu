@@ -52,8 +52,19 @@ namespace moe {
 template <int EPI>
 struct GemmCfg {
   static constexpr int TOK = 128;  // token rows per tile
-  static constexpr bool kGated = (EPI == kEpiSwiGLU);
+  // two 128-row boxes of K-major weights per stage: the gate rows and the
+  // matching up rows of the tile's 128 h columns
+  static constexpr bool kGated = (EPI == kEpiSwiGLU || EPI == kEpiPreSwiGLU);
   static constexpr bool kGather = (EPI == kEpiSwiGLU || EPI == kEpiRelu2);
+  static constexpr bool kPre = (EPI == kEpiPreSwiGLU || EPI == kEpiPreRelu2);
+  static constexpr bool kGrad = (EPI == kEpiGradSwiGLU || EPI == kEpiGradRelu2);
+  static constexpr bool kReduce = (EPI == kEpiScale || EPI == kEpiDx);
+  // the weight operand read MN-major: its 256 output columns are contiguous
+  // in memory (W2 for dh = W2^T dout, W13 for dx = W13^T da), loaded as four
+  // 64-column boxes of 64 K rows
+  static constexpr bool kBmn = kGrad || EPI == kEpiDx;
+  // a spare warp zeroes the accumulator the next kernel reduces into
+  static constexpr bool kZero = kGather || kPre;
   static constexpr int kBoxRows = kGated ? 128 : 256;
   static constexpr int kBoxes = kGated ? 2 : 1;
   static constexpr int kWRows = kBoxRows * kBoxes;
@@ -65,19 +76,22 @@ struct GemmCfg {
   static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
   static constexpr int kAccCols = 256;
   static constexpr int kTmemCols = 512;
-  // gate/up: warps 6-9 gather token rows, warp 10 zeroes the accumulator
-  // epilogue warps: the down GEMM's scatter-reduce bounds that kernel, so it
-  // runs two warps per TMEM lane quadrant, each on half of the tile's columns
-  static constexpr int kEpiWarps = EPI == kEpiScale ? 8 : 4;
-  static constexpr int kNumThreads = kGather ? 352 : 64 + 32 * kEpiWarps;
+  // epilogue warps: the reductions into the fp32 accumulator bound those
+  // kernels, so they run two warps per TMEM lane quadrant, each on half of
+  // the tile's columns
+  static constexpr int kEpiWarps = kReduce ? 8 : 4;
+  // gate/up: warps 6-9 gather token rows, warp 10 zeroes the accumulator;
+  // pre-activations: warp 6 zeroes
+  static constexpr int kZeroWarp = kGather ? 10 : 2 + kEpiWarps;
+  static constexpr int kNumThreads = kGather ? 352 : 64 + 32 * kEpiWarps + (kZero ? 32 : 0);
   static constexpr uint32_t kTxBytes = kWBytes + (kGather ? 0 : kXBytes);
   static constexpr int kBarrierBytes = 512;
-  // down GEMM: per epilogue warp a 32 x 33 fp32 transpose buffer, so the
+  // reductions: per epilogue warp a 32 x 33 fp32 transpose buffer, so the
   // reduction is issued as full 128-byte row segments
   static constexpr int kRedStride = 33;
-  static constexpr int kRedBytes = EPI == kEpiScale ? kEpiWarps * 32 * kRedStride * 4 : 0;
+  static constexpr int kRedBytes = kReduce ? kEpiWarps * 32 * kRedStride * 4 : 0;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes + kRedBytes;
-  static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(128, 256);
+  static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(128, 256, false, kBmn);
 
   static_assert(kStages >= 3, "pipeline depth");
   static_assert(kAccCols * 2 <= kTmemCols, "two accumulator buffers must fit TMEM");
@@ -216,7 +230,14 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
           }
           uint8_t* sW = smem + stage * C::kStageBytes;
           ptx::mbar_arrive_expect_tx(&full[stage], C::kTxBytes);
-          ptx::tma_load_3d(sW, tm, &full[stage], kb * 64, row0, e);
+          if (C::kBmn) {
+            // 64 K rows of the tile's 256 contiguous output columns, as four
+            // 64-column boxes 8 KB apart (the MN-major operand's chunks)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) ptx::tma_load_3d(sW + j * 8192, tm, &full[stage], row0 + 64 * j, kb * 64, e);
+          } else {
+            ptx::tma_load_3d(sW, tm, &full[stage], kb * 64, row0, e);
+          }
           if (C::kGated)
             ptx::tma_load_3d(sW + C::kBoxRows * 128, tm, &full[stage], kb * 64, args.up_row_offset + row0, e);
           if (!C::kGather) ptx::tma_load_2d(sW + C::kWBytes, &args.tm_x, &full[stage], kb * 64, tc.blk * args.block_m);
@@ -281,8 +302,11 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
-            ptx::mma_bf16(d_tmem, ptx::sw128_kmajor_desc(sX + kk * 32), ptx::sw128_kmajor_desc(sW + kk * 32),
-                          C::kIdesc, acc);
+            // B: K-major (16 K values = 32 B along the swizzled row) or
+            // MN-major (16 K rows = two 1024-byte atoms)
+            const uint64_t bdesc =
+                C::kBmn ? ptx::sw128_mnmajor_desc(sW + kk * 2048, 8192) : ptx::sw128_kmajor_desc(sW + kk * 32);
+            ptx::mma_bf16(d_tmem, ptx::sw128_kmajor_desc(sX + kk * 32), bdesc, C::kIdesc, acc);
           }
           ptx::mma_commit(&empty[stage]);
           if (++stage == C::kStages) {
@@ -367,6 +391,130 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
             dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
           }
         }
+      } else if (EPI == kEpiPreSwiGLU) {
+        // pre-activations kept for the backward (fp32: the activation's
+        // derivative is taken from them): g at column c, u at F + c
+        float* orow = static_cast<float*>(args.out) + static_cast<size_t>(p) * args.out_ld;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t g[32], u[32];
+          ptx::tmem_ld16(t_acc + c0, *reinterpret_cast<uint32_t(*)[16]>(&g[0]));
+          ptx::tmem_ld16(t_acc + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&g[16]));
+          ptx::tmem_ld16(t_acc + 128 + c0, *reinterpret_cast<uint32_t(*)[16]>(&u[0]));
+          ptx::tmem_ld16(t_acc + 128 + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&u[16]));
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) asm volatile("" : "+r"(g[j]), "+r"(u[j]));  // uses stay after the wait
+          const int col = tc.wt * 128 + c0;
+          if (col < args.n_out) {
+            uint4* dg = reinterpret_cast<uint4*>(orow + col);
+            uint4* du = reinterpret_cast<uint4*>(orow + args.up_row_offset + col);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              dg[i] = make_uint4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
+              du[i] = make_uint4(u[4 * i], u[4 * i + 1], u[4 * i + 2], u[4 * i + 3]);
+            }
+          }
+        }
+      } else if (EPI == kEpiPreRelu2) {
+        float* orow = static_cast<float*>(args.out) + static_cast<size_t>(p) * args.out_ld;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 256; c0 += 16) {
+          uint32_t a[16];
+          ptx::tmem_ld16(t_acc + c0, a);
+          ptx::tmem_wait_ld();
+          const int col = tc.wt * 256 + c0;
+          if (col < args.n_out) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(a[4 * i], a[4 * i + 1], a[4 * i + 2], a[4 * i + 3]);
+          }
+        }
+      } else if (C::kGrad) {
+        // thread = row p; TMEM columns = dhu = W2^T dout[token] for the
+        // tile's 256 h columns.  With the row's top-k weight w (0 for
+        // padding rows, 1 for the shared expert): dh = w * dhu, the
+        // activation's derivative at the stored fp32 pre-activations gives
+        // da (bf16, the operand of the dx and dW13 GEMMs), w * h goes to hw
+        // (the dW2 operand), and sum(h * dhu) over the columns is this
+        // tile's share of dL/dw for the row's slot.
+        int slot = -1;
+        float wrow = 0.0f;
+        if (!tc.shared_blk) {
+          slot = args.sorted_ids[p];
+          if (static_cast<unsigned>(slot) < static_cast<unsigned>(args.S))
+            wrow = args.topk_w[slot];
+          else
+            slot = -1;
+        } else {
+          const int t = (tc.blk - routed_blocks) * args.block_m + row;
+          wrow = t < args.T ? 1.0f : 0.0f;
+        }
+        const float* prow = args.pre + static_cast<size_t>(p) * args.out_ld;
+        uint16_t* arow = static_cast<uint16_t*>(args.out) + static_cast<size_t>(p) * args.out_ld;
+        uint16_t* hrow = args.hw + static_cast<size_t>(p) * args.n_out;
+        float part = 0.0f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 256; c0 += 32) {
+          uint32_t a[32];
+          ptx::tmem_ld16(t_acc + c0, *reinterpret_cast<uint32_t(*)[16]>(&a[0]));
+          ptx::tmem_ld16(t_acc + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&a[16]));
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) asm volatile("" : "+r"(a[j]));  // uses stay after the wait
+          const int col = tc.wt * 256 + c0;
+          if (col >= args.n_out) break;  // uniform across the warp
+          float4 pv[8], uv[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) pv[i] = reinterpret_cast<const float4*>(prow + col)[i];
+          if (EPI == kEpiGradSwiGLU) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) uv[i] = reinterpret_cast<const float4*>(prow + args.up_row_offset + col)[i];
+          }
+          const float* pg = reinterpret_cast<const float*>(pv);
+          const float* pu = reinterpret_cast<const float*>(uv);
+          uint32_t da_lo[16], da_hi[16], hv[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float d0[2], d1[2], hh[2];
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+              const int j = 2 * i + m;
+              const float dhu = __uint_as_float(a[j]);
+              const float dh = wrow * dhu;
+              float h;
+              if (EPI == kEpiGradSwiGLU) {
+                const float g = pg[j];
+                const float u = pu[j];
+                const float sg = __frcp_rn(1.0f + __expf(-g));
+                const float sl = g * sg;
+                h = sl * u;
+                d0[m] = dh * u * sg * (1.0f + g * (1.0f - sg));  // d/dg
+                d1[m] = dh * sl;                                   // d/du
+              } else {
+                const float r = fmaxf(pg[j], 0.0f);
+                h = r * r;
+                d0[m] = 2.0f * dh * r;
+                d1[m] = 0.0f;
+              }
+              hh[m] = wrow * h;
+              part += h * dhu;
+            }
+            da_lo[i] = pack_bf16x2(d0[0], d0[1]);
+            da_hi[i] = pack_bf16x2(d1[0], d1[1]);
+            hv[i] = pack_bf16x2(hh[0], hh[1]);
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            reinterpret_cast<uint4*>(arow + col)[i] =
+                make_uint4(da_lo[4 * i], da_lo[4 * i + 1], da_lo[4 * i + 2], da_lo[4 * i + 3]);
+            reinterpret_cast<uint4*>(hrow + col)[i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+            if (EPI == kEpiGradSwiGLU)
+              reinterpret_cast<uint4*>(arow + args.up_row_offset + col)[i] =
+                  make_uint4(da_hi[4 * i], da_hi[4 * i + 1], da_hi[4 * i + 2], da_hi[4 * i + 3]);
+          }
+        }
+        if (slot >= 0 && args.dtopk != nullptr) atomicAdd(args.dtopk + slot, part);
       } else if (EPI == kEpiRouter) {
         // thread = token row of the tile, TMEM columns 0..E-1 = its logits.
         // Top-k over columns in increasing id order into a list sorted by
@@ -468,7 +616,8 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
           }
         }
       } else {
-        // scatter-reduce: acc[token] += topk_weight * row (shared expert: weight 1)
+        // scatter-reduce: acc[token] += topk_weight * row (shared expert and
+        // dx rows, whose da already carries the weight: 1)
         bool valid;
         int tok;
         float wrow = 1.0f;
@@ -476,7 +625,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
           const int slot = args.sorted_ids[p];
           valid = static_cast<unsigned>(slot) < static_cast<unsigned>(args.S);
           tok = valid ? slot / args.k : 0;
-          if (valid) wrow = args.topk_w[slot];
+          if (valid && EPI == kEpiScale) wrow = args.topk_w[slot];
         } else {
           tok = (tc.blk - routed_blocks) * args.block_m + row;
           valid = tok < args.T;
@@ -524,20 +673,23 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
         aphase ^= 1u;
       }
     }
-  } else if (C::kGather && warp == 10) {
-    // ------------------------------------------------ zero this CTA's share of the down GEMM's accumulator
-    if (args.acc != nullptr) {
-      const int64_t n = args.acc_elems;
+  } else if (C::kZero && warp == C::kZeroWarp) {
+    // ------------------------------------------------ zero this CTA's share of the accumulator(s) the
+    // next kernels add into (the down GEMM's, or the backward's dx and dL/dw)
+    auto zero_share = [&](float* buf, int64_t n) {
+      if (buf == nullptr) return;
       const int64_t per = ((n + gridDim.x - 1) / gridDim.x + 3) & ~int64_t(3);
       const int64_t lo = static_cast<int64_t>(blockIdx.x) * per;
       const int64_t hi = lo + per < n ? lo + per : n;
       for (int64_t i = lo + 4 * lane; i < hi; i += 4 * kWarp) {
         if (i + 4 <= hi)
-          *reinterpret_cast<float4*>(args.acc + i) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          *reinterpret_cast<float4*>(buf + i) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         else
-          for (int64_t m = i; m < hi; ++m) args.acc[m] = 0.0f;
+          for (int64_t m = i; m < hi; ++m) buf[m] = 0.0f;
       }
-    }
+    };
+    zero_share(args.acc, args.acc_elems);
+    zero_share(args.zero2, args.zero2_elems);
   } else if (C::kGather) {
     // ------------------------------------------------ row gather of x
     constexpr int kRowsPerThread = TOK / 16;
@@ -639,7 +791,7 @@ cudaError_t launch_variant(const GemmArgs& args, int grid, cudaStream_t stream) 
 
 }  // namespace
 
-int gemm_box_rows(int epi) { return epi == kEpiSwiGLU ? 128 : 256; }
+int gemm_box_rows(int epi) { return (epi == kEpiSwiGLU || epi == kEpiPreSwiGLU) ? 128 : 256; }
 
 int64_t gemm_max_tiles(int epi, int max_routed_blocks, int n_shared_blocks, int n_out) {
   const int cols = gemm_box_rows(epi);
@@ -654,6 +806,11 @@ cudaError_t launch_grouped_gemm(int epi, const GemmArgs& a, int grid, cudaStream
     case kEpiRelu2: return launch_variant<kEpiRelu2>(a, grid, s);
     case kEpiScale: return launch_variant<kEpiScale>(a, grid, s);
     case kEpiRouter: return launch_variant<kEpiRouter>(a, grid, s);
+    case kEpiPreSwiGLU: return launch_variant<kEpiPreSwiGLU>(a, grid, s);
+    case kEpiPreRelu2: return launch_variant<kEpiPreRelu2>(a, grid, s);
+    case kEpiGradSwiGLU: return launch_variant<kEpiGradSwiGLU>(a, grid, s);
+    case kEpiGradRelu2: return launch_variant<kEpiGradRelu2>(a, grid, s);
+    case kEpiDx: return launch_variant<kEpiDx>(a, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -334,12 +334,30 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
   return desc;
 }
 
-// Instruction descriptor of kind::f16 with bf16 A and B, fp32 D, both
-// operands K-major: D format in bits [4,6), A/B formats in [7,10)/[10,13),
-// N >> 3 in [17,23), M >> 4 in [24,29).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
-         (static_cast<uint32_t>(M >> 4) << 24);
+// Shared-memory matrix descriptor of an MN-major operand tile (the M or N
+// index contiguous) in the 128-byte-swizzled canonical layout: each row of
+// 128 B holds 64 consecutive M (or N) values of one K index, 8 such rows
+// (K indices) form a 1024-byte swizzle atom, consecutive atoms along K are
+// 1024 B apart (stride byte offset) and consecutive 64-wide M (or N) chunks
+// are `mn_chunk_bytes` apart (leading byte offset).  This is what a TMA box
+// of {64 M/N values, K rows} with 128-byte swizzle writes; several boxes side
+// by side along M/N give the chunks.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint32_t mn_chunk_bytes) {
+  uint64_t desc = 0;
+  desc |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  desc |= static_cast<uint64_t>((mn_chunk_bytes >> 4) & 0x3FFFu) << 16;
+  desc |= static_cast<uint64_t>(1024u >> 4) << 32;
+  desc |= static_cast<uint64_t>(1u) << 46;
+  desc |= static_cast<uint64_t>(2u) << 61;
+  return desc;
+}
+
+// Instruction descriptor of kind::f16 with bf16 A and B, fp32 D: D format in
+// bits [4,6), A/B formats in [7,10)/[10,13), A and B major-ness in bits 15
+// and 16 (0: K-major, 1: MN-major), N >> 3 in [17,23), M >> 4 in [24,29).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn = false, bool b_mn = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 }  // namespace ptx

@@ -46,6 +46,9 @@ _SIG = {
                          _P, _P, ctypes.c_size_t, _P, _P]),
     "moe_layer": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _I, _P, _P, _I, _P, _P, _I, _I, _I,
                        _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
+    "moe_backward_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I]),
+    "moe_backward": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _P, _I, _P, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P,
+                          _P, _P, ctypes.c_size_t, _P, _P]),
     "moe_read_status": (_I, [_P, _P]),
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_last_launch_count": (_I, []),
@@ -55,7 +58,7 @@ _SIG = {
 }
 
 STAGES = ("route", "align", "gate_up_gemm", "down_gemm", "combine", "route_align", "fused_expert", "permute",
-          "router")
+          "router", "bwd_recompute", "bwd_dh_gemm", "bwd_dx_gemm", "bwd_dw13_gemm", "bwd_dw2_gemm")
 
 _lib = None
 _lock = threading.Lock()
@@ -274,6 +277,60 @@ def moe_layer(logits, x, w13, w2, k, block_m, act, topk_ids, topk_weights, sorte
         _ptr(num_tokens_post_padded), _ptr(inv_pos), _ptr(_bits(out)), _ptr(ws), ws.numel() * ws.element_size(),
         _ptr(dev_status), _stream(x.device))
     _check("moe_layer", code)
+
+
+def moe_backward_workspace_size(T, d, F, E, k, act, n_shared) -> int:
+    return int(load_library().moe_backward_workspace_size(T, d, F, E, k, act, n_shared))
+
+
+def moe_backward(x, w13, w2, topk_weights, sorted_token_ids, expert_ids, num_tokens_post_padded, act, dout,
+                 dx, dw13, dw2, ws, w13_shared=None, w2_shared=None, dw13_shared=None, dw2_shared=None,
+                 dtopk_weights=None, dev_status=None):
+    """The layer's backward (align outputs for block_m = 128): fills dx [T, d],
+    dw13 [E, n1, d], dw2 [E, d, F] (bf16) and, when given, dtopk_weights [T, k]
+    fp32 and the shared expert's weight gradients."""
+    T, d = x.shape
+    E, n1, _ = w13.shape
+    F = w2.shape[2]
+    k = topk_weights.shape[1] if topk_weights.dim() == 2 else 1
+    n_shared = 0 if w13_shared is None else 1
+    if dtopk_weights is not None and dtopk_weights.dtype != torch.float32:
+        raise ValueError("moe_backward: dtopk_weights must be fp32")
+    code = load_library().moe_backward(
+        _ptr(_bits(x)), T, d, _ptr(_bits(w13)), _ptr(_bits(w2)), E, F, _ptr(_bits(w13_shared)),
+        _ptr(_bits(w2_shared)), n_shared, _ptr(topk_weights), k, _ptr(sorted_token_ids), _ptr(expert_ids),
+        _ptr(num_tokens_post_padded), act, _ptr(_bits(dout)), _ptr(_bits(dx)), _ptr(_bits(dw13)), _ptr(_bits(dw2)),
+        _ptr(_bits(dw13_shared)), _ptr(_bits(dw2_shared)), _ptr(dtopk_weights), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(dev_status), _stream(x.device))
+    _check("moe_backward", code)
+
+
+class MoEGradBuffers:
+    """Device buffers of one layer shape's backward (plumbing only): the
+    gradients and the backward's workspace, allocated once."""
+
+    def __init__(self, T, d, F, E, k, act=ACT_SWIGLU, n_shared=0, device="cuda"):
+        dev = torch.device(device)
+        n1 = 2 * F if act == ACT_SWIGLU else F
+        self.act, self.n_shared = act, n_shared
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        self.dx = torch.empty((T, d), **bf)
+        self.dw13 = torch.empty((E, n1, d), **bf)
+        self.dw2 = torch.empty((E, d, F), **bf)
+        self.dw13_shared = torch.empty((1, n1, d), **bf) if n_shared else None
+        self.dw2_shared = torch.empty((1, d, F), **bf) if n_shared else None
+        self.dtopk = torch.empty((T, k), dtype=torch.float32, device=dev)
+        n = moe_backward_workspace_size(T, d, F, E, k, act, n_shared)
+        if n == 0:
+            raise ValueError("unsupported layer shape")
+        self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+
+    def backward(self, fwd: "MoEBuffers", x, w13, w2, dout, w13_shared=None, w2_shared=None):
+        """Gradients of the layer whose routing and align outputs fwd holds
+        (block_m = 128)."""
+        moe_backward(x, w13, w2, fwd.topk_weights, fwd.sorted_token_ids, fwd.expert_ids, fwd.ntpp, self.act,
+                     dout, self.dx, self.dw13, self.dw2, self.ws, w13_shared, w2_shared, self.dw13_shared,
+                     self.dw2_shared, self.dtopk, fwd.status)
 
 
 def moe_read_status(dev_status) -> int:

@@ -194,6 +194,11 @@ def make_inputs(cfg: MoEConfig, threads: int = 8) -> MoEInputs:
     return MoEInputs(cfg, x, logits, w13, w2, w13s, w2s, router_w)
 
 
+def grad_output(T: int, d: int, seed: int) -> np.ndarray:
+    """Seeded dL/dout for the backward: N(0, 1) in bf16 bits [T, d]."""
+    return _normal_bf16(np.random.SeedSequence(seed).spawn(1)[0], (T, d), 1.0)
+
+
 def router_inputs(T: int, d: int, E: int, seed: int, zero_rows=()):
     """Seeded router-projection inputs: x ~ N(0, 1) and W_g ~ N(0, 0.02),
     both bf16 bits ([T, d] and [E, d]); the listed token rows are zero."""

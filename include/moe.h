@@ -309,6 +309,60 @@ MOE_API moe_status moe_layer(const float* logits, int T, int E, int k,
                      uint16_t* out, void* ws, size_t ws_bytes,
                      int32_t* dev_status, moe_stream_t stream);
 
+/* Bytes of device scratch moe_backward needs: the token rows and the dL/dout
+ * rows in expert-sorted order [P_total, d] bf16 each, the gate/up
+ * pre-activations [P_total, n1] fp32, their gradient [P_total, n1] bf16,
+ * w * h [P_total, F] bf16 and the fp32 dx accumulator [T, d], each 256-byte
+ * aligned, where P_total is that of moe_workspace_size with block_m = 128
+ * and n1 = 2F (SwiGLU) or F (relu^2).  Returns 0 on invalid arguments. */
+MOE_API size_t moe_backward_workspace_size(int T, int d, int F, int E, int k, moe_act act, int n_shared);
+
+/*
+ * moe_backward -- the layer's training pass: given dL/dout, the gradients of
+ * the loss with respect to the tokens, both expert weight stacks and the
+ * top-k weights.  The computation is the grouped backward of the axolotl
+ * vendor-moe diff (src/axolotl/kernels/moe/tt_cg_gemm/cg_backward.py:
+ * `_kernel_cg_backward_dx`, the token rows' gradient from dY and each
+ * expert's weights; `_kernel_cg_backward_dw`, each expert's weight gradient
+ * summed over the rows routed to it), for the training use case of the
+ * Gemma-4 MoE note (the expert path of a training step).  With, per routed
+ * row (t, j) of expert e and its weight w = topk_weights[t, j]:
+ *   SwiGLU: [g; u] = W13_e x[t], h = silu(g) u, dh = w W2_e^T dout[t],
+ *           da = [dh u silu'(g); dh silu(g)];  relu^2: a = W13_e x[t],
+ *           h = max(a, 0)^2, da = 2 dh max(a, 0);
+ *   dx[t]        = sum_j W13_e^T da            (+ the shared expert's, w = 1)
+ *   dw13[e]      = sum over e's rows of da x[t]^T
+ *   dw2[e]       = sum over e's rows of w dout[t] h^T
+ *   dtopk[t, j]  = dout[t] . W2_e h
+ * Arguments as for moe_forward, with moe_align's outputs for block_m = 128
+ * (sorted_token_ids, expert_ids, num_tokens_post_padded; no other block
+ * size), plus:
+ *   dout          [T, d] bf16, device: dL/dout.
+ *   dx            [T, d] bf16 out.
+ *   dw13, dw2     [E, n1, d] and [E, d, F] bf16 out (experts no token was
+ *                 routed to get zeros); dw13_shared / dw2_shared [1, n1, d] /
+ *                 [1, d, F] with n_shared == 1.
+ *   dtopk_weights [T, k] fp32 out, nullable (16-byte aligned).
+ *   ws, ws_bytes  scratch of moe_backward_workspace_size bytes (no
+ *                 initial contents needed).
+ * Precision: fp32 accumulation; the recomputed pre-activations stay fp32;
+ * da and w*h are rounded to bf16 (the bf16 operands of the next GEMMs); dx is
+ * summed over its k rows in fp32 with atomics (in a timing-dependent order)
+ * and rounded once; each dW is one fp32 accumulation rounded once.
+ * Launches: two row copies, four tcgen05 GEMMs, a conversion and two
+ * per-expert weight-gradient GEMMs, all on `stream`.  Errors as for
+ * moe_forward.
+ */
+MOE_API moe_status moe_backward(const uint16_t* x, int T, int d,
+                        const uint16_t* w13, const uint16_t* w2, int E, int F,
+                        const uint16_t* w13_shared, const uint16_t* w2_shared, int n_shared,
+                        const float* topk_weights, int k,
+                        const int32_t* sorted_token_ids, const int32_t* expert_ids,
+                        const int32_t* num_tokens_post_padded, moe_act act,
+                        const uint16_t* dout, uint16_t* dx, uint16_t* dw13, uint16_t* dw2,
+                        uint16_t* dw13_shared, uint16_t* dw2_shared, float* dtopk_weights,
+                        void* ws, size_t ws_bytes, int32_t* dev_status, moe_stream_t stream);
+
 /* Synchronises `stream`, then returns the code stored in dev_status (MOE_OK
  * when 0), or MOE_ERR_CUDA if the synchronisation or the copy failed. */
 MOE_API moe_status moe_read_status(const int32_t* dev_status, moe_stream_t stream);
@@ -353,7 +407,10 @@ MOE_API moe_status moe_debug_timeouts(uint64_t wait_limit_ns, int unreachable_ar
  * (moe_route_align on a small batch), 6 fused expert kernel (moe_forward
  * with block_m <= 64: both GEMMs and the scatter-reduce; under moe_layer on
  * a small batch also the routing and align), 7 permute (x rows copied into
- * the expert-sorted order for the gate/up GEMM on CTA pairs).
+ * the expert-sorted order for the gate/up GEMM on CTA pairs, and the
+ * backward's row copies), 8 router (moe_router), and for moe_backward: 9
+ * pre-activation recompute, 10 dh GEMM with the activation's derivative,
+ * 11 dx GEMM, 12 dW13 GEMM, 13 dW2 GEMM (its conversion of dx is stage 4).
  * moe_profile_enable(1) starts a fresh record (and primes the event pool),
  * (0) stops recording and keeps what was recorded.  moe_profile_collect waits for the recorded events,
  * writes into stage_ms[i] (i < n_stages) the summed milliseconds of stage i
@@ -361,7 +418,7 @@ MOE_API moe_status moe_debug_timeouts(uint64_t wait_limit_ns, int unreachable_ar
  * release != 0 it then returns the events to the pool and clears the record
  * (release == 0 keeps them, e.g. to read a graph's events after each
  * replay).  MOE_ERR_CUDA if an event call failed. */
-#define MOE_NUM_STAGES 8
+#define MOE_NUM_STAGES 14
 MOE_API moe_status moe_profile_enable(int on);
 MOE_API moe_status moe_profile_collect(double* stage_ms, int* stage_calls, int n_stages, int release);
 

@@ -276,6 +276,12 @@ def expert_backward_values(x: np.ndarray, W13: np.ndarray, W2: np.ndarray, dy: n
     Squared ReLU: a = W13 x, h = max(a, 0)^2, da = dh * 2 max(a, 0).
     Then dx = W13^T da, dW13 = sum over rows of da x^T, dW2 = sum of dy h^T.
     """
+    da, h = expert_backward_hidden(x, W13, W2, dy, act)
+    return da @ W13, da.T @ x, dy.T @ h, h @ W2.T
+
+
+def expert_backward_hidden(x: np.ndarray, W13: np.ndarray, W2: np.ndarray, dy: np.ndarray, act: int):
+    """The hidden quantities of expert_backward_values: (da [n, n1], h [n, F])."""
     dh = dy @ W2                                   # [n, F]
     if act == ACT_SWIGLU:
         F = W13.shape[0] // 2
@@ -289,7 +295,7 @@ def expert_backward_values(x: np.ndarray, W13: np.ndarray, W2: np.ndarray, dy: n
         da = dh * 2.0 * np.maximum(a, 0.0)
     else:
         raise ValueError("unknown activation")
-    return da @ W13, da.T @ x, dy.T @ h, h @ W2.T
+    return da, h
 
 
 def backward_values(x: np.ndarray, W13: np.ndarray, W2: np.ndarray, topk_ids: np.ndarray,

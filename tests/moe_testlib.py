@@ -104,6 +104,33 @@ def compare_out(gpu_bits: np.ndarray, ref: np.ndarray, label: str = ""):
     return max_abs / rms, excess / rms, rel_l2
 
 
+# Gradients (the backward): the same bounds, plus the effect of the bf16
+# operands the kernels must feed the tensor cores.  da (for dx and dW13) and
+# w*h (for dW2) are computed in fp32 and rounded to bf16 (relative error
+# <= 2^-9 each, 2^-8 with the fp32 evaluation before it), so an element
+# c = sum_r a_r b_r of a gradient GEMM whose operand a is rounded can be off
+# by 2^-8 * sum_r |a_r b_r|: |diff| <= 2e-2 * rms + half_ulp_bf16(ref) +
+# 2^-8 * (|a|^T |b|) element-wise, relative L2 still within 5e-3.
+GRAD_OPERAND_REL = 2.0 ** -8
+
+
+def compare_grad(gpu_bits: np.ndarray, ref: np.ndarray, abs_terms: np.ndarray, label: str = ""):
+    """compare_out for a gradient whose GEMM rounds one operand to bf16;
+    abs_terms = sum_r |a_r b_r| per element (same shape as ref)."""
+    got = W.bf16_bits_to_f32(gpu_bits).astype(np.float64)
+    assert got.shape == ref.shape == abs_terms.shape, (got.shape, ref.shape, abs_terms.shape)
+    assert np.isfinite(got).all(), f"{label}: non-finite output"
+    diff = np.abs(got - ref)
+    rms = float(np.sqrt((ref ** 2).mean()))
+    assert rms > 0.0, f"{label}: degenerate oracle output"
+    allowed = OUT_MAX_ABS_REL_RMS * rms + bf16_half_ulp(ref) + GRAD_OPERAND_REL * abs_terms
+    worst = float((diff / allowed).max())
+    rel_l2 = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+    assert worst <= 1.0, f"{label}: |diff| reaches {worst:.3f} of its bound (max|diff| {diff.max() / rms:.3e} rms)"
+    assert rel_l2 <= OUT_REL_L2, f"{label}: rel L2={rel_l2:.3e}"
+    return diff.max() / rms, rel_l2
+
+
 def assert_within_ulp(a_bits: np.ndarray, b_bits: np.ndarray, max_ulp: int = 1, label: str = ""):
     """Two bf16 outputs of the same inputs agree up to the reordering of an
     fp32 sum: max_ulp bf16 ulps of the result, plus 1e-4 rms for terms that

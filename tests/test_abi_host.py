@@ -131,6 +131,35 @@ def test_forward_host_checks(lib):
     assert f(*args(T=0, x=NULL)) == 0          # T == 0: no-op
 
 
+def test_backward_host_checks(lib):
+    f = lib.moe_backward
+    p = ctypes.c_void_p(256)
+    odd = ctypes.c_void_p(258)
+    args = lambda **kw: [kw.get("x", p), kw.get("T", 4), kw.get("d", 128), p, p, kw.get("E", 8), kw.get("F", 128),
+                         kw.get("w13s", NULL), kw.get("w2s", NULL), kw.get("ns", 0), p, kw.get("k", 2), p, p, p,
+                         kw.get("act", 0), kw.get("dout", p), kw.get("dx", p), kw.get("dw13", p), p, NULL, NULL,
+                         kw.get("dtopk", NULL), kw.get("ws", p), kw.get("wsb", 1 << 40), NULL, NULL]
+    assert f(*args(d=96)) == 2                 # d % 64
+    assert f(*args(F=100)) == 2                # F % 64
+    assert f(*args(E=257)) == 2                # E > 256
+    assert f(*args(k=9, E=8)) == 1             # k > E
+    assert f(*args(act=3)) == 1                # activation
+    assert f(*args(ns=1)) == 1                 # shared expert weights / gradients missing
+    assert f(*args(dout=odd)) == 1             # misaligned
+    assert f(*args(dtopk=ctypes.c_void_p(260))) == 1   # dL/dw must be 16-byte aligned
+    assert f(*args(dw13=NULL)) == 1            # gradient output missing
+    assert f(*args(dx=NULL)) == 1
+    assert f(*args(wsb=16)) == 3               # workspace too small
+    assert f(*args(ws=NULL)) == 3              # workspace missing
+    T, d, F, E, k = 300, 256, 192, 8, 2
+    P = oracle.max_padded(T, k, E, 128)
+    need = M.moe_backward_workspace_size(T, d, F, E, k, M.ACT_SWIGLU, 0)
+    # x and dL/dout rows [P, d] bf16 each, fp32 pre-activations and bf16 da [P, 2F], w*h [P, F], fp32 dx [T, d]
+    lo = P * (2 * d * 2 + 2 * F * 4 + 2 * F * 2 + F * 2) + T * d * 4
+    assert lo <= need <= lo + 1792
+    assert M.moe_backward_workspace_size(T, d, 100, E, k, M.ACT_SWIGLU, 0) == 0
+
+
 def test_layer_host_checks(lib):
     f = lib.moe_layer
     p = ctypes.c_void_p(256)
