@@ -28,9 +28,11 @@ meet at barriers and the slowest rank's time is reported.
 Each workload also carries, measured in the same run: the end-to-end step through
 the public API with host buffers (one host-to-device copy of x and logits,
 one device-to-host copy of out per step), the dominant kernel's roofline,
-the clocks seen, the CPU oracle on a bounded token sample, and the router
+the clocks seen, the CPU oracle on a bounded token sample, the router
 (moe_router: x . W_g^T and top-k gating, the step before the layer) on its
-own with a seeded W_g.
+own with a seeded W_g, and, for the 128-row prefill workloads, the backward
+(moe_backward: dx, dW13, dW2 and dL/d topk_weights from a seeded dL/dout)
+timed the same way.
 
 --impl reference times the CPU fp64 oracle (test infrastructure) on the host
 cores on a bounded sample of the same workload; rank 0 only.
@@ -84,6 +86,7 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="all", choices=["all"] + sorted(W.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward leg (block_m = 128 workloads)")
     ap.add_argument("--single-copy", action="store_true",
                     help="one copy of the inputs and an L2 flush before every step (small device footprint, "
                          "e.g. for profiler captures)")
@@ -574,6 +577,74 @@ def measure_workload(name, args, dev, pg, world, rank, cpu_seconds):
                       g_router_steps.replay if g_router_steps is not None else None)
     del g_router, g_router_steps
 
+    # ---- the backward (moe_backward: dx, dW13, dW2, dL/dw) on the 128-row
+    # layout, with a seeded dL/dout per input copy; same timing rule ----
+    backward = None
+    if cfg.block_m == 128 and not args.no_backward:
+        grads = M.MoEGradBuffers(cfg.T, cfg.d, cfg.F, cfg.E, cfg.k, cfg.act, cfg.n_shared, dev)
+        for i, st in enumerate(sets):
+            st["dout"] = to_dev(W.grad_output(cfg.T, cfg.d, seed=cfg.seed + 50 + i))
+
+        def bwd_call(st):
+            grads.backward(buf, st["x"], st["w13"], st["w2"], st["dout"], st["w13s"], st["w2s"])
+            return M.moe_last_launch_count()
+
+        b_launches = 0
+        for i in range(args.warmup):
+            b_launches = bwd_call(sets[i % n_copies])
+        torch.cuda.synchronize(dev)
+        g_bwd = [capture(lambda st=st: bwd_call(st)) for st in sets]
+        g_bwd_steps = None
+        if rotate:
+            g_bwd_steps = capture(lambda: [bwd_call(sets[i % n_copies]) for i in range(args.steps)])
+            g_bwd_steps.replay()
+            torch.cuda.synchronize(dev)
+        bwd_ms = timed([g.replay for g in g_bwd], args.steps, g_bwd_steps.replay if g_bwd_steps is not None else None)
+        assert M.moe_read_status(buf.status) == 0, "device status set during the backward"
+        M.moe_profile_enable(True)
+        g_bprof = [capture(lambda st=st: bwd_call(st)) for st in sets]
+        M.moe_profile_enable(False)
+        b_stages = {k_: [0.0, 0] for k_ in M.STAGES}
+        for _ in range(-(-args.steps // n_copies)):
+            for g in g_bprof:
+                if not rotate:
+                    flush.zero_()
+                g.replay()
+            torch.cuda.synchronize(dev)
+            for k_, (ms, c) in M.moe_profile_collect(release=False).items():
+                b_stages[k_][0] += ms
+                b_stages[k_][1] += c
+        M.moe_profile_collect(release=True)
+        del g_bwd, g_bwd_steps, g_bprof
+        rows = cfg.T * cfg.k + cfg.T * cfg.n_shared
+        # algorithmic: dh (2 rows d F), dx (2 rows n1 d), dW13 (2 rows n1 d),
+        # dW2 (2 rows d F) = twice the forward; the recomputed gate/up
+        # pre-activations (2 rows n1 d) are reported on top
+        b_flops = 2 * cfg.flops_total()
+        recompute = 2 * rows * cfg.n1 * cfg.d
+        b_s = bwd_ms / args.steps / 1e3
+        bst = {k: round(v[0] / max(v[1], 1) * 1e3, 2) for k, v in b_stages.items() if v[1]}
+        dom = max(("bwd_recompute", "bwd_dh_gemm", "bwd_dx_gemm", "bwd_dw13_gemm", "bwd_dw2_gemm"),
+                  key=lambda k_: b_stages[k_][0])
+        dom_flops = {"bwd_recompute": recompute, "bwd_dh_gemm": 2 * rows * cfg.d * cfg.F,
+                     "bwd_dx_gemm": 2 * rows * cfg.n1 * cfg.d, "bwd_dw13_gemm": 2 * rows * cfg.n1 * cfg.d,
+                     "bwd_dw2_gemm": 2 * rows * cfg.d * cfg.F}[dom]
+        dom_s = b_stages[dom][0] / max(b_stages[dom][1], 1) / 1e3
+        peaks_b, _ = load_peaks()
+        backward = {"ms_per_step": round(bwd_ms / args.steps, 5),
+                    "value": round(world * b_flops / b_s / 1e12, 4), "unit": "TFLOPS",
+                    "algorithmic_flops": int(b_flops), "recompute_flops": int(recompute),
+                    "tflops_incl_recompute": round(world * (b_flops + recompute) / b_s / 1e12, 4),
+                    "launches_per_step": int(b_launches), "gpu_launches": int(b_launches * args.steps),
+                    "stages_us": bst,
+                    "roofline": {"bound": "tensor", "kernel": dom, "unit": "TFLOP/s",
+                                 "achieved": round(dom_flops / dom_s / 1e12, 2), "peak": peaks_b["bf16_tflops"],
+                                 "frac": round(dom_flops / dom_s / 1e12 / peaks_b["bf16_tflops"], 4),
+                                 "per_launch_us": round(dom_s * 1e6, 2), "algorithmic_flops": int(dom_flops)}}
+        del grads
+        for st in sets:
+            st.pop("dout", None)
+
     sec_per_step = total_ms / args.steps / 1e3
     value = whole_job_tflops(world, alg["flops_total"], total_ms, args.steps)
     e2e_value = whole_job_tflops(world, alg["flops_total"], e2e_ms, args.steps)
@@ -614,6 +685,8 @@ def measure_workload(name, args, dev, pg, world, rank, cpu_seconds):
         "launches_per_step": int(launches_per_step),
         "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
     }
+    if backward is not None:
+        res["backward"] = backward
     # free this workload's device memory before the next one
     del sets, buf, wg, r_logits, r_ids, r_w, flush
     torch.cuda.synchronize(dev)
@@ -651,6 +724,7 @@ def run_ours(args):
         "stages_source": h["stages_source"],
         "roofline": h["roofline"],
         "router": h["router"],
+        "backward": h.get("backward"),
         "e2e": h["e2e"],
         "gpu_launches": h["gpu_launches"],
         "clocks": h["clocks"],
