@@ -194,6 +194,48 @@ def make_inputs(cfg: MoEConfig, threads: int = 8) -> MoEInputs:
     return MoEInputs(cfg, x, logits, w13, w2, w13s, w2s, router_w)
 
 
+MX_BLOCK = 32     # K values sharing one power-of-two scale
+E4M3_MAX = 448.0  # largest finite e4m3 value
+
+
+def quantize_mxfp8(w_bits: np.ndarray):
+    """Weight-only block quantisation of a bf16 stack [E, rows, K] (bits) for
+    the fp8 expert weights: every run of 32 consecutive K values of a row
+    shares a power-of-two scale 2^s (s the smallest integer with
+    max|w| / 2^s <= 448), stored as the byte s + 127; the values w / 2^s are
+    rounded to e4m3 (round to nearest even; torch's cast).
+
+    Returns (q uint8 [E, rows, K] e4m3 bit patterns, scales uint8
+    [E, K/32, rows]) -- the scales K-block-major, so that the scales of 128
+    consecutive rows for one 64-wide K step are two rows of 128 bytes."""
+    import torch
+    w = bf16_bits_to_f32(w_bits).astype(np.float64)
+    E, R, K = w.shape
+    assert K % MX_BLOCK == 0
+    blocks = w.reshape(E, R, K // MX_BLOCK, MX_BLOCK)
+    amax = np.abs(blocks).max(axis=3)
+    with np.errstate(divide="ignore"):
+        s = np.ceil(np.log2(np.where(amax > 0, amax, 1.0) / E4M3_MAX))
+    s = np.clip(s, -126, 127).astype(np.int64)               # byte 1..254
+    scaled = blocks / np.exp2(s)[..., None]
+    q = torch.from_numpy(scaled.reshape(E, R, K).astype(np.float32)).to(torch.float8_e4m3fn)
+    q_bits = q.view(torch.uint8).numpy().copy()
+    scales = np.ascontiguousarray((s + 127).astype(np.uint8).transpose(0, 2, 1))
+    return q_bits, scales
+
+
+def fp8_weights(inp: "MoEInputs"):
+    """The fp8 form of one configuration's expert weights: (w13_q, w13_s,
+    w2_q, w2_s, w13s_q, w13s_s, w2s_q, w2s_s), the shared expert's entries
+    None without one."""
+    out = list(quantize_mxfp8(inp.w13)) + list(quantize_mxfp8(inp.w2))
+    if inp.w13_shared is not None:
+        out += list(quantize_mxfp8(inp.w13_shared)) + list(quantize_mxfp8(inp.w2_shared))
+    else:
+        out += [None] * 4
+    return tuple(out)
+
+
 def grad_output(T: int, d: int, seed: int) -> np.ndarray:
     """Seeded dL/dout for the backward: N(0, 1) in bf16 bits [T, d]."""
     return _normal_bf16(np.random.SeedSequence(seed).spawn(1)[0], (T, d), 1.0)

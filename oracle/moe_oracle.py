@@ -71,6 +71,29 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     return u32.view(np.float32).astype(np.float64)
 
 
+def e4m3_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact value of fp8 e4m3 bit patterns (uint8): sign, 4 exponent bits
+    (bias 7), 3 mantissa bits; exponent field 0 is subnormal (m * 2^-9);
+    S.1111.111 is NaN and there is no infinity (largest value 448)."""
+    b = np.asarray(bits, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 0x7).astype(np.float64)
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = np.where((e == 15) & (m == 7), np.nan, val)
+    return sign * val
+
+
+def dequant_mxfp8(q: np.ndarray, scales: np.ndarray, block: int = 32) -> np.ndarray:
+    """fp8 expert weights as fp64: w[.., r, c] = e4m3(q[.., r, c]) *
+    2^(scales[.., c // block, r] - 127), with q [..., rows, K] and the scale
+    bytes K-block-major [..., K / block, rows]."""
+    w = e4m3_to_f64(q)
+    s = np.asarray(scales, dtype=np.int64) - 127
+    per_col = np.repeat(np.swapaxes(s, -1, -2), block, axis=-1)  # [..., rows, K]
+    return w * np.exp2(per_col.astype(np.float64))
+
+
 # --------------------------------------------------------------------------
 # Route
 # --------------------------------------------------------------------------
