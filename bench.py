@@ -62,10 +62,8 @@ METRIC = "MoE layer TFLOPS and tokens/s on 1 B200; % of bf16 tensor peak / HBM r
 # --warmup 3 --no-cpu-baseline --single-copy under ncu -k <kernel>).  An
 # entry is removed whenever the kernel changes after its capture.
 NCU_TRAFFIC = {
-    ("decode", "fused_expert"): 202_819_328,
-    ("relu2", "fused_expert"): 2_642_480_832,
-    ("dsv3", "gate_up_gemm"): 1_020_184_832,
-    ("zipf", "gate_up_gemm"): 1_496_556_680,
+    ("decode", "fused_expert"): 201_748_736,
+    ("zipf", "gate_up_gemm"): 1_502_857_216,
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -87,6 +85,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward leg (block_m = 128 workloads)")
+    ap.add_argument("--fp8", action="store_true", help="with --workload NAME: also measure it with fp8 expert weights")
     ap.add_argument("--single-copy", action="store_true",
                     help="one copy of the inputs and an L2 flush before every step (small device footprint, "
                          "e.g. for profiler captures)")
@@ -373,15 +372,18 @@ def roofline(cfg, alg, stages, total_ms, steps, launches_per_step, rotate, peaks
     return roof
 
 
-def measure_workload(name, args, dev, pg, world, rank, cpu_seconds):
+def measure_workload(name, args, dev, pg, world, rank, cpu_seconds, fp8=False):
     """Every figure of one workload: device-timed steps, per-kernel times,
-    roofline, the end-to-end step, the router and the CPU oracle."""
+    roofline, the end-to-end step, the router and the CPU oracle.  With fp8,
+    the layer runs on the workload's expert weights quantised to fp8
+    (moe_layer_fp8) and only the layer itself is measured."""
     import torch
 
     from grouped_gemm_gating_b200 import moe as M
 
     cfg = W.CONFIGS[name]
     inp = W.make_inputs(cfg)
+    q8 = W.fp8_weights(inp) if fp8 else None
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
 
     def to_dev(bits):
@@ -403,6 +405,10 @@ def measure_workload(name, args, dev, pg, world, rank, cpu_seconds):
         x_v, lg_v = io_views(io)
         x_v.copy_(to_dev(inp.x))
         lg_v.copy_(torch.from_numpy(inp.logits).to(dev))
+        if fp8:
+            wq = M.Fp8Experts(*[None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+                                for a in q8])
+            return dict(io=io, x=x_v, logits=lg_v, wq=wq, w13=None, w2=None, w13s=None, w2s=None)
         return dict(io=io, x=x_v, logits=lg_v,
                     w13=to_dev(inp.w13), w2=to_dev(inp.w2),
                     w13s=to_dev(inp.w13_shared) if cfg.n_shared else None,
@@ -416,8 +422,11 @@ def measure_workload(name, args, dev, pg, world, rank, cpu_seconds):
     def step(st, xin=None, lgin=None):
         # the whole layer through the public API: route + align + forward
         # (one launch for decode batches)
-        buf.layer(st["logits"] if lgin is None else lgin, st["x"] if xin is None else xin,
-                  st["w13"], st["w2"], st["w13s"], st["w2s"], **rk)
+        if fp8:
+            buf.layer_fp8(st["logits"] if lgin is None else lgin, st["x"] if xin is None else xin, st["wq"], **rk)
+        else:
+            buf.layer(st["logits"] if lgin is None else lgin, st["x"] if xin is None else xin,
+                      st["w13"], st["w2"], st["w13s"], st["w2s"], **rk)
         return M.moe_last_launch_count()
 
     # Cold inputs between steps: the timed steps run back to back, each on one
@@ -430,6 +439,12 @@ def measure_workload(name, args, dev, pg, world, rank, cpu_seconds):
     torch.cuda.synchronize(dev)
     topk_ids = buf.topk_ids.cpu().numpy()
     alg = algorithmic(cfg, topk_ids)
+    if fp8:
+        # the weight stream is one e4m3 byte per weight plus one scale byte
+        # per 32 weights
+        wb = alg["weight_bytes"] // 2 * 33 // 32
+        alg["fused_bytes"] += wb - alg["weight_bytes"]
+        alg["weight_bytes"] = wb
     touched = alg["weight_bytes"]
     n_copies = 1 + -(-2 * l2 // touched)
     rotate = n_copies <= MAX_INPUT_COPIES and not args.single_copy
@@ -553,6 +568,28 @@ def measure_workload(name, args, dev, pg, world, rank, cpu_seconds):
     e2e_ms = timed([g.replay for g in g_e2e], args.steps, g_e2e_steps.replay if g_e2e_steps is not None else None)
     assert torch.equal(out_h.view(torch.int16), buf.out.cpu().view(torch.int16))
     del g_main, g_prof, g_e2e, g_steps, g_e2e_steps
+
+    if fp8:
+        sec_per_step = total_ms / args.steps / 1e3
+        peaks, peak_src = load_peaks()
+        res = {
+            "value": round(whole_job_tflops(world, alg["flops_total"], total_ms, args.steps), 4), "unit": "TFLOPS",
+            "ms_per_step": round(total_ms / args.steps, 5), "tokens_per_s": round(world * cfg.T / sec_per_step, 1),
+            "config": dict(job_config(cfg, world, alg["U"]), weights="fp8 e4m3, power-of-two scale per 32 K values"),
+            "stages_us": {k: round(v[0] / max(v[1], 1) * 1e3, 2) for k, v in stages.items() if v[1]},
+            "roofline": roofline(cfg, alg, stages, total_ms, args.steps, launches_per_step, rotate, peaks, peak_src),
+            "e2e": {"value": round(whole_job_tflops(world, alg["flops_total"], e2e_ms, args.steps), 4),
+                    "unit": "TFLOPS", "ms_per_step": round(e2e_ms / args.steps, 5),
+                    "h2d_bytes_per_step": int(io_bytes), "d2h_bytes_per_step": int(cfg.T * cfg.d * 2)},
+            "gpu_launches": int(launches), "launches_per_step": int(launches_per_step),
+            "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        }
+        res["roofline"]["traffic"] = None
+        res["roofline"]["traffic_vs_algorithmic"] = None
+        del sets, buf, flush
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+        return res
 
     # ---- the gate before the layer (moe_router: x . W_g^T + top-k), on its
     # own: same x copies, a seeded W_g ~ N(0, 0.02), the same timing rule ----
@@ -710,6 +747,10 @@ def run_ours(args):
     for name in names:
         cpu_s = 0.0 if args.no_cpu_baseline else (10.0 if name == head else 3.0)
         results[name] = measure_workload(name, args, dev, pg, world, rank, cpu_s)
+    if args.workload == "all" or args.fp8:
+        # the bandwidth-bound shapes again with fp8 expert weights
+        for name in [n for n in names if W.CONFIGS[n].block_m <= 64 and n != "tiny"]:
+            results[name + "_fp8"] = measure_workload(name, args, dev, pg, world, rank, 0.0, fp8=True)
     h = results[head]
     line = {
         "metric": METRIC, "value": h["value"], "unit": "TFLOPS", "n_gpus": world,
@@ -731,8 +772,8 @@ def run_ours(args):
     }
     if "cpu_baseline" in h:
         line["cpu_baseline"] = h["cpu_baseline"]
-    if len(names) > 1:
-        line["workloads"] = {n: results[n] for n in names}
+    if len(results) > 1:
+        line["workloads"] = dict(results)
     if pg is not None:
         pg.destroy_process_group()
     if rank == 0:

@@ -147,7 +147,29 @@ bool encode_2d(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, ui
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// uint8 tensor [depth, rows, inner] (inner contiguous) as a 3-D map with
+// box_inner x box_rows boxes, no swizzle; zero fill out of bounds.
+bool encode_3d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                  uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {inner, rows, depth};
+  const cuuint64_t strides[2] = {inner, rows * inner};
+  const cuuint32_t box[3] = {box_inner, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// fp8 expert weights (e4m3 values [E, rows, K] and their scale bytes
+// [E, K / 32, rows]) for the fused expert kernel.
+struct Fp8Weights {
+  const uint8_t *w13, *s13, *w2, *s2;      // routed experts
+  const uint8_t *w13s, *s13s, *w2s, *s2s;  // shared expert (n_shared == 1)
+};
 
 bool valid_block_m(int bm) { return bm == 16 || bm == 32 || bm == 64 || bm == 128; }
 
@@ -364,7 +386,7 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
                         const float* topk_weights, int k, const int32_t* sorted_token_ids,
                         const int32_t* expert_ids, const int32_t* num_tokens_post_padded, int block_m, moe_act act,
                         uint16_t* out, void* ws, int32_t* dev_status, cudaStream_t s, int* launches_io,
-                        const moe::FusedRoute* route) {
+                        const moe::FusedRoute* route, const Fp8Weights* fp8 = nullptr) {
   const int bm = block_m;
   const int64_t P_max = moe_max_padded(T, k, E, bm);
   const int64_t P_total = padded_total(T, k, E, bm, n_shared);
@@ -394,13 +416,35 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
     // loaded in boxes of the kernel's box height; W2 tiles: 128 d rows
     const uint32_t box13 = act == MOE_ACT_SWIGLU ? moe::kFusedBoxRowsGated : moe::kFusedBoxRowsRelu2;
     const uint32_t box2 = moe::kFusedBoxRowsW2;
-    if (!encode_3d(&fa.tm_w13, w13, d, n1, E, box13) || !encode_3d(&fa.tm_w2, w2, F, d, E, box2)) return MOE_ERR_CUDA;
-    if (n_shared) {
-      if (!encode_3d(&fa.tm_w13s, w13_shared, d, n1, 1, box13) || !encode_3d(&fa.tm_w2s, w2_shared, F, d, 1, box2))
+    if (fp8 != nullptr) {
+      // e4m3 weights in boxes of 64 K bytes x 128 rows; scale bytes in boxes
+      // of 128 rows x 2 K blocks
+      if (!encode_3d_u8(&fa.tm_w13, fp8->w13, d, n1, E, 64, 128) || !encode_3d_u8(&fa.tm_w2, fp8->w2, F, d, E, 64, 128) ||
+          !encode_3d_u8(&fa.tm_s13, fp8->s13, n1, d / 32, E, 128, 2) ||
+          !encode_3d_u8(&fa.tm_s2, fp8->s2, d, F / 32, E, 128, 2))
         return MOE_ERR_CUDA;
+      if (n_shared) {
+        if (!encode_3d_u8(&fa.tm_w13s, fp8->w13s, d, n1, 1, 64, 128) ||
+            !encode_3d_u8(&fa.tm_w2s, fp8->w2s, F, d, 1, 64, 128) ||
+            !encode_3d_u8(&fa.tm_s13s, fp8->s13s, n1, d / 32, 1, 128, 2) ||
+            !encode_3d_u8(&fa.tm_s2s, fp8->s2s, d, F / 32, 1, 128, 2))
+          return MOE_ERR_CUDA;
+      } else {
+        fa.tm_w13s = fa.tm_w13;
+        fa.tm_w2s = fa.tm_w2;
+        fa.tm_s13s = fa.tm_s13;
+        fa.tm_s2s = fa.tm_s2;
+      }
     } else {
-      fa.tm_w13s = fa.tm_w13;
-      fa.tm_w2s = fa.tm_w2;
+      if (!encode_3d(&fa.tm_w13, w13, d, n1, E, box13) || !encode_3d(&fa.tm_w2, w2, F, d, E, box2))
+        return MOE_ERR_CUDA;
+      if (n_shared) {
+        if (!encode_3d(&fa.tm_w13s, w13_shared, d, n1, 1, box13) || !encode_3d(&fa.tm_w2s, w2_shared, F, d, 1, box2))
+          return MOE_ERR_CUDA;
+      } else {
+        fa.tm_w13s = fa.tm_w13;
+        fa.tm_w2s = fa.tm_w2;
+      }
     }
     fa.x = x;
     fa.acc = y;
@@ -429,7 +473,7 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
     cudaError_t err;
     {
       StageScope scope(6, s);
-      err = moe::launch_fused_expert(epi, bm, route != nullptr, fa, grid < 1 ? 1 : grid, s);
+      err = moe::launch_fused_expert(epi, bm, route != nullptr, fa, grid < 1 ? 1 : grid, s, fp8 != nullptr);
     }
     if (err != cudaSuccess) return MOE_ERR_CUDA;
     ++launches;
@@ -561,6 +605,123 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
 
 }  // namespace
 
+namespace {
+
+moe_status forward_checked(const uint16_t* x, int T, int d, const uint16_t* w13, const uint16_t* w2, int E, int F,
+                       const uint16_t* w13_shared, const uint16_t* w2_shared, int n_shared,
+                       const float* topk_weights, int k, const int32_t* sorted_token_ids,
+                       const int32_t* expert_ids, const int32_t* num_tokens_post_padded, const int32_t* inv_pos,
+                       int block_m, moe_act act, uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
+                       moe_stream_t stream, const Fp8Weights* fp8) {
+  moe_status st = check_dims(T, d, F, E, k);
+  if (st != MOE_OK) return st;
+  if (!valid_block_m(block_m)) return MOE_ERR_UNSUPPORTED;
+  if (act != MOE_ACT_SWIGLU && act != MOE_ACT_RELU2) return MOE_ERR_INVALID_ARG;
+  if (n_shared != 0 && n_shared != 1) return MOE_ERR_UNSUPPORTED;
+  if (n_shared && (!w13_shared || !w2_shared)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return finish(cudaSuccess, 0);
+  if (!x || !w13 || !w2 || !topk_weights || !sorted_token_ids || !expert_ids || !num_tokens_post_padded || !out)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w13) || !aligned16(w2) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (n_shared && (!aligned16(w13_shared) || !aligned16(w2_shared))) return MOE_ERR_INVALID_ARG;
+  if (fp8 != nullptr) {
+    if (!moe::fused_expert_supported(block_m)) return MOE_ERR_UNSUPPORTED;  // block_m <= 64 only
+    if (!fp8->s13 || !fp8->s2 || !aligned16(fp8->s13) || !aligned16(fp8->s2)) return MOE_ERR_INVALID_ARG;
+    if (n_shared && (!fp8->s13s || !fp8->s2s || !aligned16(fp8->s13s) || !aligned16(fp8->s2s)))
+      return MOE_ERR_INVALID_ARG;
+  }
+  const size_t need = moe_workspace_size(T, d, F, E, k, block_m, act, n_shared);
+  if (ws == nullptr || ws_bytes < need) return MOE_ERR_WORKSPACE;
+
+  int launches = 0;
+  return forward_impl(x, T, d, w13, w2, E, F, w13_shared, w2_shared, n_shared, topk_weights, k, sorted_token_ids,
+                      expert_ids, num_tokens_post_padded, block_m, act, out, ws, dev_status,
+                      reinterpret_cast<cudaStream_t>(stream), &launches, nullptr, fp8);
+}
+
+moe_status layer_checked(const float* logits, int T, int E, int k, int n_group, int topk_group,
+                     moe_group_score group_score, int renormalize, float routed_scaling, const uint16_t* x, int d,
+                     const uint16_t* w13, const uint16_t* w2, int F, const uint16_t* w13_shared,
+                     const uint16_t* w2_shared, int n_shared, int block_m, moe_act act, int32_t* topk_ids,
+                     float* topk_weights, int32_t* sorted_token_ids, int32_t* expert_ids,
+                     int32_t* num_tokens_post_padded, int32_t* inv_pos, uint16_t* out, void* ws, size_t ws_bytes,
+                     int32_t* dev_status, moe_stream_t stream, const Fp8Weights* fp8) {
+  moe_status st = check_route_args(T, E, k, n_group, topk_group, group_score, routed_scaling);
+  if (st != MOE_OK) return st;
+  st = check_dims(T, d, F, E, k);
+  if (st != MOE_OK) return st;
+  if (!valid_block_m(block_m)) return MOE_ERR_UNSUPPORTED;
+  if (act != MOE_ACT_SWIGLU && act != MOE_ACT_RELU2) return MOE_ERR_INVALID_ARG;
+  if (n_shared != 0 && n_shared != 1) return MOE_ERR_UNSUPPORTED;
+  if (n_shared && (!w13_shared || !w2_shared)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return finish(cudaSuccess, 0);
+  if (!logits || !x || !w13 || !w2 || !topk_ids || !topk_weights || !sorted_token_ids || !expert_ids ||
+      !num_tokens_post_padded || !inv_pos || !out)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w13) || !aligned16(w2) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (n_shared && (!aligned16(w13_shared) || !aligned16(w2_shared))) return MOE_ERR_INVALID_ARG;
+  if (fp8 != nullptr) {
+    if (!moe::fused_expert_supported(block_m)) return MOE_ERR_UNSUPPORTED;  // block_m <= 64 only
+    if (!fp8->s13 || !fp8->s2 || !aligned16(fp8->s13) || !aligned16(fp8->s2)) return MOE_ERR_INVALID_ARG;
+    if (n_shared && (!fp8->s13s || !fp8->s2s || !aligned16(fp8->s13s) || !aligned16(fp8->s2s)))
+      return MOE_ERR_INVALID_ARG;
+  }
+  const size_t need = moe_workspace_size(T, d, F, E, k, block_m, act, n_shared);
+  if (ws == nullptr || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int launches = 0;
+  if (moe::fused_expert_supported(block_m) && moe::fused_routing_supported(T, k, E, n_group, block_m)) {
+    moe::FusedRoute r;
+    r.logits = logits;
+    r.n_group = n_group;
+    r.topk_group = topk_group;
+    r.group_score = static_cast<int>(group_score);
+    r.renormalize = renormalize ? 1 : 0;
+    r.routed_scaling = routed_scaling;
+    r.topk_ids = topk_ids;
+    r.topk_w = topk_weights;
+    r.sorted_ids = sorted_token_ids;
+    r.expert_ids = expert_ids;
+    r.ntpp = num_tokens_post_padded;
+    r.inv_pos = inv_pos;
+    r.P_max = static_cast<int>(moe_max_padded(T, k, E, block_m));
+    return forward_impl(x, T, d, w13, w2, E, F, w13_shared, w2_shared, n_shared, topk_weights, k, sorted_token_ids,
+                        expert_ids, num_tokens_post_padded, block_m, act, out, ws, dev_status, s, &launches, &r, fp8);
+  }
+  // separate launches: routing and align (fused when the batch is small),
+  // then the forward; the align scratch borrows the forward's accumulator
+  // region, which the forward only touches after the align has finished
+  const int P_max = static_cast<int>(moe_max_padded(T, k, E, block_m));
+  cudaError_t err;
+  if (moe::route_align_fusable(T, k, n_group)) {
+    StageScope scope(5, s);
+    err = moe::launch_route_align(logits, T, E, k, n_group, topk_group, static_cast<int>(group_score),
+                                  renormalize ? 1 : 0, routed_scaling, topk_ids, topk_weights, block_m, P_max,
+                                  sorted_token_ids, expert_ids, num_tokens_post_padded, inv_pos, dev_status, s,
+                                  &launches);
+  } else {
+    {
+      StageScope scope(0, s);
+      err = moe::launch_route(logits, T, E, k, n_group, topk_group, static_cast<int>(group_score),
+                              renormalize ? 1 : 0, routed_scaling, topk_ids, topk_weights, dev_status, s, &launches);
+    }
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    const size_t align_need = moe_align_workspace_size(T, k, E);
+    uint8_t* wsb = reinterpret_cast<uint8_t*>(round_up(reinterpret_cast<uintptr_t>(ws), kWsAlign));
+    const size_t acc_off = need - kWsAlign - round_up(static_cast<size_t>(T) * d * 4, kWsAlign);
+    if (align_need > round_up(static_cast<size_t>(T) * d * 4, kWsAlign)) return MOE_ERR_WORKSPACE;
+    StageScope scope(1, s);
+    err = moe::launch_align(topk_ids, T * k, E, block_m, P_max, sorted_token_ids, expert_ids,
+                            num_tokens_post_padded, inv_pos, reinterpret_cast<int32_t*>(wsb + acc_off), dev_status, s,
+                            &launches);
+  }
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  return forward_impl(x, T, d, w13, w2, E, F, w13_shared, w2_shared, n_shared, topk_weights, k, sorted_token_ids,
+                      expert_ids, num_tokens_post_padded, block_m, act, out, ws, dev_status, s, &launches, nullptr, fp8);
+}
+
+}  // namespace
+
 extern "C" {
 
 moe_status moe_router(const uint16_t* x, int T, int d, const uint16_t* w_gate, int E, int k, int n_group,
@@ -637,30 +798,30 @@ moe_status moe_router(const uint16_t* x, int T, int d, const uint16_t* w_gate, i
   return finish(err, launches);
 }
 
+
 moe_status moe_forward(const uint16_t* x, int T, int d, const uint16_t* w13, const uint16_t* w2, int E, int F,
                        const uint16_t* w13_shared, const uint16_t* w2_shared, int n_shared,
                        const float* topk_weights, int k, const int32_t* sorted_token_ids,
                        const int32_t* expert_ids, const int32_t* num_tokens_post_padded, const int32_t* inv_pos,
                        int block_m, moe_act act, uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
                        moe_stream_t stream) {
-  moe_status st = check_dims(T, d, F, E, k);
-  if (st != MOE_OK) return st;
-  if (!valid_block_m(block_m)) return MOE_ERR_UNSUPPORTED;
-  if (act != MOE_ACT_SWIGLU && act != MOE_ACT_RELU2) return MOE_ERR_INVALID_ARG;
-  if (n_shared != 0 && n_shared != 1) return MOE_ERR_UNSUPPORTED;
-  if (n_shared && (!w13_shared || !w2_shared)) return MOE_ERR_INVALID_ARG;
-  if (T == 0) return finish(cudaSuccess, 0);
-  if (!x || !w13 || !w2 || !topk_weights || !sorted_token_ids || !expert_ids || !num_tokens_post_padded || !out)
-    return MOE_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(w13) || !aligned16(w2) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-  if (n_shared && (!aligned16(w13_shared) || !aligned16(w2_shared))) return MOE_ERR_INVALID_ARG;
-  const size_t need = moe_workspace_size(T, d, F, E, k, block_m, act, n_shared);
-  if (ws == nullptr || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  return forward_checked(x, T, d, w13, w2, E, F, w13_shared, w2_shared, n_shared, topk_weights, k, sorted_token_ids,
+                         expert_ids, num_tokens_post_padded, inv_pos, block_m, act, out, ws, ws_bytes, dev_status,
+                         stream, nullptr);
+}
 
-  int launches = 0;
-  return forward_impl(x, T, d, w13, w2, E, F, w13_shared, w2_shared, n_shared, topk_weights, k, sorted_token_ids,
-                      expert_ids, num_tokens_post_padded, block_m, act, out, ws, dev_status,
-                      reinterpret_cast<cudaStream_t>(stream), &launches, nullptr);
+moe_status moe_forward_fp8(const uint16_t* x, int T, int d, const uint8_t* w13_q, const uint8_t* w13_scales,
+                           const uint8_t* w2_q, const uint8_t* w2_scales, int E, int F, const uint8_t* w13s_q,
+                           const uint8_t* w13s_scales, const uint8_t* w2s_q, const uint8_t* w2s_scales, int n_shared,
+                           const float* topk_weights, int k, const int32_t* sorted_token_ids,
+                           const int32_t* expert_ids, const int32_t* num_tokens_post_padded, const int32_t* inv_pos,
+                           int block_m, moe_act act, uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
+                           moe_stream_t stream) {
+  const Fp8Weights f{w13_q, w13_scales, w2_q, w2_scales, w13s_q, w13s_scales, w2s_q, w2s_scales};
+  return forward_checked(x, T, d, reinterpret_cast<const uint16_t*>(w13_q), reinterpret_cast<const uint16_t*>(w2_q),
+                         E, F, reinterpret_cast<const uint16_t*>(w13s_q), reinterpret_cast<const uint16_t*>(w2s_q),
+                         n_shared, topk_weights, k, sorted_token_ids, expert_ids, num_tokens_post_padded, inv_pos,
+                         block_m, act, out, ws, ws_bytes, dev_status, stream, &f);
 }
 
 moe_status moe_layer(const float* logits, int T, int E, int k, int n_group, int topk_group,
@@ -670,72 +831,25 @@ moe_status moe_layer(const float* logits, int T, int E, int k, int n_group, int 
                      float* topk_weights, int32_t* sorted_token_ids, int32_t* expert_ids,
                      int32_t* num_tokens_post_padded, int32_t* inv_pos, uint16_t* out, void* ws, size_t ws_bytes,
                      int32_t* dev_status, moe_stream_t stream) {
-  moe_status st = check_route_args(T, E, k, n_group, topk_group, group_score, routed_scaling);
-  if (st != MOE_OK) return st;
-  st = check_dims(T, d, F, E, k);
-  if (st != MOE_OK) return st;
-  if (!valid_block_m(block_m)) return MOE_ERR_UNSUPPORTED;
-  if (act != MOE_ACT_SWIGLU && act != MOE_ACT_RELU2) return MOE_ERR_INVALID_ARG;
-  if (n_shared != 0 && n_shared != 1) return MOE_ERR_UNSUPPORTED;
-  if (n_shared && (!w13_shared || !w2_shared)) return MOE_ERR_INVALID_ARG;
-  if (T == 0) return finish(cudaSuccess, 0);
-  if (!logits || !x || !w13 || !w2 || !topk_ids || !topk_weights || !sorted_token_ids || !expert_ids ||
-      !num_tokens_post_padded || !inv_pos || !out)
-    return MOE_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(w13) || !aligned16(w2) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-  if (n_shared && (!aligned16(w13_shared) || !aligned16(w2_shared))) return MOE_ERR_INVALID_ARG;
-  const size_t need = moe_workspace_size(T, d, F, E, k, block_m, act, n_shared);
-  if (ws == nullptr || ws_bytes < need) return MOE_ERR_WORKSPACE;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  int launches = 0;
-  if (moe::fused_expert_supported(block_m) && moe::fused_routing_supported(T, k, E, n_group, block_m)) {
-    moe::FusedRoute r;
-    r.logits = logits;
-    r.n_group = n_group;
-    r.topk_group = topk_group;
-    r.group_score = static_cast<int>(group_score);
-    r.renormalize = renormalize ? 1 : 0;
-    r.routed_scaling = routed_scaling;
-    r.topk_ids = topk_ids;
-    r.topk_w = topk_weights;
-    r.sorted_ids = sorted_token_ids;
-    r.expert_ids = expert_ids;
-    r.ntpp = num_tokens_post_padded;
-    r.inv_pos = inv_pos;
-    r.P_max = static_cast<int>(moe_max_padded(T, k, E, block_m));
-    return forward_impl(x, T, d, w13, w2, E, F, w13_shared, w2_shared, n_shared, topk_weights, k, sorted_token_ids,
-                        expert_ids, num_tokens_post_padded, block_m, act, out, ws, dev_status, s, &launches, &r);
-  }
-  // separate launches: routing and align (fused when the batch is small),
-  // then the forward; the align scratch borrows the forward's accumulator
-  // region, which the forward only touches after the align has finished
-  const int P_max = static_cast<int>(moe_max_padded(T, k, E, block_m));
-  cudaError_t err;
-  if (moe::route_align_fusable(T, k, n_group)) {
-    StageScope scope(5, s);
-    err = moe::launch_route_align(logits, T, E, k, n_group, topk_group, static_cast<int>(group_score),
-                                  renormalize ? 1 : 0, routed_scaling, topk_ids, topk_weights, block_m, P_max,
-                                  sorted_token_ids, expert_ids, num_tokens_post_padded, inv_pos, dev_status, s,
-                                  &launches);
-  } else {
-    {
-      StageScope scope(0, s);
-      err = moe::launch_route(logits, T, E, k, n_group, topk_group, static_cast<int>(group_score),
-                              renormalize ? 1 : 0, routed_scaling, topk_ids, topk_weights, dev_status, s, &launches);
-    }
-    if (err != cudaSuccess) return MOE_ERR_CUDA;
-    const size_t align_need = moe_align_workspace_size(T, k, E);
-    uint8_t* wsb = reinterpret_cast<uint8_t*>(round_up(reinterpret_cast<uintptr_t>(ws), kWsAlign));
-    const size_t acc_off = need - kWsAlign - round_up(static_cast<size_t>(T) * d * 4, kWsAlign);
-    if (align_need > round_up(static_cast<size_t>(T) * d * 4, kWsAlign)) return MOE_ERR_WORKSPACE;
-    StageScope scope(1, s);
-    err = moe::launch_align(topk_ids, T * k, E, block_m, P_max, sorted_token_ids, expert_ids,
-                            num_tokens_post_padded, inv_pos, reinterpret_cast<int32_t*>(wsb + acc_off), dev_status, s,
-                            &launches);
-  }
-  if (err != cudaSuccess) return MOE_ERR_CUDA;
-  return forward_impl(x, T, d, w13, w2, E, F, w13_shared, w2_shared, n_shared, topk_weights, k, sorted_token_ids,
-                      expert_ids, num_tokens_post_padded, block_m, act, out, ws, dev_status, s, &launches, nullptr);
+  return layer_checked(logits, T, E, k, n_group, topk_group, group_score, renormalize, routed_scaling, x, d, w13, w2,
+                       F, w13_shared, w2_shared, n_shared, block_m, act, topk_ids, topk_weights, sorted_token_ids,
+                       expert_ids, num_tokens_post_padded, inv_pos, out, ws, ws_bytes, dev_status, stream, nullptr);
+}
+
+moe_status moe_layer_fp8(const float* logits, int T, int E, int k, int n_group, int topk_group,
+                         moe_group_score group_score, int renormalize, float routed_scaling, const uint16_t* x, int d,
+                         const uint8_t* w13_q, const uint8_t* w13_scales, const uint8_t* w2_q,
+                         const uint8_t* w2_scales, int F, const uint8_t* w13s_q, const uint8_t* w13s_scales,
+                         const uint8_t* w2s_q, const uint8_t* w2s_scales, int n_shared, int block_m, moe_act act,
+                         int32_t* topk_ids, float* topk_weights, int32_t* sorted_token_ids, int32_t* expert_ids,
+                         int32_t* num_tokens_post_padded, int32_t* inv_pos, uint16_t* out, void* ws,
+                         size_t ws_bytes, int32_t* dev_status, moe_stream_t stream) {
+  const Fp8Weights f{w13_q, w13_scales, w2_q, w2_scales, w13s_q, w13s_scales, w2s_q, w2s_scales};
+  return layer_checked(logits, T, E, k, n_group, topk_group, group_score, renormalize, routed_scaling, x, d,
+                       reinterpret_cast<const uint16_t*>(w13_q), reinterpret_cast<const uint16_t*>(w2_q), F,
+                       reinterpret_cast<const uint16_t*>(w13s_q), reinterpret_cast<const uint16_t*>(w2s_q), n_shared,
+                       block_m, act, topk_ids, topk_weights, sorted_token_ids, expert_ids, num_tokens_post_padded,
+                       inv_pos, out, ws, ws_bytes, dev_status, stream, &f);
 }
 
 size_t moe_backward_workspace_size(int T, int d, int F, int E, int k, moe_act act, int n_shared) {

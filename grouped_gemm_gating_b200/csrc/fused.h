@@ -27,9 +27,14 @@ struct FusedRoute {
 struct FusedArgs {
   CUtensorMap tm_w13;   // routed gate/up (or fc1) weights, 3-D {d, N1, E}; boxes of 64 x 64 rows
                         // (SwiGLU: 64 gate rows, then the matching 64 up rows) or 64 x 128 (relu^2)
+                        // fp8 weights: uint8 e4m3, boxes of 64 x 128 rows, no swizzle
   CUtensorMap tm_w13s;  // shared expert, 3-D {d, N1, 1}, same boxes
-  CUtensorMap tm_w2;    // routed down weights, 3-D {F, d, E}, 64 x 128 boxes
+  CUtensorMap tm_w2;    // routed down weights, 3-D {F, d, E}, 64 x 128 boxes (fp8: the same, uint8)
   CUtensorMap tm_w2s;   // shared expert, 3-D {F, d, 1}
+  // fp8 weights only: the power-of-two scale bytes, K-block-major
+  // [E, K / 32, rows] as 3-D {rows, K / 32, E} maps with 128 x 2 boxes (the
+  // scales of one stage's 128 rows and 64 K values)
+  CUtensorMap tm_s13, tm_s13s, tm_s2, tm_s2s;
   const uint16_t* x;    // [T, d] bf16
   float* acc;           // [T, d] fp32 accumulator (workspace; zeroed by the kernel)
   uint16_t* out;        // [T, d] bf16
@@ -63,6 +68,6 @@ bool fused_routing_supported(int T, int k, int E, int n_group, int block_m);
 // Upper bound on the fused kernel's tiles, for grid sizing.
 int64_t fused_expert_max_tiles(int act_epi, int total_blocks_max, int F);
 cudaError_t launch_fused_expert(int act_epi, int block_m, bool route, const FusedArgs& args, int grid,
-                                cudaStream_t stream);
+                                cudaStream_t stream, bool fp8 = false);
 
 }  // namespace moe

@@ -57,6 +57,8 @@
 // down-GEMM accumulators (groups of 64 columns).  Every wait is bounded in
 // time; on expiry the kernel records MOE_ERR_DEVICE_TIMEOUT and all roles
 // leave.
+#include <cuda_fp16.h>
+
 #include <atomic>
 
 #include "align_impl.cuh"
@@ -76,7 +78,7 @@ constexpr int kRouteMaxS = 256;
 // last CTA to finish, alone: the others leave without waiting for a release.
 constexpr int kLastCtaConvertMax = 16384;
 
-template <int EPI1, int TOK, bool ROUTE>
+template <int EPI1, int TOK, bool ROUTE, bool FP8 = false>
 struct FusedCfg {
   static constexpr bool kGated = (EPI1 == kEpiSwiGLU);
   static constexpr int kH = 128;                // h columns per tile
@@ -98,14 +100,23 @@ struct FusedCfg {
   static constexpr int kRouteBytes = ROUTE ? (4 * kRouteMaxS + 3 * (MOE_MAX_EXPERTS + 1) + 5) * 4 : 0;
   static constexpr int kFixedBytes = 2 * kHBufBytes + kTokBytes + kBarrierBytes + kRouteBytes + 1024;
   static constexpr int kStagesRaw = (227 * 1024 - kFixedBytes) / kStageBytes;
-  static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+  // fp8 weights: the weight stream lands in a deeper ring of raw stages (128
+  // rows x 64 e4m3 bytes and the 2 x 128 scale bytes of those rows), which
+  // the converter warps expand into a short ring of bf16 operand stages
+  static constexpr int kStages = FP8 ? 4 : (kStagesRaw > 12 ? 12 : kStagesRaw);
+  static constexpr int kRawWBytes = 128 * 64;
+  static constexpr int kRawStageBytes = kRawWBytes + 256;
+  static constexpr int kRawRoom = 227 * 1024 - kFixedBytes - kStages * kStageBytes - 1024;
+  static constexpr int kRawStages = FP8 ? (kRawRoom / kRawStageBytes > 16 ? 16 : kRawRoom / kRawStageBytes) : 0;
+  static constexpr int kRawRegion = (kRawStages * kRawStageBytes + 1023) / 1024 * 1024;
   // Down-GEMM accumulators: groups of kGroup d tiles (64 TMEM columns) form
   // one slot of a TMEM ring, so the epilogue synchronises once per group.
   static constexpr int kGroup = 64 / TOK;
   static constexpr int kD2Raw = (512 - 2 * kAcc1) / 64;
   static constexpr int kD2Slots = kD2Raw > 8 ? 8 : kD2Raw;
-  static constexpr int kNumThreads = 320;
-  static constexpr int kSmemBytes = kStages * kStageBytes + kFixedBytes;
+  // warps: producer, MMA, 4 epilogue, 4 gather (+ 4 converters for fp8 weights)
+  static constexpr int kNumThreads = FP8 ? 448 : 320;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kRawRegion + kFixedBytes;
   static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(128, TOK);
   static_assert(TOK == 16 || TOK == 32 || TOK == 64, "token rows per tile");
   static_assert(kStageBytes % 1024 == 0 && kHBufBytes % 1024 == 0, "1024-byte aligned operand tiles");
@@ -114,7 +125,8 @@ struct FusedCfg {
   static_assert(128 % kFusedBoxRowsGated == 0 && 128 % kFusedBoxRowsRelu2 == 0 && 128 % kFusedBoxRowsW2 == 0 &&
                     kFusedBoxRowsGated % 8 == 0 && kFusedBoxRowsRelu2 % 8 == 0 && kFusedBoxRowsW2 % 8 == 0,
                 "weight boxes tile the 128-row operand on swizzle-atom boundaries");
-  static_assert((2 * kStages + 9 + 2 * kD2Slots) * 8 + 16 <= kBarrierBytes, "barrier area");
+  static_assert((2 * kStages + 9 + 2 * kD2Slots + 2 * kRawStages) * 8 + 16 <= kBarrierBytes, "barrier area");
+  static_assert(!FP8 || kRawStages >= 6, "fp8 raw-stage ring depth");
   static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
 
@@ -149,6 +161,16 @@ __device__ __forceinline__ void red_add_f32(float* p, float v) {
 }
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Two e4m3 values (the low 16 bits of `two`, element 0 in the low byte)
+// times `scale`, as two bf16 (element 0 in the low half).  e4m3 -> f16 is
+// exact, and so is the product with a power of two within range.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two, float scale) {
+  uint32_t h;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h) : "r"(two));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return pack_bf16x2(f.x * scale, f.y * scale);
+}
 
 // Named barrier 1 over the four epilogue warps, 2 over the four gather warps
 // (barrier 0 is __syncthreads).  Each warp reconverges first, as the aligned
@@ -206,13 +228,14 @@ __device__ __forceinline__ bool spin_until(const int32_t* p, int target, volatil
   return true;
 }
 
-template <int EPI1, int TOK, bool ROUTE>
-__global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
+template <int EPI1, int TOK, bool ROUTE, bool FP8>
+__global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE, FP8>::kNumThreads, 1)
     fused_expert_kernel(const __grid_constant__ FusedArgs args) {
-  using C = FusedCfg<EPI1, TOK, ROUTE>;
+  using C = FusedCfg<EPI1, TOK, ROUTE, FP8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* hbuf = smem + C::kStages * C::kStageBytes;        // [2][kHk][TOK rows x 128 B]
+  uint8_t* raw = smem + C::kStages * C::kStageBytes;         // fp8 only: [kRawStages][weights | scales]
+  uint8_t* hbuf = raw + C::kRawRegion;                        // [2][kHk][TOK rows x 128 B]
   int* tok_s = reinterpret_cast<int*>(hbuf + 2 * C::kHBufBytes);  // [2][64]
   float* w_s = reinterpret_cast<float*>(tok_s + 2 * 64);                           // [2][64]
   uint64_t* full = reinterpret_cast<uint64_t*>(w_s + 2 * 64);
@@ -224,7 +247,9 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
   uint64_t* mma_done = hb_empty + 2;
   uint64_t* d2_full = mma_done + 1;
   uint64_t* d2_empty = d2_full + C::kD2Slots;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(d2_empty + C::kD2Slots);
+  uint64_t* raw_full = d2_empty + C::kD2Slots;    // fp8: the raw stage's bytes landed
+  uint64_t* raw_empty = raw_full + C::kRawStages;  // fp8: the converters are done with it
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(raw_empty + C::kRawStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* flag = reinterpret_cast<volatile int*>(tmem_holder + 2);
   volatile int* prod_issued = reinterpret_cast<volatile int*>(tmem_holder + 3);  // stages the producer filled
@@ -234,8 +259,14 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      ptx::mbar_init(&full[s], 1 + 128);
+      // bf16 weights: the producer's bytes and the gather warps' rows; fp8:
+      // the converter threads' expanded weights and the gather warps' rows
+      ptx::mbar_init(&full[s], FP8 ? 128 + 128 : 1 + 128);
       ptx::mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < C::kRawStages; ++s) {
+      ptx::mbar_init(&raw_full[s], 1);
+      ptx::mbar_init(&raw_empty[s], 4);
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&d1_full[b], 1);
@@ -256,6 +287,10 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
     if (args.n_shared_blocks) {
       ptx::prefetch_tmap(&args.tm_w13s);
       ptx::prefetch_tmap(&args.tm_w2s);
+    }
+    if (FP8) {
+      ptx::prefetch_tmap(&args.tm_s13);
+      ptx::prefetch_tmap(&args.tm_s2);
     }
   }
   if (warp == 1) {
@@ -399,8 +434,12 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
         if (e < 0 || e >= args.E) set_status(args.status, MOE_ERR_BAD_EXPERT_ID);  // TMA fills zeros
         return e;
       };
+      // the ring this producer fills: the bf16 operand stages, or for fp8
+      // weights the raw stages (whose slots the converters hand back)
+      constexpr int kRing = FP8 ? C::kRawStages : C::kStages;
+      uint64_t* ring_free = FP8 ? raw_empty : empty;
       auto acquire = [&]() {
-        if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.wait_ns)) {
+        if (!ptx::mbar_wait_bounded(&ring_free[stage], phase ^ 1u, abort_flag, args.wait_ns)) {
           fail();
           ok = false;
         }
@@ -409,10 +448,18 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
       int issued = 0;  // stages filled so far
       auto advance = [&]() {
         ++issued;
-        if (++stage == C::kStages) {
+        if (++stage == kRing) {
           stage = 0;
           phase ^= 1u;
         }
+      };
+      // fp8: one stage = 128 weight rows x 64 e4m3 bytes and the scale bytes
+      // of those rows for the stage's two 32-wide K blocks
+      auto load_raw = [&](const CUtensorMap* tw, const CUtensorMap* ts, int kcol, int row0, int e, uint64_t pol) {
+        uint8_t* rb = raw + stage * C::kRawStageBytes;
+        ptx::mbar_arrive_expect_tx(&raw_full[stage], C::kRawStageBytes);
+        ptx::tma_load_3d_hint(rb, tw, &raw_full[stage], kcol, row0, e, pol);
+        ptx::tma_load_3d_hint(rb + C::kRawWBytes, ts, &raw_full[stage], row0, kcol / 32, e, pol);
       };
       // Streamed weight lines are used once: mark them first to leave L2.
       const uint64_t evict_first = ptx::l2_policy_evict_first();
@@ -425,11 +472,15 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
             // K block s / kGU; SwiGLU: gate rows [wt*128, +128), then up rows [F + wt*128, +128)
             const int kb = s / C::kGU;
             const int row0 = (C::kGated && s != kb * C::kGU ? args.F : 0) + t.wt * C::kH;
-            uint8_t* sW = smem + stage * C::kStageBytes;
-            ptx::mbar_arrive_expect_tx(&full[stage], C::kWBytes);
+            if constexpr (FP8) {
+              load_raw(tm, t.shared_blk ? &args.tm_s13s : &args.tm_s13, kb * 64, row0, e, evict_first);
+            } else {
+              uint8_t* sW = smem + stage * C::kStageBytes;
+              ptx::mbar_arrive_expect_tx(&full[stage], C::kWBytes);
 #pragma unroll
-            for (int r = 0; r < 128; r += C::kBoxRows)
-              ptx::tma_load_3d_hint(sW + r * 128, tm, &full[stage], kb * 64, row0 + r, e, evict_first);
+              for (int r = 0; r < 128; r += C::kBoxRows)
+                ptx::tma_load_3d_hint(sW + r * 128, tm, &full[stage], kb * 64, row0 + r, e, evict_first);
+            }
             advance();
           }
         }
@@ -441,12 +492,17 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
           for (int s = 0; s < nk2 && acquire(); ++s) {
             const int dk = s / C::kHk, kk = s - dk * C::kHk;
             const int di = d_tile(dk, rot, n_d);
-            uint8_t* sW = smem + stage * C::kStageBytes;
-            ptx::mbar_arrive_expect_tx(&full[stage], C::kWBytes);
+            if constexpr (FP8) {
+              load_raw(tm, t.shared_blk ? &args.tm_s2s : &args.tm_s2, t.wt * C::kH + kk * 64, di * 128, e,
+                       evict_first);
+            } else {
+              uint8_t* sW = smem + stage * C::kStageBytes;
+              ptx::mbar_arrive_expect_tx(&full[stage], C::kWBytes);
 #pragma unroll
-            for (int r = 0; r < 128; r += kFusedBoxRowsW2)
-              ptx::tma_load_3d_hint(sW + r * 128, tm, &full[stage], t.wt * C::kH + kk * 64, di * 128 + r, e,
-                                    evict_first);
+              for (int r = 0; r < 128; r += kFusedBoxRowsW2)
+                ptx::tma_load_3d_hint(sW + r * 128, tm, &full[stage], t.wt * C::kH + kk * 64, di * 128 + r, e,
+                                      evict_first);
+            }
             advance();
           }
         }
@@ -454,25 +510,30 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
       *prod_issued = issued;
     }
     // The last load into every stage lands before the CTA's shared memory is
-    // released.  After an abort some were never consumed, and a stage's
-    // phase completes only with the gather warps' arrivals too: they add the
-    // ones they did not make (exit_handshake), then the producer waits for
-    // the last phase of every stage it filled (at once after a normal run,
-    // where the MMA has waited for all of them).
-    exit_handshake();
-    exit_handshake();
+    // released.  After an abort some were never consumed.  bf16 weights: a
+    // stage's phase completes only with the gather warps' arrivals too, so
+    // they add the ones they did not make (exit_handshake); fp8 weights: the
+    // raw stages complete on the loaded bytes alone.  Then the producer
+    // waits for the last phase of every stage it filled (at once after a
+    // normal run, where they have all been consumed).
+    if constexpr (!FP8) {
+      exit_handshake();
+      exit_handshake();
+    }
     if (lane == 0) {
+      constexpr int kRing = FP8 ? C::kRawStages : C::kStages;
+      uint64_t* ring_full = FP8 ? raw_full : full;
       const int issued = *prod_issued;
-      int stage = issued % C::kStages;
-      uint32_t phase = static_cast<uint32_t>((issued / C::kStages) & 1);
-      for (int j = 1; j <= C::kStages && j <= issued; ++j) {
+      int stage = issued % kRing;
+      uint32_t phase = static_cast<uint32_t>((issued / kRing) & 1);
+      for (int j = 1; j <= kRing && j <= issued; ++j) {
         int st = stage - j;
         uint32_t ph = phase;
         if (st < 0) {
-          st += C::kStages;
+          st += kRing;
           ph ^= 1u;
         }
-        ptx::mbar_wait_bounded(&full[st], ph, flag, kDrainLimitNs);
+        ptx::mbar_wait_bounded(&ring_full[st], ph, flag, kDrainLimitNs);
       }
     }
   } else if (warp == 1) {
@@ -745,7 +806,7 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
         epilogue_sync();  // all reads of this tok_s / w_s buffer are done before it is rewritten
       }
     }
-  } else {
+  } else if (warp < 10) {
     // ------------------------------------------------ token-row gather
     const int gtid = threadIdx.x - 192;
     {  // zero this CTA's slice of the accumulator, then count the CTA on sync[0]
@@ -821,14 +882,70 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
       }
     }
     cp_async_wait_all();
-    // after an abort: arrive on every stage the producer filled and this
-    // thread did not, so that the producer can wait for its own loads
-    exit_handshake();
-    for (const int target = *prod_issued; arrived < target;) {
-      ptx::mbar_arrive(&full[stage]);
-      advance();
+    if constexpr (!FP8) {
+      // after an abort: arrive on every stage the producer filled and this
+      // thread did not, so that the producer can wait for its own loads
+      exit_handshake();
+      for (const int target = *prod_issued; arrived < target;) {
+        ptx::mbar_arrive(&full[stage]);
+        advance();
+      }
+      exit_handshake();
     }
-    exit_handshake();
+  } else if constexpr (FP8) {
+    // ------------------------------------------------ fp8 weights -> bf16 operand stages
+    // Every stage of this CTA (the producer's order): wait for the raw
+    // stage's bytes and for the operand stage to be free, expand the 128 x 64
+    // e4m3 values times their power-of-two scales into bf16 (exact: an e4m3
+    // value has 4 significant bits) in the 128-byte-swizzled K-major layout
+    // the tensor core reads, and hand both stages on.  Thread: rows
+    // r0 + 32 j (j < 4) of the stage, 16 K values each (q-th quarter).
+    const int ctid = static_cast<int>(threadIdx.x) - 320;
+    const int q = ctid & 3;
+    const int r0 = ctid >> 2;
+    int stage = 0, rstage = 0;
+    uint32_t phase = 0, rphase = 0;
+    const int total = n_my * (ng + nk2);
+    for (int st = 0; st < total; ++st) {
+      if (!ptx::mbar_wait_bounded(&raw_full[rstage], rphase, abort_flag, args.wait_ns) ||
+          !ptx::mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.wait_ns)) {
+        fail();
+        break;
+      }
+      const uint8_t* rb = raw + rstage * C::kRawStageBytes;
+      uint8_t* sW = smem + stage * C::kStageBytes;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = r0 + 32 * j;
+        const uint4 v = *reinterpret_cast<const uint4*>(rb + r * 64 + q * 16);
+        // scale byte b (1..254): 2^(b - 127), an fp32 with that exponent field
+        const float scale = __uint_as_float(static_cast<uint32_t>(rb[C::kRawWBytes + (q >> 1) * 128 + r]) << 23);
+        uint4 lo, hi;
+        lo.x = e4m3x2_to_bf16x2(v.x & 0xFFFFu, scale);
+        lo.y = e4m3x2_to_bf16x2(v.x >> 16, scale);
+        lo.z = e4m3x2_to_bf16x2(v.y & 0xFFFFu, scale);
+        lo.w = e4m3x2_to_bf16x2(v.y >> 16, scale);
+        hi.x = e4m3x2_to_bf16x2(v.z & 0xFFFFu, scale);
+        hi.y = e4m3x2_to_bf16x2(v.z >> 16, scale);
+        hi.z = e4m3x2_to_bf16x2(v.w & 0xFFFFu, scale);
+        hi.w = e4m3x2_to_bf16x2(v.w >> 16, scale);
+        uint8_t* row = sW + (r >> 3) * 1024 + (r & 7) * 128;
+        *reinterpret_cast<uint4*>(row + (((2 * q) ^ (r & 7)) << 4)) = lo;
+        *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ (r & 7)) << 4)) = hi;
+      }
+      ptx::fence_proxy_async_smem();  // the tensor core reads these rows next
+      ptx::mbar_arrive(&full[stage]);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&raw_empty[rstage]);
+      if (++stage == C::kStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+      if (++rstage == C::kRawStages) {
+        rstage = 0;
+        rphase ^= 1u;
+      }
+    }
   }
 
   // every warp reconverges (the idle lanes of the producer and MMA warps
@@ -894,10 +1011,10 @@ __global__ void __launch_bounds__(FusedCfg<EPI1, TOK, ROUTE>::kNumThreads, 1)
   }
 }
 
-template <int EPI1, int TOK, bool ROUTE>
+template <int EPI1, int TOK, bool ROUTE, bool FP8 = false>
 cudaError_t launch_fused_variant(const FusedArgs& args, int grid, cudaStream_t stream) {
-  using C = FusedCfg<EPI1, TOK, ROUTE>;
-  auto kern = fused_expert_kernel<EPI1, TOK, ROUTE>;
+  using C = FusedCfg<EPI1, TOK, ROUTE, FP8>;
+  auto kern = fused_expert_kernel<EPI1, TOK, ROUTE, FP8>;
   // per device, set once; concurrent first calls may both set it (idempotent)
   static std::atomic<bool> attr_done[64];
   int dev = 0;
@@ -926,8 +1043,28 @@ bool fused_routing_supported(int T, int k, int E, int n_group, int block_m) {
 }
 
 cudaError_t launch_fused_expert(int act_epi, int block_m, bool route, const FusedArgs& args, int grid,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, bool fp8) {
   const bool gated = act_epi == kEpiSwiGLU;
+  if (fp8) {
+    if (route) {
+      if (block_m != 16) return cudaErrorInvalidValue;
+      return gated ? launch_fused_variant<kEpiSwiGLU, 16, true, true>(args, grid, stream)
+                   : launch_fused_variant<kEpiRelu2, 16, true, true>(args, grid, stream);
+    }
+    switch (block_m) {
+      case 16:
+        return gated ? launch_fused_variant<kEpiSwiGLU, 16, false, true>(args, grid, stream)
+                     : launch_fused_variant<kEpiRelu2, 16, false, true>(args, grid, stream);
+      case 32:
+        return gated ? launch_fused_variant<kEpiSwiGLU, 32, false, true>(args, grid, stream)
+                     : launch_fused_variant<kEpiRelu2, 32, false, true>(args, grid, stream);
+      case 64:
+        return gated ? launch_fused_variant<kEpiSwiGLU, 64, false, true>(args, grid, stream)
+                     : launch_fused_variant<kEpiRelu2, 64, false, true>(args, grid, stream);
+      default:
+        return cudaErrorInvalidValue;
+    }
+  }
   if (route) {
     if (block_m != 16) return cudaErrorInvalidValue;
     return gated ? launch_fused_variant<kEpiSwiGLU, 16, true>(args, grid, stream)

@@ -49,6 +49,10 @@ _SIG = {
     "moe_backward_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I]),
     "moe_backward": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _P, _I, _P, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P,
                           _P, _P, ctypes.c_size_t, _P, _P]),
+    "moe_forward_fp8": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _I, _P, _I, _P, _P, _P, _P, _I,
+                             _I, _P, _P, ctypes.c_size_t, _P, _P]),
+    "moe_layer_fp8": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _I, _P, _P, _P, _P, _I, _P, _P, _P,
+                           _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
     "moe_read_status": (_I, [_P, _P]),
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_last_launch_count": (_I, []),
@@ -333,6 +337,49 @@ class MoEGradBuffers:
                      self.dw2_shared, self.dtopk, fwd.status)
 
 
+class Fp8Experts:
+    """fp8 expert weights on the device (plumbing): e4m3 bytes and the
+    K-block-major power-of-two scale bytes of w13 and w2 (and of the shared
+    expert), as uint8 tensors in the layouts include/moe.h gives."""
+
+    def __init__(self, w13_q, w13_s, w2_q, w2_s, w13s_q=None, w13s_s=None, w2s_q=None, w2s_s=None):
+        for t in (w13_q, w13_s, w2_q, w2_s):
+            if t.dtype != torch.uint8:
+                raise ValueError("fp8 weights and scales are uint8 tensors")
+        self.w13_q, self.w13_s, self.w2_q, self.w2_s = w13_q, w13_s, w2_q, w2_s
+        self.w13s_q, self.w13s_s, self.w2s_q, self.w2s_s = w13s_q, w13s_s, w2s_q, w2s_s
+        self.E, self.n1, self.d = w13_q.shape
+        self.F = w2_q.shape[2]
+        self.n_shared = 0 if w13s_q is None else 1
+
+
+def moe_forward_fp8(x, wq: Fp8Experts, topk_weights, sorted_token_ids, expert_ids, num_tokens_post_padded,
+                    inv_pos, block_m, act, out, ws, dev_status=None):
+    """moe_forward with fp8 expert weights (block_m 16, 32 or 64)."""
+    T, d = x.shape
+    k = topk_weights.shape[1] if topk_weights.dim() == 2 else 1
+    code = load_library().moe_forward_fp8(
+        _ptr(_bits(x)), T, d, _ptr(wq.w13_q), _ptr(wq.w13_s), _ptr(wq.w2_q), _ptr(wq.w2_s), wq.E, wq.F,
+        _ptr(wq.w13s_q), _ptr(wq.w13s_s), _ptr(wq.w2s_q), _ptr(wq.w2s_s), wq.n_shared, _ptr(topk_weights), k,
+        _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded), _ptr(inv_pos), block_m, act,
+        _ptr(_bits(out)), _ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_status), _stream(x.device))
+    _check("moe_forward_fp8", code)
+
+
+def moe_layer_fp8(logits, x, wq: Fp8Experts, k, block_m, act, topk_ids, topk_weights, sorted_token_ids, expert_ids,
+                  num_tokens_post_padded, inv_pos, out, ws, n_group=1, topk_group=1, group_score=GROUP_MAX,
+                  renormalize=True, routed_scaling=1.0, dev_status=None):
+    """moe_layer with fp8 expert weights (one launch for decode batches)."""
+    T, E = logits.shape
+    code = load_library().moe_layer_fp8(
+        _ptr(logits), T, E, k, n_group, topk_group, group_score, 1 if renormalize else 0, float(routed_scaling),
+        _ptr(_bits(x)), wq.d, _ptr(wq.w13_q), _ptr(wq.w13_s), _ptr(wq.w2_q), _ptr(wq.w2_s), wq.F, _ptr(wq.w13s_q),
+        _ptr(wq.w13s_s), _ptr(wq.w2s_q), _ptr(wq.w2s_s), wq.n_shared, block_m, act, _ptr(topk_ids),
+        _ptr(topk_weights), _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded), _ptr(inv_pos),
+        _ptr(_bits(out)), _ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_status), _stream(x.device))
+    _check("moe_layer_fp8", code)
+
+
 def moe_read_status(dev_status) -> int:
     """Synchronise the current stream and return the device status code."""
     return int(load_library().moe_read_status(_ptr(dev_status), _stream(dev_status.device)))
@@ -397,6 +444,18 @@ class MoEBuffers:
         moe_layer(logits, x, w13, w2, self.k, self.block_m, self.act, self.topk_ids, self.topk_weights,
                   self.sorted_token_ids, self.expert_ids, self.ntpp, self.inv_pos, self.out, self.ws, w13_shared,
                   w2_shared, n_group, topk_group, group_score, renormalize, routed_scaling, self.status)
+        return self.out
+
+    def layer_fp8(self, logits, x, wq: "Fp8Experts", n_group=1, topk_group=1, group_score=GROUP_MAX,
+                  renormalize=True, routed_scaling=1.0):
+        moe_layer_fp8(logits, x, wq, self.k, self.block_m, self.act, self.topk_ids, self.topk_weights,
+                      self.sorted_token_ids, self.expert_ids, self.ntpp, self.inv_pos, self.out, self.ws, n_group,
+                      topk_group, group_score, renormalize, routed_scaling, self.status)
+        return self.out
+
+    def forward_fp8(self, x, wq: "Fp8Experts"):
+        moe_forward_fp8(x, wq, self.topk_weights, self.sorted_token_ids, self.expert_ids, self.ntpp, self.inv_pos,
+                        self.block_m, self.act, self.out, self.ws, self.status)
         return self.out
 
     def forward(self, x, w13, w2, w13_shared=None, w2_shared=None):

@@ -236,6 +236,55 @@ MOE_API moe_status moe_forward(const uint16_t* x, int T, int d,
                        int32_t* dev_status, moe_stream_t stream);
 
 /*
+ * moe_forward_fp8 / moe_layer_fp8 -- moe_forward / moe_layer with the
+ * expert weights quantised to fp8, for the bandwidth-bound small-batch
+ * shapes.  The decode stacks on the pages run MoE experts from quantised
+ * weights (the B70 lab page's Q8_0 "Grouped Reordered-Q8" expert path,
+ * Intent; the mlxcel PR's quantised `gather_qmm` experts, Summary); here
+ * the format is weight-only MXFP8: e4m3 values, and for every run of 32
+ * consecutive K values of a weight row one power-of-two scale 2^(b - 127)
+ * stored as the byte b (1 <= b <= 254).  The kernel streams the fp8 bytes
+ * (halving the weight bytes of the bf16 layer) and expands them in shared
+ * memory to bf16 -- exactly: an e4m3 value times a power of two has at most
+ * 4 significant bits -- before the same bf16 tensor-core MMAs, so the result
+ * is the bf16 layer's on the dequantised weights.
+ *   w13_q       [E, N1, d] uint8 e4m3 (layout of moe_forward's w13).
+ *   w13_scales  [E, d / 32, N1] uint8 (K-block-major: the scales of one
+ *               32-wide block of K for all N1 rows are contiguous).
+ *   w2_q        [E, d, F] uint8 e4m3; w2_scales [E, F / 32, d] uint8.
+ *   w13s_* / w2s_*  the shared expert, same layouts with E = 1 (n_shared == 1).
+ * Everything else as for moe_forward / moe_layer.  block_m must be 16, 32 or
+ * 64 (the fused expert kernel; MOE_ERR_UNSUPPORTED otherwise).  All weight
+ * and scale pointers 16-byte aligned.
+ */
+MOE_API moe_status moe_forward_fp8(const uint16_t* x, int T, int d,
+                           const uint8_t* w13_q, const uint8_t* w13_scales,
+                           const uint8_t* w2_q, const uint8_t* w2_scales, int E, int F,
+                           const uint8_t* w13s_q, const uint8_t* w13s_scales,
+                           const uint8_t* w2s_q, const uint8_t* w2s_scales, int n_shared,
+                           const float* topk_weights, int k,
+                           const int32_t* sorted_token_ids, const int32_t* expert_ids,
+                           const int32_t* num_tokens_post_padded, const int32_t* inv_pos,
+                           int block_m, moe_act act,
+                           uint16_t* out, void* ws, size_t ws_bytes,
+                           int32_t* dev_status, moe_stream_t stream);
+
+MOE_API moe_status moe_layer_fp8(const float* logits, int T, int E, int k,
+                         int n_group, int topk_group, moe_group_score group_score,
+                         int renormalize, float routed_scaling,
+                         const uint16_t* x, int d,
+                         const uint8_t* w13_q, const uint8_t* w13_scales,
+                         const uint8_t* w2_q, const uint8_t* w2_scales, int F,
+                         const uint8_t* w13s_q, const uint8_t* w13s_scales,
+                         const uint8_t* w2s_q, const uint8_t* w2s_scales, int n_shared,
+                         int block_m, moe_act act,
+                         int32_t* topk_ids, float* topk_weights,
+                         int32_t* sorted_token_ids, int32_t* expert_ids,
+                         int32_t* num_tokens_post_padded, int32_t* inv_pos,
+                         uint16_t* out, void* ws, size_t ws_bytes,
+                         int32_t* dev_status, moe_stream_t stream);
+
+/*
  * moe_align_noalloc — moe_align for callers that cannot allocate device
  * memory.  No passage of the source pages has a counterpart: it is the same
  * sort and pad as moe_align, with the same arguments minus the workspace.
