@@ -2,6 +2,8 @@
 run the layer through the C ABI, run the oracle, and compare."""
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -101,7 +103,36 @@ def compare_out(gpu_bits: np.ndarray, ref: np.ndarray, label: str = ""):
     assert excess <= OUT_MAX_ABS_REL_RMS * rms, \
         f"{label}: max(|diff| - half_ulp) = {excess / rms:.3e} * rms > 2e-2 * rms (literal {max_abs / rms:.3e})"
     assert rel_l2 <= OUT_REL_L2, f"{label}: rel L2={rel_l2:.3e}"
+    # where the correctly rounded oracle itself meets the literal bound, the
+    # GPU output is held to the literal bound too (no half-ulp allowance)
+    rounded = W.bf16_bits_to_f32(W.f32_to_bf16_bits(ref.astype(np.float32))).astype(np.float64)
+    rounded_max = float(np.abs(rounded - ref).max()) if diff.size else 0.0
+    literal_attainable = rounded_max <= OUT_MAX_ABS_REL_RMS * rms
+    _record(label, max_abs / rms, excess / rms, rel_l2, rounded_max / rms)
+    if literal_attainable and STRICT_LITERAL and label not in LITERAL_EXEMPT:
+        assert max_abs <= OUT_MAX_ABS_REL_RMS * rms, \
+            f"{label}: max|diff| = {max_abs / rms:.3e} * rms > 2e-2 * rms (the rounded oracle: {rounded_max / rms:.3e})"
     return max_abs / rms, excess / rms, rel_l2
+
+
+# MOE_TOL_REPORT=<file>: append one JSON line per comparison (label,
+# literal max|diff|/rms, beyond half-ulp, relative L2, the rounded oracle's
+# own max deviation / rms)
+STRICT_LITERAL = os.environ.get("MOE_STRICT_LITERAL", "1") == "1"
+# Measured to miss the literal bound although the rounded oracle meets it:
+# the 128-row relu^2 layer (2.31e-2 rms literal, 0.84e-2 beyond the half
+# ulp): relu^2 makes h heavy-tailed, so rounding the bf16 operand h moves
+# the largest outputs by up to 2^-9 of a few dominant terms.
+LITERAL_EXEMPT = {"tokm_relu2"}
+
+
+def _record(label, lit, excess, rel_l2, rounded):
+    path = os.environ.get("MOE_TOL_REPORT")
+    if path:
+        import json
+        with open(path, "a") as f:
+            f.write(json.dumps({"label": label, "literal": lit, "beyond_half_ulp": excess, "rel_l2": rel_l2,
+                                "rounded_oracle": rounded}) + "\n")
 
 
 # Gradients (the backward): the same bounds, plus the effect of the bf16
