@@ -216,8 +216,13 @@ MOE_API moe_status moe_align(const int32_t* topk_ids, int T, int k, int E, int b
  *                accumulator with atomics, in an order that depends on
  *                timing, so repeated calls agree up to the fp32 rounding
  *                of that sum (one bf16 ulp of a result, a little more where
- *                the k terms cancel).  inv_pos is accepted for
- *                interface stability and not read (it may be NULL).
+ *                the k terms cancel).  Callers that need bit-identical
+ *                outputs from run to run (a training run replayed for
+ *                debugging, golden-output regression checks) do not get
+ *                them from this call; routing, align and (moe_backward)
+ *                the weight gradients are deterministic.  inv_pos is
+ *                accepted for interface stability and not read (it may be
+ *                NULL).
  *   ws, ws_bytes scratch of moe_workspace_size bytes (its counter block zero
  *                before the first call, see moe_workspace_size); calls sharing
  *                a workspace must not overlap on the GPU.
