@@ -76,10 +76,10 @@ struct GemmCfg {
   static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
   static constexpr int kAccCols = 256;
   static constexpr int kTmemCols = 512;
-  // epilogue warps: the reductions into the fp32 accumulator bound those
-  // kernels, so they run two warps per TMEM lane quadrant, each on half of
-  // the tile's columns
-  static constexpr int kEpiWarps = kReduce ? 8 : 4;
+  // epilogue warps: the reductions into the fp32 accumulator, and the
+  // backward's per-row fp32 reads and writes, bound those kernels, so they
+  // run two warps per TMEM lane quadrant, each on half of the tile's columns
+  static constexpr int kEpiWarps = (kReduce || kGrad || kPre) ? 8 : 4;
   // gate/up: warps 6-9 gather token rows, warp 10 zeroes the accumulator;
   // pre-activations: warp 6 zeroes
   static constexpr int kZeroWarp = kGather ? 10 : 2 + kEpiWarps;
@@ -329,6 +329,8 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
     // ------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int row = q * 32 + lane;
+    // with eight epilogue warps, the half of the tile's columns this warp takes
+    const int ehalf = C::kEpiWarps == 8 ? (warp - 2) >> 2 : 0;
     int abuf = 0;
     uint32_t aphase = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
@@ -396,7 +398,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
         // derivative is taken from them): g at column c, u at F + c
         float* orow = static_cast<float*>(args.out) + static_cast<size_t>(p) * args.out_ld;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32) {
+        for (int c0 = ehalf * 64; c0 < ehalf * 64 + 64; c0 += 32) {
           uint32_t g[32], u[32];
           ptx::tmem_ld16(t_acc + c0, *reinterpret_cast<uint32_t(*)[16]>(&g[0]));
           ptx::tmem_ld16(t_acc + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&g[16]));
@@ -419,7 +421,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
       } else if (EPI == kEpiPreRelu2) {
         float* orow = static_cast<float*>(args.out) + static_cast<size_t>(p) * args.out_ld;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 256; c0 += 16) {
+        for (int c0 = ehalf * 128; c0 < ehalf * 128 + 128; c0 += 16) {
           uint32_t a[16];
           ptx::tmem_ld16(t_acc + c0, a);
           ptx::tmem_wait_ld();
@@ -455,7 +457,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
         uint16_t* hrow = args.hw + static_cast<size_t>(p) * args.n_out;
         float part = 0.0f;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 256; c0 += 32) {
+        for (int c0 = ehalf * 128; c0 < ehalf * 128 + 128; c0 += 32) {
           uint32_t a[32];
           ptx::tmem_ld16(t_acc + c0, *reinterpret_cast<uint32_t(*)[16]>(&a[0]));
           ptx::tmem_ld16(t_acc + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&a[16]));
