@@ -10,7 +10,7 @@ enum EpiKind : int {
   kEpiSwiGLU = 0,      // gate/up GEMM, h = silu(gate) * up
   kEpiRelu2 = 1,       // fc1 GEMM, h = max(a, 0)^2
   kEpiScale = 2,       // down GEMM, acc[token] += topk_weight(row) * row result (fp32)
-  kEpiRouter = 3,      // router GEMM, logits = x . W_g^T (fp32), top-k gating of each row
+  kEpiRouter = 3,      // router GEMM, logits = x . W_g^T (fp32)
   // backward (token rows by TMA from the expert-sorted copies)
   kEpiPreSwiGLU = 4,   // gate/up pre-activations [g | u] of every row, fp32
   kEpiPreRelu2 = 5,    // fc1 pre-activations, fp32
@@ -56,15 +56,8 @@ struct GemmArgs {
   float* dtopk;         // grad kinds: dL/d topk_weights [T * k] (fp32 adds; zeroed by the pre kinds)
   float* zero2;         // pre kinds: a second buffer their spare warp zeroes (dtopk), zero2_elems floats
   int64_t zero2_elems;
-  // router GEMM only: fp32 logits [T, E]; when r_ids is set, the top-k of
-  // every row (ids [T, k], weights [T, k]) with the routing kernel's order
-  // (logit desc, id asc) and weights (softmax over the chosen k when
-  // r_renorm, else the full softmax at the chosen ids) x r_scaling
+  // router GEMM only: fp32 logits [T, E]
   float* logits;
-  int32_t* r_ids;
-  float* r_w;
-  int r_renorm;
-  float r_scaling;
 };
 
 // Rows of one weight TMA box (= output columns of one tile) for an epilogue.
@@ -73,7 +66,8 @@ int gemm_box_rows(int epi);
 int64_t gemm_max_tiles(int epi, int max_routed_blocks, int n_shared_blocks, int n_out);
 cudaError_t launch_grouped_gemm(int epi, const GemmArgs& args, int grid, cudaStream_t stream);
 // Router GEMM: x [T, K] (tm_x, 2-D {K, T}, 64 x 128 boxes) times W_g [E, K]
-// (tm_ws, 3-D {K, E, 1}, 256-row boxes), E <= 256, top-k k <= 16.
+// (tm_ws, 3-D {K, E, 1}, 256-row boxes), E <= 256; the routing kernel gates
+// the logits it writes (top-k k <= 16).
 constexpr int kRouterMaxE = 256;
 constexpr int kRouterMaxK = 16;
 

@@ -518,26 +518,13 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
         }
         if (slot >= 0 && args.dtopk != nullptr) atomicAdd(args.dtopk + slot, part);
       } else if (EPI == kEpiRouter) {
-        // thread = token row of the tile, TMEM columns 0..E-1 = its logits.
-        // Top-k over columns in increasing id order into a list sorted by
-        // logit (desc): a value enters only if it beats the current k-th,
-        // walks down the list past every entry it does not beat (so equal
-        // logits keep the lower id first, as the routing kernel), and every
-        // entry after it shifts down by one; one unrolled pass of selects
-        // keeps the list in registers.
+        // thread = token row of the tile, TMEM columns 0..E-1 = its logits,
+        // written out in 16-column chunks (the routing kernel gates them:
+        // a warp per token beats one thread per token working through E
+        // columns in this epilogue)
         const int t = (tc.blk - routed_blocks) * args.block_m + row;
         const bool valid = t < args.T;
-        const int E = args.E, kk = args.k;
-        float kv[kRouterMaxK];
-        int ki[kRouterMaxK];
-#pragma unroll
-        for (int j = 0; j < kRouterMaxK; ++j) {
-          kv[j] = -INFINITY;
-          ki[j] = 0;
-        }
-        float kth = -INFINITY;  // current k-th largest (-inf until k values are in)
-        float run_max = -INFINITY, run_sum = 0.0f;  // full softmax, online (no renormalisation)
-        bool finite = true;
+        const int E = args.E;
         float* lrow = args.logits + static_cast<size_t>(valid ? t : 0) * E;
 #pragma unroll 1
         for (int c0 = 0; c0 < E; c0 += 16) {
@@ -547,74 +534,16 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::kNumThreads, 1)
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) asm volatile("" : "+r"(a[jj]));  // uses stay after the wait
           if (!valid) continue;
-          // one cheap unrolled pass stores the logits and marks the columns
-          // that beat the k-th at the chunk's start; the insertion (one
-          // copy of its code) then runs over the marked columns only
-          uint32_t cand = 0;
+          if (c0 + 16 <= E && (E & 3) == 0) {
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int e = c0 + jj;
-            const float v = __uint_as_float(a[jj]);
-            if (e < E) {
-              lrow[e] = v;
-              if (!isfinite(v)) finite = false;
-              if (!args.r_renorm) {
-                if (v > run_max) {
-                  run_sum = run_sum * expf(run_max - v) + 1.0f;
-                  run_max = v;
-                } else {
-                  run_sum += expf(v - run_max);
-                }
-              }
-              if (v > kth) cand |= 1u << jj;
-            }
-          }
-          while (cand != 0) {
-            const int jj = __ffs(cand) - 1;
-            cand &= cand - 1;
-            float v = 0.0f;
+            for (int i = 0; i < 4; ++i)
+              *reinterpret_cast<float4*>(lrow + c0 + 4 * i) =
+                  make_float4(__uint_as_float(a[4 * i]), __uint_as_float(a[4 * i + 1]), __uint_as_float(a[4 * i + 2]),
+                              __uint_as_float(a[4 * i + 3]));
+          } else {
 #pragma unroll
-            for (int q = 0; q < 16; ++q)
-              if (q == jj) v = __uint_as_float(a[q]);
-            if (v > kth) {  // the k-th may have risen since the chunk started
-              float cv = v;
-              int ci = c0 + jj;
-              bool placed = false;
-#pragma unroll
-              for (int j = 0; j < kRouterMaxK; ++j) {
-                const bool take = j < kk && (placed || cv > kv[j]);
-                const float tv = kv[j];
-                const int ti = ki[j];
-                kv[j] = take ? cv : tv;
-                ki[j] = take ? ci : ti;
-                cv = take ? tv : cv;
-                ci = take ? ti : ci;
-                placed = placed || take;
-              }
-              // the list is sorted, so its k-th entry is its minimum (written as a
-              // min: a select on j == kk - 1 becomes a runtime-indexed load)
-              kth = kv[0];
-#pragma unroll
-              for (int j = 1; j < kRouterMaxK; ++j)
-                if (j < kk) kth = fminf(kth, kv[j]);
-            }
-          }
-        }
-        if (valid && !finite) set_status(args.status, MOE_ERR_NONFINITE);
-        if (valid && args.r_ids != nullptr) {
-          // weights: softmax over the chosen k (the first is the largest), or
-          // the full softmax taken at the chosen ids; then x routed_scaling
-          float z = 0.0f;
-#pragma unroll
-          for (int j = 0; j < kRouterMaxK; ++j)
-            if (j < kk) z += expf(kv[j] - kv[0]);
-#pragma unroll
-          for (int j = 0; j < kRouterMaxK; ++j) {
-            if (j < kk) {
-              const float w = args.r_renorm ? expf(kv[j] - kv[0]) / z : expf(kv[j] - run_max) / run_sum;
-              args.r_ids[static_cast<size_t>(t) * kk + j] = ki[j];
-              args.r_w[static_cast<size_t>(t) * kk + j] = w * args.r_scaling;
-            }
+            for (int jj = 0; jj < 16; ++jj)
+              if (c0 + jj < E) lrow[c0 + jj] = __uint_as_float(a[jj]);
           }
         }
       } else {

@@ -149,8 +149,8 @@ MOE_API moe_status moe_route(const float* logits, int T, int E, int k,
  * timed_forward) the block's gate maps the flattened hidden states to their
  * top-k expert ids and weights; "Fused MoE Kernel Optimization" (overview:
  * top-k gating fusion; "Token-Expert Routing" step 1) gates on those
- * logits.  Here the product runs on the tensor cores and each token's gating
- * runs in the GEMM's epilogue.
+ * logits.  Here the product runs on the tensor cores (or, for small
+ * batches, the CUDA cores) and a warp per token gates the logits.
  *   x             [T, d] bf16, device, row-major; d a multiple of 64.
  *   w_gate        [E, d] bf16, device, row-major (K = d contiguous); E <= 256.
  *   k, n_group, topk_group, group_score, renormalize, routed_scaling:
@@ -161,10 +161,10 @@ MOE_API moe_status moe_route(const float* logits, int T, int E, int k,
  *                 writes for these logits (ids bit for bit, weights up to
  *                 the rounding of the softmax sum).
  * Up to 1024 tokens (and d <= 5120) the product runs on the CUDA cores, in
- * CTAs of 8 expert rows x 16 tokens, and the routing kernel gates (two
- * launches).  Larger batches run on the tensor cores: with n_group == 1 in
- * one launch (the gating runs in the GEMM epilogue), otherwise the routing
- * kernel runs on the written logits (two launches).  T == 0 is a no-op.
+ * CTAs of 8 expert rows x 16 tokens; larger batches run on the tensor cores
+ * (128-token tiles, W_g's rows as the N = 256 operand).  Either way the
+ * routing kernel then gates the written logits (two launches).  T == 0 is a
+ * no-op.
  * Errors as for moe_route; x and w_gate must be 16-byte aligned.
  */
 MOE_API moe_status moe_router(const uint16_t* x, int T, int d, const uint16_t* w_gate, int E, int k,
