@@ -532,6 +532,8 @@ moe_status forward_impl(const uint16_t* x, int T, int d, const uint16_t* w13, co
                                        n_shared_blocks * bm, x_sorted, num_sms, s, &launches);
       }
       if (err == cudaSuccess) err = moe::launch_grouped_gemm_pair(epi1, a1, num_sms & ~1, s);
+    } else if (moe::gemm_wide_supported(epi1, bm, total_blocks_max)) {
+      err = moe::launch_grouped_gemm_wide(epi1, a1, grid, s);
     } else {
       err = moe::launch_grouped_gemm(epi1, a1, grid, s);
     }

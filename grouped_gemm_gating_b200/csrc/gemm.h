@@ -78,6 +78,13 @@ constexpr int kRouterMaxK = 16;
 bool gemm_pair_supported(int block_m, int total_blocks_max);
 cudaError_t launch_grouped_gemm_pair(int epi, const GemmArgs& args, int grid, cudaStream_t stream);
 
+// The gate/up (fc1) GEMM with gathered token rows on units of two 128-row
+// blocks of one expert (256-token tiles sharing each weight stage): args as
+// for launch_grouped_gemm; at most kWideMaxBlocks blocks per launch.
+constexpr int kWideMaxBlocks = 8192;
+bool gemm_wide_supported(int epi, int block_m, int total_blocks_max);
+cudaError_t launch_grouped_gemm_wide(int epi, const GemmArgs& args, int grid, cudaStream_t stream);
+
 // Per-expert weight gradient (backward): for every expert e (and the shared
 // expert, when present), dW_e [M, N] = sum over the rows p of e's blocks of
 // A[p, :]^T B[p, :], with A [P_total, M] and B [P_total, N] in the

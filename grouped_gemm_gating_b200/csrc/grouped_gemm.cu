@@ -13,6 +13,9 @@
 // epilogue; the down projection applies the top-k weight of each row in its
 // epilogue ("Common Pitfalls" 4: routed weights on the right rows).
 //
+// The gate/up GEMM normally runs on two-block units (grouped_gemm_wide.cu);
+// the one-block form here serves launches beyond that kernel's block limit.
+//
 // Tiles are token-major (block_m = 128): MMA M = 128 token rows, N = 256
 // weight rows (SwiGLU: 128 gate rows followed by the matching 128 up rows, so
 // one thread holds both halves of its h columns).  The down GEMM's epilogue

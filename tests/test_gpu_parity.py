@@ -236,6 +236,25 @@ def test_layer_full_size_sampled(name):
         assert (counts == 0).sum() == 8
 
 
+@pytest.mark.slow
+def test_layer_beyond_wide_gemm_block_limit_sampled():
+    """More than 8192 blocks of 128 rows (T * k over a million slots): the
+    gate/up GEMM runs on one-block tiles instead of two-block units."""
+    cfg = CFG["tiny"].with_(name="many_blocks", T=131072, d=128, F=128, E=8, k=8, block_m=128, seed=2016,
+                            logits_kind="normal")
+    inp = W.make_inputs(cfg)
+    lay = DeviceLayer(inp)
+    out = lay.run()
+    torch.cuda.synchronize()
+    assert lay.status() == 0, M.status_name(lay.status())
+    ids, w = oracle_route(inp)
+    assert M.moe_max_padded(cfg.T, cfg.k, cfg.E, cfg.block_m) // cfg.block_m > 8192
+    compare_align(lay.buf, oracle.align(ids, cfg.E, cfg.block_m), cfg.name)
+    sample = np.sort(np.random.default_rng(cfg.seed).choice(cfg.T, size=64, replace=False))
+    ref = oracle.forward(inp.x[sample], inp.w13, inp.w2, ids[sample], w[sample], cfg.act)
+    compare_out(M_bits(out)[sample], ref, cfg.name)
+
+
 def test_repeated_calls_agree_up_to_sum_order():
     """Both paths add partial sums with fp32 atomics in a timing-dependent
     order: repeated calls agree up to that reordering (a bf16 ulp of the
