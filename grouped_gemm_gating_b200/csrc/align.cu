@@ -16,8 +16,9 @@
 // the same bits.
 //   * S <= kSingleBlockMax: one 1024-thread block does histogram, scan,
 //     padding fill and the stable scatter in one launch (decode latency).
-//   * larger S: per-chunk histograms (one block per chunk), one block for
-//     the scan over (expert, chunk), and a per-chunk stable scatter.
+//   * larger S: per-chunk histograms (one block per chunk), then per chunk
+//     one block that scans all chunks' counts itself and places its slots
+//     (stable scatter).
 // Within a round of slots, the rank of a slot among equal experts comes from
 // __match_any_sync inside the warp plus an exclusive prefix over the warps.
 #include "align_impl.cuh"
@@ -72,72 +73,72 @@ __global__ void __launch_bounds__(kChunkThreads)
   for (int i = threadIdx.x; i < E; i += kChunkThreads) counts[static_cast<size_t>(c) * E + i] = cnt[i];
 }
 
-__global__ void __launch_bounds__(1024)
-    align_scan_kernel(const int32_t* __restrict__ counts, int nchunks, int S, int E, int bm, int P_max,
-                      int32_t* __restrict__ bases, int32_t* __restrict__ sorted_ids,
-                      int32_t* __restrict__ expert_ids, int32_t* ntpp) {
-  constexpr int kSlices = 1024 / MOE_MAX_EXPERTS;  // contiguous chunk ranges per expert
+// Every chunk block sums the counts of all chunks itself (per expert: the
+// total, and the part in chunks before its own), scans the padded totals
+// and so knows where its slots go; it also writes its share of the layout
+// (padding ids, block experts) and then places its slots.
+__global__ void __launch_bounds__(kScatterThreads)
+    align_place_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ counts, int nchunks, int S,
+                       int E, int bm, int P_max, int32_t* __restrict__ sorted_ids, int32_t* __restrict__ expert_ids,
+                       int32_t* ntpp, int32_t* __restrict__ inv_pos) {
+  constexpr int kWarps = kScatterThreads / 32;
+  constexpr int kSlices = kScatterThreads / MOE_MAX_EXPERTS;  // contiguous chunk ranges per expert
   __shared__ int part[kSlices][MOE_MAX_EXPERTS];
+  __shared__ int before[kSlices][MOE_MAX_EXPERTS];
   __shared__ int cnt[MOE_MAX_EXPERTS];
   __shared__ int off[MOE_MAX_EXPERTS + 1];
-  const int tid = threadIdx.x;
-  const int e = tid % MOE_MAX_EXPERTS, slice = tid / MOE_MAX_EXPERTS;
-  const int per = (nchunks + kSlices - 1) / kSlices;
-  const int c_lo = slice * per, c_hi = min(nchunks, c_lo + per);
-  pdl_wait();
-  pdl_launch_dependents();
-  // threads over experts (coalesced loads), each summing one chunk range
-  int sum = 0;
-  if (e < E) {
-#pragma unroll 8
-    for (int c = c_lo; c < c_hi; ++c) sum += counts[static_cast<size_t>(c) * E + e];
-  }
-  part[slice][e] = sum;
-  __syncthreads();
-  if (tid < E) {
-    int total = 0;
-#pragma unroll
-    for (int s2 = 0; s2 < kSlices; ++s2) total += part[s2][tid];
-    cnt[tid] = total;
-  }
-  __syncthreads();
-  if (tid < 32) warp_padded_scan(cnt, off, E, bm, tid);
-  __syncthreads();
-  // chunk bases: the expert's offset, the earlier slices, then this range
-  if (e < E) {
-    int run = off[e];
-    for (int s2 = 0; s2 < slice; ++s2) run += part[s2][e];
-#pragma unroll 8
-    for (int c = c_lo; c < c_hi; ++c) {
-      bases[static_cast<size_t>(c) * E + e] = run;
-      run += counts[static_cast<size_t>(c) * E + e];
-    }
-    // padding inside this expert's last block, split over the slices
-    for (int p = off[e] + cnt[e] + slice; p < off[e + 1]; p += kSlices) sorted_ids[p] = S;
-  }
-  if (tid == 0) *ntpp = off[E];
-  for (int p = off[E] + tid; p < P_max; p += blockDim.x) sorted_ids[p] = S;
-  for (int b = tid; b < P_max / bm; b += blockDim.x) expert_ids[b] = block_expert(off, E, b * bm);
-}
-
-__global__ void __launch_bounds__(kScatterThreads)
-    align_scatter_kernel(const int32_t* __restrict__ ids, int S, int E, const int32_t* __restrict__ bases,
-                         int32_t* __restrict__ sorted_ids, int32_t* __restrict__ inv_pos) {
-  constexpr int kWarps = kScatterThreads / 32;
   __shared__ int run[MOE_MAX_EXPERTS];
   __shared__ int tot[MOE_MAX_EXPERTS];
   __shared__ int wcnt[kWarps][MOE_MAX_EXPERTS];
   const int c = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int e = tid % MOE_MAX_EXPERTS, slice = tid / MOE_MAX_EXPERTS;
+  const int per = (nchunks + kSlices - 1) / kSlices;
+  const int c_lo = slice * per, c_hi = min(nchunks, c_lo + per);
+  for (int i = tid; i < kWarps * MOE_MAX_EXPERTS; i += kScatterThreads) (&wcnt[0][0])[i] = 0;
   pdl_wait();
   pdl_launch_dependents();
-  for (int i = threadIdx.x; i < E; i += kScatterThreads) run[i] = bases[static_cast<size_t>(c) * E + i];
-  for (int i = threadIdx.x; i < kWarps * MOE_MAX_EXPERTS; i += kScatterThreads) (&wcnt[0][0])[i] = 0;
+  // threads over experts (coalesced loads), each summing one chunk range
+  int sum = 0, pre = 0;
+  if (e < E) {
+#pragma unroll 8
+    for (int cc = c_lo; cc < c_hi; ++cc) {
+      const int v = counts[static_cast<size_t>(cc) * E + e];
+      sum += v;
+      pre += cc < c ? v : 0;
+    }
+  }
+  part[slice][e] = sum;
+  before[slice][e] = pre;
+  __syncthreads();
+  if (tid < E) {
+    int total = 0, b = 0;
+#pragma unroll
+    for (int s2 = 0; s2 < kSlices; ++s2) {
+      total += part[s2][tid];
+      b += before[s2][tid];
+    }
+    cnt[tid] = total;
+    tot[tid] = b;
+  }
+  __syncthreads();
+  if (tid < 32) warp_padded_scan(cnt, off, E, bm, tid);
+  __syncthreads();
+  if (tid < E) run[tid] = off[tid] + tot[tid];
+  // this block's share of the layout: padding inside experts' last blocks,
+  // the tail past the padded total, the block experts
+  if (c == 0 && tid == 0) *ntpp = off[E];
+  for (int e2 = c; e2 < E; e2 += gridDim.x)
+    for (int p = off[e2] + cnt[e2] + tid; p < off[e2 + 1]; p += kScatterThreads) sorted_ids[p] = S;
+  for (int p = off[E] + c * kScatterThreads + tid; p < P_max; p += gridDim.x * kScatterThreads) sorted_ids[p] = S;
+  for (int b = c * kScatterThreads + tid; b < P_max / bm; b += gridDim.x * kScatterThreads)
+    expert_ids[b] = block_expert(off, E, b * bm);
   __syncthreads();
   const int end = min(S, (c + 1) * kChunk);
   for (int base = c * kChunk; base < end; base += kScatterThreads) {
-    const int s = base + threadIdx.x;
-    const int e = s < end ? load_expert(ids, s, S, E, nullptr) : -1;
-    scatter_round<kWarps>(e, s, wcnt, run, tot, E, sorted_ids, inv_pos);
+    const int s = base + tid;
+    const int ex = s < end ? load_expert(ids, s, S, E, nullptr) : -1;
+    scatter_round<kWarps>(ex, s, wcnt, run, tot, E, sorted_ids, inv_pos);
   }
 }
 
@@ -157,16 +158,13 @@ cudaError_t launch_align(const int32_t* topk_ids, int S, int E, int block_m, int
   }
   const int nchunks = align_num_chunks(S);
   int32_t* counts = ws;
-  int32_t* bases = ws + static_cast<size_t>(nchunks) * E;
   cudaError_t err = launch_pdl(align_count_kernel, dim3(nchunks), dim3(kChunkThreads), 0, stream, topk_ids, S, E,
                                counts, status);
   if (err != cudaSuccess) return err;
-  err = launch_pdl(align_scan_kernel, dim3(1), dim3(1024), 0, stream, static_cast<const int32_t*>(counts), nchunks,
-                   S, E, block_m, P_max, bases, sorted_ids, expert_ids, ntpp);
-  if (err != cudaSuccess) return err;
-  err = launch_pdl(align_scatter_kernel, dim3(nchunks), dim3(kScatterThreads), 0, stream, topk_ids, S, E,
-                   static_cast<const int32_t*>(bases), sorted_ids, inv_pos);
-  *launches += 3;
+  err = launch_pdl(align_place_kernel, dim3(nchunks), dim3(kScatterThreads), 0, stream, topk_ids,
+                   static_cast<const int32_t*>(counts), nchunks, S, E, block_m, P_max, sorted_ids, expert_ids, ntpp,
+                   inv_pos);
+  *launches += 2;
   return err;
 }
 

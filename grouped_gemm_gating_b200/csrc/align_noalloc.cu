@@ -8,8 +8,8 @@
 // the device and break the capture), and plugins whose host framework owns
 // every allocation.  Such callers cannot provide moe_align's workspace.
 //
-// The multi-block align path needs per-chunk expert counts and bases; here
-// they live in a file-scope static __device__ array of fixed size, which
+// The multi-block align path needs per-chunk expert counts; here they live
+// in a file-scope static __device__ array of fixed size, which
 // every GPU that loads this library holds until the process exits.
 #include <cuda.h>
 
@@ -23,8 +23,8 @@ void record_launches(int n);
 
 namespace {
 
-// 256 Ki int32 = 1 MiB: counts and bases of ceil(T*k / 2048) chunks x E
-// experts, i.e. ceil(T*k / 2048) * E <= 131072.
+// 256 Ki int32 = 1 MiB: counts of ceil(T*k / 2048) chunks x E experts,
+// i.e. ceil(T*k / 2048) * E <= 262144.
 constexpr size_t kScratchInts = 262144;
 static __device__ __align__(256) int32_t g_align_scratch[kScratchInts];
 
@@ -105,8 +105,8 @@ extern "C" MOE_API moe_status moe_align_noalloc(const int32_t* topk_ids, int T, 
   const int S = T * k;
   const int64_t P_max = moe_max_padded(T, k, E, block_m);
   int launches = 0;
-  // The count kernel overwrites every count it owns and the scan kernel
-  // every base, so no part of the scratch has to start at zero.
+  // The count kernel overwrites every count it owns, so no part of the
+  // scratch has to start at zero.
   cudaError_t err = moe::launch_align(topk_ids, S, E, block_m, static_cast<int>(P_max), sorted_token_ids,
                                       expert_ids, num_tokens_post_padded, inv_pos, ws, dev_status,
                                       reinterpret_cast<cudaStream_t>(stream), &launches);

@@ -291,7 +291,7 @@ size_t moe_align_workspace_size(int T, int k, int E) {
   const int64_t S = static_cast<int64_t>(T) * k;
   if (S >= (int64_t(1) << 30)) return 0;
   if (moe::align_uses_single_block(static_cast<int>(S))) return 0;
-  return static_cast<size_t>(moe::align_num_chunks(static_cast<int>(S))) * E * 2 * sizeof(int32_t);
+  return static_cast<size_t>(moe::align_num_chunks(static_cast<int>(S))) * E * sizeof(int32_t);  // per-chunk counts
 }
 
 size_t moe_workspace_size(int T, int d, int F, int E, int k, int block_m, moe_act act, int n_shared) {

@@ -298,7 +298,7 @@ MOE_API moe_status moe_layer_fp8(const float* logits, int T, int E, int k,
  * graph, a plugin whose host framework owns every allocation) cannot supply
  * moe_align's workspace; this entry point keeps the multi-block path's
  * scratch in a fixed 1 MiB static device array instead.
- *   Limit: ceil(T*k / 2048) * E <= 131072 (e.g. T*k <= 2^21 at E = 128);
+ *   Limit: ceil(T*k / 2048) * E <= 262144 (e.g. T*k <= 2^22 at E = 128);
  *   larger problems return MOE_ERR_UNSUPPORTED and launch nothing.
  *   Every GPU that loads the library holds the 1 MiB until the process exits.
  *   The first call on a device looks up the array's device address (one

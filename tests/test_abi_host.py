@@ -65,7 +65,7 @@ def test_workspace_sizes(lib):
     assert M.moe_workspace_size(T, d + 32, F, E, k, bm, M.ACT_SWIGLU, 0) == 0   # d % 64
     assert M.moe_workspace_size(T, d, F, 300, k, bm, M.ACT_SWIGLU, 0) == 0      # E > 256
     assert M.moe_align_workspace_size(3, 8, 128) == 0                           # single block
-    assert M.moe_align_workspace_size(16384, 8, 128) == (131072 // 2048) * 128 * 8
+    assert M.moe_align_workspace_size(16384, 8, 128) == (131072 // 2048) * 128 * 4
 
 
 def test_status_strings(lib):

@@ -42,8 +42,8 @@ def _no_alloc(ids, E, bm, status):
 
 
 # the first case fills the static scratch exactly: ceil(T*k / 2048) * E =
-# 1024 * 128 = 131072 chunk x expert entries
-@pytest.mark.parametrize("T,E,k,bm", [(262144, 128, 8, 128), (16384, 128, 8, 128), (9000, 64, 2, 16),
+# 2048 * 128 = 262144 chunk x expert entries
+@pytest.mark.parametrize("T,E,k,bm", [(524288, 128, 8, 128), (16384, 128, 8, 128), (9000, 64, 2, 16),
                                       (5000, 256, 8, 64), (3, 128, 8, 16)])
 def test_noalloc_align_matches_workspace_align_twice(T, E, k, bm):
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -56,8 +56,8 @@ def test_noalloc_align_matches_workspace_align_twice(T, E, k, bm):
             assert np.array_equal(a, b), f"call {call}: {name} differs"
 
 
-@pytest.mark.parametrize("T,k,E", [((1 << 18) + 1, 8, 128),   # one slot past the limit: 1025 * 128 entries
-                                   (1 << 18, 16, 256)])       # ceil(T*k/2048) * E = 524288 > 131072
+@pytest.mark.parametrize("T,k,E", [((1 << 19) + 1, 8, 128),   # one slot past the limit: 2049 * 128 entries
+                                   (1 << 18, 16, 256)])       # ceil(T*k/2048) * E = 524288 > 262144
 def test_noalloc_align_rejects_sizes_beyond_the_static_scratch(T, k, E):
     ids = torch.zeros((1, 1), dtype=torch.int32, device="cuda")
     lib = M.load_library()
