@@ -63,7 +63,7 @@ METRIC = "MoE layer TFLOPS and tokens/s on 1 B200; % of bf16 tensor peak / HBM r
 # entry is removed whenever the kernel changes after its capture.
 NCU_TRAFFIC = {
     ("decode", "fused_expert"): 201_748_736,
-    ("zipf", "gate_up_gemm"): None,
+    ("zipf", "gate_up_gemm"): 1_549_468_416,
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
