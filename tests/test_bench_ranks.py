@@ -94,3 +94,52 @@ def test_algorithmic_counts_the_shared_expert():
     a = bench.algorithmic(cfg, ids)
     assert a["flops_total"] == a["flops_routed"] + 2 * cfg.T * 3 * cfg.d * cfg.F
     assert a["weight_bytes"] == (cfg.E + 1) * (2 * cfg.F * cfg.d + cfg.d * cfg.F) * 2
+
+
+def test_roofline_of_a_tensor_bound_kernel_recomputes_against_the_burst_peak():
+    """frac = algorithmic FLOPs / per-launch time / burst bf16 peak; the
+    sustained fraction beside it; the DRAM traffic ratio from the stored
+    ncu figure."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+
+    import bench
+    from grouped_gemm_gating_b200 import workloads as W
+    cfg = W.CONFIGS["zipf"]
+    ids = (np.arange(cfg.T * cfg.k, dtype=np.int32) % 120).reshape(cfg.T, cfg.k)
+    alg = bench.algorithmic(cfg, ids)
+    peaks = {"hbm_gbs": 6534.8, "bf16_tflops": 1649.5, "bf16_tflops_sustained": 1390.6}
+    stages = {"gate_up_gemm": (7.5, 10), "down_gemm": (4.8, 10), "fused_expert": (0.0, 0)}
+    r = bench.roofline(cfg, alg, stages, total_ms=13.0, steps=10, launches_per_step=6, rotate=True, peaks=peaks,
+                       peak_src="measured")
+    fl = alg["gate_up_gemm"][0]
+    assert r["bound"] == "tensor" and r["kernel"] == "gate_up_gemm" and r["peak"] == 1649.5
+    assert r["per_launch_us"] == pytest.approx(750.0)
+    assert r["achieved"] == pytest.approx(fl / 750e-6 / 1e12, rel=1e-4)
+    assert r["frac"] == pytest.approx(r["achieved"] / 1649.5, abs=1e-4)
+    assert r["frac_of_sustained_peak"] == pytest.approx(r["achieved"] / 1390.6, abs=1e-4)
+    assert r["traffic"] == bench.NCU_TRAFFIC[("zipf", "gate_up_gemm")]
+    assert r["traffic_vs_algorithmic"] == pytest.approx(r["traffic"] / alg["gate_up_gemm"][1], abs=1e-3)
+
+
+def test_roofline_of_the_one_kernel_decode_step_is_hbm_bound():
+    """The decode step is one kernel: its launch time is the back-to-back
+    step time, its numerator the streamed bytes, its denominator the
+    measured copy bandwidth (and the nominal 8 TB/s beside it)."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+
+    import bench
+    from grouped_gemm_gating_b200 import workloads as W
+    cfg = W.CONFIGS["decode"]
+    ids = (np.arange(cfg.T * cfg.k, dtype=np.int32) % 21).reshape(cfg.T, cfg.k)
+    alg = bench.algorithmic(cfg, ids)
+    peaks = {"hbm_gbs": 6534.8, "bf16_tflops": 1649.5, "bf16_tflops_sustained": 1390.6}
+    stages = {"gate_up_gemm": (0.0, 0), "down_gemm": (0.0, 0), "fused_expert": (0.46, 10)}
+    r = bench.roofline(cfg, alg, stages, total_ms=0.42, steps=10, launches_per_step=1, rotate=True, peaks=peaks,
+                       peak_src="measured")
+    assert r["bound"] == "hbm" and r["kernel"] == "fused_expert" and r["peak"] == 6534.8
+    assert r["per_launch_us"] == pytest.approx(42.0)
+    assert r["achieved"] == pytest.approx(alg["fused_bytes"] / 42e-6 / 1e9, rel=1e-4)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6534.8, abs=1e-4)
+    assert r["frac_of_nominal_hbm"] == pytest.approx(r["achieved"] / bench.NOMINAL_HBM_GBS, abs=1e-4)
