@@ -10,8 +10,10 @@
 // weight rows.  Each K step stages the 256 weight rows once (TMA) and the
 // unit's token rows (cp.async gather, up to 256), and the MMA thread issues
 // two M = 128, N = 256 MMAs that share the weight operand: per SM a 64-wide
-// K step moves 64 KB for two 128 x 256 products instead of 48 KB for one,
-// which is what bounds the one-block kernel when the K loop streams from L2.
+// K step writes 64 KB into shared memory (and the MMAs read 96 KB) for two
+// 128 x 256 products, against 48 KB (and 48 KB) for one in the one-block
+// kernel.  Shared-memory traffic, staging writes plus operand reads, is what
+// bounds these single-CTA GEMMs.
 // The two accumulators fill all 512 TMEM columns, so the accumulator is not
 // double-buffered: at the end of a tile the eight epilogue warps drain block
 // 0's accumulator, then block 1's; the MMA thread starts the next tile's
